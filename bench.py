@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE-layer forward (tokens/s) on 1..N B200s.
+
+A step is one full layer forward (router -> top-k -> permute -> grouped SwiGLU
+FFN -> combine) over one batch of synthetic tokens. Default workload: the
+decode-shaped layer (H=2048, E=128, top-8, I=768, MXFP4 experts, bf16
+activations, uniform routing) at T=64 tokens; T=1, T=8 and the prefill-shaped
+NVFP4 layer (T=4096, Zipf-skewed routing) are reported alongside under "extra".
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and a device
+synchronise, timed with CUDA events on the launching stream, max over ranks.
+Every step replays a CUDA graph of the layer on one of NSETS copies of the
+expert weights (and one of NSETS activation batches), so consecutive steps
+read weights that are not in L2 ("inputs larger than L2").
+Multi-GPU: replicas only (the layer has no exchange step); value = tokens of
+all ranks / max time.
+
+--impl reference times the CPU oracle (the plain C reference of the same math)
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+NSETS = 16
+L2_BYTES = 126 * 2**20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------- workload
+
+
+def active_expert_bytes(idx: torch.Tensor, layer) -> int:
+    """Bytes of the experts that received at least one token (codes + scales)."""
+    E = layer.E
+    used = torch.bincount(idx.reshape(-1).long(), minlength=E) > 0
+    per = synthetic.expert_bytes(layer.fmt, layer.H, layer.I)
+    return int(used.sum().item()) * per
+
+
+class LayerBench:
+    """One layer configuration: NSETS weight copies, NSETS token batches, a graph per pair."""
+
+    def __init__(self, moe, cfg: str, T: int, device, seed: int = 0, nsets: int = NSETS):
+        self.moe, self.cfg, self.T, self.dev = moe, cfg, T, device
+        c = synthetic.CONFIGS[cfg]
+        self.k, self.y32 = c["k"], c["y_fp32"]
+        base = synthetic.make_layer(cfg, seed, device=device)
+        self.layer = base
+        self.sets = [base] + [self._clone(base) for _ in range(nsets - 1)]
+        self.experts = [moe.Experts.from_layer(s) for s in self.sets]
+        self.xs = [synthetic.make_tokens(T, base.H, seed=100 + i, device=device) for i in range(nsets)]
+        self.ws = torch.empty(moe.moe_workspace_size(T, base.H, base.I, base.E, self.k, self.y32),
+                              dtype=torch.uint8, device=device)
+        self.out = torch.empty(T, base.H, dtype=torch.bfloat16, device=device)
+        self.idx = [torch.empty(T, self.k, dtype=torch.int32, device=device) for _ in range(nsets)]
+        self.w = [torch.empty(T, self.k, dtype=torch.float32, device=device) for _ in range(nsets)]
+        self.graphs = None
+
+    @staticmethod
+    def _clone(l):
+        c = l.to(l.wr.device)
+        for n in ("w13", "w2", "w13_scale", "w2_scale"):
+            t = getattr(c, n)
+            if t is not None:
+                setattr(c, n, t.clone())
+        return c
+
+    def call(self, i: int):
+        j = i % len(self.sets)
+        s = self.sets[j]
+        self.moe.moe_layer_forward(self.xs[j], s.wr, self.k, self.experts[j], bias=s.bias, y_fp32=self.y32,
+                                   ws=self.ws, out=self.out, idx_out=self.idx[j], w_out=self.w[j])
+
+    def capture(self):
+        self.graphs = []
+        st = torch.cuda.Stream(self.dev)
+        st.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(st):
+            for j in range(len(self.sets)):   # warm the launch paths before capture
+                self.call(j)
+        torch.cuda.current_stream(self.dev).wait_stream(st)
+        torch.cuda.synchronize(self.dev)
+        for j in range(len(self.sets)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.call(j)
+            self.graphs.append(g)
+        torch.cuda.synchronize(self.dev)
+
+    def step(self, i: int):
+        self.graphs[i % len(self.graphs)].replay()
+
+    def algorithmic_bytes(self, i: int) -> int:
+        """Router weights + active experts + x in + out (SURVEY 8(d) definition)."""
+        j = i % len(self.sets)
+        s = self.sets[j]
+        router = s.wr.numel() * s.wr.element_size()
+        return router + active_expert_bytes(self.idx[j], s) + 2 * self.T * s.H * 2
+
+    def flops(self) -> float:
+        s = self.layer
+        return 2.0 * self.T * s.H * s.E + self.T * self.k * 6.0 * s.H * s.I
+
+
+def time_steps(fn, K: int, W: int, device, barrier=None):
+    for i in range(W):
+        fn(i)
+    torch.cuda.synchronize(device)
+    if barrier:
+        barrier()
+    st = torch.cuda.current_stream(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for i in range(K):
+        fn(W + i)
+    e1.record(st)
+    torch.cuda.synchronize(device)
+    if barrier:
+        barrier()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def time_ffn_only(moe, lb: LayerBench, K: int, W: int, device):
+    """Average duration of the grouped FFN call (gate/up + down launches) on the same data."""
+    T, k = lb.T, lb.k
+    P = T * k
+    j0 = 0
+    # permuted operands per set, prepared once (untimed)
+    prep = []
+    for j in range(len(lb.sets)):
+        off, sp, pr, xp = moe.moe_permute(lb.idx[j], lb.layer.E, lb.xs[j])
+        prep.append((xp, off))
+    y = torch.empty(P, lb.layer.H, dtype=torch.float32 if lb.y32 else torch.bfloat16, device=device)
+    ws = torch.empty(P * lb.layer.I * 2 + 256, dtype=torch.uint8, device=device)
+
+    def fn(i):
+        j = i % len(prep)
+        moe.moe_grouped_ffn(prep[j][0], prep[j][1], lb.experts[j], y_fp32=lb.y32, ws=ws)
+
+    sec = time_steps(fn, K, W, device)
+    nbytes = []
+    for j in range(len(lb.sets)):
+        nbytes.append(active_expert_bytes(lb.idx[j], lb.sets[j]) + 2 * P * lb.layer.H * 2)
+    # average algorithmic bytes over the rotation, weighted like the timed calls
+    avg_bytes = sum(nbytes[(W + i) % len(nbytes)] for i in range(K)) / K
+    return sec / K, avg_bytes
+
+
+def source_sha():
+    h = hashlib.sha256()
+    for f in ("ffn_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "expert_ffn_layer_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(key: str):
+    p = os.path.join(ROOT, "profiles", "ffn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("src_sha") != source_sha():
+            return None
+        return d.get(key)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------------------------- arms
+
+
+def cpu_oracle_tokens_per_s(cfg: str, T: int, budget_s: float = 12.0):
+    import oracle
+
+    L = synthetic.make_layer(cfg, 0)
+    xs = [synthetic.make_tokens(T, L.H, seed=100 + i) for i in range(4)]
+    n = 0
+    t0 = time.time()
+    while True:
+        oracle.layer_forward(xs[n % len(xs)], L)
+        n += 1
+        if time.time() - t0 > budget_s:
+            break
+    dt = time.time() - t0
+    return n * T / dt, oracle.threads(), f"{n} full {cfg} layer forward(s) at T={T} ({dt:.1f} s)"
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    tps, cores, sample = cpu_oracle_tokens_per_s("decode", 64, budget_s=max(5.0, 2.0 * args.steps))
+    line = {
+        "impl": "reference", "metric": "moe_layer_tokens_per_s", "value": tps, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 64 / tps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": "decode-shaped MoE layer, MXFP4 experts, T=64",
+                                        "H": 2048, "E": 128, "k": 8, "I": 768, "T": 64},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, device):
+    import expert_ffn_layer_top_b200 as moe
+
+    barrier = None
+    if world > 1:
+        import torch.distributed as dist
+
+        def barrier():
+            dist.barrier(device_ids=[device.index])
+
+    hbm, bf16_tf, peak_kind = _peaks()
+    lb = LayerBench(moe, "decode", 64, device)
+    lb.capture()
+    extra = {}
+    launches_per_step = 9   # router 2 + permute 4 + FFN 2 + combine 1
+    with ClockSampler(device.index) as clk:
+        sec = time_steps(lb.step, args.steps, args.warmup, device, barrier)
+    clocks = clk.summary()
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([sec], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        sec = float(t.item())
+    tokens = lb.T * args.steps * world
+    value = tokens / sec
+    ms = sec / args.steps * 1e3
+    # layer roofline context (algorithmic bytes of the steps just timed)
+    alg = [lb.algorithmic_bytes(args.warmup + i) for i in range(min(args.steps, NSETS))]
+    layer_gbs = (sum(alg) / len(alg)) / (ms * 1e-3) / 1e9
+
+    # dominant kernel: the grouped FFN call, timed alone with events on the same rotation
+    ffn_s, ffn_bytes = time_ffn_only(moe, lb, max(args.steps, 20), args.warmup, device)
+    achieved = ffn_bytes / ffn_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic_for("decode64_bytes_per_call"), "kernel": "grouped SwiGLU FFN (ffn_tc_kernel up + down)",
+                "peak_kind": peak_kind, "layer_achieved_gbs": layer_gbs}
+
+    # end to end through the C ABI with host buffers: pinned x in, out back, every step
+    xh = [x.cpu().pin_memory() for x in lb.xs]
+    oh = torch.empty(lb.T, lb.layer.H, dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(lb.xs[0])
+
+    def e2e_step(i):
+        j = i % NSETS
+        xd.copy_(xh[j], non_blocking=True)
+        s = lb.sets[j]
+        moe.moe_layer_forward(xd, s.wr, lb.k, lb.experts[j], bias=s.bias, ws=lb.ws, out=lb.out)
+        oh.copy_(lb.out, non_blocking=True)
+
+    e2e_sec = time_steps(e2e_step, args.steps, args.warmup, device, barrier)
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([e2e_sec], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_sec = float(t.item())
+    e2e = {"value": tokens / e2e_sec, "unit": "tokens/s", "h2d_bytes_per_step": lb.T * lb.layer.H * 2,
+           "d2h_bytes_per_step": lb.T * lb.layer.H * 2}
+
+    # side measurements (not the headline): other batch sizes and the prefill-shaped layer
+    if not args.quick:
+        for cfg, T in (("decode", 1), ("decode", 8), ("prefill", 4096)):
+            b = lb if (cfg == "decode" and T == 64) else LayerBench(moe, cfg, T, device,
+                                                                     nsets=NSETS if cfg == "decode" else 4)
+            b.capture()
+            s = time_steps(b.step, max(10, args.steps // 2), args.warmup, device, barrier)
+            ms_b = s / max(10, args.steps // 2) * 1e3
+            n_alg = [b.algorithmic_bytes(args.warmup + i) for i in range(min(8, len(b.sets)))]
+            gbs = sum(n_alg) / len(n_alg) / (ms_b * 1e-3) / 1e9
+            extra[f"{cfg}_T{T}"] = {"tokens_per_s": T / (ms_b * 1e-3) * world, "ms_per_layer": ms_b,
+                                    "layer_gbs": gbs, "frac_hbm": gbs / hbm,
+                                    "tflops": b.flops() / (ms_b * 1e-3) / 1e12,
+                                    "frac_bf16_peak": b.flops() / (ms_b * 1e-3) / 1e12 / bf16_tf}
+            del b
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tps, cores, sample = cpu_oracle_tokens_per_s("decode", 64)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    line = {
+        "metric": "moe_layer_tokens_per_s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 math on MXFP4 weights",
+        "data": "synthetic (seeded; weights N(0,0.02) quantised, x N(0,1))",
+        "config": {"workload": "decode-shaped MoE layer, MXFP4 experts, T=64", "H": 2048, "E": 128, "k": 8,
+                   "I": 768, "T": 64, "parallelism": f"replicas x{world}",
+                   "l2": f"{NSETS} rotating weight copies + activation batches (weights touched per step > L2)"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks, "extra": extra,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--quick", action="store_true", help="headline workload only")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

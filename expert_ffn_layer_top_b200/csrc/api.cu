@@ -1,0 +1,371 @@
+// C-ABI entry points of libmoe (declared in include/moe.h): argument checks,
+// workspace carving, TMA descriptor construction and kernel launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+static thread_local char t_err[512] = "no error";
+
+moe_status set_error(moe_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+moe_status set_cuda_error(cudaError_t e, const char *what) {
+    snprintf(t_err, sizeof(t_err), "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+    return e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA;
+}
+
+int num_sms(int device) {
+    static int cache[64] = {0};
+    if (device < 0 || device >= 64) return 148;
+    if (!cache[device]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || v <= 0) v = 148;
+        cache[device] = v;
+    }
+    return cache[device];
+}
+
+static int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return 0;
+    return d;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                      const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled_t encode_fn() {
+    static PFN_encodeTiled_t fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled_t>(p);
+    });
+    return fn;
+}
+
+moe_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+                     const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle sw) {
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return set_error(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (reinterpret_cast<uintptr_t>(base) & 15) return set_error(MOE_ERR_INVALID_ARG, "TMA base not 16-byte aligned");
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) {
+            s[i] = strides_bytes[i];
+            if (s[i] % 16) return set_error(MOE_ERR_INVALID_ARG, "TMA stride %llu not a multiple of 16",
+                                            (unsigned long long)s[i]);
+        }
+    }
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(base), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(MOE_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ helpers
+
+static int elem_bytes_x2(int fmt) {   // bytes per element, times 2
+    return fmt == MOE_BF16 ? 4 : fmt == MOE_FP8_E4M3_K128 ? 2 : 1;
+}
+
+struct Strides {
+    int64_t w13, w13s, w2, w2s;
+};
+
+static Strides default_strides(const moe_experts &x) {
+    Strides s;
+    const int64_t r13 = 2LL * x.I, r2 = x.H;
+    s.w13 = x.w13_estride ? x.w13_estride : r13 * x.H * elem_bytes_x2(x.fmt) / 2;
+    s.w13s = x.w13s_estride ? x.w13s_estride : r13 * scale_rowbytes(x.fmt, x.H);
+    s.w2 = x.w2_estride ? x.w2_estride : r2 * x.I * elem_bytes_x2(x.fmt) / 2;
+    s.w2s = x.w2s_estride ? x.w2s_estride : r2 * scale_rowbytes(x.fmt, x.I);
+    return s;
+}
+
+static moe_status check_experts(const moe_experts *x) {
+    if (!x) return set_error(MOE_ERR_INVALID_ARG, "experts is NULL");
+    if (x->fmt < MOE_BF16 || x->fmt > MOE_NVFP4) return set_error(MOE_ERR_UNSUPPORTED, "unknown weight format %d", x->fmt);
+    if (x->E <= 0 || x->E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d outside 1..%d", x->E, kMaxExperts);
+    if (x->H <= 0 || x->I <= 0 || x->H % 128 || x->I % 128)
+        return set_error(MOE_ERR_UNSUPPORTED, "H=%d and I=%d must be positive multiples of 128", x->H, x->I);
+    if (!x->w13 || !x->w2) return set_error(MOE_ERR_INVALID_ARG, "expert weights are NULL");
+    if (x->fmt != MOE_BF16 && (!x->w13_scale || !x->w2_scale))
+        return set_error(MOE_ERR_INVALID_ARG, "scale planes are NULL");
+    if (x->fmt == MOE_NVFP4 && (!x->w13_tscale || !x->w2_tscale))
+        return set_error(MOE_ERR_INVALID_ARG, "NVFP4 tensor scales are NULL");
+    const Strides s = default_strides(*x);
+    if ((s.w13 | s.w2 | s.w13s | s.w2s) & 15) return set_error(MOE_ERR_INVALID_ARG, "expert strides not 16-byte aligned");
+    const uintptr_t a = reinterpret_cast<uintptr_t>(x->w13) | reinterpret_cast<uintptr_t>(x->w2) |
+                        reinterpret_cast<uintptr_t>(x->w13_scale) | reinterpret_cast<uintptr_t>(x->w2_scale);
+    if (a & 15) return set_error(MOE_ERR_INVALID_ARG, "expert arrays not 16-byte aligned");
+    return MOE_OK;
+}
+
+// Build the weight tensor map of one phase: 3D (K bytes|elements, rows, entries).
+static moe_status weight_tmap(CUtensorMap *m, int fmt, const void *base, int rows, int K, int64_t estride,
+                              int entries) {
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    CUtensorMapDataType dt;
+    CUtensorMapSwizzle sw;
+    if (fmt == MOE_BF16) {
+        dt = CU_TENSOR_MAP_DATA_TYPE_UINT16;
+        dims[0] = K;
+        strides[0] = 2ULL * K;
+        box[0] = 64;
+        sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    } else if (fmt == MOE_FP8_E4M3_K128) {
+        dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+        dims[0] = K;
+        strides[0] = K;
+        box[0] = 128;
+        sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    } else {
+        dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+        dims[0] = K / 2;
+        strides[0] = K / 2;
+        box[0] = 64;
+        sw = CU_TENSOR_MAP_SWIZZLE_64B;
+    }
+    dims[1] = rows;
+    dims[2] = entries;
+    strides[1] = estride;
+    box[1] = 64;
+    box[2] = 1;
+    return make_tmap(m, dt, 3, base, dims, strides, box, sw);
+}
+
+static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, int BN) {
+    uint64_t dims[2] = {(uint64_t)K, (uint64_t)(rows > 0 ? rows : 1)};
+    uint64_t strides[1] = {2ULL * K};
+    uint32_t box[2] = {64, (uint32_t)BN};
+    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static size_t ffn_ws_bytes(int n_rows, int I) { return align_up((size_t)n_rows * I * 2, 256); }
+
+// grouped FFN with explicit h buffer
+static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *x,
+                                   void *y_perm, int y_is_fp32, void *h, cudaStream_t st) {
+    if (n_rows == 0) return MOE_OK;
+    const Strides s = default_strides(*x);
+    const int nent = x->expert_map ? (int)(x->n_entries > 0 ? x->n_entries : x->E) : x->E;
+    const int BN = choose_bn(n_rows, x->E);
+    const int nsm = num_sms(current_device());
+    CUtensorMap wmap, bmap;
+    moe_status r;
+    FfnParams p;
+    memset(&p, 0, sizeof(p));
+    p.offsets = offsets;
+    p.expert_map = x->expert_map;
+    p.E = x->E;
+    p.H = x->H;
+    p.I = x->I;
+    p.n_rows = n_rows;
+    // ---- gate/up + SwiGLU
+    if ((r = weight_tmap(&wmap, x->fmt, x->w13, 2 * x->I, x->H, s.w13, nent)) != MOE_OK) return r;
+    if ((r = act_tmap(&bmap, x_perm, n_rows, x->H, BN)) != MOE_OK) return r;
+    p.K = x->H;
+    p.m_tiles = x->I / 64;
+    p.scale_base = reinterpret_cast<const uint8_t *>(x->w13_scale);
+    p.s_estride = s.w13s;
+    p.s_rowbytes = scale_rowbytes(x->fmt, x->H);
+    p.tscale = x->w13_tscale;
+    p.out = h;
+    p.out_fp32 = 0;
+    if ((r = launch_ffn_phase(kPhaseUp, x->fmt, BN, wmap, bmap, p, nsm, st)) != MOE_OK) return r;
+    // ---- down projection
+    if ((r = weight_tmap(&wmap, x->fmt, x->w2, x->H, x->I, s.w2, nent)) != MOE_OK) return r;
+    if ((r = act_tmap(&bmap, h, n_rows, x->I, BN)) != MOE_OK) return r;
+    p.K = x->I;
+    p.m_tiles = x->H / 128;
+    p.scale_base = reinterpret_cast<const uint8_t *>(x->w2_scale);
+    p.s_estride = s.w2s;
+    p.s_rowbytes = scale_rowbytes(x->fmt, x->I);
+    p.tscale = x->w2_tscale;
+    p.out = y_perm;
+    p.out_fp32 = y_is_fp32;
+    return launch_ffn_phase(kPhaseDown, x->fmt, BN, wmap, bmap, p, nsm, st);
+}
+
+// workspace layout of moe_layer_forward
+struct LayerWs {
+    size_t router, idx, w, offsets, sorted, pair_row, perm, x_perm, h, y, total;
+};
+
+static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
+    LayerWs L;
+    const size_t P = (size_t)T * k;
+    size_t o = 0;
+    L.router = o; o += align_up(router_ws_bytes(T, H, E), 256);
+    L.idx = o; o += align_up(P * 4, 256);
+    L.w = o; o += align_up(P * 4, 256);
+    L.offsets = o; o += align_up((size_t)(E + 1) * 4, 256);
+    L.sorted = o; o += align_up(P * 4, 256);
+    L.pair_row = o; o += align_up(P * 4, 256);
+    L.perm = o; o += align_up(permute_ws_bytes(T, k, E), 256);
+    L.x_perm = o; o += align_up(P * H * 2, 256);
+    L.h = o; o += ffn_ws_bytes((int)P, I);
+    L.y = o; o += align_up(P * H * (y32 ? 4 : 2), 256);
+    L.total = o;
+    return L;
+}
+
+moe_status cache_resolve_and_map(struct expert_cache *c, int layer, const int32_t *idx, int T, int k,
+                                 const moe_experts *shape, moe_experts *dev_view, cudaStream_t st);
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_last_error_string(void) { return t_err; }
+
+const char *moe_version(void) { return "libmoe 0.1 (sm_100a)"; }
+
+moe_status moe_device_error(int *code) {
+    if (!code) return set_error(MOE_ERR_INVALID_ARG, "code is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return set_cuda_error(e, "device synchronize");
+    int v = 0, z = 0;
+    e = cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_dev_error, &z, sizeof(int));
+    if (e != cudaSuccess) return set_cuda_error(e, "device error word");
+    *code = v;
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32) {
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return 0;
+    return layer_ws(T, H, I, E, k, y_is_fp32).total;
+}
+
+moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
+                          int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+    if (T < 0 || H <= 0 || H % 8) return set_error(MOE_ERR_INVALID_ARG, "bad T=%d or H=%d", T, H);
+    if (E < 1 || E > kMaxRouterExperts || k < 1 || k > kMaxTopK || k > E)
+        return set_error(MOE_ERR_UNSUPPORTED, "router needs 1<=k<=%d, k<=E<=%d (E=%d k=%d)", kMaxTopK,
+                         kMaxRouterExperts, E, k);
+    if (T == 0) return MOE_OK;
+    if (!x || !wr || !idx || !w || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    return launch_router(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, logits, ws, ws_bytes,
+                         num_sms(current_device()), (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+                       int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+    if (T < 0 || k < 1 || k > kMaxTopK || E < 1 || E > kMaxExperts)
+        return set_error(MOE_ERR_INVALID_ARG, "bad T/k/E (%d %d %d)", T, k, E);
+    if (!offsets) return set_error(MOE_ERR_INVALID_ARG, "offsets is NULL");
+    if (T > 0 && (!idx || !sorted_pair || !pair_row || (x_perm && !x) || !ws))
+        return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (x_perm && (H <= 0 || H % 8)) return set_error(MOE_ERR_INVALID_ARG, "H must be a positive multiple of 8");
+    if (x_perm && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(x_perm)) & 15))
+        return set_error(MOE_ERR_INVALID_ARG, "x and x_perm must be 16-byte aligned");
+    return launch_permute(idx, T, k, E, x, H, offsets, sorted_pair, pair_row, x_perm, ws, ws_bytes,
+                          (cudaStream_t)stream);
+}
+
+moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
+                           void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status r = check_experts(experts);
+    if (r != MOE_OK) return r;
+    if (n_rows < 0) return set_error(MOE_ERR_INVALID_ARG, "n_rows < 0");
+    if (n_rows == 0) return MOE_OK;
+    if (!x_perm || !offsets || !y_perm || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (ws_bytes < ffn_ws_bytes(n_rows, experts->I)) return set_error(MOE_ERR_OOM, "FFN workspace too small");
+    if ((reinterpret_cast<uintptr_t>(x_perm) | reinterpret_cast<uintptr_t>(ws)) & 15)
+        return set_error(MOE_ERR_INVALID_ARG, "x_perm and ws must be 16-byte aligned");
+    return grouped_ffn_impl(x_perm, n_rows, offsets, experts, y_perm, y_is_fp32, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
+                          moe_stream_t stream) {
+    if (fmt < MOE_BF16 || fmt > MOE_NVFP4) return set_error(MOE_ERR_UNSUPPORTED, "unknown format %d", fmt);
+    const int kq = fmt == MOE_FP8_E4M3_K128 ? 128 : fmt == MOE_MXFP4 ? 32 : fmt == MOE_NVFP4 ? 16 : 8;
+    if (rows < 0 || K <= 0 || K % kq) return set_error(MOE_ERR_INVALID_ARG, "K=%d must be a multiple of %d", K, kq);
+    if (rows == 0) return MOE_OK;
+    if (!w || !out || (fmt != MOE_BF16 && !scale)) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return set_error(MOE_ERR_INVALID_ARG, "w and out must be 16-byte aligned");
+    return launch_dequant(fmt, w, scale, tscale, rows, K, out, (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
+                       int H, void *out, moe_stream_t stream) {
+    if (T < 0 || k < 1 || k > kMaxTopK || H <= 0 || H % 8) return set_error(MOE_ERR_INVALID_ARG, "bad T/k/H");
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !pair_row || !w || !out) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(y_perm) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return set_error(MOE_ERR_INVALID_ARG, "y_perm and out must be 16-byte aligned");
+    return launch_combine(y_perm, y_is_fp32, pair_row, w, T, k, H, out, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp32, const float *bias, int k,
+                             const moe_experts *experts, struct expert_cache *cache, int layer, int y_is_fp32,
+                             void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+    if (!experts) return set_error(MOE_ERR_INVALID_ARG, "experts is NULL");
+    const int E = experts->E, H = experts->H, I = experts->I;
+    if (T < 0) return set_error(MOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) return MOE_OK;
+    if (!cache) {
+        moe_status r = check_experts(experts);
+        if (r != MOE_OK) return r;
+    } else if (experts->E <= 0 || H % 128 || I % 128) {
+        return set_error(MOE_ERR_UNSUPPORTED, "bad layer shape");
+    }
+    if (!x || !wr || !out || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    const LayerWs L = layer_ws(T, H, I, E, k, y_is_fp32);
+    if (ws_bytes < L.total) return set_error(MOE_ERR_OOM, "workspace %zu < %zu bytes", ws_bytes, L.total);
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOE_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *b = reinterpret_cast<uint8_t *>(ws);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(b + L.idx);
+    float *w = w_out ? w_out : reinterpret_cast<float *>(b + L.w);
+    int32_t *offsets = reinterpret_cast<int32_t *>(b + L.offsets);
+    int32_t *sorted = reinterpret_cast<int32_t *>(b + L.sorted);
+    int32_t *prow = reinterpret_cast<int32_t *>(b + L.pair_row);
+    moe_status r = moe_route_topk(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router,
+                                  L.idx - L.router, stream);
+    if (r != MOE_OK) return r;
+    r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, b + L.x_perm, b + L.perm, L.x_perm - L.perm, stream);
+    if (r != MOE_OK) return r;
+    moe_experts view = *experts;
+    if (cache) {
+        r = cache_resolve_and_map(cache, layer, idx, T, k, experts, &view, st);
+        if (r != MOE_OK) return r;
+        if ((r = check_experts(&view)) != MOE_OK) return r;
+    }
+    r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+    if (r != MOE_OK) return r;
+    return moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Gate-weighted combine (un-permute): out[t] = sum_j w[t,j] * y_perm[pair_row[t*k+j]],
+// accumulated in fp32 in order of j and rounded once to bf16. The pages give no
+// combine formula; this is the standard weighted sum of the k expert outputs.
+// One block per token, 8 channels (16-byte bf16 / 32-byte fp32 loads) per thread.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+template <bool Y32>
+__global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y_perm,
+                                                     const int32_t *__restrict__ pair_row,
+                                                     const float *__restrict__ w, int k, int H,
+                                                     __nv_bfloat16 *__restrict__ out) {
+    const int t = blockIdx.x;
+    __shared__ int rows[kMaxTopK];
+    __shared__ float ws[kMaxTopK];
+    if (threadIdx.x < k) {
+        rows[threadIdx.x] = pair_row[(int64_t)t * k + threadIdx.x];
+        ws[threadIdx.x] = w[(int64_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int64_t base = (int64_t)rows[j] * H + c;
+            const float wj = ws[j];
+            if (Y32) {
+                const float4 a = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(y_perm) + base);
+                const float4 b =
+                    *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(y_perm) + base + 4);
+                acc[0] += wj * a.x; acc[1] += wj * a.y; acc[2] += wj * a.z; acc[3] += wj * a.w;
+                acc[4] += wj * b.x; acc[5] += wj * b.y; acc[6] += wj * b.z; acc[7] += wj * b.w;
+            } else {
+                const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(y_perm) + base);
+                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(p2[i]);
+                    acc[2 * i] += wj * f.x;
+                    acc[2 * i + 1] += wj * f.y;
+                }
+            }
+        }
+        uint4 o;
+        __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o2[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(out + (int64_t)t * H + c) = o;
+    }
+}
+
+moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
+                          int H, void *out, cudaStream_t st) {
+    if (T == 0) return MOE_OK;
+    int threads = H / 8;
+    if (threads > 256) threads = 256;
+    threads = (threads + 31) / 32 * 32;
+    if (y_is_fp32)
+        combine_kernel<true><<<T, threads, 0, st>>>(y_perm, pair_row, w, k, H, reinterpret_cast<__nv_bfloat16 *>(out));
+    else
+        combine_kernel<false><<<T, threads, 0, st>>>(y_perm, pair_row, w, k, H, reinterpret_cast<__nv_bfloat16 *>(out));
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "combine launch");
+}
+
+}  // namespace moe

@@ -1,0 +1,70 @@
+// Internal declarations shared by the host-side translation units of libmoe.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;   // grouped FFN / permutation limit
+constexpr int kMaxRouterExperts = 256;
+constexpr int kMaxTopK = 16;
+constexpr int kPhaseUp = 0;
+constexpr int kPhaseDown = 1;
+
+struct FfnParams {
+    const int32_t *offsets;     // [E+1]
+    const int32_t *expert_map;  // nullable [E]
+    int E, H, I;
+    int K;                      // reduction dimension of this phase (H or I)
+    int m_tiles;                // I/64 (up) or H/128 (down)
+    int stages;                 // pipeline depth, set by the launcher
+    const uint8_t *scale_base;  // scale plane of this phase's tensor (nullable for bf16)
+    int64_t s_estride;          // bytes between experts in the scale plane
+    int s_rowbytes;             // scale bytes per weight row
+    const float *tscale;        // nvfp4 per-expert tensor scale, else nullable
+    void *out;                  // up: h bf16 [n_rows][I]; down: y [n_rows][H]
+    int out_fp32;
+    int n_rows;
+};
+
+// error reporting (thread-local message), defined in api.cu
+moe_status set_error(moe_status s, const char *fmt, ...);
+moe_status set_cuda_error(cudaError_t e, const char *what);
+
+int num_sms(int device);
+int choose_bn(int n_rows, int E);
+int scale_rowbytes(int fmt, int K);
+
+moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap,
+                            FfnParams p, int num_sms, cudaStream_t st);
+
+moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
+                          cudaStream_t st);
+
+// router (router.cu)
+size_t router_ws_bytes(int T, int H, int E);
+moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
+                         int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes, int nsm,
+                         cudaStream_t st);
+
+// permutation (permute.cu)
+size_t permute_ws_bytes(int T, int k, int E);
+moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+                          int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
+                          cudaStream_t st);
+
+// combine (combine.cu)
+moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
+                          int H, void *out, cudaStream_t st);
+
+// tensor maps (api.cu)
+moe_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+                     const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle sw);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace moe

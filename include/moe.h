@@ -1,0 +1,226 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) MoE-layer library (libmoe.so).
+ *
+ * One hot path: the forward pass of a mixture-of-experts layer over
+ * quantised experts, plus the device expert cache that lets an expert pool
+ * larger than device memory stream from pinned host memory.
+ *
+ * Sources. The pages describing the serving engine this layer comes from give
+ * the problem, not the kernels:
+ *   [P3] winzheng.com, "FreeToken ... 753B local inference MoE":
+ *        section "Why Now of All Times" - each token activates a few routed
+ *        experts per layer (top-k routing); most experts can stay in host
+ *        memory and be loaded on demand;
+ *        section "FreeToken's Three-Layer Mechanism" - double-buffered
+ *        streaming overlapping weight movement with compute, and a global
+ *        LRU expert cache reusing high-frequency experts.
+ *   [P4] aimodeling.com, "FreeToken: UC Berkeley Brings 753B GLM-5.2 MoE
+ *        Inference to Consumer Hardware": section "Three Engineering Cores"
+ *        (the same LRU cache and double-buffered streaming) and section
+ *        "Reported Numbers and Ecosystem Position" (expert formats MXFP4,
+ *        NVFP4, FP8 and BF16).
+ * The pages give no router, gating, FFN or combine formula; this library
+ * implements the standard top-k softmax SwiGLU MoE layer:
+ *   logits = x.Wr (+ bias), rounded once to fp32 from an fp64 sum;
+ *   idx = top-k logits (ties to the lower expert index);
+ *   w = softmax over the k selected logits;
+ *   y_p = W2_e . (silu(Wg_e . x_t) * (Wu_e . x_t)) for each pair p = (t, j);
+ *   out_t = sum_j w[t,j] y_(t,j).
+ *
+ * Conventions for every call:
+ *   - All pointers are device pointers unless marked "host".
+ *   - The caller owns every buffer passed in. The library allocates nothing on
+ *     the hot path; scratch comes from the caller's workspace `ws` of at least
+ *     moe_workspace_size() bytes (256-byte aligned).
+ *   - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream). The only host synchronisation is
+ *     inside moe_layer_forward when a cache is given (the miss list is read
+ *     back once per call).
+ *   - Every call returns a moe_status; moe_last_error_string() gives a
+ *     thread-local message for the last failure. There is no CPU fallback:
+ *     unsupported shapes or formats return MOE_ERR_UNSUPPORTED.
+ *   - Layouts are row-major. bf16 values are passed as raw 16-bit patterns.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned buffer */
+    MOE_ERR_UNSUPPORTED = 2, /* shape or format outside the kernel set */
+    MOE_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    MOE_ERR_OOM = 4,         /* workspace too small, or a cache allocation failed */
+    MOE_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired */
+    MOE_ERR_CACHE_FULL = 6   /* the cache cannot hold one call's working set */
+} moe_status;
+
+/* Stored expert-weight formats ([P4] "Reported Numbers and Ecosystem Position").
+ * For a tensor [R, K] (K = reduction dimension, contiguous):
+ *   MOE_BF16          codes: bf16 [R][K]; no scales.
+ *   MOE_FP8_E4M3_K128 codes: E4M3 bytes [R][K]; scale: fp32 [R][K/128].
+ *   MOE_MXFP4         codes: E2M1, two per byte, low nibble = lower K index, [R][K/2];
+ *                     scale: E8M0 bytes [R][K/32].
+ *   MOE_NVFP4         codes: as MXFP4; scale: E4M3 bytes [R][K/16];
+ *                     tscale: one fp32 per expert and tensor. */
+typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3 } moe_wfmt;
+
+/* The experts of one layer.
+ *   w13: gate and up projections, per expert [2I][H] (gate rows 0..I-1, then up rows).
+ *   w2:  down projection, per expert [H][I].
+ *   *_scale: scale planes as above (NULL for MOE_BF16).
+ *   *_tscale: [E] fp32 per-expert tensor scales (MOE_NVFP4 only, else NULL);
+ *             always indexed by the logical expert id.
+ *   *_estride: bytes from expert e to expert e+1 in each array; 0 = densely
+ *             packed. Codes, scales and strides must be 16-byte aligned.
+ *   expert_map: optional device [E] int32; when set, expert e's data is the
+ *             expert_map[e]-th entry of the strided arrays (used by the cache).
+ *   n_entries: number of entries in the strided arrays when expert_map is
+ *             set (0 = E). */
+typedef struct {
+    int fmt; /* moe_wfmt */
+    int E, H, I;
+    const void *w13;
+    const void *w13_scale;
+    const float *w13_tscale;
+    const void *w2;
+    const void *w2_scale;
+    const float *w2_tscale;
+    int64_t w13_estride, w13s_estride, w2_estride, w2s_estride;
+    const int32_t *expert_map;
+    int n_entries;
+} moe_experts;
+
+/* Router logits + top-k + softmax gating ([P3] "Why Now of All Times": a token
+ * activates k routed experts).
+ *   x: bf16 [T][H]; wr: [H][E], fp32 if wr_is_fp32 else bf16; bias: nullable fp32 [E].
+ *   Logits are the fp64 sum of x*Wr rounded once to fp32, plus bias (one fp32 add).
+ *   idx: int32 [T][k] in descending logit order, ties to the lower expert index.
+ *   w: fp32 [T][k], softmax over the k selected logits. logits: nullable fp32 [T][E].
+ *   ws: scratch of moe_workspace_size(T, H, ...) bytes (fp64 partial sums).
+ *   Requires 1 <= k <= 16, k <= E <= 256, H % 8 == 0. T == 0 is a no-op. */
+moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
+                          int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* Token-to-expert permutation (the dispatch implied by [P3] "Why Now of All
+ * Times"): a counting sort of the T*k pairs p = t*k + j by expert, stable in p.
+ *   offsets: int32 [E+1], exclusive scan of per-expert counts (offsets[E] = T*k).
+ *   sorted_pair: int32 [T*k], the pairs in expert order; pair_row: its inverse.
+ *   x_perm (nullable): bf16 [T*k][H], row r = x[sorted_pair[r] / k], with the
+ *     columns of every aligned group of 8 stored in the order 0,4,1,5,2,6,3,7
+ *     (the operand layout of moe_grouped_ffn).
+ *   Bit-exact and deterministic. Requires H % 8 == 0. */
+moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+                       int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Grouped SwiGLU expert FFN over the permuted rows ([P4] formats): for every
+ * expert e and row r in [offsets[e], offsets[e+1]):
+ *   h = silu(Wg_e . x_perm[r]) * (Wu_e . x_perm[r]), rounded to bf16;
+ *   y_perm[r] = W2_e . h   (bf16, or fp32 if y_is_fp32).
+ *   x_perm: bf16 [n_rows][H] in the interleaved layout written by moe_permute.
+ *   y_perm: [n_rows][H], natural column order.
+ *   ws: scratch for h ([n_rows][I] bf16).
+ *   Requires H % 128 == 0, I % 128 == 0, E <= 1024. n_rows == 0 is a no-op. */
+moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
+                           void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Gate-weighted combine: out[t] = sum_{j<k} w[t,j] * y_perm[pair_row[t*k+j]],
+ * accumulated in fp32 in order of j, rounded to bf16.
+ *   y_perm: [T*k][H] bf16 or fp32 (y_is_fp32); out: bf16 [T][H]. H % 8 == 0. */
+moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
+                       int H, void *out, moe_stream_t stream);
+
+/* Dequantise one expert tensor [rows][K] stored in `fmt` ([P4] formats) to bf16
+ * [rows][K] (row-major, natural K order), with the same decode the grouped FFN
+ * applies to its weight tiles. Exact for BF16 and MXFP4 (within bf16 range);
+ * NVFP4 ((E2M1 * E4M3) * tscale) and FP8 (E4M3 * fp32 scale) are rounded to
+ * bf16. w/scale as in moe_experts for a single expert; tscale: host value
+ * (NVFP4 only). K must be a multiple of the format's block (128/32/16/8). */
+moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
+                          moe_stream_t stream);
+
+struct expert_cache;
+
+/* The whole layer: route -> permute -> grouped FFN -> combine.
+ *   cache: nullable. When set, `experts` gives the layer's shape and format
+ *     only, the weights come from the cache's device slots for `layer`, and
+ *     missing experts are streamed from the cache's pinned host pool first
+ *     (one host synchronisation per call to read the miss list).
+ *   idx_out, w_out: nullable copies of the routing.
+ *   y_is_fp32: keep the expert outputs in fp32 before the combine. */
+moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp32, const float *bias, int k,
+                             const moe_experts *experts, struct expert_cache *cache, int layer, int y_is_fp32,
+                             void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* Scratch bytes needed by moe_layer_forward / moe_route_topk / moe_permute /
+ * moe_grouped_ffn for these sizes (an upper bound; host-only, no CUDA call). */
+size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32);
+
+/* ---------------------------------------------------------------- cache */
+/* Device LRU expert cache with streaming from pinned host memory ([P3]
+ * "FreeToken's Three-Layer Mechanism"; [P4] "Three Engineering Cores").
+ * The slot pool is one device allocation of capacity_bytes / slot_bytes slots,
+ * each holding one expert's w13, w2 and scales. The table (slot of each
+ * (layer, expert), owner and recency of each slot) lives on the device and is
+ * updated by a kernel; misses are copied host->device with cudaMemcpyAsync on
+ * the cache's own copy stream, and the compute stream waits on an event.
+ * Policy: ascending expert ids within a call; a miss takes the lowest free
+ * slot, else evicts the least recently referenced slot not referenced by this
+ * call or the previous one. */
+
+/* host_layers: host array [n_layers] of layer descriptions whose code/scale
+ * pointers are host pointers into page-locked (pinned) memory; all layers
+ * share fmt, E, H, I. The library allocates the slot pool, the table, a copy
+ * stream and events on `device`. The library keeps the pointers, not copies. */
+moe_status expert_cache_init(struct expert_cache **cache, size_t capacity_bytes, int n_layers,
+                             const moe_experts *host_layers, int device);
+
+/* Load the listed experts of `layer` (host array ids[n]) ahead of use, on the
+ * copy stream, without counting hits or misses. Synchronises with `stream`
+ * once to read back the loads the table update decided. */
+moe_status expert_cache_prefetch(struct expert_cache *cache, int layer, const int32_t *ids, int n,
+                                 moe_stream_t stream);
+
+/* Free slots: layer -1 = every slot; n -1 = all experts of `layer`; else the
+ * n listed experts (host array). Synchronous. */
+moe_status expert_cache_evict(struct expert_cache *cache, int layer, const int32_t *ids, int n);
+
+/* Counters since init: hits and misses of layer-forward calls, bytes copied
+ * host->device, and seconds the copy stream spent copying (event-timed). */
+moe_status expert_cache_stats(struct expert_cache *cache, uint64_t *hits, uint64_t *misses, uint64_t *bytes_h2d,
+                              double *copy_s);
+
+/* Device slot of (layer, e), or -1 (synchronous read; for tests and tools). */
+moe_status expert_cache_slot_of(struct expert_cache *cache, int layer, int e, int32_t *slot);
+
+/* Waits for outstanding copies and frees everything the cache allocated. */
+moe_status expert_cache_destroy(struct expert_cache *cache);
+
+/* ---------------------------------------------------------------- misc */
+
+/* Thread-local message describing the last failing call on this thread. */
+const char *moe_last_error_string(void);
+
+/* Reads and clears the device error word set by bounded waits and in-kernel
+ * checks (0 = none; 1 = a wait timed out; 2 = bad argument seen on device).
+ * Synchronises the device. */
+moe_status moe_device_error(int *code);
+
+/* Library version, for logs. */
+const char *moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

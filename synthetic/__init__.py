@@ -10,6 +10,7 @@ from .gen import (  # noqa: F401
     LayerInputs,
     WFMT,
     make_layer,
+    make_router,
     make_tokens,
     zipf_bias,
     expert_bytes,

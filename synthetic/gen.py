@@ -189,6 +189,16 @@ def make_tokens(T: int, H: int, seed: int, device="cpu", sub: int = 0) -> torch.
     return torch.randn(T, H, generator=g, device=device).to(torch.bfloat16)
 
 
+def make_router(cfg: str | dict, seed: int = 0, device="cpu", layer: int = 0):
+    """(wr, bias) of one layer, identical to the ones make_layer draws for the same arguments."""
+    c = dict(CONFIGS[cfg]) if isinstance(cfg, str) else dict(cfg)
+    H, E_ = c["H"], c["E"]
+    wr = torch.randn(H, E_, generator=_gen(seed, "wr", layer * 4096, device), device=device) * 0.02
+    wr = wr.float() if c.get("wr_fp32") else wr.to(torch.bfloat16)
+    bias = zipf_bias(E_, c["zipf"], H, seed + 7919 * layer, device) if c.get("zipf") else None
+    return wr, bias
+
+
 def make_layer(cfg: str | dict, seed: int = 0, device="cpu", E: Optional[int] = None,
                fmt: Optional[str] = None, layer: int = 0) -> LayerInputs:
     """All parameters of one layer of workload ``cfg`` (weights drawn N(0, 0.02), then encoded)."""

@@ -1,0 +1,297 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs. Integer outputs must match bit-exactly; floating-point
+outputs within TOL = 2e-2 of max|oracle| per tensor (tighter where stated)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from gpu_util import TOL, bf16_np, deinterleave_cols, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import expert_ffn_layer_top_b200 as m
+
+    return m
+
+
+def _ulp_close(a, b, ulps=1):
+    a = np.asarray(a, np.float32)
+    b = np.asarray(b, np.float32)
+    return np.all(np.abs(a - b) <= ulps * np.spacing(np.maximum(np.abs(a), np.abs(b))))
+
+
+# ----------------------------------------------------------------------------- decode
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp8", "mxfp4", "nvfp4"])
+def test_dequantize_matches_oracle(moe, fmt):
+    rows, K = 64, 256
+    g = torch.Generator().manual_seed(3)
+    t = 1.0
+    s = None
+    if fmt == "bf16":
+        w = torch.randn(rows, K, generator=g).to(torch.bfloat16)
+    elif fmt == "mxfp4":
+        w = torch.randint(0, 256, (rows, K // 2), dtype=torch.uint8, generator=g)
+        # scales spanning subnormal results (small), the common range, and > 2^1 (second multiply)
+        s = torch.randint(0, 200, (rows, K // 32), dtype=torch.uint8, generator=g)
+        s[0, :4] = torch.tensor([0, 1, 128, 129], dtype=torch.uint8)
+    elif fmt == "nvfp4":
+        w = torch.randint(0, 256, (rows, K // 2), dtype=torch.uint8, generator=g)
+        s = torch.randint(0, 0x7F, (rows, K // 16), dtype=torch.uint8, generator=g)   # incl. 0 and subnormals
+        t = 0.37
+    else:
+        w = torch.randint(0, 256, (rows, K), dtype=torch.uint8, generator=g)
+        w[(w & 0x7F) == 0x7F] = 0x7E                                                   # no NaN codes
+        s = (torch.rand(rows, K // 128, generator=g) + 0.5) * 1e-3
+    got = moe.moe_dequantize(fmt, w.cuda(), None if s is None else s.cuda(), t, rows, K).float().cpu()
+    ref = torch.from_numpy(oracle.dequant(fmt, w, s, tscale=t, rows=rows, K=K))
+    if fmt == "fp8":
+        assert rel_err(got, ref) < 2 ** -7
+        assert torch.allclose(got, ref, rtol=2 ** -7, atol=0)
+    else:
+        # exact: the same binary32 value, rounded once to bf16
+        assert torch.equal(got, ref.to(torch.bfloat16).float())
+
+
+# ----------------------------------------------------------------------------- router
+
+
+ROUTER_CASES = [("tiny", 16), ("decode", 1), ("decode", 8), ("decode", 64), ("prefill", 4096), ("large", 32),
+                ("large", 1000)]
+
+
+@pytest.mark.parametrize("cfg,T", ROUTER_CASES)
+def test_router_parity(moe, cfg, T):
+    wr, bias = synthetic.make_router(cfg, seed=1)
+    k = synthetic.CONFIGS[cfg]["k"]
+    x = synthetic.make_tokens(T, wr.shape[0], seed=1)
+    idx_o, w_o, lg_o = oracle.route(x, wr, k, bias=bias)
+    idx, w, lg = moe.moe_route_topk(x.cuda(), wr.cuda(), k, bias=None if bias is None else bias.cuda(),
+                                    want_logits=True)
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert _ulp_close(lg.cpu().numpy(), lg_o, 1)
+    assert np.allclose(w.cpu().numpy(), w_o, rtol=0, atol=2e-6)
+
+
+def test_router_ties_and_equal_logits(moe):
+    wr, _ = synthetic.make_router("tiny", seed=2)
+    wr = wr.clone()
+    wr[:, 5] = wr[:, 2]
+    x = synthetic.make_tokens(33, wr.shape[0], seed=2)
+    idx_o, w_o, _ = oracle.route(x, wr, 8)
+    idx, w = moe.moe_route_topk(x.cuda(), wr.cuda(), 8)
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    idx, w = moe.moe_route_topk(x.cuda(), torch.zeros_like(wr).cuda(), 3)
+    assert (idx.cpu().numpy() == np.arange(3)).all()
+    assert np.allclose(w.cpu().numpy(), 1 / 3, atol=1e-7)
+
+
+# ----------------------------------------------------------------------------- permutation
+
+
+def _rand_idx(T, k, E, seed):
+    g = np.random.default_rng(seed)
+    if T == 0:
+        return np.zeros((0, k), np.int32)
+    return np.argsort(g.random((T, E)), axis=1)[:, :k].astype(np.int32)
+
+
+@pytest.mark.parametrize("T,k,E", [(16, 2, 8), (1, 8, 128), (64, 8, 128), (4096, 8, 128), (8192, 6, 256),
+                                   (5, 3, 40), (0, 8, 128)])
+def test_permute_parity(moe, T, k, E):
+    idx = _rand_idx(T, k, E, T + k)
+    H = 256
+    x = synthetic.make_tokens(max(T, 1), H, seed=3)[:T]
+    off_o, sp_o, pr_o = oracle.permute(idx, E)
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), E, x.cuda())
+    assert np.array_equal(off.cpu().numpy(), off_o)
+    assert np.array_equal(sp.cpu().numpy(), sp_o)
+    assert np.array_equal(pr.cpu().numpy(), pr_o)
+    if T:
+        got = deinterleave_cols(xp.view(torch.int16).cpu().numpy())
+        want = x.view(torch.int16).numpy()[sp_o // k]
+        assert np.array_equal(got, want)
+
+
+def test_permute_single_expert_takes_everything(moe):
+    T, E = 300, 16
+    idx = np.full((T, 1), 7, np.int32)
+    off, sp, pr, _ = moe.moe_permute(torch.from_numpy(idx).cuda(), E)
+    off = off.cpu().numpy()
+    assert off[7] == 0 and off[8] == T and off[-1] == T
+    assert np.array_equal(sp.cpu().numpy(), np.arange(T))
+
+
+# ----------------------------------------------------------------------------- combine
+
+
+@pytest.mark.parametrize("y_fp32", [False, True])
+def test_combine_parity(moe, y_fp32):
+    g = torch.Generator().manual_seed(5)
+    T, k, H = 37, 4, 512
+    y = torch.randn(T * k, H, generator=g)
+    y = y if y_fp32 else y.to(torch.bfloat16)
+    pr = torch.randperm(T * k, generator=g).to(torch.int32)
+    w = torch.rand(T, k, generator=g)
+    ref = oracle.combine(y.float().numpy(), pr.numpy(), w.numpy(), T, k)
+    out = moe.moe_combine(y.cuda(), pr.cuda(), w.cuda())
+    assert rel_err(bf16_np(out), ref) < 4e-3
+
+
+# ----------------------------------------------------------------------------- grouped FFN
+
+
+FFN_CASES = [(fmt, T) for fmt in ("bf16", "fp8", "mxfp4", "nvfp4") for T in (40, 100, 200, 600)]
+
+
+@pytest.mark.parametrize("fmt,T", FFN_CASES)
+def test_grouped_ffn_parity(moe, fmt, T):
+    """T = 40/100/200/600 with E = 8, k = 2 exercises token tiles of 16/32/64/128."""
+    cfg = dict(H=256, E=8, k=2, I=256, fmt=fmt, wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=7)
+    x = synthetic.make_tokens(T, 256, seed=7)
+    idx = _rand_idx(T, 2, 8, T)
+    off_o, sp_o, pr_o = oracle.permute(idx, 8)
+    y_o, h_o = oracle.ffn(x, L, off_o, sp_o, 2, want_h=True)
+    Ld = L.to("cuda")
+    ex = moe.Experts.from_layer(Ld)
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), 8, x.cuda())
+    ws = torch.empty(T * 2 * 256 * 2 + 256, dtype=torch.uint8, device="cuda")
+    y = moe.moe_grouped_ffn(xp, off, ex, ws=ws)
+    torch.cuda.synchronize()
+    h = ws[: T * 2 * 256 * 2].view(torch.bfloat16).view(T * 2, 256)
+    h_got = deinterleave_cols(h.float().cpu().numpy())
+    assert rel_err(h_got, h_o) < TOL, "gate/up + SwiGLU"
+    assert rel_err(bf16_np(y), y_o) < TOL, "down projection"
+    assert moe.moe_device_error() == 0
+
+
+def test_grouped_ffn_fp32_output(moe):
+    cfg = dict(H=256, E=8, k=2, I=256, fmt="nvfp4", wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=8)
+    x = synthetic.make_tokens(50, 256, seed=8)
+    idx = _rand_idx(50, 2, 8, 50)
+    off_o, sp_o, _ = oracle.permute(idx, 8)
+    y_o = oracle.ffn(x, L, off_o, sp_o, 2)
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), 8, x.cuda())
+    y = moe.moe_grouped_ffn(xp, off, moe.Experts.from_layer(L.to("cuda")), y_fp32=True)
+    assert y.dtype == torch.float32
+    assert rel_err(y.cpu().numpy(), y_o) < TOL
+
+
+# ----------------------------------------------------------------------------- whole layer
+
+
+def _layer_check(moe, L, x, y_fp32=False, sample=None):
+    """Run the layer on the GPU; compare routing bit-exactly and outputs (all or sampled rows)."""
+    Ld = L.to("cuda")
+    T = x.shape[0]
+    idx = torch.empty(T, L.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, L.k, dtype=torch.float32, device="cuda")
+    out = moe.moe_layer_forward(x.cuda(), Ld.wr, L.k, moe.Experts.from_layer(Ld), bias=Ld.bias, y_fp32=y_fp32,
+                                idx_out=idx, w_out=w)
+    torch.cuda.synchronize()
+    idx_o, w_o, _ = oracle.route(x, L.wr, L.k, bias=L.bias, with_logits=False)
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert np.allclose(w.cpu().numpy(), w_o, atol=2e-6, rtol=0)
+    got = bf16_np(out)
+    if sample is None:
+        ref = oracle.layer_forward(x, L)["out"]
+        err = rel_err(got, ref)
+    else:
+        ref = oracle.token_rows(x, L, idx_o, w_o, sample)
+        err = rel_err(got[sample], ref)
+    assert err < TOL, f"layer output error {err:.3e}"
+    assert moe.moe_device_error() == 0
+    return err
+
+
+def test_layer_tiny(moe):
+    L = synthetic.make_layer("tiny", 0)
+    x = synthetic.make_tokens(16, L.H, 0)
+    _layer_check(moe, L, x)
+
+
+@pytest.fixture(scope="module")
+def decode_layer():
+    return synthetic.make_layer("decode", 0)
+
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_layer_decode_mxfp4(moe, decode_layer, T):
+    x = synthetic.make_tokens(T, 2048, seed=10 + T)
+    _layer_check(moe, decode_layer, x)
+
+
+@pytest.fixture(scope="module")
+def prefill_layer():
+    return synthetic.make_layer("prefill", 0)
+
+
+def test_layer_prefill_nvfp4_reduced_batch(moe, prefill_layer):
+    x = synthetic.make_tokens(256, 2048, seed=11)
+    _layer_check(moe, prefill_layer, x)
+
+
+def test_layer_prefill_nvfp4_full_size_sampled(moe, prefill_layer):
+    x = synthetic.make_tokens(4096, 2048, seed=12)
+    _layer_check(moe, prefill_layer, x, sample=[0, 1, 777, 2048, 4095])
+
+
+@pytest.fixture(scope="module")
+def large_layer():
+    # 3.6 GB of NVFP4 experts: generated on the GPU, copied to the host for the oracle
+    return synthetic.make_layer("large", 0, device="cuda").to("cpu")
+
+
+def test_layer_large_decode_sampled(moe, large_layer):
+    x = synthetic.make_tokens(32, 4096, seed=13)
+    _layer_check(moe, large_layer, x, y_fp32=True, sample=[0, 17, 31])
+
+
+def test_layer_large_prefill_sampled(moe, large_layer):
+    x = synthetic.make_tokens(8192, 4096, seed=14)
+    _layer_check(moe, large_layer, x, y_fp32=True, sample=[0, 4096, 8191])
+
+
+def test_layer_one_hot_expert_and_k1(moe):
+    """k = 1 and a bias that sends every token to expert 3: one expert gets every row."""
+    cfg = dict(H=256, E=16, k=1, I=256, fmt="mxfp4", wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=15)
+    L.bias = torch.zeros(16)
+    L.bias[3] = 100.0
+    x = synthetic.make_tokens(300, 256, seed=15)
+    _layer_check(moe, L, x)
+
+
+def test_layer_empty_batch(moe):
+    L = synthetic.make_layer("tiny", 0).to("cuda")
+    x = torch.empty(0, L.H, dtype=torch.bfloat16, device="cuda")
+    out = moe.moe_layer_forward(x, L.wr, L.k, moe.Experts.from_layer(L))
+    assert out.shape == (0, L.H)
+
+
+def test_layer_is_deterministic(moe):
+    L = synthetic.make_layer("tiny", 0).to("cuda")
+    x = synthetic.make_tokens(16, L.H, 0).cuda()
+    a = moe.moe_layer_forward(x, L.wr, L.k, moe.Experts.from_layer(L))
+    b = moe.moe_layer_forward(x, L.wr, L.k, moe.Experts.from_layer(L))
+    assert torch.equal(a, b)
+
+
+def test_bad_arguments_are_rejected(moe):
+    L = synthetic.make_layer("tiny", 0).to("cuda")
+    x = synthetic.make_tokens(4, L.H, 0).cuda()
+    bad = moe.Experts("bf16", 8, 200, 512, L.w13, L.w2)       # H not a multiple of 128
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_layer_forward(x, L.wr, L.k, bad)
+    assert ei.value.name == "UNSUPPORTED"
+    with pytest.raises(moe.MoeError):
+        moe.moe_route_topk(x, L.wr, 17)                        # k > 16
