@@ -55,57 +55,65 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every 20 ms
+    during the timed region (read-only queries; no setting is changed)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+
+    def _handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            p = torch.cuda.get_device_properties(self.device)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+
+    def _run(self):
+        import pynvml
+
+        while not self._stop.is_set():
+            try:
+                self.samples.append(pynvml.nvmlDeviceGetClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            import pynvml
+
+            self._h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
         except Exception:
-            self.proc = None
+            self._h = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        if self._h is not None:
+            self._t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = self.samples
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(sm)}
 
 
 # ------------------------------------------------------------------------------------------- workload
@@ -128,8 +136,11 @@ class LayerBench:
         self.k, self.y32 = c["k"], c["y_fp32"]
         base = synthetic.make_layer(cfg, seed, device=device)
         self.layer = base
-        self.sets = [base] + [self._clone(base) for _ in range(nsets - 1)]
-        self.experts = [moe.Experts.from_layer(s) for s in self.sets]
+        # weights are prepacked once into the tiled layout (model-load work, not timed)
+        tiled = moe.moe_prepack(moe.Experts.from_layer(base))
+        del base.w13, base.w2, base.w13_scale, base.w2_scale
+        self.sets = [base] * nsets
+        self.experts = [tiled] + [self._clone(moe, tiled) for _ in range(nsets - 1)]
         self.xs = [synthetic.make_tokens(T, base.H, seed=100 + i, device=device) for i in range(nsets)]
         self.ws = torch.empty(moe.moe_workspace_size(T, base.H, base.I, base.E, self.k, self.y32),
                               dtype=torch.uint8, device=device)
@@ -139,13 +150,10 @@ class LayerBench:
         self.graphs = None
 
     @staticmethod
-    def _clone(l):
-        c = l.to(l.wr.device)
-        for n in ("w13", "w2", "w13_scale", "w2_scale"):
-            t = getattr(c, n)
-            if t is not None:
-                setattr(c, n, t.clone())
-        return c
+    def _clone(moe, ex):
+        """The same tiled weights at another address (defeats L2 reuse across steps)."""
+        return moe.Experts(ex.fmt, ex.E, ex.H, ex.I, ex.w13.clone(), ex.w2.clone(), None, None, ex.w13_tscale,
+                           ex.w2_tscale, layout=ex.layout)
 
     def call(self, i: int):
         j = i % len(self.sets)
@@ -173,7 +181,7 @@ class LayerBench:
         self.graphs[i % len(self.graphs)].replay()
 
     def algorithmic_bytes(self, i: int) -> int:
-        """Router weights + active experts + x in + out (SURVEY 8(d) definition)."""
+        """Algorithmic bytes of one layer: router weights + experts with >= 1 token + x in + out."""
         j = i % len(self.sets)
         s = self.sets[j]
         router = s.wr.numel() * s.wr.element_size()
@@ -301,7 +309,7 @@ def run_ours(args, rank, world, device):
     lb.capture()
     extra = {}
     launches_per_step = 9   # router 2 + permute 4 + FFN 2 + combine 1
-    with ClockSampler(device.index) as clk:
+    with ClockSampler(device) as clk:
         sec = time_steps(lb.step, args.steps, args.warmup, device, barrier)
     clocks = clk.summary()
     if world > 1:
@@ -383,14 +391,27 @@ def run_ours(args, rank, world, device):
         print(json.dumps(line), flush=True)
 
 
+def run_profile(args, device):
+    """W + K plain (non-graph) layer forwards of one workload; for ncu launch lists."""
+    import expert_ffn_layer_top_b200 as moe
+
+    cfg, T = args.profile.split(":")
+    lb = LayerBench(moe, cfg, int(T), device, nsets=4)
+    for i in range(args.warmup + args.steps):
+        lb.call(i)
+    torch.cuda.synchronize(device)
+    print(json.dumps({"profile": args.profile, "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile", default=None, help="plain launches of one workload (cfg:T, e.g. decode:64) for ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -402,6 +423,9 @@ def main():
         return
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.profile:
+        run_profile(args, device)
+        return
     if world > 1:
         import datetime
 

@@ -18,6 +18,10 @@ from ._lib import (  # noqa: F401
     moe_grouped_ffn,
     moe_layer_forward,
     moe_permute,
+    moe_prepack,
+    moe_prepacked_expert_bytes,
+    LAYOUT_STANDARD,
+    LAYOUT_TILED,
     moe_route_topk,
     moe_version,
     moe_workspace_size,

@@ -33,7 +33,7 @@ class _Experts(C.Structure):
         ("w2", _P), ("w2_scale", _P), ("w2_tscale", _P),
         ("w13_estride", C.c_int64), ("w13s_estride", C.c_int64),
         ("w2_estride", C.c_int64), ("w2s_estride", C.c_int64),
-        ("expert_map", _P), ("n_entries", C.c_int),
+        ("expert_map", _P), ("n_entries", C.c_int), ("layout", C.c_int),
     ]
 
 
@@ -64,6 +64,10 @@ def lib():
             L.moe_layer_forward.restype = st
             L.moe_layer_forward.argtypes = [_P, _I, _P, _I, _P, _I, C.POINTER(_Experts), _P, _I, _I, _P, _P, _P,
                                             _P, C.c_size_t, _P]
+            L.moe_prepacked_expert_bytes.restype = C.c_size_t
+            L.moe_prepacked_expert_bytes.argtypes = [_I, _I, _I, _I]
+            L.moe_prepack.restype = st
+            L.moe_prepack.argtypes = [C.POINTER(_Experts), _P, _P, _P]
             L.moe_workspace_size.restype = C.c_size_t
             L.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
             L.expert_cache_init.restype = st
@@ -131,18 +135,41 @@ class Experts:
     """A layer's experts (a moe_experts descriptor plus the tensors it points at)."""
 
     def __init__(self, fmt: str, E: int, H: int, I: int, w13, w2, w13_scale=None, w2_scale=None,
-                 w13_tscale=None, w2_tscale=None, strides=(0, 0, 0, 0), expert_map=None, n_entries=0):
-        self.fmt, self.E, self.H, self.I = fmt, E, H, I
+                 w13_tscale=None, w2_tscale=None, strides=(0, 0, 0, 0), expert_map=None, n_entries=0,
+                 layout: int = 0):
+        self.fmt, self.E, self.H, self.I, self.layout = fmt, E, H, I, layout
+        self.w13, self.w2, self.w13_scale, self.w2_scale = w13, w2, w13_scale, w2_scale
+        self.w13_tscale, self.w2_tscale = w13_tscale, w2_tscale
         self._keep = [w13, w2, w13_scale, w2_scale, w13_tscale, w2_tscale, expert_map]
         self.c = _Experts(FMT[fmt], E, H, I, _ptr(w13), _ptr(w13_scale), _ptr(w13_tscale), _ptr(w2), _ptr(w2_scale),
                           _ptr(w2_tscale), strides[0], strides[1], strides[2], strides[3], _ptr(expert_map),
-                          n_entries)
+                          n_entries, layout)
 
     @classmethod
     def from_layer(cls, layer) -> "Experts":
         """From an object with fmt/E/H/I/w13/w2/*_scale/*_tscale tensor attributes."""
         return cls(layer.fmt, layer.E, layer.H, layer.I, layer.w13, layer.w2, layer.w13_scale, layer.w2_scale,
                    layer.w13_tscale, layer.w2_tscale)
+
+
+LAYOUT_STANDARD, LAYOUT_TILED = 0, 1
+
+
+def moe_prepacked_expert_bytes(fmt: str, H: int, I: int, which: int) -> int:
+    return int(lib().moe_prepacked_expert_bytes(FMT[fmt], H, I, which))
+
+
+def moe_prepack(experts: Experts) -> Experts:
+    """Tiled (prepacked) copy of standard-layout device experts (see moe_prepack in moe.h)."""
+    _need_cuda(experts.w13, experts.w2)
+    dev = experts.w13.device
+    b13 = moe_prepacked_expert_bytes(experts.fmt, experts.H, experts.I, 0)
+    b2 = moe_prepacked_expert_bytes(experts.fmt, experts.H, experts.I, 1)
+    o13 = torch.empty(experts.E * b13, dtype=torch.uint8, device=dev)
+    o2 = torch.empty(experts.E * b2, dtype=torch.uint8, device=dev)
+    _check(lib().moe_prepack(C.byref(experts.c), _ptr(o13), _ptr(o2), _stream()))
+    return Experts(experts.fmt, experts.E, experts.H, experts.I, o13, o2, None, None, experts.w13_tscale,
+                   experts.w2_tscale, layout=LAYOUT_TILED)
 
 
 def moe_route_topk(x: torch.Tensor, wr: torch.Tensor, k: int, bias: Optional[torch.Tensor] = None,

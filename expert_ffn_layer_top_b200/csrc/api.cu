@@ -97,6 +97,12 @@ struct Strides {
 
 static Strides default_strides(const moe_experts &x) {
     Strides s;
+    if (x.layout == MOE_LAYOUT_TILED) {
+        s.w13 = x.w13_estride ? x.w13_estride : (int64_t)prepacked_expert_bytes(x.fmt, x.H, x.I, 0);
+        s.w2 = x.w2_estride ? x.w2_estride : (int64_t)prepacked_expert_bytes(x.fmt, x.H, x.I, 1);
+        s.w13s = s.w2s = 0;
+        return s;
+    }
     const int64_t r13 = 2LL * x.I, r2 = x.H;
     s.w13 = x.w13_estride ? x.w13_estride : r13 * x.H * elem_bytes_x2(x.fmt) / 2;
     s.w13s = x.w13s_estride ? x.w13s_estride : r13 * scale_rowbytes(x.fmt, x.H);
@@ -109,17 +115,20 @@ static moe_status check_experts(const moe_experts *x) {
     if (!x) return set_error(MOE_ERR_INVALID_ARG, "experts is NULL");
     if (x->fmt < MOE_BF16 || x->fmt > MOE_NVFP4) return set_error(MOE_ERR_UNSUPPORTED, "unknown weight format %d", x->fmt);
     if (x->E <= 0 || x->E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d outside 1..%d", x->E, kMaxExperts);
-    if (x->H <= 0 || x->I <= 0 || x->H % 128 || x->I % 128)
-        return set_error(MOE_ERR_UNSUPPORTED, "H=%d and I=%d must be positive multiples of 128", x->H, x->I);
+    if (x->H <= 0 || x->I <= 0 || x->H % 256 || x->I % 256)
+        return set_error(MOE_ERR_UNSUPPORTED, "H=%d and I=%d must be positive multiples of 256", x->H, x->I);
     if (!x->w13 || !x->w2) return set_error(MOE_ERR_INVALID_ARG, "expert weights are NULL");
-    if (x->fmt != MOE_BF16 && (!x->w13_scale || !x->w2_scale))
+    if (x->layout != MOE_LAYOUT_STANDARD && x->layout != MOE_LAYOUT_TILED)
+        return set_error(MOE_ERR_INVALID_ARG, "unknown layout %d", x->layout);
+    if (x->layout == MOE_LAYOUT_STANDARD && x->fmt != MOE_BF16 && (!x->w13_scale || !x->w2_scale))
         return set_error(MOE_ERR_INVALID_ARG, "scale planes are NULL");
     if (x->fmt == MOE_NVFP4 && (!x->w13_tscale || !x->w2_tscale))
         return set_error(MOE_ERR_INVALID_ARG, "NVFP4 tensor scales are NULL");
     const Strides s = default_strides(*x);
     if ((s.w13 | s.w2 | s.w13s | s.w2s) & 15) return set_error(MOE_ERR_INVALID_ARG, "expert strides not 16-byte aligned");
-    const uintptr_t a = reinterpret_cast<uintptr_t>(x->w13) | reinterpret_cast<uintptr_t>(x->w2) |
-                        reinterpret_cast<uintptr_t>(x->w13_scale) | reinterpret_cast<uintptr_t>(x->w2_scale);
+    uintptr_t a = reinterpret_cast<uintptr_t>(x->w13) | reinterpret_cast<uintptr_t>(x->w2);
+    if (x->layout == MOE_LAYOUT_STANDARD)
+        a |= reinterpret_cast<uintptr_t>(x->w13_scale) | reinterpret_cast<uintptr_t>(x->w2_scale);
     if (a & 15) return set_error(MOE_ERR_INVALID_ARG, "expert arrays not 16-byte aligned");
     return MOE_OK;
 }
@@ -185,8 +194,16 @@ static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t
     p.H = x->H;
     p.I = x->I;
     p.n_rows = n_rows;
+    const bool tiled = x->layout == MOE_LAYOUT_TILED;
+    p.tiled = tiled;
+    memset(&wmap, 0, sizeof(wmap));   // unused by the tiled kernels
     // ---- gate/up + SwiGLU
-    if ((r = weight_tmap(&wmap, x->fmt, x->w13, 2 * x->I, x->H, s.w13, nent)) != MOE_OK) return r;
+    if (tiled) {
+        p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
+        p.w_estride = s.w13;
+    } else if ((r = weight_tmap(&wmap, x->fmt, x->w13, 2 * x->I, x->H, s.w13, nent)) != MOE_OK) {
+        return r;
+    }
     if ((r = act_tmap(&bmap, x_perm, n_rows, x->H, BN)) != MOE_OK) return r;
     p.K = x->H;
     p.m_tiles = x->I / 64;
@@ -198,7 +215,12 @@ static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t
     p.out_fp32 = 0;
     if ((r = launch_ffn_phase(kPhaseUp, x->fmt, BN, wmap, bmap, p, nsm, st)) != MOE_OK) return r;
     // ---- down projection
-    if ((r = weight_tmap(&wmap, x->fmt, x->w2, x->H, x->I, s.w2, nent)) != MOE_OK) return r;
+    if (tiled) {
+        p.wbase = reinterpret_cast<const uint8_t *>(x->w2);
+        p.w_estride = s.w2;
+    } else if ((r = weight_tmap(&wmap, x->fmt, x->w2, x->H, x->I, s.w2, nent)) != MOE_OK) {
+        return r;
+    }
     if ((r = act_tmap(&bmap, h, n_rows, x->I, BN)) != MOE_OK) return r;
     p.K = x->I;
     p.m_tiles = x->H / 128;
@@ -317,6 +339,25 @@ moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscal
     return launch_dequant(fmt, w, scale, tscale, rows, K, out, (cudaStream_t)stream);
 }
 
+size_t moe_prepacked_expert_bytes(int fmt, int H, int I, int which) {
+    if (fmt < MOE_BF16 || fmt > MOE_NVFP4 || H <= 0 || I <= 0 || H % 256 || I % 256 || (which != 0 && which != 1))
+        return 0;
+    return prepacked_expert_bytes(fmt, H, I, which);
+}
+
+moe_status moe_prepack(const moe_experts *in, void *out_w13, void *out_w2, moe_stream_t stream) {
+    moe_status r = check_experts(in);
+    if (r != MOE_OK) return r;
+    if (in->layout != MOE_LAYOUT_STANDARD || in->expert_map)
+        return set_error(MOE_ERR_INVALID_ARG, "moe_prepack needs standard-layout experts without expert_map");
+    if (!out_w13 || !out_w2 || ((reinterpret_cast<uintptr_t>(out_w13) | reinterpret_cast<uintptr_t>(out_w2)) & 15))
+        return set_error(MOE_ERR_INVALID_ARG, "outputs must be non-NULL and 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((r = launch_prepack(*in, 0, out_w13, (int64_t)prepacked_expert_bytes(in->fmt, in->H, in->I, 0), st)) != MOE_OK)
+        return r;
+    return launch_prepack(*in, 1, out_w2, (int64_t)prepacked_expert_bytes(in->fmt, in->H, in->I, 1), st);
+}
+
 moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
                        int H, void *out, moe_stream_t stream) {
     if (T < 0 || k < 1 || k > kMaxTopK || H <= 0 || H % 8) return set_error(MOE_ERR_INVALID_ARG, "bad T/k/H");
@@ -338,7 +379,7 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     if (!cache) {
         moe_status r = check_experts(experts);
         if (r != MOE_OK) return r;
-    } else if (experts->E <= 0 || H % 128 || I % 128) {
+    } else if (experts->E <= 0 || H % 256 || I % 256) {
         return set_error(MOE_ERR_UNSUPPORTED, "bad layer shape");
     }
     if (!x || !wr || !out || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");

@@ -35,7 +35,7 @@
 #include "internal.h"
 
 struct expert_cache {
-    int device = 0, n_layers = 0, E = 0, H = 0, I = 0, fmt = 0;
+    int device = 0, n_layers = 0, E = 0, H = 0, I = 0, fmt = 0, layout = 0;
     size_t sz[4] = {0, 0, 0, 0};      // per-expert bytes: w13, w13 scales, w2, w2 scales
     size_t off[4] = {0, 0, 0, 0};     // offsets inside a slot
     size_t slot_bytes = 0;
@@ -359,6 +359,7 @@ moe_status cache_resolve_and_map(expert_cache *c, int layer, const int32_t *idx,
     view->w13_estride = view->w13s_estride = view->w2_estride = view->w2s_estride = (int64_t)c->slot_bytes;
     view->expert_map = c->d_slot_of + (size_t)layer * c->E;
     view->n_entries = c->n_slots;
+    view->layout = c->layout;
     if (c->fmt == MOE_NVFP4) {
         view->w13_tscale = c->d_ts13 + (size_t)layer * c->E;
         view->w2_tscale = c->d_ts2 + (size_t)layer * c->E;
@@ -377,11 +378,11 @@ moe_status expert_cache_init(struct expert_cache **out, size_t capacity_bytes, i
     if (!out || !host_layers || n_layers <= 0) return set_error(MOE_ERR_INVALID_ARG, "bad cache arguments");
     *out = nullptr;
     const moe_experts &l0 = host_layers[0];
-    if (l0.fmt < MOE_BF16 || l0.fmt > MOE_NVFP4 || l0.E <= 0 || l0.E > kMaxExperts || l0.H % 128 || l0.I % 128)
+    if (l0.fmt < MOE_BF16 || l0.fmt > MOE_NVFP4 || l0.E <= 0 || l0.E > kMaxExperts || l0.H % 256 || l0.I % 256)
         return set_error(MOE_ERR_UNSUPPORTED, "unsupported layer shape for the cache");
     for (int l = 1; l < n_layers; ++l) {
         const moe_experts &x = host_layers[l];
-        if (x.fmt != l0.fmt || x.E != l0.E || x.H != l0.H || x.I != l0.I)
+        if (x.fmt != l0.fmt || x.E != l0.E || x.H != l0.H || x.I != l0.I || x.layout != l0.layout)
             return set_error(MOE_ERR_INVALID_ARG, "cache layers must share format and shape");
     }
     const char *fault = getenv("MOE_FAULT");
@@ -398,10 +399,16 @@ moe_status expert_cache_init(struct expert_cache **out, size_t capacity_bytes, i
     c->layers.assign(host_layers, host_layers + n_layers);
     if (fault && strncmp(fault, "h2d_fail@", 9) == 0) c->fault_h2d_at = atol(fault + 9);
     const int fmt = l0.fmt;
-    c->sz[0] = part_bytes(fmt, 2 * c->I, c->H, false);
-    c->sz[1] = fmt == MOE_BF16 ? 0 : part_bytes(fmt, 2 * c->I, c->H, true);
-    c->sz[2] = part_bytes(fmt, c->H, c->I, false);
-    c->sz[3] = fmt == MOE_BF16 ? 0 : part_bytes(fmt, c->H, c->I, true);
+    c->layout = l0.layout;
+    if (c->layout == MOE_LAYOUT_TILED) {   // scales travel inside the prepacked blobs
+        c->sz[0] = prepacked_expert_bytes(fmt, c->H, c->I, 0);
+        c->sz[2] = prepacked_expert_bytes(fmt, c->H, c->I, 1);
+    } else {
+        c->sz[0] = part_bytes(fmt, 2 * c->I, c->H, false);
+        c->sz[1] = fmt == MOE_BF16 ? 0 : part_bytes(fmt, 2 * c->I, c->H, true);
+        c->sz[2] = part_bytes(fmt, c->H, c->I, false);
+        c->sz[3] = fmt == MOE_BF16 ? 0 : part_bytes(fmt, c->H, c->I, true);
+    }
     size_t o = 0;
     for (int i = 0; i < 4; ++i) {
         c->off[i] = o;

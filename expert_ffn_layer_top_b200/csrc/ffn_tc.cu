@@ -11,17 +11,24 @@
 //   * M tile = 128 weight rows. UP: 64 gate rows + the 64 matching up rows, so
 //     one MMA produces both halves of the SwiGLU for 64 channels. DOWN: 128 rows.
 //   * N tile = BN permuted rows (tokens) of one expert, BN in {16,32,64,128}.
-//   * K stage = 128 elements.
-//   * Warp roles (512 threads, one CTA per SM, persistent over work items):
-//       warp 0      TMA producer: raw weight tile (swizzled), activation tile
-//                   (128-byte swizzle), and per tile the scale block (bulk copy).
+//   * K stage = 128 elements; stages are handled in groups of kG = 2 (16 MMAs).
+//   * Warp roles (768 threads, one CTA per SM, persistent over work items):
+//       warp 0      producer: per stage one bulk copy of the prepacked weight
+//                   blob (or TMA boxes + a per-tile scale copy for row-major
+//                   weights) and a TMA box of activations (128-byte swizzle).
 //       warp 1      owns TMEM; one lane issues tcgen05.mma (A from TMEM,
-//                   B from shared memory) and tcgen05.commit.
+//                   B from shared memory).
 //       warps 4-7   epilogue: tcgen05.ld of the fp32 accumulator, SwiGLU (UP)
 //                   or scaling (DOWN), stores.
-//       warps 8-15  decoders: raw codes + scales -> exact bf16 (or bf16-rounded
-//                   for FP8) weights, written straight into TMEM with
-//                   tcgen05.st, so decoded weights never touch shared memory.
+//       warps 8-23  decoders: codes + scales -> exact bf16 (bf16-rounded for
+//                   FP8) weights, written straight into TMEM with tcgen05.st,
+//                   so decoded weights never touch shared memory.
+//   * A tcgen05.mma of this shape costs ~52 cycles whatever N <= 64, and each
+//     tcgen05.commit or wait-plus-fence in the issuing thread stalls the
+//     tensor pipe for ~100+ cycles, so the issuing thread synchronises once
+//     per group: it waits for the decoders of the group's last stage, issues
+//     16 MMAs, and commits once to the group's barrier, which then frees both
+//     the group's shared-memory stages and its TMEM slots.
 //   * K order inside every 8-element group is 0,4,1,5,2,6,3,7 in both
 //     operands: one shift/multiply/mask then decodes an FP4 pair (k, k+4).
 //   * Every wait is bounded; on timeout the CTA sets the device error word,
@@ -31,23 +38,25 @@
 
 namespace moe {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 768;
+constexpr int kDecWarps = 16;       // warps 8..23
 constexpr int kBK = 128;            // K elements per stage
-constexpr int kMaxStages = 4;
-constexpr int kACol = 0;            // TMEM columns [0, 64*stages): A stages
-constexpr int kAccCol = 256;        // TMEM columns [256, 256+2*BN): accumulators
+constexpr int kG = 2;               // stages per MMA group (one commit, one wait)
+constexpr int kMaxStages = 16;      // shared-memory ring (multiple of kG)
+constexpr int kMaxAStages = 6;      // TMEM ring of decoded weight tiles (64 columns each, multiple of kG)
 constexpr int kXchStride = 17;      // padded row of the gate/up exchange buffer
 
+// Per weight row and K stage (128 elements): code bytes and scale bytes.
 template <int FMT>
 struct RawFmt;
 template <>
-struct RawFmt<MOE_MXFP4> { static constexpr int kRowBytes = 64; };   // 128 e4m1 codes
+struct RawFmt<MOE_MXFP4> { static constexpr int kRowBytes = 64, kScaleBytes = 4; };   // 4 E8M0 (block 32)
 template <>
-struct RawFmt<MOE_NVFP4> { static constexpr int kRowBytes = 64; };
+struct RawFmt<MOE_NVFP4> { static constexpr int kRowBytes = 64, kScaleBytes = 8; };   // 8 E4M3 (block 16)
 template <>
-struct RawFmt<MOE_FP8_E4M3_K128> { static constexpr int kRowBytes = 128; };
+struct RawFmt<MOE_FP8_E4M3_K128> { static constexpr int kRowBytes = 128, kScaleBytes = 4; };   // 1 fp32
 template <>
-struct RawFmt<MOE_BF16> { static constexpr int kRowBytes = 256; };
+struct RawFmt<MOE_BF16> { static constexpr int kRowBytes = 256, kScaleBytes = 0; };
 
 // bf16x2 multiply (exact for the power-of-two and short-significand factors used here).
 __device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
@@ -83,10 +92,15 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t v) {
     return __uint_as_float(pat) * 0x1p120f;
 }
 
+// bf16x2 factor 2^126 * 2^(s-127) for an E8M0 scale s <= 128; for s > 128 the
+// factor saturates at 2^127 and a second factor 2^(s-128) completes it.
+__device__ __forceinline__ uint32_t mx_factor(uint32_t s8) { return bf16x2_splat_bits((s8 <= 128 ? s8 + 126 : 254u) << 7); }
+__device__ __forceinline__ uint32_t mx_factor2(uint32_t s8) { return bf16x2_splat_bits((s8 > 128 ? s8 - 1 : 127u) << 7); }
+
 struct FfnSmem {
-    uint64_t full[kMaxStages];
-    uint64_t adec[kMaxStages];
-    uint64_t empty[kMaxStages];
+    uint64_t full[kMaxStages];                 // stage landed (producer expect_tx + copies)
+    uint64_t gdone[kMaxStages / kG];           // group's MMAs complete (frees its stages and TMEM slots)
+    uint64_t adec[kMaxAStages];                // stage decoded into TMEM (one arrive per decoder warp)
     uint64_t accfull[2];
     uint64_t accempty[2];
     uint64_t scfull[2];
@@ -122,21 +136,30 @@ __device__ __forceinline__ ItemInfo decode_item(const FfnSmem &sm, const FfnPara
     return it;
 }
 
-template <int FMT, int PHASE, int BN>
+// TILED: the weights were prepacked by moe_prepack into one contiguous blob per
+// (M tile, K stage) - 128 rows of codes, 16-byte chunk-major, followed by the
+// rows' scales for that stage - and each stage arrives with one bulk copy.
+// Otherwise the codes come from the row-major tensor through a 3D TMA box and
+// the scales through one bulk copy per tile.
+template <int FMT, int PHASE, int BN, bool TILED>
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap bmap, FfnParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     constexpr int RB = RawFmt<FMT>::kRowBytes;
-    constexpr int RAWB = 128 * RB;              // raw weight bytes per stage
+    constexpr int SBY = RawFmt<FMT>::kScaleBytes;
+    constexpr int RAWB = 128 * RB;                          // code bytes per stage
+    constexpr int SB = RAWB + (TILED ? 128 * SBY : 0);      // smem bytes per stage (codes [+ scales])
     constexpr int BSTAGE = BN * 256;            // activation bytes per stage (two 64-column atoms)
 
     // ---- shared memory carve-up (1024-aligned operand regions)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int nst = p.stages;
+    const int nst = p.stages;                 // multiple of kG
+    const int na = p.astages;                 // TMEM A stages, multiple of kG
+    const int nsg = nst / kG;                 // groups in the shared-memory ring
     uint8_t *bstage = base;
     uint8_t *rawst = bstage + nst * BSTAGE;
-    uint8_t *scbuf = rawst + nst * RAWB;
-    const int scb_bytes = 128 * p.s_rowbytes;   // per buffer (0 for bf16)
+    uint8_t *scbuf = rawst + nst * SB;
+    const int scb_bytes = TILED ? 0 : 128 * p.s_rowbytes;   // per tile buffer (standard layout only)
     float *xch = reinterpret_cast<float *>(scbuf + 2 * ((scb_bytes + 15) & ~15));
     FfnSmem &sm = *reinterpret_cast<FfnSmem *>(reinterpret_cast<uint8_t *>(xch) +
                                               (PHASE == kPhaseUp ? 64 * kXchStride * 4 : 0));
@@ -146,16 +169,14 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
 
     // ---- set-up: barriers (thread 0), TMEM (warp 1), tile prefix (warp 2)
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.adec[s], 8);
-            mbar_init(&sm.empty[s], 1);
-        }
+        for (int s = 0; s < kMaxStages; ++s) mbar_init(&sm.full[s], 1);
+        for (int g = 0; g < kMaxStages / kG; ++g) mbar_init(&sm.gdone[g], 1);
+        for (int s = 0; s < kMaxAStages; ++s) mbar_init(&sm.adec[s], kDecWarps);
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sm.accfull[a], 1);
             mbar_init(&sm.accempty[a], 128);
             mbar_init(&sm.scfull[a], 1);
-            mbar_init(&sm.scempty[a], 8);
+            mbar_init(&sm.scempty[a], kDecWarps);
         }
         mbar_init(&sm.mmadone, 1);
         mbar_init(&sm.xfull, 64);
@@ -164,7 +185,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&wmap);
+        if (!TILED) tma_prefetch_desc(&wmap);
         tma_prefetch_desc(&bmap);
     }
     if (warp == 1) {
@@ -197,15 +218,15 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     tc_fence_after();
 
     const uint32_t tmem = sm.tmem_base;
+    const uint32_t acc_col = (uint32_t)na * 64;   // accumulators follow the A ring
     const int total = sm.total_items;
-    const int KB = p.K / kBK;
+    const int KB = p.K / kBK;                     // multiple of kG
 
     if (warp == 0) {
-        // =================================================== TMA producer
+        // =================================================== producer
         if (lane == 0) {
-            int kc = 0, lt = 0;
-            int issued_mask = 0;                 // stages with a load whose completion was not yet awaited here
-            uint32_t issued_par[kMaxStages] = {0, 0, 0, 0};
+            int kc = 0, lt = 0, s = 0;           // kc: stages issued so far
+            uint32_t ph = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
                 const ItemInfo it = decode_item(sm, p, item, BN);
@@ -213,7 +234,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 int rowA, rowB;
                 if (PHASE == kPhaseUp) { rowA = it.m * 64; rowB = p.I + it.m * 64; }
                 else { rowA = it.m * 128; rowB = rowA + 64; }
-                if (FMT != MOE_BF16) {
+                if (FMT != MOE_BF16 && !TILED) {
                     const int sb = lt & 1;
                     if (!mbar_wait(&sm.scempty[sb], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     mbar_expect_tx(&sm.scfull[sb], 128 * p.s_rowbytes);
@@ -223,14 +244,17 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     bulk_load(dst + 64 * p.s_rowbytes, sbase + (int64_t)rowB * p.s_rowbytes, 64 * p.s_rowbytes,
                               &sm.scfull[sb]);
                 }
-                for (int kb = 0; kb < KB; ++kb, ++kc) {
-                    const int s = kc % nst;
-                    const uint32_t ph = (kc / nst) & 1;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+                for (int kb = 0; kb < KB; ++kb) {
+                    // a group's stages are reused once the group's MMAs completed
+                    if ((s & (kG - 1)) == 0 && !mbar_wait(&sm.gdone[s / kG], ph ^ 1, abort_flag)) { ok = false; break; }
                     uint64_t *fb = &sm.full[s];
-                    mbar_expect_tx(fb, RAWB + BSTAGE);
-                    uint8_t *raw = rawst + s * RAWB;
-                    if (FMT == MOE_BF16) {
+                    mbar_expect_tx(fb, SB + BSTAGE);
+                    uint8_t *raw = rawst + s * SB;
+                    if (TILED) {
+                        const uint8_t *src = p.wbase + (int64_t)slot * p.w_estride +
+                                             ((int64_t)it.m * KB + kb) * SB;
+                        bulk_load(raw, src, SB, fb);
+                    } else if (FMT == MOE_BF16) {
                         // two 64-column boxes per 64-row half
                         tma_load_3d(raw + 0 * 8192, &wmap, fb, kb * kBK, rowA, slot);
                         tma_load_3d(raw + 1 * 8192, &wmap, fb, kb * kBK + 64, rowA, slot);
@@ -244,15 +268,15 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     uint8_t *bs = bstage + s * BSTAGE;
                     tma_load_2d(bs, &bmap, fb, kb * kBK, it.row0);
                     tma_load_2d(bs + BN * 128, &bmap, fb, kb * kBK + 64, it.row0);
-                    issued_mask |= 1 << s;
-                    issued_par[s] = ph;
+                    ++kc;
+                    if (++s == nst) { s = 0; ph ^= 1; }
                 }
             }
-            // drain: never leave the CTA while a copy into its shared memory is in flight
-            for (int s = 0; s < nst; ++s) {
-                if (!(issued_mask & (1 << s))) continue;
+            // drain: never leave the CTA while a copy into its shared memory is in
+            // flight - wait for the completion of the last min(kc, nst) stages issued
+            for (int j = kc - 1; j >= 0 && j >= kc - nst; --j) {
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full[s], issued_par[s])) {
+                while (!mbar_try_wait(&sm.full[j % nst], (j / nst) & 1)) {
                     if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
                 }
             }
@@ -261,27 +285,36 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         // =================================================== MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-            int kc = 0, lt = 0;
+            const uint32_t desc_hi = (uint32_t)(smem_desc_sw128(0) >> 32);
+            const uint32_t desc_lo0 = (uint32_t)smem_desc_sw128(smem_u32(bstage));
+            int s = 0, sa = 0, lt = 0;
+            uint32_t pha = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
                 const int a = lt & 1;
                 if (!mbar_wait(&sm.accempty[a], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t dcol = tmem + kAccCol + a * BN;
-                for (int kb = 0; kb < KB; ++kb, ++kc) {
-                    const int s = kc % nst;
-                    const uint32_t ph = (kc / nst) & 1;
-                    if (!mbar_wait(&sm.adec[s], ph, abort_flag)) { ok = false; break; }
-                    if (!mbar_wait(&sm.full[s], ph, abort_flag)) { ok = false; break; }
+                const uint32_t dcol = tmem + acc_col + a * BN;
+                for (int kb = 0; kb < KB; kb += kG) {
+                    // the decoders arrive stage by stage, so the group's last stage implies the rest;
+                    // they waited for its activation tiles too
+                    if (!mbar_wait(&sm.adec[sa + kG - 1], pha, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t bsa = smem_u32(bstage + s * BSTAGE);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t atm = tmem + kACol + s * 64 + i * 8;
-                        const uint32_t baddr = bsa + (i >> 2) * (BN * 128) + (i & 3) * 32;
-                        mma_bf16_ts(dcol, atm, smem_desc_sw128(baddr), idesc, (kb | i) != 0);
+                    for (int g = 0; g < kG; ++g) {
+                        const uint32_t lo = desc_lo0 + ((uint32_t)((s + g) * BSTAGE) >> 4);
+                        const uint32_t atm = tmem + (sa + g) * 64;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            mma_bf16_ts_lohi(dcol, atm + i * 8,
+                                             lo + (((i >> 2) * (BN * 128) + (i & 3) * 32) >> 4), desc_hi, idesc,
+                                             (kb | g | i) != 0);
                     }
-                    mma_commit(&sm.empty[s]);
+                    mma_commit(&sm.gdone[s / kG]);
+                    s += kG;
+                    if (s == nst) s = 0;
+                    sa += kG;
+                    if (sa == na) { sa = 0; pha ^= 1; }
                 }
                 if (!ok) break;
                 mma_commit(&sm.accfull[a]);
@@ -306,7 +339,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
             tc_fence_after();
             float osc = 1.0f;
             if (FMT == MOE_NVFP4) osc = p.tscale[it.e] * 128.0f;   // decoded codes carry 2^-7
-            const uint32_t acc = tmem + ((uint32_t)(q * 32) << 16) + kAccCol + a * BN;
+            const uint32_t acc = tmem + ((uint32_t)(q * 32) << 16) + acc_col + a * BN;
             if (PHASE == kPhaseUp) {
                 // rows 0-63: gate of channel c0+row; rows 64-127: up of the same channel
                 const int ch = it.m * 64 + (lrow & 63);
@@ -364,97 +397,92 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         }
     } else if (warp >= 8) {
         // =================================================== decoders
+        // 16 warps: warp (8 + dw) owns TMEM lane quarter q = dw % 4 (rows 32q..32q+31)
+        // and the 32 K elements [32*sub, 32*sub + 32) of every stage, sub = dw / 4.
         const int dw = warp - 8;
-        const int q = dw & 3;          // TMEM lane quarter (warp % 4)
-        const int hf = dw >> 2;        // which 64-wide half of the K stage
+        const int q = dw & 3;
+        const int sub = dw >> 2;
         const int m = q * 32 + lane;   // M-tile row
         const int rh = m >> 6, rr = m & 63;
-        int kc = 0, lt = 0;
+        int lt = 0, s = 0, sa = 0, gstart = 0;   // gstart: groups started
+        uint32_t ph = 0, pha = 0;
+        int lag_slot = 0;                        // group (gstart - na/kG) whose MMAs must have completed
+        uint32_t lag_ph = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
             const int sb = lt & 1;
             const uint8_t *scrow = scbuf + sb * ((scb_bytes + 15) & ~15) + m * p.s_rowbytes;
-            if (FMT != MOE_BF16) {
+            if (FMT != MOE_BF16 && !TILED) {
                 if (!mbar_wait(&sm.scfull[sb], (lt >> 1) & 1, abort_flag)) { ok = false; break; }
             }
-            for (int kb = 0; kb < KB; ++kb, ++kc) {
-                const int s = kc % nst;
-                const uint32_t ph = (kc / nst) & 1;
+            for (int kb = 0; kb < KB; ++kb) {
+                if ((sa & (kG - 1)) == 0) {
+                    // new group: its TMEM slots were last used by the group na/kG groups back
+                    if (gstart >= na / kG) {
+                        if (!mbar_wait(&sm.gdone[lag_slot], lag_ph, abort_flag)) { ok = false; break; }
+                        if (++lag_slot == nsg) { lag_slot = 0; lag_ph ^= 1; }
+                    }
+                    ++gstart;
+                }
                 if (!mbar_wait(&sm.full[s], ph, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint8_t *raw = rawst + s * RAWB;
-                uint32_t o[32];
+                const uint8_t *raw = rawst + s * SB;
+                // 16-byte chunk c of this thread's row, and its scales for this stage
+                auto chunk = [&](int c) -> uint4 {
+                    const uint8_t *a;
+                    if (TILED) a = raw + ((c * 128 + m) << 4);
+                    else if (FMT == MOE_MXFP4 || FMT == MOE_NVFP4) a = raw + rh * (RAWB / 2) + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4);
+                    else if (FMT == MOE_FP8_E4M3_K128) a = raw + rh * (RAWB / 2) + rr * 128 + ((c ^ (rr & 7)) << 4);
+                    else a = raw + (rh * 2 + (c >> 3)) * 8192 + rr * 128 + (((c & 7) ^ (rr & 7)) << 4);
+                    return *reinterpret_cast<const uint4 *>(a);
+                };
+                const uint8_t *scs = TILED ? raw + RAWB + m * SBY : scrow + kb * SBY;
+                uint32_t o[16];
                 if (FMT == MOE_MXFP4 || FMT == MOE_NVFP4) {
-                    // row rr of half rh: 64 bytes, 16-byte chunks swizzled by ((rr >> 1) & 3)
-                    const uint8_t *row = raw + rh * (RAWB / 2) + rr * 64;
-                    bool big_any = false;
-                    uint32_t f[4];   // bf16x2 factor per 16-element quarter of this thread's 64 elements
+                    const uint4 v = chunk(sub);                 // 32 codes = 4 groups of 8
+                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
                     if (FMT == MOE_MXFP4) {
-                        const uint32_t sc2 = *reinterpret_cast<const uint16_t *>(scrow + kb * 4 + hf * 2);
-                        bool big = false;
-#pragma unroll
-                        for (int b = 0; b < 2; ++b) {
-                            const uint32_t s8 = (sc2 >> (8 * b)) & 0xFF;
-                            big |= s8 > 128;
-                            // 2^126 * 2^(s-127) = 2^(s-1): bf16 exponent field s + 126
-                            const uint32_t fb = (s8 <= 128 ? (s8 + 126) : 254u) << 7;
-                            f[2 * b] = f[2 * b + 1] = bf16x2_splat_bits(fb);
-                        }
-                        big_any = __any_sync(0xffffffffu, big);
-                        if (big_any) {
-                            // rare: scales above 2^1 need a second exact multiply
-#pragma unroll
-                            for (int c = 0; c < 2; ++c) {
-                                const uint4 v = *reinterpret_cast<const uint4 *>(
-                                    row + (((2 * hf + c) ^ ((rr >> 1) & 3)) << 4));
-                                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                                for (int g = 0; g < 4; ++g) {
-                                    uint32_t pr[4];
-                                    e2m1x8_to_bf16_pattern(wv[g], pr);
-                                    const int b = (c * 4 + g) >> 2;
-                                    const uint32_t s8 = (sc2 >> (8 * b)) & 0xFF;
-                                    const uint32_t f2 = bf16x2_splat_bits((s8 > 128 ? (s8 - 128 + 127) : 127u) << 7);
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) o[(c * 4 + g) * 4 + j] = bmul2(bmul2(pr[j], f[2 * b]), f2);
-                                }
-                            }
-                        }
-                    } else {
-                        const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(scrow + kb * 8 + hf * 4);
-#pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            // 2^126 * e4m3 * 2^-7 (the 2^7 is restored in the epilogue with the tensor scale)
-                            const float sv = e4m3_to_f32((sc4 >> (8 * b)) & 0xFF) * 0x1p119f;
-                            const __nv_bfloat16 bs = __float2bfloat16_rn(sv);
-                            f[b] = bf16x2_splat_bits(*reinterpret_cast<const uint16_t *>(&bs));
-                        }
-                    }
-                    if (!(FMT == MOE_MXFP4 && big_any)) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(row + (((2 * hf + c) ^ ((rr >> 1) & 3)) << 4));
-                        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+                        const uint32_t s8 = scs[sub];               // one E8M0 block of 32
+                        const uint32_t f = mx_factor(s8);
+                        const bool big = __any_sync(0xffffffffu, s8 > 128);
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
                             uint32_t pr[4];
                             e2m1x8_to_bf16_pattern(wv[g], pr);
-                            const int gi = c * 4 + g;                      // 8-group index 0..7
-                            const uint32_t fac = (FMT == MOE_MXFP4) ? f[(gi >> 2) * 2] : f[gi >> 1];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) o[gi * 4 + j] = bmul2(pr[j], fac);
+                            for (int j = 0; j < 4; ++j) o[g * 4 + j] = bmul2(pr[j], f);
+                        }
+                        if (big) {   // rare: scales above 2^1 need a second exact multiply
+                            const uint32_t f2 = mx_factor2(s8);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) o[j] = bmul2(o[j], f2);
+                        }
+                    } else {
+                        const uint32_t sc2 = *reinterpret_cast<const uint16_t *>(scs + 2 * sub);   // two blocks of 16
+                        uint32_t f[2];
+#pragma unroll
+                        for (int b = 0; b < 2; ++b) {
+                            // 2^126 * e4m3 * 2^-7 (the 2^7 is restored in the epilogue with the tensor scale)
+                            const float sv = e4m3_to_f32((sc2 >> (8 * b)) & 0xFF) * 0x1p119f;
+                            const __nv_bfloat16 bs = __float2bfloat16_rn(sv);
+                            f[b] = bf16x2_splat_bits(*reinterpret_cast<const uint16_t *>(&bs));
+                        }
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            uint32_t pr[4];
+                            e2m1x8_to_bf16_pattern(wv[g], pr);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) o[g * 4 + j] = bmul2(pr[j], f[g >> 1]);
                         }
                     }
-                    }
                 } else if (FMT == MOE_FP8_E4M3_K128) {
-                    const uint8_t *row = raw + rh * (RAWB / 2) + rr * 128;
-                    const float sc = reinterpret_cast<const float *>(scrow)[kb];
+                    const float sc = *reinterpret_cast<const float *>(scs);
                     // 2^120 * scale, rounded to bf16 (the one inexact step of this format)
                     const __nv_bfloat16 bs = __float2bfloat16_rn(sc * 0x1p120f);
                     const uint32_t fac = bf16x2_splat_bits(*reinterpret_cast<const uint16_t *>(&bs));
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(row + (((4 * hf + c) ^ (rr & 7)) << 4));
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 v = chunk(2 * sub + c);
                         // v.x,v.y = K 16c..16c+7 ; v.z,v.w = 16c+8..16c+15
                         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -470,30 +498,31 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                         }
                     }
                 } else {
-                    // bf16: box hf holds K 64*hf..64*hf+63 of this half's rows, 128-byte swizzle
-                    const uint8_t *row = raw + (rh * 2 + hf) * 8192 + rr * 128;
+                    // bf16: K 32*sub..32*sub+31 are chunks 4*sub..4*sub+3
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (rr & 7)) << 4));
-                        const uint4 iv = interleave8(v);
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 iv = interleave8(chunk(4 * sub + c));
                         o[c * 4 + 0] = iv.x;
                         o[c * 4 + 1] = iv.y;
                         o[c * 4 + 2] = iv.z;
                         o[c * 4 + 3] = iv.w;
                     }
                 }
-                tmem_st32(tmem + ((uint32_t)(q * 32) << 16) + kACol + s * 64 + hf * 32, o);
+                tmem_st16(tmem + ((uint32_t)(q * 32) << 16) + sa * 64 + sub * 16, o);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.adec[s]);
+                if (lane == 0) mbar_arrive(&sm.adec[sa]);
+                if (++s == nst) { s = 0; ph ^= 1; }
+                if (++sa == na) { sa = 0; pha ^= 1; }
             }
             if (!ok) break;
-            if (FMT != MOE_BF16) {
+            if (FMT != MOE_BF16 && !TILED) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.scempty[sb]);
             }
         }
+        (void)pha;
     }
 
     tc_fence_before();
@@ -582,12 +611,17 @@ moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscal
 
 // ------------------------------------------------------------------ host side
 
-static size_t ffn_smem_bytes(int fmt, int phase, int BN, int stages, int s_rowbytes) {
-    const int rb = fmt == MOE_BF16 ? 256 : fmt == MOE_FP8_E4M3_K128 ? 128 : 64;
+int stage_scale_bytes(int fmt) {
+    return fmt == MOE_MXFP4 ? 4 : fmt == MOE_NVFP4 ? 8 : fmt == MOE_FP8_E4M3_K128 ? 4 : 0;
+}
+int stage_code_bytes(int fmt) { return fmt == MOE_BF16 ? 256 : fmt == MOE_FP8_E4M3_K128 ? 128 : 64; }
+
+static size_t ffn_smem_bytes(int fmt, int phase, int BN, int stages, int s_rowbytes, bool tiled) {
+    const int rb = stage_code_bytes(fmt);
     size_t b = 1024;                                     // alignment slack
     b += (size_t)stages * BN * 256;
-    b += (size_t)stages * 128 * rb;
-    b += 2 * (size_t)((128 * s_rowbytes + 15) & ~15);
+    b += (size_t)stages * 128 * (rb + (tiled ? stage_scale_bytes(fmt) : 0));
+    if (!tiled) b += 2 * (size_t)((128 * s_rowbytes + 15) & ~15);
     if (phase == kPhaseUp) b += 64 * kXchStride * 4;
     b += sizeof(FfnSmem);
     return b;
@@ -596,7 +630,7 @@ static size_t ffn_smem_bytes(int fmt, int phase, int BN, int stages, int s_rowby
 template <int FMT, int PHASE, int BN>
 static cudaError_t launch_one(const CUtensorMap &wmap, const CUtensorMap &bmap, const FfnParams &p, int grid,
                               size_t smem, cudaStream_t st) {
-    auto kfn = ffn_tc_kernel<FMT, PHASE, BN>;
+    auto kfn = p.tiled ? ffn_tc_kernel<FMT, PHASE, BN, true> : ffn_tc_kernel<FMT, PHASE, BN, false>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kfn<<<grid, kThreads, smem, st>>>(wmap, bmap, p);
@@ -645,17 +679,27 @@ int scale_rowbytes(int fmt, int K) {
 // Launch one phase. The tensor maps are built by the caller (api.cu).
 moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap,
                             FfnParams p, int num_sms, cudaStream_t st) {
+    if (p.K % (kBK * kG)) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", p.K, kBK * kG);
     int stages = kMaxStages;
     size_t smem = 0;
-    for (; stages >= 2; --stages) {
-        smem = ffn_smem_bytes(fmt, phase, BN, stages, p.s_rowbytes);
+    for (; stages >= kG; stages -= kG) {
+        smem = ffn_smem_bytes(fmt, phase, BN, stages, p.s_rowbytes, p.tiled != 0);
         if (smem <= 227 * 1024) break;
     }
-    if (stages < 2) return set_error(MOE_ERR_UNSUPPORTED, "FFN tile does not fit in shared memory");
+    if (stages < kG) return set_error(MOE_ERR_UNSUPPORTED, "FFN tile does not fit in shared memory");
     // The CTA allocates all 512 TMEM columns: ask for enough shared memory that a
     // second CTA can never be co-resident on the SM (it would only block in alloc).
     if (smem < 120 * 1024) smem = 120 * 1024;
     p.stages = stages;
+    // TMEM: A ring of 64-column stages, then two accumulators of BN columns
+    int na = (512 - 2 * BN) / 64;
+    if (na > kMaxAStages) na = kMaxAStages;
+    // The decoders wait on the group barrier of the group na/kG back; with at
+    // least as many shared-memory groups as TMEM groups no barrier can complete
+    // twice before that wait, so the parity check cannot alias.
+    if (na > stages) na = stages;
+    na -= na % kG;
+    p.astages = na;
     // upper bound of work items; the kernel reads the exact count from the offsets
     const int64_t tiles_ub = (int64_t)p.n_rows / BN + p.E;
     const int64_t items_ub = tiles_ub * p.m_tiles;

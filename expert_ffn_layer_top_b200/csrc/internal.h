@@ -21,7 +21,8 @@ struct FfnParams {
     int E, H, I;
     int K;                      // reduction dimension of this phase (H or I)
     int m_tiles;                // I/64 (up) or H/128 (down)
-    int stages;                 // pipeline depth, set by the launcher
+    int stages;                 // shared-memory ring depth, set by the launcher
+    int astages;                // TMEM ring depth (decoded weight stages), set by the launcher
     const uint8_t *scale_base;  // scale plane of this phase's tensor (nullable for bf16)
     int64_t s_estride;          // bytes between experts in the scale plane
     int s_rowbytes;             // scale bytes per weight row
@@ -29,6 +30,9 @@ struct FfnParams {
     void *out;                  // up: h bf16 [n_rows][I]; down: y [n_rows][H]
     int out_fp32;
     int n_rows;
+    int tiled;                  // weights prepacked (moe_prepack): one blob per (M tile, K stage)
+    const uint8_t *wbase;       // tiled: this phase's prepacked tensor
+    int64_t w_estride;          // tiled: bytes between experts
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -36,6 +40,10 @@ moe_status set_error(moe_status s, const char *fmt, ...);
 moe_status set_cuda_error(cudaError_t e, const char *what);
 
 int num_sms(int device);
+int stage_scale_bytes(int fmt);
+int stage_code_bytes(int fmt);
+size_t prepacked_expert_bytes(int fmt, int H, int I, int which);
+moe_status launch_prepack(const moe_experts &in, int which, void *out, int64_t out_estride, cudaStream_t st);
 int choose_bn(int n_rows, int E);
 int scale_rowbytes(int fmt, int K);
 

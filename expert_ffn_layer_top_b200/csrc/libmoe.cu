@@ -5,4 +5,5 @@
 #include "permute.cu"
 #include "combine.cu"
 #include "ffn_tc.cu"
+#include "prepack.cu"
 #include "cache.cu"

@@ -73,6 +73,13 @@ typedef enum {
  *                     tscale: one fp32 per expert and tensor. */
 typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3 } moe_wfmt;
 
+/* Memory layout of the expert codes. STANDARD: row-major as described above.
+ * TILED: produced by moe_prepack; for every (M tile, 128-wide K stage) one
+ * contiguous blob holding the 128 weight rows' codes (16-byte chunk-major) and
+ * then their scales for that stage, so a stage is one bulk copy. The values
+ * are the same; only the byte order differs. */
+typedef enum { MOE_LAYOUT_STANDARD = 0, MOE_LAYOUT_TILED = 1 } moe_layout;
+
 /* The experts of one layer.
  *   w13: gate and up projections, per expert [2I][H] (gate rows 0..I-1, then up rows).
  *   w2:  down projection, per expert [H][I].
@@ -84,7 +91,10 @@ typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3
  *   expert_map: optional device [E] int32; when set, expert e's data is the
  *             expert_map[e]-th entry of the strided arrays (used by the cache).
  *   n_entries: number of entries in the strided arrays when expert_map is
- *             set (0 = E). */
+ *             set (0 = E).
+ *   layout:   MOE_LAYOUT_STANDARD (the arrays above) or MOE_LAYOUT_TILED
+ *             (w13/w2 hold moe_prepack output, scales included; *_scale and
+ *             the scale strides are ignored; *_estride 0 = densely packed). */
 typedef struct {
     int fmt; /* moe_wfmt */
     int E, H, I;
@@ -97,6 +107,7 @@ typedef struct {
     int64_t w13_estride, w13s_estride, w2_estride, w2s_estride;
     const int32_t *expert_map;
     int n_entries;
+    int layout; /* moe_layout */
 } moe_experts;
 
 /* Router logits + top-k + softmax gating ([P3] "Why Now of All Times": a token
@@ -130,7 +141,7 @@ moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, i
  *   x_perm: bf16 [n_rows][H] in the interleaved layout written by moe_permute.
  *   y_perm: [n_rows][H], natural column order.
  *   ws: scratch for h ([n_rows][I] bf16).
- *   Requires H % 128 == 0, I % 128 == 0, E <= 1024. n_rows == 0 is a no-op. */
+ *   Requires H % 256 == 0, I % 256 == 0, E <= 1024. n_rows == 0 is a no-op. */
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
                            void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -148,6 +159,17 @@ moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_ro
  * (NVFP4 only). K must be a multiple of the format's block (128/32/16/8). */
 moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           moe_stream_t stream);
+
+/* Bytes of one expert's prepacked w13 (which = 0) or w2 (which = 1). */
+size_t moe_prepacked_expert_bytes(int fmt, int H, int I, int which);
+
+/* Rewrite a layer's experts from MOE_LAYOUT_STANDARD into MOE_LAYOUT_TILED
+ * (a device-side byte permutation, done once when weights are loaded).
+ *   in: standard-layout experts (device pointers; expert_map must be NULL).
+ *   out_w13, out_w2: device buffers of E * moe_prepacked_expert_bytes(...) bytes,
+ *   16-byte aligned. The result is used through a moe_experts with
+ *   layout = MOE_LAYOUT_TILED, w13 = out_w13, w2 = out_w2 (tscales unchanged). */
+moe_status moe_prepack(const moe_experts *in, void *out_w13, void *out_w2, moe_stream_t stream);
 
 struct expert_cache;
 

@@ -113,6 +113,25 @@ def test_explicit_prefetch_turns_misses_into_hits(moe, stack):
     cache.close()
 
 
+def test_tiled_host_pool_streams_and_matches(moe, stack):
+    """Host pool in the prepacked (tiled) layout: two copies per miss, same results."""
+    layers, host, dev = stack
+    tiled_host = []
+    for L in dev:
+        t = moe.moe_prepack(moe.Experts.from_layer(L))
+        tiled_host.append(moe.Experts(t.fmt, t.E, t.H, t.I, t.w13.cpu().pin_memory(), t.w2.cpu().pin_memory(),
+                                      layout=moe.LAYOUT_TILED))
+    cache = moe.ExpertCache(1 << 30, tiled_host, device=0)
+    for l in range(L_):
+        x = synthetic.make_tokens(T_, H_, seed=40 + l).cuda()
+        shape = moe.Experts.from_layer(dev[l])
+        out_c = moe.moe_layer_forward(x, dev[l].wr, K_, shape, cache=cache, layer=l)
+        out_r = moe.moe_layer_forward(x, dev[l].wr, K_, shape)
+        assert torch.equal(out_c, out_r)
+    assert cache.stats()["misses"] > 0
+    cache.close()
+
+
 def test_cache_full_is_reported(moe, stack):
     layers, host, dev = stack
     slot_bytes = sum(((t.numel() * t.element_size() // E_) + 255) // 256 * 256

@@ -148,12 +148,14 @@ def test_combine_parity(moe, y_fp32):
 # ----------------------------------------------------------------------------- grouped FFN
 
 
-FFN_CASES = [(fmt, T) for fmt in ("bf16", "fp8", "mxfp4", "nvfp4") for T in (40, 100, 200, 600)]
+FFN_CASES = [(fmt, T, tiled) for fmt in ("bf16", "fp8", "mxfp4", "nvfp4") for T in (40, 100, 200, 600)
+             for tiled in (False, True)]
 
 
-@pytest.mark.parametrize("fmt,T", FFN_CASES)
-def test_grouped_ffn_parity(moe, fmt, T):
-    """T = 40/100/200/600 with E = 8, k = 2 exercises token tiles of 16/32/64/128."""
+@pytest.mark.parametrize("fmt,T,tiled", FFN_CASES)
+def test_grouped_ffn_parity(moe, fmt, T, tiled):
+    """T = 40/100/200/600 with E = 8, k = 2 exercises token tiles of 16/32/64/128,
+    on row-major weights and on weights prepacked into the tiled layout."""
     cfg = dict(H=256, E=8, k=2, I=256, fmt=fmt, wr_fp32=False)
     L = synthetic.make_layer(cfg, seed=7)
     x = synthetic.make_tokens(T, 256, seed=7)
@@ -162,6 +164,8 @@ def test_grouped_ffn_parity(moe, fmt, T):
     y_o, h_o = oracle.ffn(x, L, off_o, sp_o, 2, want_h=True)
     Ld = L.to("cuda")
     ex = moe.Experts.from_layer(Ld)
+    if tiled:
+        ex = moe.moe_prepack(ex)
     off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), 8, x.cuda())
     ws = torch.empty(T * 2 * 256 * 2 + 256, dtype=torch.uint8, device="cuda")
     y = moe.moe_grouped_ffn(xp, off, ex, ws=ws)
@@ -189,14 +193,17 @@ def test_grouped_ffn_fp32_output(moe):
 # ----------------------------------------------------------------------------- whole layer
 
 
-def _layer_check(moe, L, x, y_fp32=False, sample=None):
+def _layer_check(moe, L, x, y_fp32=False, sample=None, tiled=True):
     """Run the layer on the GPU; compare routing bit-exactly and outputs (all or sampled rows)."""
     Ld = L.to("cuda")
     T = x.shape[0]
     idx = torch.empty(T, L.k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, L.k, dtype=torch.float32, device="cuda")
-    out = moe.moe_layer_forward(x.cuda(), Ld.wr, L.k, moe.Experts.from_layer(Ld), bias=Ld.bias, y_fp32=y_fp32,
-                                idx_out=idx, w_out=w)
+    ex = moe.Experts.from_layer(Ld)
+    if tiled:
+        ex = moe.moe_prepack(ex)
+        del Ld.w13, Ld.w2          # keep device memory low for the large layer
+    out = moe.moe_layer_forward(x.cuda(), Ld.wr, L.k, ex, bias=Ld.bias, y_fp32=y_fp32, idx_out=idx, w_out=w)
     torch.cuda.synchronize()
     idx_o, w_o, _ = oracle.route(x, L.wr, L.k, bias=L.bias, with_logits=False)
     assert np.array_equal(idx.cpu().numpy(), idx_o)
@@ -213,10 +220,11 @@ def _layer_check(moe, L, x, y_fp32=False, sample=None):
     return err
 
 
-def test_layer_tiny(moe):
+@pytest.mark.parametrize("tiled", [False, True])
+def test_layer_tiny(moe, tiled):
     L = synthetic.make_layer("tiny", 0)
     x = synthetic.make_tokens(16, L.H, 0)
-    _layer_check(moe, L, x)
+    _layer_check(moe, L, x, tiled=tiled)
 
 
 @pytest.fixture(scope="module")
@@ -228,6 +236,11 @@ def decode_layer():
 def test_layer_decode_mxfp4(moe, decode_layer, T):
     x = synthetic.make_tokens(T, 2048, seed=10 + T)
     _layer_check(moe, decode_layer, x)
+
+
+def test_layer_decode_mxfp4_standard_layout(moe, decode_layer):
+    x = synthetic.make_tokens(64, 2048, seed=9)
+    _layer_check(moe, decode_layer, x, tiled=False)
 
 
 @pytest.fixture(scope="module")
