@@ -165,9 +165,12 @@ class LayerBench:
         self.graphs = []
         st = torch.cuda.Stream(self.dev)
         st.wait_stream(torch.cuda.current_stream(self.dev))
+        n0 = self.moe.moe_kernel_launch_count()
         with torch.cuda.stream(st):
             for j in range(len(self.sets)):   # warm the launch paths before capture
                 self.call(j)
+        # kernels one layer call enqueues (the captured graphs replay exactly these)
+        self.launches_per_call = (self.moe.moe_kernel_launch_count() - n0) / len(self.sets)
         torch.cuda.current_stream(self.dev).wait_stream(st)
         torch.cuda.synchronize(self.dev)
         for j in range(len(self.sets)):
@@ -308,7 +311,7 @@ def run_ours(args, rank, world, device):
     lb = LayerBench(moe, "decode", 64, device)
     lb.capture()
     extra = {}
-    launches_per_step = 9   # router 2 + permute 4 + FFN 2 + combine 1
+    launches_per_step = lb.launches_per_call
     with ClockSampler(device) as clk:
         sec = time_steps(lb.step, args.steps, args.warmup, device, barrier)
     clocks = clk.summary()
@@ -384,7 +387,7 @@ def run_ours(args, rank, world, device):
         "config": {"workload": "decode-shaped MoE layer, MXFP4 experts, T=64", "H": 2048, "E": 128, "k": 8,
                    "I": 768, "T": 64, "parallelism": f"replicas x{world}",
                    "l2": f"{NSETS} rotating weight copies + activation batches (weights touched per step > L2)"},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clocks, "extra": extra,
     }
     if rank == 0:

@@ -24,5 +24,6 @@ from ._lib import (  # noqa: F401
     LAYOUT_TILED,
     moe_route_topk,
     moe_version,
+    moe_kernel_launch_count,
     moe_workspace_size,
 )

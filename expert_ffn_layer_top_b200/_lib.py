@@ -89,6 +89,8 @@ def lib():
             L.moe_device_error.argtypes = [C.POINTER(C.c_int)]
             L.moe_version.restype = C.c_char_p
             L.moe_version.argtypes = []
+            L.moe_kernel_launch_count.restype = C.c_uint64
+            L.moe_kernel_launch_count.argtypes = []
             _lib_handle = L
     return _lib_handle
 
@@ -115,6 +117,11 @@ def _need_cuda(*ts):
 
 def moe_version() -> str:
     return lib().moe_version().decode()
+
+
+def moe_kernel_launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(lib().moe_kernel_launch_count())
 
 
 def moe_device_error() -> int:

@@ -269,6 +269,8 @@ const char *moe_last_error_string(void) { return t_err; }
 
 const char *moe_version(void) { return "libmoe 0.1 (sm_100a)"; }
 
+uint64_t moe_kernel_launch_count(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
+
 moe_status moe_device_error(int *code) {
     if (!code) return set_error(MOE_ERR_INVALID_ARG, "code is NULL");
     cudaError_t e = cudaDeviceSynchronize();

@@ -334,6 +334,7 @@ moe_status cache_resolve_and_map(expert_cache *c, int layer, const int32_t *idx,
     if (layer < 0 || layer >= c->n_layers) return set_error(MOE_ERR_INVALID_ARG, "layer %d out of range", layer);
     if (shape->E != c->E || shape->H != c->H || shape->I != c->I || shape->fmt != c->fmt)
         return set_error(MOE_ERR_INVALID_ARG, "layer shape differs from the cache's");
+    count_launch();
     lru_kernel<<<1, 32, 0, st>>>(table_of(c), layer, idx, T * k, 0, 1, c->d_io);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) e = cudaEventRecord(c->ev_lru, st);
@@ -471,6 +472,7 @@ moe_status expert_cache_init(struct expert_cache **out, size_t capacity_bytes, i
         }
     }
     const int n = (int)std::max<size_t>(std::max<size_t>((size_t)L * E, S), (size_t)L * lw);
+    count_launch();
     lru_init_kernel<<<(n + 255) / 256, 256>>>(table_of(c));
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return fail(e, "cache init");
     *out = c;
@@ -485,6 +487,7 @@ moe_status expert_cache_prefetch(struct expert_cache *c, int layer, const int32_
     // the previous call's readback is complete (it was synchronised), so io is free
     c->h_io[0] = n;
     memcpy(c->h_io + 1, ids, sizeof(int32_t) * n);
+    count_launch();
     lru_kernel<<<1, 32, 0, st>>>(table_of(c), layer, nullptr, 0, 1, 0, c->d_io);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) e = cudaEventRecord(c->ev_lru, st);
@@ -506,6 +509,7 @@ moe_status expert_cache_evict(struct expert_cache *c, int layer, const int32_t *
     if (e != cudaSuccess) return set_cuda_error(e, "copy stream");
     c->h_io[0] = (layer < 0 || n < 0) ? -1 : n;
     if (layer >= 0 && n > 0) memcpy(c->h_io + 1, ids, sizeof(int32_t) * n);
+    count_launch();
     lru_evict_kernel<<<1, 32>>>(table_of(c), layer, c->d_io);
     e = cudaGetLastError();
     if (e == cudaSuccess) e = cudaDeviceSynchronize();

@@ -58,6 +58,7 @@ moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair
     int threads = H / 8;
     if (threads > 256) threads = 256;
     threads = (threads + 31) / 32 * 32;
+    count_launch();
     if (y_is_fp32)
         combine_kernel<true><<<T, threads, 0, st>>>(y_perm, pair_row, w, k, H, reinterpret_cast<__nv_bfloat16 *>(out));
     else

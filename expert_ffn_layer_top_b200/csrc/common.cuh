@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -17,6 +19,11 @@ namespace moe {
 // found on the device. Read and cleared by moe_device_error(). The library is
 // one translation unit (libmoe.cu), so this is the only definition.
 __device__ int g_dev_error = 0;
+
+// Kernels enqueued by the library in this process (all devices and streams),
+// returned by moe_kernel_launch_count().
+static std::atomic<unsigned long long> g_kernel_launches{0};
+inline void count_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, then give up and flag
 

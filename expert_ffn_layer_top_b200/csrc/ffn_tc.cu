@@ -13,9 +13,13 @@
 //   * N tile = BN permuted rows (tokens) of one expert, BN in {16,32,64,128}.
 //   * K stage = 128 elements; stages are handled in groups of kG = 2 (16 MMAs).
 //   * Warp roles (768 threads, one CTA per SM, persistent over work items):
-//       warp 0      producer: per stage one bulk copy of the prepacked weight
-//                   blob (or TMA boxes + a per-tile scale copy for row-major
-//                   weights) and a TMA box of activations (128-byte swizzle).
+//       warp 0      code producer: per stage one bulk copy of the prepacked
+//                   weight blob (or TMA boxes + a per-tile scale copy for
+//                   row-major weights) into a deep ring whose slots are freed
+//                   as soon as the decoders have read them.
+//       warp 2      activation producer: per group the TMA boxes of the
+//                   activation tiles (128-byte swizzle), freed by the group's
+//                   MMA completion.
 //       warp 1      owns TMEM; one lane issues tcgen05.mma (A from TMEM,
 //                   B from shared memory).
 //       warps 4-7   epilogue: tcgen05.ld of the fp32 accumulator, SwiGLU (UP)
@@ -28,7 +32,7 @@
 //     tensor pipe for ~100+ cycles, so the issuing thread synchronises once
 //     per group: it waits for the decoders of the group's last stage, issues
 //     16 MMAs, and commits once to the group's barrier, which then frees both
-//     the group's shared-memory stages and its TMEM slots.
+//     the group's activation tiles and its TMEM slots.
 //   * K order inside every 8-element group is 0,4,1,5,2,6,3,7 in both
 //     operands: one shift/multiply/mask then decodes an FP4 pair (k, k+4).
 //   * Every wait is bounded; on timeout the CTA sets the device error word,
@@ -42,7 +46,8 @@ constexpr int kThreads = 768;
 constexpr int kDecWarps = 16;       // warps 8..23
 constexpr int kBK = 128;            // K elements per stage
 constexpr int kG = 2;               // stages per MMA group (one commit, one wait)
-constexpr int kMaxStages = 16;      // shared-memory ring (multiple of kG)
+constexpr int kMaxStages = 16;      // code ring (stages)
+constexpr int kMaxBGroups = 8;      // activation ring (groups of kG stages)
 constexpr int kMaxAStages = 6;      // TMEM ring of decoded weight tiles (64 columns each, multiple of kG)
 constexpr int kXchStride = 17;      // padded row of the gate/up exchange buffer
 
@@ -98,8 +103,10 @@ __device__ __forceinline__ uint32_t mx_factor(uint32_t s8) { return bf16x2_splat
 __device__ __forceinline__ uint32_t mx_factor2(uint32_t s8) { return bf16x2_splat_bits((s8 > 128 ? s8 - 1 : 127u) << 7); }
 
 struct FfnSmem {
-    uint64_t full[kMaxStages];                 // stage landed (producer expect_tx + copies)
-    uint64_t gdone[kMaxStages / kG];           // group's MMAs complete (frees its stages and TMEM slots)
+    uint64_t rfull[kMaxStages];                // code stage landed (producer expect_tx + copies)
+    uint64_t rempty[kMaxStages];               // code stage read by all decoder warps
+    uint64_t bfull[kMaxBGroups];               // activation tiles of a group landed
+    uint64_t gdone[kMaxBGroups];               // group's MMAs complete (frees its activation tiles and TMEM slots)
     uint64_t adec[kMaxAStages];                // stage decoded into TMEM (one arrive per decoder warp)
     uint64_t accfull[2];
     uint64_t accempty[2];
@@ -150,15 +157,16 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     constexpr int RAWB = 128 * RB;                          // code bytes per stage
     constexpr int SB = RAWB + (TILED ? 128 * SBY : 0);      // smem bytes per stage (codes [+ scales])
     constexpr int BSTAGE = BN * 256;            // activation bytes per stage (two 64-column atoms)
+    constexpr int BGROUP = kG * BSTAGE;         // activation bytes per group
 
     // ---- shared memory carve-up (1024-aligned operand regions)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int nst = p.stages;                 // multiple of kG
-    const int na = p.astages;                 // TMEM A stages, multiple of kG
-    const int nsg = nst / kG;                 // groups in the shared-memory ring
+    const int nr = p.stages;                  // code ring depth (stages)
+    const int nbg = p.bgroups;                // activation ring depth (groups)
+    const int na = p.astages;                 // TMEM A stages, multiple of kG, na / kG <= nbg
     uint8_t *bstage = base;
-    uint8_t *rawst = bstage + nst * BSTAGE;
-    uint8_t *scbuf = rawst + nst * SB;
+    uint8_t *rawst = bstage + nbg * BGROUP;
+    uint8_t *scbuf = rawst + nr * SB;
     const int scb_bytes = TILED ? 0 : 128 * p.s_rowbytes;   // per tile buffer (standard layout only)
     float *xch = reinterpret_cast<float *>(scbuf + 2 * ((scb_bytes + 15) & ~15));
     FfnSmem &sm = *reinterpret_cast<FfnSmem *>(reinterpret_cast<uint8_t *>(xch) +
@@ -167,10 +175,16 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     const int warp = warp_id(), lane = lane_id();
     volatile int *abort_flag = &sm.abort_flag;
 
-    // ---- set-up: barriers (thread 0), TMEM (warp 1), tile prefix (warp 2)
+    // ---- set-up: barriers (thread 0), TMEM (warp 1), tile prefix (warp 3)
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMaxStages; ++s) mbar_init(&sm.full[s], 1);
-        for (int g = 0; g < kMaxStages / kG; ++g) mbar_init(&sm.gdone[g], 1);
+        for (int s = 0; s < kMaxStages; ++s) {
+            mbar_init(&sm.rfull[s], 1);
+            mbar_init(&sm.rempty[s], kDecWarps);
+        }
+        for (int g = 0; g < kMaxBGroups; ++g) {
+            mbar_init(&sm.bfull[g], 1);
+            mbar_init(&sm.gdone[g], 1);
+        }
         for (int s = 0; s < kMaxAStages; ++s) mbar_init(&sm.adec[s], kDecWarps);
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sm.accfull[a], 1);
@@ -184,15 +198,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
-        if (!TILED) tma_prefetch_desc(&wmap);
-        tma_prefetch_desc(&bmap);
-    }
+    if (warp == 0 && lane == 0 && !TILED) tma_prefetch_desc(&wmap);
+    if (warp == 2 && lane == 0) tma_prefetch_desc(&bmap);
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == 2) {
+    if (warp == 3) {
         int run = 0;
         if (lane == 0) sm.tile_start[0] = 0;
         for (int e0 = 0; e0 < p.E; e0 += 32) {
@@ -223,7 +235,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     const int KB = p.K / kBK;                     // multiple of kG
 
     if (warp == 0) {
-        // =================================================== producer
+        // =================================================== code producer
+        // Codes (and, tiled, their scales) stream through their own ring; a slot
+        // is refilled as soon as the 16 decoder warps have read it.
         if (lane == 0) {
             int kc = 0, lt = 0, s = 0;           // kc: stages issued so far
             uint32_t ph = 0;
@@ -245,10 +259,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                               &sm.scfull[sb]);
                 }
                 for (int kb = 0; kb < KB; ++kb) {
-                    // a group's stages are reused once the group's MMAs completed
-                    if ((s & (kG - 1)) == 0 && !mbar_wait(&sm.gdone[s / kG], ph ^ 1, abort_flag)) { ok = false; break; }
-                    uint64_t *fb = &sm.full[s];
-                    mbar_expect_tx(fb, SB + BSTAGE);
+                    if (!mbar_wait(&sm.rempty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+                    uint64_t *fb = &sm.rfull[s];
+                    mbar_expect_tx(fb, SB);
                     uint8_t *raw = rawst + s * SB;
                     if (TILED) {
                         const uint8_t *src = p.wbase + (int64_t)slot * p.w_estride +
@@ -265,18 +278,46 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                         tma_load_3d(raw, &wmap, fb, kcoord, rowA, slot);
                         tma_load_3d(raw + RAWB / 2, &wmap, fb, kcoord, rowB, slot);
                     }
-                    uint8_t *bs = bstage + s * BSTAGE;
-                    tma_load_2d(bs, &bmap, fb, kb * kBK, it.row0);
-                    tma_load_2d(bs + BN * 128, &bmap, fb, kb * kBK + 64, it.row0);
                     ++kc;
-                    if (++s == nst) { s = 0; ph ^= 1; }
+                    if (++s == nr) { s = 0; ph ^= 1; }
                 }
             }
             // drain: never leave the CTA while a copy into its shared memory is in
-            // flight - wait for the completion of the last min(kc, nst) stages issued
-            for (int j = kc - 1; j >= 0 && j >= kc - nst; --j) {
+            // flight - wait for the completion of the last min(kc, nr) stages issued
+            for (int j = kc - 1; j >= 0 && j >= kc - nr; --j) {
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full[j % nst], (j / nst) & 1)) {
+                while (!mbar_try_wait(&sm.rfull[j % nr], (j / nr) & 1)) {
+                    if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // =================================================== activation producer
+        // One barrier per group of kG stages; a group's tiles are refilled once
+        // the group's MMAs have completed.
+        if (lane == 0) {
+            int gc = 0, bg = 0;                  // gc: groups issued so far
+            uint32_t bph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const ItemInfo it = decode_item(sm, p, item, BN);
+                for (int kb = 0; kb < KB; kb += kG) {
+                    if (!mbar_wait(&sm.gdone[bg], bph ^ 1, abort_flag)) { ok = false; break; }
+                    uint64_t *fb = &sm.bfull[bg];
+                    mbar_expect_tx(fb, BGROUP);
+                    uint8_t *bs = bstage + bg * BGROUP;
+#pragma unroll
+                    for (int g = 0; g < kG; ++g) {
+                        tma_load_2d(bs + g * BSTAGE, &bmap, fb, (kb + g) * kBK, it.row0);
+                        tma_load_2d(bs + g * BSTAGE + BN * 128, &bmap, fb, (kb + g) * kBK + 64, it.row0);
+                    }
+                    ++gc;
+                    if (++bg == nbg) { bg = 0; bph ^= 1; }
+                }
+            }
+            for (int j = gc - 1; j >= 0 && j >= gc - nbg; --j) {
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(&sm.bfull[j % nbg], (j / nbg) & 1)) {
                     if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
                 }
             }
@@ -287,8 +328,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
             constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
             const uint32_t desc_hi = (uint32_t)(smem_desc_sw128(0) >> 32);
             const uint32_t desc_lo0 = (uint32_t)smem_desc_sw128(smem_u32(bstage));
-            int s = 0, sa = 0, lt = 0;
-            uint32_t pha = 0;
+            int bg = 0, sa = 0, lt = 0;
+            uint32_t bph = 0, pha = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
                 const int a = lt & 1;
@@ -296,13 +337,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t dcol = tmem + acc_col + a * BN;
                 for (int kb = 0; kb < KB; kb += kG) {
-                    // the decoders arrive stage by stage, so the group's last stage implies the rest;
-                    // they waited for its activation tiles too
+                    // decoders arrive stage by stage, so the group's last stage implies the rest
                     if (!mbar_wait(&sm.adec[sa + kG - 1], pha, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(&sm.bfull[bg], bph, abort_flag)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int g = 0; g < kG; ++g) {
-                        const uint32_t lo = desc_lo0 + ((uint32_t)((s + g) * BSTAGE) >> 4);
+                        const uint32_t lo = desc_lo0 + ((uint32_t)(bg * BGROUP + g * BSTAGE) >> 4);
                         const uint32_t atm = tmem + (sa + g) * 64;
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
@@ -310,9 +351,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                                              lo + (((i >> 2) * (BN * 128) + (i & 3) * 32) >> 4), desc_hi, idesc,
                                              (kb | g | i) != 0);
                     }
-                    mma_commit(&sm.gdone[s / kG]);
-                    s += kG;
-                    if (s == nst) s = 0;
+                    mma_commit(&sm.gdone[bg]);
+                    if (++bg == nbg) { bg = 0; bph ^= 1; }
                     sa += kG;
                     if (sa == na) { sa = 0; pha ^= 1; }
                 }
@@ -405,7 +445,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         const int m = q * 32 + lane;   // M-tile row
         const int rh = m >> 6, rr = m & 63;
         int lt = 0, s = 0, sa = 0, gstart = 0;   // gstart: groups started
-        uint32_t ph = 0, pha = 0;
+        uint32_t ph = 0;
         int lag_slot = 0;                        // group (gstart - na/kG) whose MMAs must have completed
         uint32_t lag_ph = 0;
         bool ok = true;
@@ -420,11 +460,11 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     // new group: its TMEM slots were last used by the group na/kG groups back
                     if (gstart >= na / kG) {
                         if (!mbar_wait(&sm.gdone[lag_slot], lag_ph, abort_flag)) { ok = false; break; }
-                        if (++lag_slot == nsg) { lag_slot = 0; lag_ph ^= 1; }
+                        if (++lag_slot == nbg) { lag_slot = 0; lag_ph ^= 1; }
                     }
                     ++gstart;
                 }
-                if (!mbar_wait(&sm.full[s], ph, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&sm.rfull[s], ph, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint8_t *raw = rawst + s * SB;
                 // 16-byte chunk c of this thread's row, and its scales for this stage
@@ -512,9 +552,12 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.adec[sa]);
-                if (++s == nst) { s = 0; ph ^= 1; }
-                if (++sa == na) { sa = 0; pha ^= 1; }
+                if (lane == 0) {
+                    mbar_arrive(&sm.adec[sa]);
+                    mbar_arrive(&sm.rempty[s]);   // codes read: the slot can be refilled
+                }
+                if (++s == nr) { s = 0; ph ^= 1; }
+                if (++sa == na) sa = 0;
             }
             if (!ok) break;
             if (FMT != MOE_BF16 && !TILED) {
@@ -522,7 +565,6 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 if (lane == 0) mbar_arrive(&sm.scempty[sb]);
             }
         }
-        (void)pha;
     }
 
     tc_fence_before();
@@ -605,6 +647,7 @@ moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscal
         case MOE_MXFP4: dequant_kernel<MOE_MXFP4><<<blocks, 256, 0, st>>>(wp, sp, tscale, rows, K, op); break;
         default: dequant_kernel<MOE_NVFP4><<<blocks, 256, 0, st>>>(wp, sp, tscale, rows, K, op); break;
     }
+    count_launch();
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "dequant launch");
 }
@@ -616,10 +659,10 @@ int stage_scale_bytes(int fmt) {
 }
 int stage_code_bytes(int fmt) { return fmt == MOE_BF16 ? 256 : fmt == MOE_FP8_E4M3_K128 ? 128 : 64; }
 
-static size_t ffn_smem_bytes(int fmt, int phase, int BN, int stages, int s_rowbytes, bool tiled) {
+static size_t ffn_smem_bytes(int fmt, int phase, int BN, int stages, int bgroups, int s_rowbytes, bool tiled) {
     const int rb = stage_code_bytes(fmt);
     size_t b = 1024;                                     // alignment slack
-    b += (size_t)stages * BN * 256;
+    b += (size_t)bgroups * kG * BN * 256;
     b += (size_t)stages * 128 * (rb + (tiled ? stage_scale_bytes(fmt) : 0));
     if (!tiled) b += 2 * (size_t)((128 * s_rowbytes + 15) & ~15);
     if (phase == kPhaseUp) b += 64 * kXchStride * 4;
@@ -633,6 +676,7 @@ static cudaError_t launch_one(const CUtensorMap &wmap, const CUtensorMap &bmap, 
     auto kfn = p.tiled ? ffn_tc_kernel<FMT, PHASE, BN, true> : ffn_tc_kernel<FMT, PHASE, BN, false>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     kfn<<<grid, kThreads, smem, st>>>(wmap, bmap, p);
     return cudaGetLastError();
 }
@@ -680,25 +724,33 @@ int scale_rowbytes(int fmt, int K) {
 moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap,
                             FfnParams p, int num_sms, cudaStream_t st) {
     if (p.K % (kBK * kG)) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", p.K, kBK * kG);
+    // TMEM: A ring of 64-column stages, then two accumulators of BN columns
+    int na = (512 - 2 * BN) / 64;
+    if (na > kMaxAStages) na = kMaxAStages;
+    na -= na % kG;
+    // Activation ring: one group more than the TMEM ring holds. The decoders
+    // wait on the group barrier of the group na/kG back; with at least that many
+    // activation groups no barrier can complete twice before that wait, so the
+    // parity check cannot alias.
+    int bgroups = na / kG + 1;
+    if (bgroups > kMaxBGroups) bgroups = kMaxBGroups;
     int stages = kMaxStages;
     size_t smem = 0;
-    for (; stages >= kG; stages -= kG) {
-        smem = ffn_smem_bytes(fmt, phase, BN, stages, p.s_rowbytes, p.tiled != 0);
-        if (smem <= 227 * 1024) break;
+    for (;;) {
+        for (stages = kMaxStages; stages >= 2; --stages) {
+            smem = ffn_smem_bytes(fmt, phase, BN, stages, bgroups, p.s_rowbytes, p.tiled != 0);
+            if (smem <= 227 * 1024) break;
+        }
+        if (stages >= 2) break;
+        if (bgroups == 1) return set_error(MOE_ERR_UNSUPPORTED, "FFN tile does not fit in shared memory");
+        --bgroups;
+        if (na > bgroups * kG) na = bgroups * kG;
     }
-    if (stages < kG) return set_error(MOE_ERR_UNSUPPORTED, "FFN tile does not fit in shared memory");
     // The CTA allocates all 512 TMEM columns: ask for enough shared memory that a
     // second CTA can never be co-resident on the SM (it would only block in alloc).
     if (smem < 120 * 1024) smem = 120 * 1024;
     p.stages = stages;
-    // TMEM: A ring of 64-column stages, then two accumulators of BN columns
-    int na = (512 - 2 * BN) / 64;
-    if (na > kMaxAStages) na = kMaxAStages;
-    // The decoders wait on the group barrier of the group na/kG back; with at
-    // least as many shared-memory groups as TMEM groups no barrier can complete
-    // twice before that wait, so the parity check cannot alias.
-    if (na > stages) na = stages;
-    na -= na % kG;
+    p.bgroups = bgroups;
     p.astages = na;
     // upper bound of work items; the kernel reads the exact count from the offsets
     const int64_t tiles_ub = (int64_t)p.n_rows / BN + p.E;

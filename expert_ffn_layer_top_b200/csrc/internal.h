@@ -23,6 +23,7 @@ struct FfnParams {
     int m_tiles;                // I/64 (up) or H/128 (down)
     int stages;                 // shared-memory ring depth, set by the launcher
     int astages;                // TMEM ring depth (decoded weight stages), set by the launcher
+    int bgroups;                // activation ring depth (groups of stages), set by the launcher
     const uint8_t *scale_base;  // scale plane of this phase's tensor (nullable for bf16)
     int64_t s_estride;          // bytes between experts in the scale plane
     int s_rowbytes;             // scale bytes per weight row

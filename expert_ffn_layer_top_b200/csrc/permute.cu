@@ -110,6 +110,82 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t *__r
     }
 }
 
+// Small batches (P <= kSmallP, E <= kSmallE): the whole counting sort in one
+// block - histogram, scan, then the chunks of 1024 pairs in order, each pair
+// placed at its expert's running position + its rank among equal experts of
+// earlier warps of the chunk + its rank inside its warp.
+constexpr int kSmallP = 8192;
+constexpr int kSmallE = 256;
+
+__global__ void __launch_bounds__(kChunk) perm_small_kernel(const int32_t *__restrict__ idx, int P, int E,
+                                                           int32_t *__restrict__ offsets,
+                                                           int32_t *__restrict__ sorted_pair,
+                                                           int32_t *__restrict__ pair_row) {
+    __shared__ int32_t cnt[kSmallE];
+    __shared__ int32_t run[kSmallE];
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t wcnt[kChunk / 32][kSmallE];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    for (int e = tid; e < E; e += kChunk) cnt[e] = 0;
+    __syncthreads();
+    for (int p = tid; p < P; p += kChunk) {
+        const int e = idx[p];
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        else flag_error(2);
+    }
+    __syncthreads();
+    // exclusive scan over experts (E <= 256: the first 8 warps hold one expert per lane)
+    int c = (tid < E) ? cnt[tid] : 0;
+    int incl = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    if (lane == 31) wsum[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int s = wsum[lane];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, s, d);
+            if (lane >= d) s += v;
+        }
+        wsum[lane] = s;   // inclusive over warps
+    }
+    __syncthreads();
+    if (tid < E) {
+        const int excl = incl - c + (wid > 0 ? wsum[wid - 1] : 0);
+        offsets[tid] = excl;
+        run[tid] = excl;
+    }
+    if (tid == 0) offsets[E] = P;
+    for (int c0 = 0; c0 < P; c0 += kChunk) {
+        for (int i = tid; i < (kChunk / 32) * E; i += kChunk) (&wcnt[0][0])[(i / E) * kSmallE + (i % E)] = 0;
+        __syncthreads();
+        const int p = c0 + tid;
+        int e = (p < P) ? idx[p] : -1 - lane;
+        if (p < P && (e < 0 || e >= E)) e = -1 - lane;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank_w = __popc(peers & ((1u << lane) - 1u));
+        if (e >= 0 && rank_w == 0) wcnt[wid][e] = __popc(peers);
+        __syncthreads();
+        if (e >= 0) {
+            int rank = run[e] + rank_w;
+            for (int w2 = 0; w2 < wid; ++w2) rank += wcnt[w2][e];
+            sorted_pair[rank] = p;
+            pair_row[p] = rank;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += kChunk) {
+            int add = 0;
+            for (int w2 = 0; w2 < kChunk / 32; ++w2) add += wcnt[w2][ee];
+            run[ee] += add;
+        }
+        __syncthreads();
+    }
+}
+
 __global__ void __launch_bounds__(256) perm_gather_kernel(const uint4 *__restrict__ x, int H8, int k,
                                                          const int32_t *__restrict__ sorted_pair, int P,
                                                          uint4 *__restrict__ x_perm) {
@@ -130,27 +206,37 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
         cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
         return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "memset offsets");
     }
-    const int C = (P + kChunk - 1) / kChunk;
-    const size_t half = align_up((size_t)C * E * sizeof(int32_t), 256);
-    if (ws_bytes < 2 * half) return set_error(MOE_ERR_OOM, "permute workspace too small");
-    int32_t *counts = reinterpret_cast<int32_t *>(ws);
-    int32_t *bases = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + half);
-    perm_count_kernel<<<C, kChunk, E * sizeof(int32_t), st>>>(idx, P, E, counts);
-    perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, C, E, P, bases, offsets);
-    const size_t sm_scatter = (size_t)(kChunk / 32) * E * sizeof(int32_t);
-    if (sm_scatter > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)sm_scatter);
-        if (e != cudaSuccess) return set_cuda_error(e, "scatter smem attribute");
+    cudaError_t e;
+    if (P <= kSmallP && E <= kSmallE) {
+        count_launch();
+        perm_small_kernel<<<1, kChunk, 0, st>>>(idx, P, E, offsets, sorted_pair, pair_row);
+    } else {
+        const int C = (P + kChunk - 1) / kChunk;
+        const size_t half = align_up((size_t)C * E * sizeof(int32_t), 256);
+        if (ws_bytes < 2 * half) return set_error(MOE_ERR_OOM, "permute workspace too small");
+        int32_t *counts = reinterpret_cast<int32_t *>(ws);
+        int32_t *bases = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + half);
+        count_launch();
+        perm_count_kernel<<<C, kChunk, E * sizeof(int32_t), st>>>(idx, P, E, counts);
+        count_launch();
+        perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, C, E, P, bases, offsets);
+        const size_t sm_scatter = (size_t)(kChunk / 32) * E * sizeof(int32_t);
+        if (sm_scatter > 48 * 1024) {
+            e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sm_scatter);
+            if (e != cudaSuccess) return set_cuda_error(e, "scatter smem attribute");
+        }
+        count_launch();
+        perm_scatter_kernel<<<C, kChunk, sm_scatter, st>>>(idx, P, E, bases, sorted_pair, pair_row);
     }
-    perm_scatter_kernel<<<C, kChunk, sm_scatter, st>>>(idx, P, E, bases, sorted_pair, pair_row);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "permute launch");
     if (x_perm) {
         const int H8 = H / 8;
         const int64_t total = (int64_t)P * H8;
         int blocks = (int)((total + 255) / 256);
         if (blocks > 148 * 16) blocks = 148 * 16;
+        count_launch();
         perm_gather_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4 *>(x), H8, k, sorted_pair, P,
                                                    reinterpret_cast<uint4 *>(x_perm));
         e = cudaGetLastError();

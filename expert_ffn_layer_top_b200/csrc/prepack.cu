@@ -74,6 +74,7 @@ moe_status launch_prepack(const moe_experts &in, int which, void *out, int64_t o
     const uint8_t *s = reinterpret_cast<const uint8_t *>(which == 0 ? in.w13_scale : in.w2_scale);
     const int64_t total = (int64_t)in.E * mt * KB * 128;
     const int blocks = (int)((total + 255) / 256);
+    count_launch();
     prepack_kernel<<<blocks, 256, 0, st>>>(w, w_es, s, s_es, in.E, in.I, K, which, mt, KB, RB, SBY, row_bytes,
                                            s_row_bytes, reinterpret_cast<uint8_t *>(out), out_estride);
     cudaError_t e = cudaGetLastError();

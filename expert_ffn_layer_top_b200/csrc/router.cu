@@ -9,11 +9,15 @@
 // Experts are ranked by logit (descending, ties to the lower index) and the
 // gate weights are a softmax over the k selected logits.
 //
-// Kernel 1 (partial): a block owns 16 tokens x all experts x one slice of H;
-// the slice count is chosen so small batches still fill the GPU. fp64 partial
-// sums go to the workspace. Kernel 2 (finish): one warp per token adds the
+// Up to 256 tokens: one launch of 8-CTA clusters that split H, reduce through
+// distributed shared memory and finish with one warp per token (below).
+// Larger batches: kernel 1 (partial) - a block owns 16 tokens x all experts x
+// one slice of H, the slice count chosen so the grid fills the GPU, fp64 partial
+// sums to the workspace; kernel 2 (finish) - one warp per token adds the
 // partials in slice order, rounds, adds the bias, selects the top k with warp
 // shuffles and writes idx, w (and optionally the logits).
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -192,10 +196,255 @@ __global__ void __launch_bounds__(256) router_finish_kernel(const double *__rest
     }
 }
 
+// Warp-wide top-k of the logits held as v[i] for expert lane + 32 i (experts
+// >= E excluded), descending, ties to the lower expert index; lane 0 writes
+// idx and the softmax over the selected logits.
+__device__ __forceinline__ void topk_softmax_warp(float (&v)[kMaxRouterExperts / 32], int E, int k, int lane,
+                                                  int32_t *idx_row, float *w_row) {
+    constexpr int kPer = kMaxRouterExperts / 32;
+    bool taken[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) taken[i] = lane + 32 * i >= E;
+    float selv[kMaxTopK];
+    int seli[kMaxTopK];
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            if (!taken[i] && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
+        }
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+#pragma unroll
+        for (int i = 0; i < kPer; ++i)
+            if (lane + 32 * i == bi) taken[i] = true;
+        selv[j] = bv;
+        seli[j] = bi;
+    }
+    if (lane == 0) {
+        const float l0 = selv[0];
+        float z = 0.0f;
+        for (int j = 0; j < k; ++j) z += expf(selv[j] - l0);
+        for (int j = 0; j < k; ++j) {
+            idx_row[j] = seli[j];
+            w_row[j] = expf(selv[j] - l0) / z;
+        }
+    }
+}
+
+// Small batches (T <= 256): one kernel, clusters of 8 CTAs. The 8 CTAs of a
+// cluster share a tile of TT tokens and split H into 8 contiguous slices; CTA r
+// streams rows [r H/8, (r+1) H/8) of Wr into shared memory with bulk copies (a
+// ring of chunks) and keeps fp64 sums for (token, expert) in registers: thread
+// (g, e) owns expert e for every token of the tile over the g-th part of each
+// chunk. The G parts are added in g order inside the CTA, then the 8 CTA sums in
+// rank order through distributed shared memory, so the result is one fixed
+// fp64 summation order. One warp per token rounds, biases and selects the top k.
+constexpr int kRCl = 8;              // CTAs per cluster (H slices)
+constexpr int kRClThreads = 256;
+constexpr int kRClChunkMax = 24576;  // bytes of Wr per ring chunk
+constexpr int kRClRing = 4;
+constexpr int kTokenKernelMaxT = 256;
+
+struct RouterClusterShape {
+    int TT;      // tokens per cluster tile (1, 2, 4, 8 or 16)
+    int Ep;      // E rounded up to a warp
+    int G;       // row groups per chunk (kRClThreads / Ep)
+    int hs;      // rows per CTA (H / 8)
+    int RC;      // rows per chunk
+    int nch;     // chunks per CTA
+    size_t smem;
+};
+
+static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClusterShape *sh) {
+    if (T > kTokenKernelMaxT || H % kRCl) return false;
+    const int eb = wr_is_fp32 ? 4 : 2;
+    if ((E * eb) % 16) return false;
+    sh->Ep = (E + 31) / 32 * 32;
+    sh->G = kRClThreads / sh->Ep;
+    sh->hs = H / kRCl;
+    int TT = 1;
+    while (TT < 16 && (T + TT - 1) / TT > 18) TT *= 2;
+    sh->TT = TT;
+    int rc = kRClChunkMax / (E * eb);
+    if (rc > sh->hs) rc = sh->hs;
+    int p = 1;
+    while (p * 2 <= rc) p *= 2;
+    while (p >= sh->G && (sh->hs % p || p % sh->G)) p /= 2;
+    if (p < sh->G || p < 1) return false;
+    sh->RC = p;
+    sh->nch = sh->hs / p;
+    const size_t ring = (size_t)kRClRing * p * E * eb;
+    const size_t red = (size_t)TT * kRClThreads * sizeof(double);
+    sh->smem = 64 + (ring > red ? ring : red) + (size_t)sh->hs * TT * sizeof(double);
+    return sh->smem <= 200 * 1024;
+}
+
+template <bool WR32, int TT>
+__global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
+    router_cluster_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, const void *__restrict__ wr, int E,
+                          int Ep, int G, int RC, int nch, const float *__restrict__ bias, int k,
+                          int32_t *__restrict__ idx, float *__restrict__ w, float *__restrict__ logits) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    constexpr int eb = WR32 ? 4 : 2;
+    extern __shared__ __align__(128) uint8_t rsm[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(rsm);            // [kRClRing]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(rsm + 48);
+    const int hs = H / kRCl;
+    const size_t chunk_bytes = (size_t)RC * E * eb;
+    const size_t ring = (size_t)kRClRing * chunk_bytes;
+    const size_t red_bytes = (size_t)TT * kRClThreads * sizeof(double);
+    uint8_t *wring = rsm + 64;
+    double *red = reinterpret_cast<double *>(rsm + 64);              // aliases the ring after the loop
+    double *xs = reinterpret_cast<double *>(rsm + 64 + (ring > red_bytes ? ring : red_bytes));   // [hs][TT]
+
+    const int tid = threadIdx.x;
+    const int rank = (int)cluster.block_rank();
+    const int t0 = blockIdx.y * TT;
+    const int h0 = rank * hs;
+    const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wr) + (size_t)h0 * E * eb;
+
+    if (tid == 0) {
+        for (int b = 0; b < kRClRing; ++b) mbar_init(&full[b], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        for (int c = 0; c < nch && c < kRClRing; ++c) {
+            mbar_expect_tx(&full[c], (uint32_t)chunk_bytes);
+            bulk_load(wring + c * chunk_bytes, wsrc + c * chunk_bytes, (uint32_t)chunk_bytes, &full[c]);
+        }
+    }
+    // x tile -> shared, as fp64 (exact), layout [h][tt]; tokens past T are zero
+    for (int i = tid; i < hs * TT; i += kRClThreads) {
+        const int tt = i / hs, h = i - tt * hs;
+        const int t = t0 + tt;
+        xs[h * TT + tt] = t < T ? (double)__bfloat162float(x[(int64_t)t * H + h0 + h]) : 0.0;
+    }
+    __syncthreads();
+
+    const int e = tid % Ep, g = tid / Ep;
+    const bool active = g < G && e < E;
+    const int rows_g = RC / G;
+    double acc[TT];
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) acc[tt] = 0.0;
+    for (int c = 0; c < nch; ++c) {
+        const int b = c % kRClRing;
+        mbar_wait(&full[b], (uint32_t)((c / kRClRing) & 1), abort_flag);
+        if (active) {
+            const uint8_t *wc = wring + b * chunk_bytes;
+            const int rb = g * rows_g;
+#pragma unroll 4
+            for (int r = rb; r < rb + rows_g; ++r) {
+                const double wv = WR32 ? (double)reinterpret_cast<const float *>(wc)[(size_t)r * E + e]
+                                       : (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(wc)[(size_t)r * E + e]);
+                const double *xr = xs + (size_t)(c * RC + r) * TT;
+                if constexpr (TT == 1) {
+                    acc[0] = fma(xr[0], wv, acc[0]);
+                } else {
+#pragma unroll
+                    for (int tt = 0; tt < TT; tt += 2) {
+                        const double2 xv = *reinterpret_cast<const double2 *>(xr + tt);
+                        acc[tt] = fma(xv.x, wv, acc[tt]);
+                        acc[tt + 1] = fma(xv.y, wv, acc[tt + 1]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && c + kRClRing < nch) {
+            mbar_expect_tx(&full[b], (uint32_t)chunk_bytes);
+            bulk_load(wring + b * chunk_bytes, wsrc + (size_t)(c + kRClRing) * chunk_bytes, (uint32_t)chunk_bytes,
+                      &full[b]);
+        }
+    }
+    // CTA sum over the row groups, in g order: red[tt][g * Ep + e]
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) red[tt * kRClThreads + tid] = acc[tt];
+    __syncthreads();
+    if (tid < E) {
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+            double s = red[tt * kRClThreads + tid];
+            for (int gg = 1; gg < G; ++gg) s += red[tt * kRClThreads + gg * Ep + tid];
+            red[tt * kRClThreads + tid] = s;
+        }
+    }
+    cluster.sync();
+    // cluster sum in rank order; token tt of the tile is finished by CTA tt % 8, warp tt / 8
+    constexpr int kPer = kMaxRouterExperts / 32;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int tt = rank + kRCl * warp;
+    if (tt < TT && t0 + tt < T) {
+        const int t = t0 + tt;
+        float v[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int ee = lane + 32 * i;
+            v[i] = 0.0f;
+            if (ee < E) {
+                double parts[kRCl];
+#pragma unroll
+                for (int q = 0; q < kRCl; ++q) parts[q] = cluster.map_shared_rank(red, q)[tt * kRClThreads + ee];
+                double sum = parts[0];
+#pragma unroll
+                for (int q = 1; q < kRCl; ++q) sum += parts[q];
+                float l = (float)sum;
+                if (bias) l = l + bias[ee];
+                v[i] = l;
+                if (logits) logits[(int64_t)t * E + ee] = l;
+            }
+        }
+        topk_softmax_warp(v, E, k, lane, idx + (int64_t)t * k, w + (int64_t)t * k);
+    }
+    cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
+}
+
+template <bool WR32, int TT>
+static cudaError_t launch_router_cluster_t(const RouterClusterShape &sh, const void *x, int T, int H, const void *wr,
+                                           int E, const float *bias, int k, int32_t *idx, float *w, float *logits,
+                                           cudaStream_t st) {
+    auto kern = router_cluster_kernel<WR32, TT>;
+    if (sh.smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh.smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid(kRCl, (T + TT - 1) / TT);
+    count_launch();
+    kern<<<grid, kRClThreads, sh.smem, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, sh.Ep, sh.G,
+                                             sh.RC, sh.nch, bias, k, idx, w, logits);
+    return cudaGetLastError();
+}
+
+template <bool WR32>
+static cudaError_t launch_router_cluster(const RouterClusterShape &sh, const void *x, int T, int H, const void *wr,
+                                         int E, const float *bias, int k, int32_t *idx, float *w, float *logits,
+                                         cudaStream_t st) {
+    switch (sh.TT) {
+    case 1: return launch_router_cluster_t<WR32, 1>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+    case 2: return launch_router_cluster_t<WR32, 2>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+    case 4: return launch_router_cluster_t<WR32, 4>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+    case 8: return launch_router_cluster_t<WR32, 8>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+    default: return launch_router_cluster_t<WR32, 16>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+    }
+}
+
 moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                          int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes, int nsm,
                          cudaStream_t st) {
     if (T == 0) return MOE_OK;
+    RouterClusterShape sh;
+    if (router_cluster_shape(T, H, E, wr_is_fp32, &sh) && (reinterpret_cast<uintptr_t>(wr) & 15) == 0) {
+        cudaError_t e = wr_is_fp32 ? launch_router_cluster<true>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st)
+                                   : launch_router_cluster<false>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+        return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "router_cluster launch");
+    }
     int S, slice;
     router_split(T, H, &S, &slice);
     (void)nsm;
@@ -203,6 +452,7 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
     if (ws_bytes < need) return set_error(MOE_ERR_OOM, "router workspace too small (%zu < %zu)", ws_bytes, need);
     double *part = reinterpret_cast<double *>(ws);
     dim3 grid((T + kTT - 1) / kTT, S);
+    count_launch();
     if (wr_is_fp32)
         router_partial_kernel<true><<<grid, kRThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr,
                                                                E, slice, part);
@@ -211,6 +461,7 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
                                                                 wr, E, slice, part);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "router_partial launch");
+    count_launch();
     router_finish_kernel<<<(T + 7) / 8, 256, 0, st>>>(part, S, T, E, bias, k, idx, w, logits);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "router_finish launch");

@@ -242,6 +242,12 @@ moe_status moe_device_error(int *code);
 /* Library version, for logs. */
 const char *moe_version(void);
 
+/* Number of kernels this library has enqueued in this process, on every device
+ * and stream, since it was loaded (a running count; the difference across a
+ * region is the launch count of that region). No counterpart in the pages:
+ * launch accounting for benchmarks. Never fails. */
+uint64_t moe_kernel_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,14 +63,19 @@ def test_dequantize_matches_oracle(moe, fmt):
 # ----------------------------------------------------------------------------- router
 
 
-ROUTER_CASES = [("tiny", 16), ("decode", 1), ("decode", 8), ("decode", 64), ("prefill", 4096), ("large", 32),
-                ("large", 1000)]
+ROUTER_CASES = [("tiny", 16), ("decode", 1), ("decode", 2), ("decode", 8), ("decode", 64), ("decode", 130),
+                ("decode", 256), ("decode", 257), ("prefill", 4096), ("large", 32), ("large", 200), ("large", 1000),
+                # odd shapes: 40 fp32 experts (one warp holds 64 expert slots), 12 bf16 experts (24-byte
+                # rows), H with an odd number of rows per eighth
+                (dict(H=512, E=40, k=5, wr_fp32=True, zipf=None), 77),
+                (dict(H=1024, E=12, k=3, wr_fp32=False, zipf=None), 50),
+                (dict(H=520, E=40, k=4, wr_fp32=False, zipf=None), 9)]
 
 
 @pytest.mark.parametrize("cfg,T", ROUTER_CASES)
 def test_router_parity(moe, cfg, T):
     wr, bias = synthetic.make_router(cfg, seed=1)
-    k = synthetic.CONFIGS[cfg]["k"]
+    k = (synthetic.CONFIGS[cfg] if isinstance(cfg, str) else cfg)["k"]
     x = synthetic.make_tokens(T, wr.shape[0], seed=1)
     idx_o, w_o, lg_o = oracle.route(x, wr, k, bias=bias)
     idx, w, lg = moe.moe_route_topk(x.cuda(), wr.cuda(), k, bias=None if bias is None else bias.cuda(),
