@@ -18,6 +18,7 @@ from ._lib import (  # noqa: F401
     moe_grouped_ffn,
     moe_layer_forward,
     moe_permute,
+    moe_permute_static,
     moe_prepack,
     moe_prepacked_expert_bytes,
     LAYOUT_STANDARD,

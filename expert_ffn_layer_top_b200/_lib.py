@@ -55,6 +55,8 @@ def lib():
             L.moe_route_topk.argtypes = [_P, _I, _I, _P, _I, _P, _I, _I, _P, _P, _P, _P, C.c_size_t, _P]
             L.moe_permute.restype = st
             L.moe_permute.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, C.c_size_t, _P]
+            L.moe_permute_static.restype = st
+            L.moe_permute_static.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P]
             L.moe_grouped_ffn.restype = st
             L.moe_grouped_ffn.argtypes = [_P, _I, _P, C.POINTER(_Experts), _P, _I, _P, C.c_size_t, _P]
             L.moe_combine.restype = st
@@ -208,6 +210,22 @@ def moe_permute(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = None, ws:
         ws = _ws(moe_workspace_size(T, max(H, 8), 128, E, k), dev)
     _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(x), H, _ptr(offsets), _ptr(sp), _ptr(pr), _ptr(x_perm),
                              _ptr(ws), ws.numel(), _stream()))
+    return offsets, sp[:P], pr[:P], (x_perm[:P] if x_perm is not None else None)
+
+
+def moe_permute_static(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = None):
+    """moe_permute with the library's fixed device scratch instead of a workspace."""
+    _need_cuda(idx, x)
+    T, k = idx.shape
+    dev = idx.device
+    P = T * k
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sp = torch.empty(max(P, 1), dtype=torch.int32, device=dev)
+    pr = torch.empty(max(P, 1), dtype=torch.int32, device=dev)
+    H = x.shape[1] if x is not None else 0
+    x_perm = torch.empty(max(P, 1), H, dtype=torch.bfloat16, device=dev) if x is not None else None
+    _check(lib().moe_permute_static(_ptr(idx), T, k, E, _ptr(x), H, _ptr(offsets), _ptr(sp), _ptr(pr),
+                                    _ptr(x_perm), _stream()))
     return offsets, sp[:P], pr[:P], (x_perm[:P] if x_perm is not None else None)
 
 

@@ -42,6 +42,37 @@ static int current_device() {
     return d;
 }
 
+// ------------------------------------------------------------------ fixed permutation scratch
+
+// Scratch of moe_permute_static: a module-scope device array, so every device
+// the library is loaded on has its own copy and nothing is allocated per call.
+static __device__ __align__(256) uint8_t g_permute_scratch[MOE_PERMUTE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxScratchDevices = 64;
+static void *g_permute_scratch_addr[kMaxScratchDevices];
+static std::mutex g_permute_scratch_mu;
+
+// Device address of the current device's scratch array, looked up on the first
+// call on that device and kept.
+static moe_status permute_scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return set_cuda_error(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxScratchDevices)
+        return set_error(MOE_ERR_UNSUPPORTED, "device %d: fixed scratch covers devices 0..%d", dev,
+                         kMaxScratchDevices - 1);
+    std::lock_guard<std::mutex> lock(g_permute_scratch_mu);
+    if (!g_permute_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress((void **)&p, g_permute_scratch);
+        if (e != cudaSuccess) return set_cuda_error(e, "cudaGetSymbolAddress(permute scratch)");
+        if (!p) return set_error(MOE_ERR_CUDA, "permute scratch has no device address");
+        g_permute_scratch_addr[dev] = p;
+    }
+    *out = g_permute_scratch_addr[dev];
+    return MOE_OK;
+}
+
 // ------------------------------------------------------------------ tensor maps
 
 typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -314,6 +345,21 @@ moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, i
         return set_error(MOE_ERR_INVALID_ARG, "x and x_perm must be 16-byte aligned");
     return launch_permute(idx, T, k, E, x, H, offsets, sorted_pair, pair_row, x_perm, ws, ws_bytes,
                           (cudaStream_t)stream);
+}
+
+moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+                              int32_t *sorted_pair, int32_t *pair_row, void *x_perm, moe_stream_t stream) {
+    if (T < 0 || k < 1 || k > kMaxTopK || E < 1 || E > kMaxExperts)
+        return set_error(MOE_ERR_INVALID_ARG, "bad T/k/E (%d %d %d)", T, k, E);
+    const size_t need = permute_scratch_bytes(T, k, E);
+    if (need > MOE_PERMUTE_STATIC_SCRATCH_BYTES)
+        return set_error(MOE_ERR_UNSUPPORTED, "T=%d k=%d E=%d needs %zu scratch bytes; the fixed scratch holds %u", T,
+                         k, E, need, (unsigned)MOE_PERMUTE_STATIC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    moe_status r = permute_scratch_address(&scratch);
+    if (r != MOE_OK) return r;
+    return moe_permute(idx, T, k, E, x, H, offsets, sorted_pair, pair_row, x_perm, scratch,
+                       MOE_PERMUTE_STATIC_SCRATCH_BYTES, stream);
 }
 
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,

@@ -62,6 +62,7 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
 
 // permutation (permute.cu)
 size_t permute_ws_bytes(int T, int k, int E);
+size_t permute_scratch_bytes(int T, int k, int E);
 moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
                           int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
                           cudaStream_t st);

@@ -186,6 +186,15 @@ __global__ void __launch_bounds__(kChunk) perm_small_kernel(const int32_t *__res
     }
 }
 
+// Workspace bytes launch_permute actually uses for these sizes: none on the
+// one-block path, else the per-chunk counters and bases.
+size_t permute_scratch_bytes(int T, int k, int E) {
+    const int64_t P = (int64_t)T * k;
+    if (P == 0 || (P <= kSmallP && E <= kSmallE)) return 0;
+    const int64_t C = (P + kChunk - 1) / kChunk;
+    return align_up((size_t)C * E * sizeof(int32_t), 256) * 2;
+}
+
 __global__ void __launch_bounds__(256) perm_gather_kernel(const uint4 *__restrict__ x, int H8, int k,
                                                          const int32_t *__restrict__ sorted_pair, int P,
                                                          uint4 *__restrict__ x_perm) {

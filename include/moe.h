@@ -134,6 +134,28 @@ moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, i
                        int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
 
+/* moe_permute without a caller workspace: the same permutation, bit for bit,
+ * with the scratch taken from a fixed device array inside the library instead
+ * of `ws`. The pages have no counterpart; it exists for callers that cannot
+ * hand over device memory (no allocation happens anywhere on this path).
+ *   Scratch limit: MOE_PERMUTE_STATIC_SCRATCH_BYTES per device. Sizes whose
+ *   scratch would exceed it (two arrays of ceil(T*k/1024)*E int32, each rounded
+ *   up to 256 bytes; none when T*k <= 8192 and E <= 256) are rejected with
+ *   MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *   No word of the scratch has to start at zero: every per-chunk counter and
+ *   base is written before it is read within one call, so nothing is cleared.
+ *   Set-up: the first call on a device looks the array's device address up
+ *   (one runtime call, not a stream operation); make that first call before
+ *   any stream capture on that device.
+ *   Concurrency: every call on a device shares the one array, so calls whose
+ *   kernels may overlap (different streams, or different host threads without
+ *   ordering) race on it; serialise them on one stream.
+ *   Arguments, layouts, ownership and the other errors are those of
+ *   moe_permute. */
+#define MOE_PERMUTE_STATIC_SCRATCH_BYTES (1u << 20)
+moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+                              int32_t *sorted_pair, int32_t *pair_row, void *x_perm, moe_stream_t stream);
+
 /* Grouped SwiGLU expert FFN over the permuted rows ([P4] formats): for every
  * expert e and row r in [offsets[e], offsets[e+1]):
  *   h = silu(Wg_e . x_perm[r]) * (Wu_e . x_perm[r]), rounded to bf16;
