@@ -225,7 +225,8 @@ def time_ffn_only(moe, lb: LayerBench, K: int, W: int, device):
         off, sp, pr, xp = moe.moe_permute(lb.idx[j], lb.layer.E, lb.xs[j])
         prep.append((xp, off))
     y = torch.empty(P, lb.layer.H, dtype=torch.float32 if lb.y32 else torch.bfloat16, device=device)
-    ws = torch.empty(P * lb.layer.I * 2 + 256, dtype=torch.uint8, device=device)
+    ws = torch.empty(moe.moe_workspace_size(P, lb.layer.H, lb.layer.I, lb.layer.E, 1, lb.y32), dtype=torch.uint8,
+                     device=device)
 
     def fn(i):
         j = i % len(prep)
@@ -242,7 +243,7 @@ def time_ffn_only(moe, lb: LayerBench, K: int, W: int, device):
 
 def source_sha():
     h = hashlib.sha256()
-    for f in ("ffn_tc.cu", "common.cuh"):
+    for f in ("ffn_tc.cu", "ffn_mx.cu", "common.cuh"):
         with open(os.path.join(ROOT, "expert_ffn_layer_top_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -332,7 +333,7 @@ def run_ours(args, rank, world, device):
     ffn_s, ffn_bytes = time_ffn_only(moe, lb, max(args.steps, 20), args.warmup, device)
     achieved = ffn_bytes / ffn_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": traffic_for("decode64_bytes_per_call"), "kernel": "grouped SwiGLU FFN (ffn_tc_kernel up + down)",
+                "traffic": traffic_for("decode64_bytes_per_call"), "kernel": "grouped SwiGLU FFN call (MXFP4 block-scaled: mx_quant_kernel + ffn_mx_kernel up + down)",
                 "peak_kind": peak_kind, "layer_achieved_gbs": layer_gbs}
 
     # end to end through the C ABI with host buffers: pinned x in, out back, every step

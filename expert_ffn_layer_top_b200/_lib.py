@@ -235,7 +235,7 @@ def moe_grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, experts: Expert
     n = x_perm.shape[0]
     y = torch.empty(max(n, 1), experts.H, dtype=torch.float32 if y_fp32 else torch.bfloat16, device=x_perm.device)
     if ws is None:
-        ws = _ws(n * experts.I * 2 + 256, x_perm.device)
+        ws = _ws(moe_workspace_size(max(n, 1), experts.H, experts.I, experts.E, 1, y_fp32), x_perm.device)
     _check(lib().moe_grouped_ffn(_ptr(x_perm), n, _ptr(offsets), C.byref(experts.c), _ptr(y), int(y_fp32), _ptr(ws),
                                  ws.numel(), _stream()))
     return y[:n]

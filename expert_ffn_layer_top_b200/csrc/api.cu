@@ -205,7 +205,98 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
     return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-static size_t ffn_ws_bytes(int n_rows, int I) { return align_up((size_t)n_rows * I * 2, 256); }
+// Scratch of the grouped FFN. Decoding path: h, bf16 [n][I] at offset 0.
+// Block-scaled MXFP4 path: E4M3 hi/lo planes of the permuted activations
+// [2][n][H] and of h [2][n][I], and the scale atoms of both.
+struct FfnWs {
+    size_t qx, q2, sf1, sf2, total;
+};
+
+static FfnWs ffn_ws(int n, int H, int I, int E) {
+    FfnWs W;
+    size_t o = 0;
+    W.qx = o; o += align_up((size_t)2 * n * H, 256);
+    W.q2 = o; o += align_up((size_t)2 * n * I, 256);
+    W.sf1 = o; o += mx_sf_bytes(n, H, E);
+    W.sf2 = o; o += mx_sf_bytes(n, I, E);
+    W.total = o > align_up((size_t)n * I * 2, 256) ? o : align_up((size_t)n * I * 2, 256);
+    return W;
+}
+
+static size_t ffn_ws_bytes(int n_rows, int H, int I, int E) { return ffn_ws(n_rows, H, I, E).total; }
+
+static bool is_mx(const moe_experts &x) { return x.fmt == MOE_MXFP4 && x.layout == MOE_LAYOUT_TILED; }
+
+// 4D map over prepacked MXFP4 codes: (128 codes, 128 rows, blocks of one
+// expert, experts or cache slots); TMA spreads every 16 codes over 16 bytes.
+static moe_status mx_weight_tmap(CUtensorMap *m, const void *base, int blocks, int64_t estride, int entries) {
+    if ((reinterpret_cast<uintptr_t>(base) & 31) || (estride & 31))
+        return set_error(MOE_ERR_UNSUPPORTED, "prepacked MXFP4 experts need 32-byte aligned bases and strides");
+    uint64_t dims[4] = {128, 128, (uint64_t)blocks, (uint64_t)entries};
+    uint64_t strides[3] = {64, (uint64_t)kMxBlobBytes, (uint64_t)estride};
+    uint32_t box[4] = {128, 128, 1, 1};
+    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, base, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// 3D map over E4M3 hi/lo planes [2][n][K]: boxes of 128 K bytes x BN rows.
+static moe_status mx_act_tmap(CUtensorMap *m, const void *base, int n, int K, int BN) {
+    uint64_t dims[3] = {(uint64_t)K, (uint64_t)n, 2};
+    uint64_t strides[2] = {(uint64_t)K, (uint64_t)n * K};
+    uint32_t box[3] = {128, (uint32_t)BN, 1};
+    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Block-scaled MXFP4 grouped FFN. The activations are quantised first: gathered
+// from token rows x[sorted_pair[r] / k] (gather != 0) or read from x_perm.
+static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sorted_pair, int k, int n_rows,
+                              const int32_t *offsets, const moe_experts *x, void *y_perm, int y_is_fp32, void *ws,
+                              cudaStream_t st) {
+    if (n_rows == 0) return MOE_OK;
+    const int E = x->E, H = x->H, I = x->I;
+    const Strides s = default_strides(*x);
+    const int nent = x->expert_map ? (int)(x->n_entries > 0 ? x->n_entries : E) : E;
+    const int BN = choose_bn_mx(n_rows, E);
+    const int nsm = num_sms(current_device());
+    const FfnWs W = ffn_ws(n_rows, H, I, E);
+    uint8_t *b = reinterpret_cast<uint8_t *>(ws);
+    moe_status r = launch_mx_quant(x_src, gather, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.qx, b + W.sf1,
+                                   nsm, st);
+    if (r != MOE_OK) return r;
+    CUtensorMap wmap, bmap;
+    MxParams p;
+    memset(&p, 0, sizeof(p));
+    p.offsets = offsets;
+    p.expert_map = x->expert_map;
+    p.E = E;
+    p.H = H;
+    p.I = I;
+    p.n_rows = n_rows;
+    // ---- gate/up + SwiGLU, h quantised for the down pass
+    if ((r = mx_weight_tmap(&wmap, x->w13, (I / 64) * (H / 128), s.w13, nent)) != MOE_OK) return r;
+    if ((r = mx_act_tmap(&bmap, b + W.qx, n_rows, H, BN)) != MOE_OK) return r;
+    p.K = H;
+    p.m_tiles = I / 64;
+    p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
+    p.w_estride = s.w13;
+    p.sfb = b + W.sf1;
+    p.q_out = b + W.q2;
+    p.sfb_out = b + W.sf2;
+    if ((r = launch_mx_phase(kPhaseUp, BN, wmap, bmap, p, nsm, st)) != MOE_OK) return r;
+    // ---- down projection
+    if ((r = mx_weight_tmap(&wmap, x->w2, (H / 128) * (I / 128), s.w2, nent)) != MOE_OK) return r;
+    if ((r = mx_act_tmap(&bmap, b + W.q2, n_rows, I, BN)) != MOE_OK) return r;
+    p.K = I;
+    p.m_tiles = H / 128;
+    p.wbase = reinterpret_cast<const uint8_t *>(x->w2);
+    p.w_estride = s.w2;
+    p.sfb = b + W.sf2;
+    p.q_out = nullptr;
+    p.sfb_out = nullptr;
+    p.out = y_perm;
+    p.out_fp32 = y_is_fp32;
+    return launch_mx_phase(kPhaseDown, BN, wmap, bmap, p, nsm, st);
+}
 
 // grouped FFN with explicit h buffer
 static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *x,
@@ -281,7 +372,7 @@ static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
     L.pair_row = o; o += align_up(P * 4, 256);
     L.perm = o; o += align_up(permute_ws_bytes(T, k, E), 256);
     L.x_perm = o; o += align_up(P * H * 2, 256);
-    L.h = o; o += ffn_ws_bytes((int)P, I);
+    L.h = o; o += ffn_ws_bytes((int)P, H, I, E);
     L.y = o; o += align_up(P * H * (y32 ? 4 : 2), 256);
     L.total = o;
     return L;
@@ -289,6 +380,7 @@ static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
 
 moe_status cache_resolve_and_map(struct expert_cache *c, int layer, const int32_t *idx, int T, int k,
                                  const moe_experts *shape, moe_experts *dev_view, cudaStream_t st);
+int cache_layout(const struct expert_cache *c);
 
 }  // namespace moe
 
@@ -369,9 +461,14 @@ moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offset
     if (n_rows < 0) return set_error(MOE_ERR_INVALID_ARG, "n_rows < 0");
     if (n_rows == 0) return MOE_OK;
     if (!x_perm || !offsets || !y_perm || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
-    if (ws_bytes < ffn_ws_bytes(n_rows, experts->I)) return set_error(MOE_ERR_OOM, "FFN workspace too small");
+    const size_t need = is_mx(*experts) ? ffn_ws_bytes(n_rows, experts->H, experts->I, experts->E)
+                                        : align_up((size_t)n_rows * experts->I * 2, 256);
+    if (ws_bytes < need) return set_error(MOE_ERR_OOM, "FFN workspace too small (%zu < %zu)", ws_bytes, need);
     if ((reinterpret_cast<uintptr_t>(x_perm) | reinterpret_cast<uintptr_t>(ws)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "x_perm and ws must be 16-byte aligned");
+    if (is_mx(*experts))
+        return mx_ffn_impl(x_perm, 0, nullptr, 1, n_rows, offsets, experts, y_perm, y_is_fp32, ws,
+                           (cudaStream_t)stream);
     return grouped_ffn_impl(x_perm, n_rows, offsets, experts, y_perm, y_is_fp32, ws, (cudaStream_t)stream);
 }
 
@@ -444,7 +541,11 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     moe_status r = moe_route_topk(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router,
                                   L.idx - L.router, stream);
     if (r != MOE_OK) return r;
-    r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, b + L.x_perm, b + L.perm, L.x_perm - L.perm, stream);
+    // The block-scaled MXFP4 path gathers the token rows itself while quantising them.
+    const int layout = cache ? cache_layout(cache) : experts->layout;
+    const bool mx = experts->fmt == MOE_MXFP4 && layout == MOE_LAYOUT_TILED;
+    r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, mx ? nullptr : b + L.x_perm, b + L.perm,
+                    L.x_perm - L.perm, stream);
     if (r != MOE_OK) return r;
     moe_experts view = *experts;
     if (cache) {
@@ -452,7 +553,11 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
         if (r != MOE_OK) return r;
         if ((r = check_experts(&view)) != MOE_OK) return r;
     }
-    r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+    if (is_mx(view) != mx) return set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
+    if (mx)
+        r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+    else
+        r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
     if (r != MOE_OK) return r;
     return moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
 }

@@ -368,6 +368,8 @@ moe_status cache_resolve_and_map(expert_cache *c, int layer, const int32_t *idx,
     return MOE_OK;
 }
 
+int cache_layout(const struct expert_cache *c) { return c->layout; }
+
 }  // namespace moe
 
 using namespace moe;

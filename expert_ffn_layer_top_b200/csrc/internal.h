@@ -36,6 +36,27 @@ struct FfnParams {
     int64_t w_estride;          // tiled: bytes between experts
 };
 
+// Block-scaled MXFP4 path (ffn_mx.cu): weights prepacked by moe_prepack, E4M3
+// hi/lo activations with per-tile scale atoms.
+constexpr int kMxBlobBytes = 128 * 64 + 512;   // prepacked MXFP4 bytes per (M tile, K stage)
+
+struct MxParams {
+    const int32_t *offsets;     // [E+1]
+    const int32_t *expert_map;  // nullable [E]
+    int E, H, I;
+    int K;                      // reduction dimension of this phase (H or I)
+    int m_tiles;                // I/64 (up) or H/128 (down)
+    int stages;                 // shared-memory ring depth, set by the launcher
+    int n_rows;
+    const uint8_t *wbase;       // this phase's prepacked tensor (codes + scale atoms per (M tile, stage))
+    int64_t w_estride;          // bytes between experts (or cache slots)
+    const uint8_t *sfb;         // activation scale atoms [tiles][K/128][512]
+    void *out;                  // down: y [n_rows][H] (bf16 or fp32)
+    int out_fp32;
+    uint8_t *q_out;             // up: E4M3 hi/lo planes of h [2][n_rows][I]
+    uint8_t *sfb_out;           // up: scale atoms of h [tiles][I/128][512]
+};
+
 // error reporting (thread-local message), defined in api.cu
 moe_status set_error(moe_status s, const char *fmt, ...);
 moe_status set_cuda_error(cudaError_t e, const char *what);
@@ -50,6 +71,14 @@ int scale_rowbytes(int fmt, int K);
 
 moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap,
                             FfnParams p, int num_sms, cudaStream_t st);
+
+int choose_bn_mx(int n_rows, int E);
+size_t mx_tiles_ub(int n_rows, int E);
+size_t mx_sf_bytes(int n_rows, int K, int E);
+moe_status launch_mx_phase(int phase, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap, MxParams p,
+                           int num_sms, cudaStream_t st);
+moe_status launch_mx_quant(const void *src, int gather, const int32_t *sorted_pair, int k, int P, int K,
+                           const int32_t *offsets, int E, int BN, void *q, void *sfb, int num_sms, cudaStream_t st);
 
 moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           cudaStream_t st);

@@ -5,5 +5,6 @@
 #include "permute.cu"
 #include "combine.cu"
 #include "ffn_tc.cu"
+#include "ffn_mx.cu"
 #include "prepack.cu"
 #include "cache.cu"

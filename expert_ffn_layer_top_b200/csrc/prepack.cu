@@ -1,12 +1,18 @@
 // Prepacking of expert weights into the tiled layout read by the grouped FFN.
 //
 // For every expert, M tile and 128-wide K stage the tiled layout holds one
-// contiguous blob: the 128 weight rows of the tile (gate/up: 64 gate rows then
-// the 64 matching up rows; down: 128 consecutive rows) as 16-byte chunks in
-// chunk-major order (chunk c of row r at (c*128 + r)*16), followed by each
-// row's scales for that stage. The grouped FFN then moves a stage with one
-// bulk copy and its decoder threads read consecutive 16-byte chunks without
-// bank conflicts. Values are untouched: this is a byte permutation.
+// contiguous blob with the 128 weight rows of the tile (gate/up: 64 gate rows
+// then the 64 matching up rows; down: 128 consecutive rows):
+//   BF16, FP8, NVFP4: the codes as 16-byte chunks in chunk-major order (chunk c
+//     of row r at (c*128 + r)*16), then each row's scales for that stage. The
+//     decoding FFN moves a stage with one bulk copy and its decoder threads
+//     read consecutive chunks without bank conflicts.
+//   MXFP4: the codes row after row (row r at r*64, natural K order), read by a
+//     TMA box that spreads them into the block-scaled MMA's operand layout,
+//     then a 512-byte scale atom: the E8M0 scale of row r and 32-block j of
+//     the stage at byte (r % 32)*16 + (r / 32)*4 + j, the arrangement tcgen05.cp
+//     moves into TMEM.
+// Values are untouched: this is a byte permutation.
 #include "common.cuh"
 #include "internal.h"
 
@@ -35,7 +41,7 @@ size_t prepacked_expert_bytes(int fmt, int H, int I, int which) {
 // One thread per (expert, M tile, K stage, tile row).
 __global__ void prepack_kernel(const uint8_t *__restrict__ w, int64_t w_estride, const uint8_t *__restrict__ scale,
                                int64_t s_estride, int E, int I, int K, int which, int m_tiles, int KB, int RB,
-                               int SBY, int row_bytes, int s_row_bytes, uint8_t *__restrict__ out,
+                               int SBY, int row_bytes, int s_row_bytes, int mx, uint8_t *__restrict__ out,
                                int64_t out_estride) {
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)E * m_tiles * KB * 128;
@@ -50,10 +56,16 @@ __global__ void prepack_kernel(const uint8_t *__restrict__ w, int64_t w_estride,
     const int64_t SB = 128LL * (RB + SBY);
     uint8_t *blob = out + e * out_estride + ((int64_t)m * KB + kb) * SB;
     const uint8_t *src = w + e * w_estride + (int64_t)row * row_bytes + (int64_t)kb * RB;
+    const uint8_t *ss = scale + e * s_estride + (int64_t)row * s_row_bytes + (int64_t)kb * SBY;
+    if (mx) {   // RB = 64, SBY = 4
+        for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4 *>(blob + r * 64 + c * 16) = *reinterpret_cast<const uint4 *>(src + c * 16);
+        for (int j = 0; j < 4; ++j) blob[128 * 64 + (r & 31) * 16 + (r >> 5) * 4 + j] = ss[j];
+        return;
+    }
     for (int c = 0; c < RB / 16; ++c)
         *reinterpret_cast<uint4 *>(blob + ((c * 128 + r) << 4)) = *reinterpret_cast<const uint4 *>(src + c * 16);
     if (SBY) {
-        const uint8_t *ss = scale + e * s_estride + (int64_t)row * s_row_bytes + (int64_t)kb * SBY;
         for (int i = 0; i < SBY; ++i) blob[128 * RB + r * SBY + i] = ss[i];
     }
     (void)K;
@@ -76,7 +88,8 @@ moe_status launch_prepack(const moe_experts &in, int which, void *out, int64_t o
     const int blocks = (int)((total + 255) / 256);
     count_launch();
     prepack_kernel<<<blocks, 256, 0, st>>>(w, w_es, s, s_es, in.E, in.I, K, which, mt, KB, RB, SBY, row_bytes,
-                                           s_row_bytes, reinterpret_cast<uint8_t *>(out), out_estride);
+                                           s_row_bytes, in.fmt == MOE_MXFP4, reinterpret_cast<uint8_t *>(out),
+                                           out_estride);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "prepack launch");
 }

@@ -75,9 +75,12 @@ typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3
 
 /* Memory layout of the expert codes. STANDARD: row-major as described above.
  * TILED: produced by moe_prepack; for every (M tile, 128-wide K stage) one
- * contiguous blob holding the 128 weight rows' codes (16-byte chunk-major) and
- * then their scales for that stage, so a stage is one bulk copy. The values
- * are the same; only the byte order differs. */
+ * contiguous blob holding the tile's 128 weight rows. BF16/FP8/NVFP4: codes
+ * 16-byte chunk-major, then the rows' scales for that stage (one bulk copy per
+ * stage). MXFP4: codes row after row (64 bytes per row), then a 512-byte atom
+ * with the scale of row r and 32-block j at byte (r%32)*16 + (r/32)*4 + j; this
+ * layout runs the block-scaled tensor-core path (bases and strides 32-byte
+ * aligned). The values are the same; only the byte order differs. */
 typedef enum { MOE_LAYOUT_STANDARD = 0, MOE_LAYOUT_TILED = 1 } moe_layout;
 
 /* The experts of one layer.
@@ -162,7 +165,10 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
  *   y_perm[r] = W2_e . h   (bf16, or fp32 if y_is_fp32).
  *   x_perm: bf16 [n_rows][H] in the interleaved layout written by moe_permute.
  *   y_perm: [n_rows][H], natural column order.
- *   ws: scratch for h ([n_rows][I] bf16).
+ *   ws: scratch; moe_workspace_size(n_rows, H, I, E, 1, y_is_fp32) bytes
+ *   always suffice. Row-major or BF16/FP8/NVFP4 experts keep h there
+ *   ([n_rows][I] bf16, operand column order); prepacked MXFP4 experts keep the
+ *   E4M3 hi/lo split of x_perm and of h (bf16-exact) and their scale atoms.
  *   Requires H % 256 == 0, I % 256 == 0, E <= 1024. n_rows == 0 is a no-op. */
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
                            void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);

@@ -132,6 +132,26 @@ def test_tiled_host_pool_streams_and_matches(moe, stack):
     cache.close()
 
 
+def test_mxfp4_prepacked_cache_matches_resident(moe):
+    """Prepacked MXFP4 experts run the block-scaled path; through the cache they
+    are addressed by slot, and the result must not change."""
+    cfg = dict(H=H_, E=E_, k=K_, I=I_, fmt="mxfp4", wr_fp32=False)
+    dev = [synthetic.make_layer(cfg, seed=31, layer=l).to("cuda") for l in range(2)]
+    packed = [moe.moe_prepack(moe.Experts.from_layer(L)) for L in dev]
+    host = [moe.Experts(t.fmt, t.E, t.H, t.I, t.w13.cpu().pin_memory(), t.w2.cpu().pin_memory(),
+                        layout=moe.LAYOUT_TILED) for t in packed]
+    cache = moe.ExpertCache(1 << 30, host, device=0)
+    for step in range(3):
+        for l in range(2):
+            x = synthetic.make_tokens(T_, H_, seed=70 + 5 * step + l).cuda()
+            out_c = moe.moe_layer_forward(x, dev[l].wr, K_, moe.Experts.from_layer(dev[l]), cache=cache, layer=l)
+            out_r = moe.moe_layer_forward(x, dev[l].wr, K_, packed[l])
+            torch.cuda.synchronize()
+            assert torch.equal(out_c, out_r), (step, l)
+    assert moe.moe_device_error() == 0
+    cache.close()
+
+
 def test_cache_full_is_reported(moe, stack):
     layers, host, dev = stack
     slot_bytes = sum(((t.numel() * t.element_size() // E_) + 255) // 256 * 256

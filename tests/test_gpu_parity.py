@@ -154,13 +154,17 @@ def test_combine_parity(moe, y_fp32):
 
 
 FFN_CASES = [(fmt, T, tiled) for fmt in ("bf16", "fp8", "mxfp4", "nvfp4") for T in (40, 100, 200, 600)
-             for tiled in (False, True)]
+             for tiled in (False, True)] + [("mxfp4", 24, True), ("mxfp4", 9, True)]
 
 
 @pytest.mark.parametrize("fmt,T,tiled", FFN_CASES)
 def test_grouped_ffn_parity(moe, fmt, T, tiled):
     """T = 40/100/200/600 with E = 8, k = 2 exercises token tiles of 16/32/64/128,
-    on row-major weights and on weights prepacked into the tiled layout."""
+    on row-major weights and on weights prepacked into the tiled layout.
+    Prepacked MXFP4 runs the block-scaled path (token tiles of 8/16/32/64; T = 9
+    and 24 give tiles of 8 with ragged tails), whose h never exists in bf16:
+    there the down-projection output is compared."""
+    mx = fmt == "mxfp4" and tiled
     cfg = dict(H=256, E=8, k=2, I=256, fmt=fmt, wr_fp32=False)
     L = synthetic.make_layer(cfg, seed=7)
     x = synthetic.make_tokens(T, 256, seed=7)
@@ -172,13 +176,18 @@ def test_grouped_ffn_parity(moe, fmt, T, tiled):
     if tiled:
         ex = moe.moe_prepack(ex)
     off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), 8, x.cuda())
-    ws = torch.empty(T * 2 * 256 * 2 + 256, dtype=torch.uint8, device="cuda")
-    y = moe.moe_grouped_ffn(xp, off, ex, ws=ws)
-    torch.cuda.synchronize()
-    h = ws[: T * 2 * 256 * 2].view(torch.bfloat16).view(T * 2, 256)
-    h_got = deinterleave_cols(h.float().cpu().numpy())
-    assert rel_err(h_got, h_o) < TOL, "gate/up + SwiGLU"
-    assert rel_err(bf16_np(y), y_o) < TOL, "down projection"
+    if mx:
+        y = moe.moe_grouped_ffn(xp, off, ex)
+        torch.cuda.synchronize()
+    else:
+        ws = torch.empty(T * 2 * 256 * 2 + 256, dtype=torch.uint8, device="cuda")
+        y = moe.moe_grouped_ffn(xp, off, ex, ws=ws)
+        torch.cuda.synchronize()
+        h = ws[: T * 2 * 256 * 2].view(torch.bfloat16).view(T * 2, 256)
+        h_got = deinterleave_cols(h.float().cpu().numpy())
+        assert rel_err(h_got, h_o) < TOL, "gate/up + SwiGLU"
+    err = rel_err(bf16_np(y), y_o)
+    assert err < TOL, f"down projection: error {err:.3e}, device error word {moe.moe_device_error()}"
     assert moe.moe_device_error() == 0
 
 
