@@ -227,24 +227,28 @@ static size_t ffn_ws_bytes(int n_rows, int H, int I, int E) { return ffn_ws(n_ro
 
 static bool is_mx(const moe_experts &x) { return x.fmt == MOE_MXFP4 && x.layout == MOE_LAYOUT_TILED; }
 
-// 4D map over prepacked MXFP4 codes: (128 codes, 128 rows, blocks of one
-// expert, experts or cache slots); TMA spreads every 16 codes over 16 bytes.
-static moe_status mx_weight_tmap(CUtensorMap *m, const void *base, int blocks, int64_t estride, int entries) {
+// 4D map over prepacked MXFP4 codes: (128 codes, 128 rows, K blocks of all M
+// tiles of one expert, experts or cache slots); a box is `sub` consecutive K
+// blocks. TMA spreads every 16 codes over 16 bytes.
+static moe_status mx_weight_tmap(CUtensorMap *m, const void *base, int blocks, int64_t estride, int entries,
+                                 int sub) {
     if ((reinterpret_cast<uintptr_t>(base) & 31) || (estride & 31))
         return set_error(MOE_ERR_UNSUPPORTED, "prepacked MXFP4 experts need 32-byte aligned bases and strides");
     uint64_t dims[4] = {128, 128, (uint64_t)blocks, (uint64_t)entries};
-    uint64_t strides[3] = {64, (uint64_t)kMxBlobBytes, (uint64_t)estride};
-    uint32_t box[4] = {128, 128, 1, 1};
+    uint64_t strides[3] = {64, (uint64_t)kMxCodeBlockBytes, (uint64_t)estride};
+    uint32_t box[4] = {128, 128, (uint32_t)sub, 1};
     return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, base, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// 3D map over E4M3 hi/lo planes [2][n][K]: boxes of 128 K bytes x BN rows.
-static moe_status mx_act_tmap(CUtensorMap *m, const void *base, int n, int K, int BN) {
-    uint64_t dims[3] = {(uint64_t)K, (uint64_t)n, 2};
-    uint64_t strides[2] = {(uint64_t)K, (uint64_t)n * K};
-    uint32_t box[3] = {128, (uint32_t)BN, 1};
-    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+// 4D map over the E4M3 hi/lo planes [2][n][K] viewed as (128 bytes of a K
+// block, row, plane, K block): one box holds, for `sub` consecutive K blocks,
+// BN hi rows followed by the same BN lo rows.
+static moe_status mx_act_tmap(CUtensorMap *m, const void *base, int n, int K, int BN, int sub) {
+    uint64_t dims[4] = {128, (uint64_t)n, 2, (uint64_t)(K / 128)};
+    uint64_t strides[3] = {(uint64_t)K, (uint64_t)n * K, 128};
+    uint32_t box[4] = {128, (uint32_t)BN, 2, (uint32_t)sub};
+    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Block-scaled MXFP4 grouped FFN. The activations are quantised first: gathered
@@ -273,8 +277,10 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.I = I;
     p.n_rows = n_rows;
     // ---- gate/up + SwiGLU, h quantised for the down pass
-    if ((r = mx_weight_tmap(&wmap, x->w13, (I / 64) * (H / 128), s.w13, nent)) != MOE_OK) return r;
-    if ((r = mx_act_tmap(&bmap, b + W.qx, n_rows, H, BN)) != MOE_OK) return r;
+    int sub = mx_stage_blocks(kPhaseUp, BN, H);
+    if (sub == 0) return set_error(MOE_ERR_UNSUPPORTED, "H=%d: no stage split for the MXFP4 path", H);
+    if ((r = mx_weight_tmap(&wmap, x->w13, (I / 64) * (H / 128), s.w13, nent, sub)) != MOE_OK) return r;
+    if ((r = mx_act_tmap(&bmap, b + W.qx, n_rows, H, BN, sub)) != MOE_OK) return r;
     p.K = H;
     p.m_tiles = I / 64;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
@@ -284,8 +290,10 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.sfb_out = b + W.sf2;
     if ((r = launch_mx_phase(kPhaseUp, BN, wmap, bmap, p, nsm, st)) != MOE_OK) return r;
     // ---- down projection
-    if ((r = mx_weight_tmap(&wmap, x->w2, (H / 128) * (I / 128), s.w2, nent)) != MOE_OK) return r;
-    if ((r = mx_act_tmap(&bmap, b + W.q2, n_rows, I, BN)) != MOE_OK) return r;
+    sub = mx_stage_blocks(kPhaseDown, BN, I);
+    if (sub == 0) return set_error(MOE_ERR_UNSUPPORTED, "I=%d: no stage split for the MXFP4 path", I);
+    if ((r = mx_weight_tmap(&wmap, x->w2, (H / 128) * (I / 128), s.w2, nent, sub)) != MOE_OK) return r;
+    if ((r = mx_act_tmap(&bmap, b + W.q2, n_rows, I, BN, sub)) != MOE_OK) return r;
     p.K = I;
     p.m_tiles = H / 128;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w2);

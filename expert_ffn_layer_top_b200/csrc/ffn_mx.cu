@@ -14,18 +14,9 @@
 // one MMA with N = 2 BN yields both products (the lo rows carry scale s - 4),
 // and the epilogue adds column j and column BN + j.
 //
-// Per item (N tile of BN rows of one expert x one M tile of 128 weight rows):
-//   warp 0      producer: per 128-wide K stage, one TMA box of FP4 codes
-//               (128 rows x 128 codes), one bulk copy of their scale atom, two
-//               TMA boxes of E4M3 activations (hi rows, lo rows) and one bulk
-//               copy of the activation scale atom, all on the stage's barrier.
-//   warp 1      TMEM owner and MMA issuer: two tcgen05.cp (scale atoms ->
-//               TMEM), four MMAs of K = 32, one commit that frees the stage.
-//   warp 2      per-expert tile prefix at start-up.
-//   warps 4-7   epilogue. DOWN: y = acc_hi + acc_lo. UP: gate/up rows meet
-//               through shared memory, h = silu(g) u is rounded to bf16 and
-//               split into the E4M3 hi/lo operand of the DOWN pass, with its
-//               scale atom, by the warp holding the 32 channels of a block.
+// Work item: an N tile of BN rows of one expert x one M tile of 128 weight rows
+// (UP: 64 gate rows and the matching 64 up rows; DOWN: 128 rows). The warp
+// roles are described at the kernel.
 // A scale atom is 512 bytes: byte (r % 32) * 16 + (r / 32) * 4 + j holds the
 // scale of operand row r and K block j of the stage; tcgen05.cp 32x128b.warpx4
 // puts atom row l into TMEM lanes l, l+32, l+64, l+96 (4 columns), which is
@@ -40,10 +31,9 @@
 
 namespace moe {
 
-constexpr int kMxThreads = 256;
+constexpr int kMxThreads = 384;
 constexpr int kMxBK = 128;                    // K elements per stage
 constexpr int kMxCodeBytes = 128 * 64;        // packed FP4 codes of one (M tile, stage)
-constexpr int kMxBlob = kMxBlobBytes;          // prepacked bytes per (M tile, stage): codes + scale atom
 constexpr int kMxMaxStages = 12;
 constexpr int kMxSfSlots = 4;                 // TMEM scale slots (8 columns each)
 constexpr int kMxSfCol = 256;                 // first TMEM column of the scale slots
@@ -224,10 +214,10 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
 struct MxSmem {
     uint64_t full[kMxMaxStages];
     uint64_t empty[kMxMaxStages];
-    uint64_t accfull[2];
-    uint64_t accempty[2];
-    uint64_t mmadone;
-    uint64_t xfull, xempty;
+    uint64_t accfull[2];      // both MMA warps commit
+    uint64_t accempty[2];     // the epilogue group of that buffer (128 threads)
+    uint64_t mmadone[2];
+    uint64_t xfull[2], xempty[2];   // gate/up exchange, per epilogue group
     uint32_t tmem_base;
     int abort_flag;
     int total_items;
@@ -255,22 +245,35 @@ __device__ __forceinline__ MxItem mx_item(const MxSmem &sm, const MxParams &p, i
     return it;
 }
 
+// Warp roles (384 threads, one CTA per SM, persistent over items):
+//   warp 0      producer; a stage is SUB consecutive 128-wide K blocks: one
+//               TMA box of FP4 codes (SUB blocks deep), one 4D TMA box of the
+//               E4M3 hi/lo rows, one bulk copy of each side's SUB scale atoms.
+//   warps 1, 3  MMA issuers; warp 1 takes the even stages of every item, warp 3
+//               the odd ones, each into its own accumulator, so one warp's
+//               waits, commits and scale copies overlap the other's MMAs. The
+//               epilogue adds the two accumulators. Warp 1 owns TMEM.
+//   warp 2      per-expert tile prefix at start-up.
+//   warps 4-7   epilogue of even items (accumulator buffer 0);
+//   warps 8-11  epilogue of odd items (buffer 1).
+// TMEM columns: accumulator (buffer a, MMA warp w) at (2a + w) N; scale slots
+// of MMA warp w at kMxSfCol + 32 w.
 template <int PHASE, int BN>
 __global__ void __launch_bounds__(kMxThreads, 1)
 ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap bmap, MxParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     constexpr int N = 2 * BN;                     // MMA N: hi rows then lo rows
-    constexpr int A_BYTES = 128 * 128;            // FP4 codes spread to one byte each
-    constexpr int B_BYTES = N * 128;
-    constexpr int STAGE = A_BYTES + B_BYTES + 1024;
-    // the transaction count of the FP4 box is its packed size: 4 bits per code
-    constexpr uint32_t TX = A_BYTES / 2 + B_BYTES + 1024;
+    constexpr int A_BYTES = 128 * 128;            // FP4 codes of one K block, one byte each in shared memory
+    constexpr int B_BYTES = N * 128;              // E4M3 rows of one K block
+    const int SUB = p.sub;
+    const int STAGE = SUB * (A_BYTES + B_BYTES + 1024);
+    const uint32_t TX = (uint32_t)SUB * (A_BYTES / 2 + B_BYTES + 1024);   // FP4 boxes count packed bytes
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int ns = p.stages;
-    float *xch = reinterpret_cast<float *>(base + ns * STAGE);
+    float *xch = reinterpret_cast<float *>(base + ns * STAGE);   // [2 groups][64][kMxXch]
     MxSmem &sm = *reinterpret_cast<MxSmem *>(reinterpret_cast<uint8_t *>(xch) +
-                                            (PHASE == kPhaseUp ? 64 * kMxXch * 4 : 0));
+                                            (PHASE == kPhaseUp ? 2 * 64 * kMxXch * 4 : 0));
     const int warp = warp_id(), lane = lane_id();
     volatile int *abort_flag = &sm.abort_flag;
 
@@ -280,12 +283,12 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
             mbar_init(&sm.empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&sm.accfull[a], 1);
+            mbar_init(&sm.accfull[a], 2);
             mbar_init(&sm.accempty[a], 128);
+            mbar_init(&sm.mmadone[a], 1);
+            mbar_init(&sm.xfull[a], 64);
+            mbar_init(&sm.xempty[a], 64);
         }
-        mbar_init(&sm.mmadone, 1);
-        mbar_init(&sm.xfull, 64);
-        mbar_init(&sm.xempty, 64);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -321,7 +324,8 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
 
     const uint32_t tmem = sm.tmem_base;
     const int total = sm.total_items;
-    const int KB = p.K / kMxBK;
+    const int KB = p.K / kMxBK;      // 128-wide K blocks
+    const int NST = KB / SUB;        // stages per item (>= 2)
 
     if (warp == 0) {
         // =================================================== producer
@@ -332,18 +336,19 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
                 const MxItem it = mx_item(sm, p, item, BN);
                 const int slot = p.expert_map ? p.expert_map[it.e] : it.e;
-                const uint8_t *wexp = p.wbase + (int64_t)slot * p.w_estride;
-                for (int kb = 0; kb < KB; ++kb) {
+                const uint8_t *sfa = p.wbase + (int64_t)slot * p.w_estride + (int64_t)p.m_tiles * KB * kMxCodeBytes;
+                for (int st = 0; st < NST; ++st) {
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
                     uint64_t *fb = &sm.full[s];
-                    uint8_t *st = base + s * STAGE;
+                    uint8_t *sp = base + s * STAGE;
+                    const int kb = st * SUB;
                     const int blk = it.m * KB + kb;
                     mbar_expect_tx(fb, TX);
-                    tma_load_4d(st, &wmap, fb, 0, 0, blk, slot);
-                    bulk_load(st + A_BYTES + B_BYTES, wexp + (int64_t)blk * kMxBlob + kMxCodeBytes, 512, fb);
-                    tma_load_3d(st + A_BYTES, &bmap, fb, kb * kMxBK, it.row0, 0);
-                    tma_load_3d(st + A_BYTES + BN * 128, &bmap, fb, kb * kMxBK, it.row0, 1);
-                    bulk_load(st + A_BYTES + B_BYTES + 512, p.sfb + ((int64_t)it.rt * KB + kb) * 512, 512, fb);
+                    tma_load_4d(sp, &wmap, fb, 0, 0, blk, slot);
+                    tma_load_4d(sp + SUB * A_BYTES, &bmap, fb, 0, it.row0, 0, kb);
+                    bulk_load(sp + SUB * (A_BYTES + B_BYTES), sfa + (int64_t)blk * 512, SUB * 512, fb);
+                    bulk_load(sp + SUB * (A_BYTES + B_BYTES) + SUB * 512, p.sfb + ((int64_t)it.rt * KB + kb) * 512,
+                              SUB * 512, fb);
                     ++issued;
                     if (++s == ns) { s = 0; ph ^= 1; }
                 }
@@ -356,74 +361,94 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 }
             }
         }
-    } else if (warp == 1) {
-        // =================================================== MMA issuer
+    } else if (warp == 1 || warp == 3) {
+        // =================================================== MMA issuers
+        const int w = warp >> 1;   // 0: even stages, 1: odd stages
         if (lane == 0) {
-            int s = 0, lt = 0, sc = 0;
-            uint32_t ph = 0;
+            int g = 0, lt = 0, sc = 0;   // g: stages of earlier items (ring position)
             bool ok = true;
             const uint32_t base_u32 = smem_u32(base);
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
                 const int a = lt & 1;
                 if (!mbar_wait(&sm.accempty[a], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem + a * N;
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&sm.full[s], ph, abort_flag)) { ok = false; break; }
+                const uint32_t d = tmem + (uint32_t)((2 * a + w) * N);
+                bool first = true;
+                for (int st = w; st < NST; st += 2) {
+                    const int gs = g + st;
+                    const int s = gs % ns;
+                    if (!mbar_wait(&sm.full[s], (uint32_t)((gs / ns) & 1), abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t st = base_u32 + s * STAGE;
-                    const uint32_t sfa = tmem + kMxSfCol + sc * 8, sfb = sfa + 4;
-                    tmem_cp_atom(sfa, sf_atom_desc(st + A_BYTES + B_BYTES));
-                    tmem_cp_atom(sfb, sf_atom_desc(st + A_BYTES + B_BYTES + 512));
-                    const uint64_t adesc = smem_desc_sw128(st);
-                    const uint64_t bdesc = smem_desc_sw128(st + A_BYTES);
+                    const uint32_t sp = base_u32 + s * STAGE;
+                    const uint32_t sfa_s = sp + SUB * (A_BYTES + B_BYTES), sfb_s = sfa_s + SUB * 512;
+                    for (int i = 0; i < SUB; ++i) {
+                        const uint32_t sfa = tmem + kMxSfCol + 32 * w + sc * 8, sfb = sfa + 4;
+                        tmem_cp_atom(sfa, sf_atom_desc(sfa_s + i * 512));
+                        tmem_cp_atom(sfb, sf_atom_desc(sfb_s + i * 512));
+                        const uint64_t adesc = smem_desc_sw128(sp + i * A_BYTES);
+                        const uint64_t bdesc = smem_desc_sw128(sp + SUB * A_BYTES + i * B_BYTES);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mma_mx(d, adesc + (uint64_t)((j * 32) >> 4), bdesc + (uint64_t)((j * 32) >> 4),
-                               idesc_mx(N, (uint32_t)j), sfa | ((uint32_t)j << 30), sfb | ((uint32_t)j << 30),
-                               (kb | j) != 0);
+                        for (int j = 0; j < 4; ++j) {
+                            mma_mx(d, adesc + (uint64_t)((j * 32) >> 4), bdesc + (uint64_t)((j * 32) >> 4),
+                                   idesc_mx(N, (uint32_t)j), sfa | ((uint32_t)j << 30), sfb | ((uint32_t)j << 30),
+                                   !first);
+                            first = false;
+                        }
+                        if (++sc == kMxSfSlots) sc = 0;
+                    }
                     mma_commit(&sm.empty[s]);
-                    if (++s == ns) { s = 0; ph ^= 1; }
-                    if (++sc == kMxSfSlots) sc = 0;
                 }
                 if (!ok) break;
                 mma_commit(&sm.accfull[a]);
+                g += NST;
             }
-            mma_commit(&sm.mmadone);
+            mma_commit(&sm.mmadone[w]);
             const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(&sm.mmadone, 0)) {
+            while (!mbar_try_wait(&sm.mmadone[w], 0)) {
                 if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
             }
         }
     } else if (warp >= 4) {
         // =================================================== epilogue
+        const int grp = (warp - 4) >> 2;   // 0: warps 4-7 (even items), 1: warps 8-11 (odd items)
         const int q = warp & 3;
-        const int lrow = q * 32 + lane;   // TMEM lane == M-tile row
-        int lt = 0, xc = 0;
+        const int lrow = q * 32 + lane;    // TMEM lane == M-tile row
+        float *xg = xch + grp * 64 * kMxXch;
+        int lt = grp, xc = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
+        for (int item = blockIdx.x + grp * gridDim.x; item < total && ok; item += 2 * gridDim.x, lt += 2) {
             const MxItem it = mx_item(sm, p, item, BN);
-            const int a = lt & 1;
+            const int a = grp;
             if (!mbar_wait(&sm.accfull[a], (lt >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t acc = tmem + ((uint32_t)(q * 32) << 16) + a * N;
+            const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(2 * a * N);
+            const uint32_t acc1 = acc0 + N;
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
             for (int c0 = 0; c0 < BN && ok; c0 += CH, ++xc) {
-                // sum of the hi and lo columns of tokens c0..c0+CH-1
+                // hi + lo columns of both accumulators for tokens c0..c0+CH-1
                 float val[16];
                 {
-                    uint32_t vh[16], vl[16];
+                    uint32_t v0[16], v1[16];
                     if (BN < 16) {
-                        tmem_ld16(acc, vh);   // columns 0..BN-1 hi, BN..2BN-1 lo
+                        tmem_ld16(acc0, v0);   // columns 0..BN-1 hi, BN..2BN-1 lo
+                        tmem_ld16(acc1, v1);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) val[j] = j < CH ? __uint_as_float(vh[j]) + __uint_as_float(vh[(j + BN) & 15]) : 0.0f;
+                        for (int j = 0; j < 16; ++j)
+                            val[j] = j < CH ? (__uint_as_float(v0[j]) + __uint_as_float(v0[(j + BN) & 15])) +
+                                                  (__uint_as_float(v1[j]) + __uint_as_float(v1[(j + BN) & 15]))
+                                            : 0.0f;
                     } else {
-                        tmem_ld16(acc + c0, vh);
-                        tmem_ld16(acc + BN + c0, vl);
+                        uint32_t u0[16], u1[16];
+                        tmem_ld16(acc0 + c0, v0);
+                        tmem_ld16(acc0 + BN + c0, u0);
+                        tmem_ld16(acc1 + c0, v1);
+                        tmem_ld16(acc1 + BN + c0, u1);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) val[j] = __uint_as_float(vh[j]) + __uint_as_float(vl[j]);
+                        for (int j = 0; j < 16; ++j)
+                            val[j] = (__uint_as_float(v0[j]) + __uint_as_float(u0[j])) +
+                                     (__uint_as_float(v1[j]) + __uint_as_float(u1[j]));
                     }
                 }
                 if (PHASE == kPhaseDown) {
@@ -438,16 +463,16 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     }
                 } else if (q >= 2) {
                     // up rows: hand the values to the warp holding the matching gate rows
-                    if (!mbar_wait(&sm.xempty, (xc & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(&sm.xempty[grp], (xc & 1) ^ 1, abort_flag)) { ok = false; break; }
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) xch[(lrow - 64) * kMxXch + j] = val[j];
-                    mbar_arrive(&sm.xfull);
+                    for (int j = 0; j < CH; ++j) xg[(lrow - 64) * kMxXch + j] = val[j];
+                    mbar_arrive(&sm.xfull[grp]);
                 } else {
-                    if (!mbar_wait(&sm.xfull, xc & 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(&sm.xfull[grp], xc & 1, abort_flag)) { ok = false; break; }
                     float u[16];
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) u[j] = xch[lrow * kMxXch + j];
-                    mbar_arrive(&sm.xempty);
+                    for (int j = 0; j < CH; ++j) u[j] = xg[lrow * kMxXch + j];
+                    mbar_arrive(&sm.xempty[grp]);
                     // channel ch = 64 m + 32 q + lane: this warp holds one 32-block of h
                     const int ch = it.m * 64 + lrow;
                     const int blk = ch >> 5;                // 32-block along I
@@ -456,9 +481,8 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     for (int j = 0; j < CH; ++j) {
                         const float g = val[j];
                         const float hv = __bfloat162float(__float2bfloat16_rn(g / (1.0f + __expf(-g)) * u[j]));
-                        float amax = fabsf(hv);
-#pragma unroll
-                        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+                        // block maximum: non-negative floats order like their bit patterns
+                        const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv))));
                         const int s = mx_block_exp(amax);
                         const float inv = __uint_as_float((uint32_t)(254 - s) << 23);
                         const float x = hv * inv;
@@ -496,8 +520,7 @@ int choose_bn_mx(int n_rows, int E) {
     const int avg = (n_rows + E - 1) / (E > 0 ? E : 1);
     if (avg <= 8) return 8;
     if (avg <= 16) return 16;
-    if (avg <= 32) return 32;
-    return 64;
+    return 32;
 }
 
 size_t mx_tiles_ub(int n_rows, int E) {
@@ -507,9 +530,9 @@ size_t mx_tiles_ub(int n_rows, int E) {
 
 size_t mx_sf_bytes(int n_rows, int K, int E) { return align_up(mx_tiles_ub(n_rows, E) * (K / kMxBK) * 512, 256); }
 
-static size_t mx_smem_bytes(int phase, int BN, int stages) {
-    const size_t stage = 128 * 128 + (size_t)2 * BN * 128 + 1024;
-    return 1024 + stages * stage + (phase == kPhaseUp ? 64 * kMxXch * 4 : 0) + sizeof(MxSmem);
+static size_t mx_smem_bytes(int phase, int BN, int sub, int stages) {
+    const size_t stage = (size_t)sub * (128 * 128 + (size_t)2 * BN * 128 + 1024);
+    return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 64 * kMxXch * 4 : 0) + sizeof(MxSmem);
 }
 
 template <int PHASE, int BN>
@@ -529,17 +552,31 @@ static cudaError_t mx_launch_bn(int BN, const CUtensorMap &wmap, const CUtensorM
     switch (BN) {
         case 8: return mx_launch_one<PHASE, 8>(wmap, bmap, p, grid, smem, st);
         case 16: return mx_launch_one<PHASE, 16>(wmap, bmap, p, grid, smem, st);
-        case 32: return mx_launch_one<PHASE, 32>(wmap, bmap, p, grid, smem, st);
-        default: return mx_launch_one<PHASE, 64>(wmap, bmap, p, grid, smem, st);
+        default: return mx_launch_one<PHASE, 32>(wmap, bmap, p, grid, smem, st);
     }
+}
+
+// K blocks per stage: the largest of 4, 3, 2, 1 that divides the block count,
+// leaves at least two stages per item (one per MMA warp) and at least four
+// stages in the ring.
+int mx_stage_blocks(int phase, int BN, int K) {
+    const int KB = K / kMxBK;
+    for (int sub = 4; sub >= 1; --sub) {
+        if (KB % sub || KB / sub < 2) continue;
+        if (mx_smem_bytes(phase, BN, sub, 4) <= 220 * 1024) return sub;
+    }
+    return 0;
 }
 
 moe_status launch_mx_phase(int phase, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap, MxParams p,
                            int num_sms, cudaStream_t st) {
     if (p.K % kMxBK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", p.K, kMxBK);
+    const int sub = mx_stage_blocks(phase, BN, p.K);
+    if (sub == 0) return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no stage split for the MXFP4 path", p.K);
+    p.sub = sub;
     int stages = kMxMaxStages;
-    while (stages > 2 && mx_smem_bytes(phase, BN, stages) > 200 * 1024) --stages;
-    size_t smem = mx_smem_bytes(phase, BN, stages);
+    while (stages > 4 && mx_smem_bytes(phase, BN, sub, stages) > 220 * 1024) --stages;
+    size_t smem = mx_smem_bytes(phase, BN, sub, stages);
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: it allocates all 512 TMEM columns
     p.stages = stages;
     const int64_t items_ub = ((int64_t)p.n_rows / BN + p.E) * p.m_tiles;

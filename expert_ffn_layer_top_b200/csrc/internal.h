@@ -38,7 +38,7 @@ struct FfnParams {
 
 // Block-scaled MXFP4 path (ffn_mx.cu): weights prepacked by moe_prepack, E4M3
 // hi/lo activations with per-tile scale atoms.
-constexpr int kMxBlobBytes = 128 * 64 + 512;   // prepacked MXFP4 bytes per (M tile, K stage)
+constexpr int kMxCodeBlockBytes = 128 * 64;   // prepacked MXFP4 codes of one (M tile, 128-wide K block)
 
 struct MxParams {
     const int32_t *offsets;     // [E+1]
@@ -47,8 +47,9 @@ struct MxParams {
     int K;                      // reduction dimension of this phase (H or I)
     int m_tiles;                // I/64 (up) or H/128 (down)
     int stages;                 // shared-memory ring depth, set by the launcher
+    int sub;                    // 128-wide K blocks per stage, set by the launcher
     int n_rows;
-    const uint8_t *wbase;       // this phase's prepacked tensor (codes + scale atoms per (M tile, stage))
+    const uint8_t *wbase;       // this phase's prepacked tensor (code blocks, then scale atoms)
     int64_t w_estride;          // bytes between experts (or cache slots)
     const uint8_t *sfb;         // activation scale atoms [tiles][K/128][512]
     void *out;                  // down: y [n_rows][H] (bf16 or fp32)
@@ -73,6 +74,7 @@ moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap,
                             FfnParams p, int num_sms, cudaStream_t st);
 
 int choose_bn_mx(int n_rows, int E);
+int mx_stage_blocks(int phase, int BN, int K);
 size_t mx_tiles_ub(int n_rows, int E);
 size_t mx_sf_bytes(int n_rows, int K, int E);
 moe_status launch_mx_phase(int phase, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap, MxParams p,
