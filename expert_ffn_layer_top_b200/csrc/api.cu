@@ -277,10 +277,10 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.I = I;
     p.n_rows = n_rows;
     // ---- gate/up + SwiGLU, h quantised for the down pass
-    int sub = mx_stage_blocks(kPhaseUp, BN, H);
-    if (sub == 0) return set_error(MOE_ERR_UNSUPPORTED, "H=%d: no stage split for the MXFP4 path", H);
-    if ((r = mx_weight_tmap(&wmap, x->w13, (I / 64) * (H / 128), s.w13, nent, sub)) != MOE_OK) return r;
-    if ((r = mx_act_tmap(&bmap, b + W.qx, n_rows, H, BN, sub)) != MOE_OK) return r;
+    MxPlan pl;
+    if (!mx_plan(kPhaseUp, BN, H, &pl)) return set_error(MOE_ERR_UNSUPPORTED, "H=%d: no MXFP4 pipeline plan", H);
+    if ((r = mx_weight_tmap(&wmap, x->w13, (I / 64) * (H / 128), s.w13, nent, pl.sub)) != MOE_OK) return r;
+    if ((r = mx_act_tmap(&bmap, b + W.qx, n_rows, H, BN, pl.sub)) != MOE_OK) return r;
     p.K = H;
     p.m_tiles = I / 64;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
@@ -290,10 +290,9 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.sfb_out = b + W.sf2;
     if ((r = launch_mx_phase(kPhaseUp, BN, wmap, bmap, p, nsm, st)) != MOE_OK) return r;
     // ---- down projection
-    sub = mx_stage_blocks(kPhaseDown, BN, I);
-    if (sub == 0) return set_error(MOE_ERR_UNSUPPORTED, "I=%d: no stage split for the MXFP4 path", I);
-    if ((r = mx_weight_tmap(&wmap, x->w2, (H / 128) * (I / 128), s.w2, nent, sub)) != MOE_OK) return r;
-    if ((r = mx_act_tmap(&bmap, b + W.q2, n_rows, I, BN, sub)) != MOE_OK) return r;
+    if (!mx_plan(kPhaseDown, BN, I, &pl)) return set_error(MOE_ERR_UNSUPPORTED, "I=%d: no MXFP4 pipeline plan", I);
+    if ((r = mx_weight_tmap(&wmap, x->w2, (H / 128) * (I / 128), s.w2, nent, pl.sub)) != MOE_OK) return r;
+    if ((r = mx_act_tmap(&bmap, b + W.q2, n_rows, I, BN, pl.sub)) != MOE_OK) return r;
     p.K = I;
     p.m_tiles = H / 128;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w2);

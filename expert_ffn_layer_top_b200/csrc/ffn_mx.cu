@@ -31,12 +31,11 @@
 
 namespace moe {
 
-constexpr int kMxThreads = 384;
+constexpr int kMxThreads = 512;
 constexpr int kMxBK = 128;                    // K elements per stage
 constexpr int kMxCodeBytes = 128 * 64;        // packed FP4 codes of one (M tile, stage)
 constexpr int kMxMaxStages = 12;
 constexpr int kMxSfSlots = 4;                 // TMEM scale slots (8 columns each)
-constexpr int kMxSfCol = 256;                 // first TMEM column of the scale slots
 constexpr int kMxXch = 17;
 
 // ------------------------------------------------------------------ device helpers
@@ -216,7 +215,7 @@ struct MxSmem {
     uint64_t empty[kMxMaxStages];
     uint64_t accfull[2];      // both MMA warps commit
     uint64_t accempty[2];     // the epilogue group of that buffer (128 threads)
-    uint64_t mmadone[2];
+    uint64_t mmadone[4];
     uint64_t xfull[2], xempty[2];   // gate/up exchange, per epilogue group
     uint32_t tmem_base;
     int abort_flag;
@@ -245,29 +244,36 @@ __device__ __forceinline__ MxItem mx_item(const MxSmem &sm, const MxParams &p, i
     return it;
 }
 
-// Warp roles (384 threads, one CTA per SM, persistent over items):
-//   warp 0      producer; a stage is SUB consecutive 128-wide K blocks: one
-//               TMA box of FP4 codes (SUB blocks deep), one 4D TMA box of the
-//               E4M3 hi/lo rows, one bulk copy of each side's SUB scale atoms.
-//   warps 1, 3  MMA issuers; warp 1 takes the even stages of every item, warp 3
-//               the odd ones, each into its own accumulator, so one warp's
-//               waits, commits and scale copies overlap the other's MMAs. The
-//               epilogue adds the two accumulators. Warp 1 owns TMEM.
-//   warp 2      per-expert tile prefix at start-up.
+// Warp roles (512 threads, one CTA per SM, persistent over items). The K
+// stages of an item are dealt round-robin to NP independent pipelines: pipeline
+// w (producer warp w, MMA warp 12 + w, its own ring of slots and its own
+// accumulators) handles stages w, w + NP, ... of every item, in order. One
+// producer fills and one issuer drains each slot, both in order, so every
+// parity wait on a slot barrier is exactly one phase after the previous one.
+//   warps 0-3   producers: per stage (SUB consecutive 128-wide K blocks) one
+//               TMA box of FP4 codes, one bulk copy of their scale atoms, one
+//               4D TMA box of the E4M3 hi/lo rows, one bulk copy of their scale
+//               atoms. Warp 2 also builds the per-expert tile prefix first.
+//   warps 12-15 MMA issuers (warp 12 owns TMEM).
 //   warps 4-7   epilogue of even items (accumulator buffer 0);
-//   warps 8-11  epilogue of odd items (buffer 1).
-// TMEM columns: accumulator (buffer a, MMA warp w) at (2a + w) N; scale slots
-// of MMA warp w at kMxSfCol + 32 w.
+//   warps 8-11  epilogue of odd items (buffer 1). The epilogue adds the NP
+//               pipelines' accumulators.
+// TMEM columns: accumulator (buffer a, pipeline w) at (a NW + w) N; four scale
+// slots of 8 columns per pipeline from 2 NW N on.
 template <int PHASE, int BN>
 __global__ void __launch_bounds__(kMxThreads, 1)
 ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap bmap, MxParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     constexpr int N = 2 * BN;                     // MMA N: hi rows then lo rows
+    constexpr int NW = N <= 32 ? 4 : 2;           // pipelines TMEM has room for
     constexpr int A_BYTES = 128 * 128;            // FP4 codes of one K block, one byte each in shared memory
     constexpr int B_BYTES = N * 128;              // E4M3 rows of one K block
     const int SUB = p.sub;
     const int STAGE = SUB * (A_BYTES + B_BYTES + 1024);
     const uint32_t TX = (uint32_t)SUB * (A_BYTES / 2 + B_BYTES + 1024);   // FP4 boxes count packed bytes
+    const uint32_t SFCOL = 2 * NW * N;                                   // first scale slot column
+    const int NP = p.pipes;                       // pipelines (divides the stages per item, <= NW)
+    const int NSW = p.stages / NP;                // slots per pipeline
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int ns = p.stages;
@@ -277,26 +283,29 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     const int warp = warp_id(), lane = lane_id();
     volatile int *abort_flag = &sm.abort_flag;
 
+    const int KB = p.K / kMxBK;      // 128-wide K blocks
+    const int NST = KB / SUB;        // stages per item
+    const int PER = NST / NP;        // stages per item and pipeline
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMxMaxStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&sm.accfull[a], 2);
+            mbar_init(&sm.accfull[a], NP);
             mbar_init(&sm.accempty[a], 128);
-            mbar_init(&sm.mmadone[a], 1);
             mbar_init(&sm.xfull[a], 64);
             mbar_init(&sm.xempty[a], 64);
         }
+        for (int w = 0; w < 4; ++w) mbar_init(&sm.mmadone[w], 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp < 4 && warp < NP && lane == 0) {
         tma_prefetch_desc(&wmap);
         tma_prefetch_desc(&bmap);
     }
-    if (warp == 1) {
+    if (warp == 12) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
@@ -324,21 +333,21 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
 
     const uint32_t tmem = sm.tmem_base;
     const int total = sm.total_items;
-    const int KB = p.K / kMxBK;      // 128-wide K blocks
-    const int NST = KB / SUB;        // stages per item (>= 2)
 
-    if (warp == 0) {
-        // =================================================== producer
-        if (lane == 0) {
-            int issued = 0, s = 0;
-            uint32_t ph = 0;
+    if (warp < 4) {
+        // =================================================== producer of pipeline w
+        const int w = warp;
+        if (lane == 0 && w < NP) {
+            int loc = 0;   // stages this pipeline has issued
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
                 const MxItem it = mx_item(sm, p, item, BN);
                 const int slot = p.expert_map ? p.expert_map[it.e] : it.e;
                 const uint8_t *sfa = p.wbase + (int64_t)slot * p.w_estride + (int64_t)p.m_tiles * KB * kMxCodeBytes;
-                for (int st = 0; st < NST; ++st) {
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+                for (int st = w; st < NST; st += NP, ++loc) {
+                    const int s = w * NSW + loc % NSW;
+                    const uint32_t round = (uint32_t)(loc / NSW);
+                    if (!mbar_wait(&sm.empty[s], (round & 1) ^ 1, abort_flag)) { ok = false; break; }
                     uint64_t *fb = &sm.full[s];
                     uint8_t *sp = base + s * STAGE;
                     const int kb = st * SUB;
@@ -349,58 +358,52 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     bulk_load(sp + SUB * (A_BYTES + B_BYTES), sfa + (int64_t)blk * 512, SUB * 512, fb);
                     bulk_load(sp + SUB * (A_BYTES + B_BYTES) + SUB * 512, p.sfb + ((int64_t)it.rt * KB + kb) * 512,
                               SUB * 512, fb);
-                    ++issued;
-                    if (++s == ns) { s = 0; ph ^= 1; }
                 }
             }
             // never leave while a copy into this CTA's shared memory is in flight
-            for (int j = issued - 1; j >= 0 && j >= issued - ns; --j) {
+            for (int j = loc - 1; j >= 0 && j >= loc - NSW; --j) {
+                const int s = w * NSW + j % NSW;
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full[j % ns], (j / ns) & 1)) {
+                while (!mbar_try_wait(&sm.full[s], (uint32_t)((j / NSW) & 1))) {
                     if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
                 }
             }
         }
-    } else if (warp == 1 || warp == 3) {
-        // =================================================== MMA issuers
-        const int w = warp >> 1;   // 0: even stages, 1: odd stages
-        if (lane == 0) {
-            int g = 0, lt = 0, sc = 0;   // g: stages of earlier items (ring position)
+    } else if (warp >= 12) {
+        // =================================================== MMA issuer of pipeline w
+        const int w = warp - 12;
+        if (lane == 0 && w < NP) {
+            int loc = 0, lt = 0, sc = 0;
             bool ok = true;
             const uint32_t base_u32 = smem_u32(base);
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
                 const int a = lt & 1;
                 if (!mbar_wait(&sm.accempty[a], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)((2 * a + w) * N);
-                bool first = true;
-                for (int st = w; st < NST; st += 2) {
-                    const int gs = g + st;
-                    const int s = gs % ns;
-                    if (!mbar_wait(&sm.full[s], (uint32_t)((gs / ns) & 1), abort_flag)) { ok = false; break; }
+                const uint32_t d = tmem + (uint32_t)((a * NW + w) * N);
+                for (int k = 0; k < PER; ++k, ++loc) {
+                    const int s = w * NSW + loc % NSW;
+                    if (!mbar_wait(&sm.full[s], (uint32_t)((loc / NSW) & 1), abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sp = base_u32 + s * STAGE;
                     const uint32_t sfa_s = sp + SUB * (A_BYTES + B_BYTES), sfb_s = sfa_s + SUB * 512;
                     for (int i = 0; i < SUB; ++i) {
-                        const uint32_t sfa = tmem + kMxSfCol + 32 * w + sc * 8, sfb = sfa + 4;
+                        const uint32_t sfa = tmem + SFCOL + 32 * w + sc * 8, sfb = sfa + 4;
                         tmem_cp_atom(sfa, sf_atom_desc(sfa_s + i * 512));
                         tmem_cp_atom(sfb, sf_atom_desc(sfb_s + i * 512));
                         const uint64_t adesc = smem_desc_sw128(sp + i * A_BYTES);
                         const uint64_t bdesc = smem_desc_sw128(sp + SUB * A_BYTES + i * B_BYTES);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
+                        for (int j = 0; j < 4; ++j)
                             mma_mx(d, adesc + (uint64_t)((j * 32) >> 4), bdesc + (uint64_t)((j * 32) >> 4),
                                    idesc_mx(N, (uint32_t)j), sfa | ((uint32_t)j << 30), sfb | ((uint32_t)j << 30),
-                                   !first);
-                            first = false;
-                        }
+                                   (k | i | j) != 0);
                         if (++sc == kMxSfSlots) sc = 0;
                     }
                     mma_commit(&sm.empty[s]);
                 }
                 if (!ok) break;
                 mma_commit(&sm.accfull[a]);
-                g += NST;
             }
             mma_commit(&sm.mmadone[w]);
             const uint64_t t0 = globaltimer();
@@ -408,7 +411,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
             }
         }
-    } else if (warp >= 4) {
+    } else {
         // =================================================== epilogue
         const int grp = (warp - 4) >> 2;   // 0: warps 4-7 (even items), 1: warps 8-11 (odd items)
         const int q = warp & 3;
@@ -421,34 +424,29 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
             const int a = grp;
             if (!mbar_wait(&sm.accfull[a], (lt >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(2 * a * N);
-            const uint32_t acc1 = acc0 + N;
+            const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NW * N);
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
             for (int c0 = 0; c0 < BN && ok; c0 += CH, ++xc) {
-                // hi + lo columns of both accumulators for tokens c0..c0+CH-1
+                // hi + lo columns of the pipelines' accumulators for tokens c0..c0+CH-1
                 float val[16];
-                {
-                    uint32_t v0[16], v1[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) val[j] = 0.0f;
+                for (int w = 0; w < NP; ++w) {
+                    const uint32_t acc = acc0 + w * N;
+                    uint32_t v[16];
                     if (BN < 16) {
-                        tmem_ld16(acc0, v0);   // columns 0..BN-1 hi, BN..2BN-1 lo
-                        tmem_ld16(acc1, v1);
+                        tmem_ld16(acc, v);   // columns 0..BN-1 hi, BN..2BN-1 lo
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            val[j] = j < CH ? (__uint_as_float(v0[j]) + __uint_as_float(v0[(j + BN) & 15])) +
-                                                  (__uint_as_float(v1[j]) + __uint_as_float(v1[(j + BN) & 15]))
-                                            : 0.0f;
+                            if (j < CH) val[j] += __uint_as_float(v[j]) + __uint_as_float(v[(j + BN) & 15]);
                     } else {
-                        uint32_t u0[16], u1[16];
-                        tmem_ld16(acc0 + c0, v0);
-                        tmem_ld16(acc0 + BN + c0, u0);
-                        tmem_ld16(acc1 + c0, v1);
-                        tmem_ld16(acc1 + BN + c0, u1);
+                        uint32_t u[16];
+                        tmem_ld16(acc + c0, v);
+                        tmem_ld16(acc + BN + c0, u);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            val[j] = (__uint_as_float(v0[j]) + __uint_as_float(u0[j])) +
-                                     (__uint_as_float(v1[j]) + __uint_as_float(u1[j]));
+                        for (int j = 0; j < 16; ++j) val[j] += __uint_as_float(v[j]) + __uint_as_float(u[j]);
                     }
                 }
                 if (PHASE == kPhaseDown) {
@@ -511,7 +509,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == 12) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ host side
@@ -556,29 +554,42 @@ static cudaError_t mx_launch_bn(int BN, const CUtensorMap &wmap, const CUtensorM
     }
 }
 
-// K blocks per stage: the largest of 4, 3, 2, 1 that divides the block count,
-// leaves at least two stages per item (one per MMA warp) and at least four
-// stages in the ring.
-int mx_stage_blocks(int phase, int BN, int K) {
+// Stage size, pipelines and ring depth of one phase: one 128-wide K block per
+// stage if possible (else two), as many pipelines as divide the stages of an
+// item and fit TMEM (4 for N <= 32, else 2), and at least two slots per
+// pipeline in at most 220 KiB of shared memory. Returns false if none fits.
+bool mx_plan(int phase, int BN, int K, MxPlan *pl) {
     const int KB = K / kMxBK;
-    for (int sub = 4; sub >= 1; --sub) {
-        if (KB % sub || KB / sub < 2) continue;
-        if (mx_smem_bytes(phase, BN, sub, 4) <= 220 * 1024) return sub;
+    const int nw = 2 * BN <= 32 ? 4 : 2;
+    for (int sub = 1; sub <= 2; ++sub) {
+        if (KB % sub) continue;
+        const int nst = KB / sub;
+        int fit = kMxMaxStages;
+        while (fit > 0 && mx_smem_bytes(phase, BN, sub, fit) > 220 * 1024) --fit;
+        for (int np = nw < nst ? nw : nst; np >= 1; --np) {
+            if (nst % np) continue;
+            int nsw = fit / np;
+            if (nsw > 4) nsw = 4;
+            if (nsw < 2) continue;
+            pl->sub = sub;
+            pl->pipes = np;
+            pl->stages = np * nsw;
+            return true;
+        }
     }
-    return 0;
+    return false;
 }
 
 moe_status launch_mx_phase(int phase, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap, MxParams p,
                            int num_sms, cudaStream_t st) {
     if (p.K % kMxBK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", p.K, kMxBK);
-    const int sub = mx_stage_blocks(phase, BN, p.K);
-    if (sub == 0) return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no stage split for the MXFP4 path", p.K);
-    p.sub = sub;
-    int stages = kMxMaxStages;
-    while (stages > 4 && mx_smem_bytes(phase, BN, sub, stages) > 220 * 1024) --stages;
-    size_t smem = mx_smem_bytes(phase, BN, sub, stages);
+    MxPlan pl;
+    if (!mx_plan(phase, BN, p.K, &pl)) return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no pipeline plan for MXFP4", p.K);
+    p.sub = pl.sub;
+    p.pipes = pl.pipes;
+    p.stages = pl.stages;
+    size_t smem = mx_smem_bytes(phase, BN, pl.sub, pl.stages);
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: it allocates all 512 TMEM columns
-    p.stages = stages;
     const int64_t items_ub = ((int64_t)p.n_rows / BN + p.E) * p.m_tiles;
     const int grid = (int)(items_ub < num_sms ? (items_ub > 0 ? items_ub : 1) : num_sms);
     cudaError_t e = phase == kPhaseUp ? mx_launch_bn<kPhaseUp>(BN, wmap, bmap, p, grid, smem, st)

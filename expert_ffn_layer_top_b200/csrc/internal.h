@@ -48,6 +48,7 @@ struct MxParams {
     int m_tiles;                // I/64 (up) or H/128 (down)
     int stages;                 // shared-memory ring depth, set by the launcher
     int sub;                    // 128-wide K blocks per stage, set by the launcher
+    int pipes;                  // independent producer/MMA pipelines, set by the launcher
     int n_rows;
     const uint8_t *wbase;       // this phase's prepacked tensor (code blocks, then scale atoms)
     int64_t w_estride;          // bytes between experts (or cache slots)
@@ -74,7 +75,10 @@ moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap,
                             FfnParams p, int num_sms, cudaStream_t st);
 
 int choose_bn_mx(int n_rows, int E);
-int mx_stage_blocks(int phase, int BN, int K);
+struct MxPlan {
+    int sub, pipes, stages;
+};
+bool mx_plan(int phase, int BN, int K, MxPlan *pl);
 size_t mx_tiles_ub(int n_rows, int E);
 size_t mx_sf_bytes(int n_rows, int K, int E);
 moe_status launch_mx_phase(int phase, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap, MxParams p,
