@@ -24,24 +24,43 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const int64_t base = (int64_t)rows[j] * H + c;
-            const float wj = ws[j];
+        // eight rows at a time: all loads issued first, then added in order of j
+        for (int j0 = 0; j0 < k; j0 += 8) {
             if (Y32) {
-                const float4 a = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(y_perm) + base);
-                const float4 b =
-                    *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(y_perm) + base + 4);
-                acc[0] += wj * a.x; acc[1] += wj * a.y; acc[2] += wj * a.z; acc[3] += wj * a.w;
-                acc[4] += wj * b.x; acc[5] += wj * b.y; acc[6] += wj * b.z; acc[7] += wj * b.w;
-            } else {
-                const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(y_perm) + base);
-                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                float4 a[8], b[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(p2[i]);
-                    acc[2 * i] += wj * f.x;
-                    acc[2 * i + 1] += wj * f.y;
-                }
+                for (int jj = 0; jj < 8; ++jj)
+                    if (j0 + jj < k) {
+                        const float *src = reinterpret_cast<const float *>(y_perm) + (int64_t)rows[j0 + jj] * H + c;
+                        a[jj] = *reinterpret_cast<const float4 *>(src);
+                        b[jj] = *reinterpret_cast<const float4 *>(src + 4);
+                    }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    if (j0 + jj < k) {
+                        const float wj = ws[j0 + jj];
+                        acc[0] += wj * a[jj].x; acc[1] += wj * a[jj].y; acc[2] += wj * a[jj].z; acc[3] += wj * a[jj].w;
+                        acc[4] += wj * b[jj].x; acc[5] += wj * b[jj].y; acc[6] += wj * b[jj].z; acc[7] += wj * b[jj].w;
+                    }
+            } else {
+                uint4 v[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    if (j0 + jj < k)
+                        v[jj] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(y_perm) +
+                                                                (int64_t)rows[j0 + jj] * H + c);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    if (j0 + jj < k) {
+                        const float wj = ws[j0 + jj];
+                        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v[jj]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = __bfloat1622float2(p2[i]);
+                            acc[2 * i] += wj * f.x;
+                            acc[2 * i + 1] += wj * f.y;
+                        }
+                    }
             }
         }
         uint4 o;

@@ -36,7 +36,7 @@ constexpr int kMxBK = 128;                    // K elements per stage
 constexpr int kMxCodeBytes = 128 * 64;        // packed FP4 codes of one (M tile, stage)
 constexpr int kMxMaxStages = 12;
 constexpr int kMxSfSlots = 4;                 // TMEM scale slots (8 columns each)
-constexpr int kMxXch = 17;
+constexpr int kMxXch = 9;    // padded row of the gate/up exchange (8 values)
 
 // ------------------------------------------------------------------ device helpers
 
@@ -178,31 +178,41 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
         const int tile = s_tile[lo] + rel / BN, n = rel % BN;
         const uint4 *srow = src + (int64_t)(gather ? sorted_pair[r] / k : r) * K8;
         uint8_t *atom0 = sfb + (int64_t)tile * KB * 512;
-        for (int c = lane; c < K8; c += 32) {
-            uint4 u = srow[c];
-            if (!gather) u = deinterleave8(u);
-            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-            float v[8];
-            float amax = 0.0f;
+        // four 16-byte chunks per lane in flight, then each is split
+        for (int c0 = lane; c0 < K8; c0 += 128) {
+            uint4 uu[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (c0 + 32 * i < K8) uu[i] = srow[c0 + 32 * i];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[i]));
-                v[2 * i] = f.x;
-                v[2 * i + 1] = f.y;
-                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            const int s = mx_block_exp(amax);
-            uint2 h2, l2;
-            mx_split8(v, s, h2, l2);
-            *reinterpret_cast<uint2 *>(q + (int64_t)r * K + c * 8) = h2;
-            *reinterpret_cast<uint2 *>(q + ((int64_t)P + r) * K + c * 8) = l2;
-            if ((c & 3) == 0) {
-                const int b = c >> 2;   // 32-block index along K
-                uint8_t *atom = atom0 + (b >> 2) * 512;
-                atom[atom_offset(n, b & 3)] = (uint8_t)s;
-                atom[atom_offset(n + BN, b & 3)] = (uint8_t)(s - 4);
+                const int c = c0 + 32 * i;
+                if (c >= K8) break;   // warp-uniform: K8 is a multiple of 32
+                uint4 u = uu[i];
+                if (!gather) u = deinterleave8(u);
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+                float v[8];
+                float amax = 0.0f;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[h]));
+                    v[2 * h] = f.x;
+                    v[2 * h + 1] = f.y;
+                    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                }
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                const int s = mx_block_exp(amax);
+                uint2 h2, l2;
+                mx_split8(v, s, h2, l2);
+                *reinterpret_cast<uint2 *>(q + (int64_t)r * K + c * 8) = h2;
+                *reinterpret_cast<uint2 *>(q + ((int64_t)P + r) * K + c * 8) = l2;
+                if ((c & 3) == 0) {
+                    const int b = c >> 2;   // 32-block along K
+                    uint8_t *atom = atom0 + (b >> 2) * 512;
+                    atom[atom_offset(n, b & 3)] = (uint8_t)s;
+                    atom[atom_offset(n + BN, b & 3)] = (uint8_t)(s - 4);
+                }
             }
         }
     }
@@ -277,9 +287,9 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int ns = p.stages;
-    float *xch = reinterpret_cast<float *>(base + ns * STAGE);   // [2 groups][64][kMxXch]
+    float *xch = reinterpret_cast<float *>(base + ns * STAGE);   // [2 groups][2 halves][64][kMxXch]
     MxSmem &sm = *reinterpret_cast<MxSmem *>(reinterpret_cast<uint8_t *>(xch) +
-                                            (PHASE == kPhaseUp ? 2 * 64 * kMxXch * 4 : 0));
+                                            (PHASE == kPhaseUp ? 2 * 128 * kMxXch * 4 : 0));
     const int warp = warp_id(), lane = lane_id();
     volatile int *abort_flag = &sm.abort_flag;
 
@@ -294,8 +304,8 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sm.accfull[a], NP);
             mbar_init(&sm.accempty[a], 128);
-            mbar_init(&sm.xfull[a], 64);
-            mbar_init(&sm.xempty[a], 64);
+            mbar_init(&sm.xfull[a], 128);
+            mbar_init(&sm.xempty[a], 128);
         }
         for (int w = 0; w < 4; ++w) mbar_init(&sm.mmadone[w], 1);
         sm.abort_flag = 0;
@@ -416,7 +426,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         const int grp = (warp - 4) >> 2;   // 0: warps 4-7 (even items), 1: warps 8-11 (odd items)
         const int q = warp & 3;
         const int lrow = q * 32 + lane;    // TMEM lane == M-tile row
-        float *xg = xch + grp * 64 * kMxXch;
+        float *xg = xch + grp * 128 * kMxXch;
         int lt = grp, xc = 0;
         bool ok = true;
         for (int item = blockIdx.x + grp * gridDim.x; item < total && ok; item += 2 * gridDim.x, lt += 2) {
@@ -426,24 +436,30 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
             tc_fence_after();
             const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NW * N);
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
+            constexpr int HCH = CH / 2;             // UP: tokens per warp of a gate/up pair
             for (int c0 = 0; c0 < BN && ok; c0 += CH, ++xc) {
                 // hi + lo columns of the pipelines' accumulators for tokens c0..c0+CH-1
                 float val[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) val[j] = 0.0f;
-                for (int w = 0; w < NP; ++w) {
-                    const uint32_t acc = acc0 + w * N;
-                    uint32_t v[16];
-                    if (BN < 16) {
-                        tmem_ld16(acc, v);   // columns 0..BN-1 hi, BN..2BN-1 lo
-                        tmem_wait_ld();
+                if (BN < 16) {
+                    uint32_t v[4][16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (j < CH) val[j] += __uint_as_float(v[j]) + __uint_as_float(v[(j + BN) & 15]);
-                    } else {
-                        uint32_t u[16];
-                        tmem_ld16(acc + c0, v);
-                        tmem_ld16(acc + BN + c0, u);
+                    for (int w = 0; w < 4; ++w)
+                        if (w < NP) tmem_ld16(acc0 + w * N, v[w]);   // columns 0..BN-1 hi, BN..2BN-1 lo
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        if (w < NP) {
+#pragma unroll
+                            for (int j = 0; j < CH; ++j)
+                                val[j] += __uint_as_float(v[w][j]) + __uint_as_float(v[w][(j + BN) & 15]);
+                        }
+                } else {
+                    for (int w = 0; w < NP; ++w) {
+                        uint32_t v[16], u[16];
+                        tmem_ld16(acc0 + w * N + c0, v);
+                        tmem_ld16(acc0 + w * N + BN + c0, u);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j) val[j] += __uint_as_float(v[j]) + __uint_as_float(u[j]);
@@ -459,26 +475,34 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                             else reinterpret_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(val[j]);
                         }
                     }
-                } else if (q >= 2) {
-                    // up rows: hand the values to the warp holding the matching gate rows
-                    if (!mbar_wait(&sm.xempty[grp], (xc & 1) ^ 1, abort_flag)) { ok = false; break; }
-#pragma unroll
-                    for (int j = 0; j < CH; ++j) xg[(lrow - 64) * kMxXch + j] = val[j];
-                    mbar_arrive(&sm.xfull[grp]);
                 } else {
-                    if (!mbar_wait(&sm.xfull[grp], xc & 1, abort_flag)) { ok = false; break; }
-                    float u[16];
+                    // Warp q < 2 holds the gate rows of channels 32 q..32 q+31 of this M tile,
+                    // warp q + 2 the up rows of the same channels. The gate warp finishes
+                    // tokens 0..HCH-1 of the chunk and the up warp tokens HCH..CH-1; each
+                    // hands the other the values of the other half through shared memory.
+                    const bool gate = q < 2;
+                    const int pr = q & 1;
+                    if (!mbar_wait(&sm.xempty[grp], (xc & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    float *mine = xg + ((gate ? 0 : 64) + pr * 32 + lane) * kMxXch;
+                    const float *theirs = xg + ((gate ? 64 : 0) + pr * 32 + lane) * kMxXch;
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) u[j] = xg[lrow * kMxXch + j];
+                    for (int j = 0; j < HCH; ++j) mine[j] = val[gate ? HCH + j : j];
+                    mbar_arrive(&sm.xfull[grp]);
+                    if (!mbar_wait(&sm.xfull[grp], xc & 1, abort_flag)) { ok = false; break; }
+                    float other[8];
+#pragma unroll
+                    for (int j = 0; j < HCH; ++j) other[j] = theirs[j];
                     mbar_arrive(&sm.xempty[grp]);
-                    // channel ch = 64 m + 32 q + lane: this warp holds one 32-block of h
-                    const int ch = it.m * 64 + lrow;
+                    const int t0 = gate ? 0 : HCH;   // first token of this warp's half
+                    // channel ch = 64 m + 32 pr + lane: this warp holds one 32-block of h
+                    const int ch = it.m * 64 + pr * 32 + lane;
                     const int blk = ch >> 5;                // 32-block along I
                     uint8_t *atom = p.sfb_out + ((int64_t)it.rt * (p.I / kMxBK) + (blk >> 2)) * 512;
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) {
-                        const float g = val[j];
-                        const float hv = __bfloat162float(__float2bfloat16_rn(g / (1.0f + __expf(-g)) * u[j]));
+                    for (int j = 0; j < HCH; ++j) {
+                        const float g = gate ? val[j] : other[j];
+                        const float uu = gate ? other[j] : val[HCH + j];
+                        const float hv = __bfloat162float(__float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * uu));
                         // block maximum: non-negative floats order like their bit patterns
                         const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv))));
                         const int s = mx_block_exp(amax);
@@ -488,13 +512,14 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                         const __half_raw hr = __nv_cvt_fp8_to_halfraw(hb, __NV_E4M3);
                         const float hf = __half2float(*reinterpret_cast<const __half *>(&hr));
                         const __nv_fp8_storage_t lb = __nv_cvt_float_to_fp8((x - hf) * 16.0f, __NV_SATFINITE, __NV_E4M3);
-                        if (c0 + j < it.nvalid) {
-                            const int64_t row = it.row0 + c0 + j;
+                        const int tok = c0 + t0 + j;
+                        if (tok < it.nvalid) {
+                            const int64_t row = it.row0 + tok;
                             p.q_out[row * p.I + ch] = hb;
                             p.q_out[((int64_t)p.n_rows + row) * p.I + ch] = lb;
                             if (lane == 0) {
-                                atom[atom_offset(c0 + j, blk & 3)] = (uint8_t)s;
-                                atom[atom_offset(c0 + j + BN, blk & 3)] = (uint8_t)(s - 4);
+                                atom[atom_offset(tok, blk & 3)] = (uint8_t)s;
+                                atom[atom_offset(tok + BN, blk & 3)] = (uint8_t)(s - 4);
                             }
                         }
                     }
@@ -530,7 +555,7 @@ size_t mx_sf_bytes(int n_rows, int K, int E) { return align_up(mx_tiles_ub(n_row
 
 static size_t mx_smem_bytes(int phase, int BN, int sub, int stages) {
     const size_t stage = (size_t)sub * (128 * 128 + (size_t)2 * BN * 128 + 1024);
-    return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 64 * kMxXch * 4 : 0) + sizeof(MxSmem);
+    return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 128 * kMxXch * 4 : 0) + sizeof(MxSmem);
 }
 
 template <int PHASE, int BN>

@@ -133,8 +133,80 @@ __global__ void __launch_bounds__(kRThreads) router_partial_kernel(const __nv_bf
     }
 }
 
-__device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
-    return v1 > v2 || (v1 == v2 && i1 < i2);
+// Exact widening to fp64 by moving the bit fields (the exponent is rebiased by
+// 1023 - 127 = 896); zeros and subnormals take the conversion instruction.
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
+    if ((b & 0x7F80u) == 0) return (double)__uint_as_float(b << 16);
+    const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + (896u << 20));
+    return __hiloint2double((int)hi, 0);
+}
+
+__device__ __forceinline__ double f32_bits_to_f64(uint32_t f) {
+    if ((f & 0x7F800000u) == 0) return (double)__uint_as_float(f);
+    const uint32_t hi = (f & 0x80000000u) | (((f & 0x7FFFFFFFu) >> 3) + (896u << 20));
+    return __hiloint2double((int)hi, (int)(f << 29));
+}
+
+// Order-preserving 32-bit key of an fp32 logit (larger logit, larger key);
+// -0 is folded into +0 so that equal logits always tie.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+    const uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Warp-wide top-k of the logits held as v[i] for expert lane + 32 i (experts
+// >= E excluded), descending, ties to the lower expert index, and the softmax
+// over the k selected logits. Each round takes the largest key with one
+// redux.sync and, among the lanes holding it, the lowest expert with a second;
+// the selection stays in registers. Lanes j < k write idx_row[j], w_row[j].
+__device__ __forceinline__ void topk_softmax_warp(float (&v)[kMaxRouterExperts / 32], int E, int k, int lane,
+                                                  int32_t *idx_row, float *w_row) {
+    constexpr int kPer = kMaxRouterExperts / 32;
+    uint32_t key[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) key[i] = lane + 32 * i < E ? logit_key(v[i]) : 0u;
+    float selv[kMaxTopK];
+    int seli[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        selv[j] = 0.0f;
+        seli[j] = 0;
+        if (j < k) {
+            // this lane's best remaining expert (lowest index among equal keys)
+            uint32_t bk = 0u;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i)
+                if (key[i] > bk) { bk = key[i]; bi = lane + 32 * i; }
+            const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+            const int win = (int)__reduce_min_sync(0xffffffffu, bk == mk ? (uint32_t)bi : 0x7fffffffu);
+#pragma unroll
+            for (int i = 0; i < kPer; ++i)
+                if (lane + 32 * i == win) key[i] = 0u;   // taken
+            selv[j] = key_logit(mk);
+            seli[j] = win;
+        }
+    }
+    // softmax over the selected logits, summed in selection order
+    const float l0 = selv[0];
+    float z = 0.0f, mine = 0.0f;
+    int myidx = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < k) {
+            const float e = expf(selv[j] - l0);
+            z += e;
+            if (j == lane) { mine = e; myidx = seli[j]; }
+        }
+    }
+    if (lane < k) {
+        idx_row[lane] = myidx;
+        w_row[lane] = mine / z;
+    }
 }
 
 __global__ void __launch_bounds__(256) router_finish_kernel(const double *__restrict__ part, int S, int T, int E,
@@ -146,11 +218,9 @@ __global__ void __launch_bounds__(256) router_finish_kernel(const double *__rest
     if (t >= T) return;
     constexpr int kPer = kMaxRouterExperts / 32;
     float v[kPer];
-    bool taken[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
-        taken[i] = true;
         v[i] = 0.0f;
         if (e < E) {
             double sum = 0.0;
@@ -158,84 +228,10 @@ __global__ void __launch_bounds__(256) router_finish_kernel(const double *__rest
             float l = (float)sum;
             if (bias) l = l + bias[e];
             v[i] = l;
-            taken[i] = false;
             if (logits) logits[(int64_t)t * E + e] = l;
         }
     }
-    float selv[kMaxTopK];
-    int seli[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int e = lane + 32 * i;
-            if (!taken[i] && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
-        }
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-        // owner marks it taken
-#pragma unroll
-        for (int i = 0; i < kPer; ++i)
-            if (lane + 32 * i == bi) taken[i] = true;
-        selv[j] = bv;
-        seli[j] = bi;
-    }
-    if (lane == 0) {
-        const float l0 = selv[0];
-        float z = 0.0f;
-        for (int j = 0; j < k; ++j) z += expf(selv[j] - l0);
-        for (int j = 0; j < k; ++j) {
-            idx[(int64_t)t * k + j] = seli[j];
-            w[(int64_t)t * k + j] = expf(selv[j] - l0) / z;
-        }
-    }
-}
-
-// Warp-wide top-k of the logits held as v[i] for expert lane + 32 i (experts
-// >= E excluded), descending, ties to the lower expert index; lane 0 writes
-// idx and the softmax over the selected logits.
-__device__ __forceinline__ void topk_softmax_warp(float (&v)[kMaxRouterExperts / 32], int E, int k, int lane,
-                                                  int32_t *idx_row, float *w_row) {
-    constexpr int kPer = kMaxRouterExperts / 32;
-    bool taken[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) taken[i] = lane + 32 * i >= E;
-    float selv[kMaxTopK];
-    int seli[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int e = lane + 32 * i;
-            if (!taken[i] && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
-        }
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-#pragma unroll
-        for (int i = 0; i < kPer; ++i)
-            if (lane + 32 * i == bi) taken[i] = true;
-        selv[j] = bv;
-        seli[j] = bi;
-    }
-    if (lane == 0) {
-        const float l0 = selv[0];
-        float z = 0.0f;
-        for (int j = 0; j < k; ++j) z += expf(selv[j] - l0);
-        for (int j = 0; j < k; ++j) {
-            idx_row[j] = seli[j];
-            w_row[j] = expf(selv[j] - l0) / z;
-        }
-    }
+    topk_softmax_warp(v, E, k, lane, idx + (int64_t)t * k, w + (int64_t)t * k);
 }
 
 // Small batches (T <= 256): one kernel, clusters of 8 CTAs. The 8 CTAs of a
@@ -254,8 +250,8 @@ constexpr int kTokenKernelMaxT = 256;
 
 struct RouterClusterShape {
     int TT;      // tokens per cluster tile (1, 2, 4, 8 or 16)
-    int Ep;      // E rounded up to a warp
-    int G;       // row groups per chunk (kRClThreads / Ep)
+    int EPP;     // expert pairs per row group, rounded up to a warp
+    int G;       // row groups per chunk (kRClThreads / EPP)
     int hs;      // rows per CTA (H / 8)
     int RC;      // rows per chunk
     int nch;     // chunks per CTA
@@ -263,11 +259,11 @@ struct RouterClusterShape {
 };
 
 static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClusterShape *sh) {
-    if (T > kTokenKernelMaxT || H % kRCl) return false;
+    if (T > kTokenKernelMaxT || H % kRCl || E % 2) return false;
     const int eb = wr_is_fp32 ? 4 : 2;
     if ((E * eb) % 16) return false;
-    sh->Ep = (E + 31) / 32 * 32;
-    sh->G = kRClThreads / sh->Ep;
+    sh->EPP = (E / 2 + 31) / 32 * 32;
+    sh->G = kRClThreads / sh->EPP;
     sh->hs = H / kRCl;
     int TT = 1;
     while (TT < 16 && (T + TT - 1) / TT > 18) TT *= 2;
@@ -281,7 +277,7 @@ static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClus
     sh->RC = p;
     sh->nch = sh->hs / p;
     const size_t ring = (size_t)kRClRing * p * E * eb;
-    const size_t red = (size_t)TT * kRClThreads * sizeof(double);
+    const size_t red = (size_t)TT * sh->G * 2 * sh->EPP * sizeof(double);
     sh->smem = 64 + (ring > red ? ring : red) + (size_t)sh->hs * TT * sizeof(double);
     return sh->smem <= 200 * 1024;
 }
@@ -289,7 +285,7 @@ static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClus
 template <bool WR32, int TT>
 __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     router_cluster_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, const void *__restrict__ wr, int E,
-                          int Ep, int G, int RC, int nch, const float *__restrict__ bias, int k,
+                          int EPP, int G, int RC, int nch, const float *__restrict__ bias, int k,
                           int32_t *__restrict__ idx, float *__restrict__ w, float *__restrict__ logits) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -300,7 +296,8 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     const int hs = H / kRCl;
     const size_t chunk_bytes = (size_t)RC * E * eb;
     const size_t ring = (size_t)kRClRing * chunk_bytes;
-    const size_t red_bytes = (size_t)TT * kRClThreads * sizeof(double);
+    const int E2 = 2 * EPP;                                        // expert slots per row group
+    const size_t red_bytes = (size_t)TT * G * E2 * sizeof(double);
     uint8_t *wring = rsm + 64;
     double *red = reinterpret_cast<double *>(rsm + 64);              // aliases the ring after the loop
     double *xs = reinterpret_cast<double *>(rsm + 64 + (ring > red_bytes ? ring : red_bytes));   // [hs][TT]
@@ -324,35 +321,58 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     for (int i = tid; i < hs * TT; i += kRClThreads) {
         const int tt = i / hs, h = i - tt * hs;
         const int t = t0 + tt;
-        xs[h * TT + tt] = t < T ? (double)__bfloat162float(x[(int64_t)t * H + h0 + h]) : 0.0;
+        xs[h * TT + tt] =
+            t < T ? bf16_bits_to_f64(reinterpret_cast<const uint16_t *>(x)[(int64_t)t * H + h0 + h]) : 0.0;
     }
     __syncthreads();
 
-    const int e = tid % Ep, g = tid / Ep;
-    const bool active = g < G && e < E;
+    // thread (g, ep) owns experts 2 ep and 2 ep + 1 for every token of the tile over
+    // rows [g rows_g, (g + 1) rows_g) of each chunk; NA independent fp64 sums per
+    // (token, expert) keep at least 8 FMA chains in flight, added in order at the end
+    const int ep = tid % EPP, g = tid / EPP;
+    const bool active = g < G && 2 * ep < E;
     const int rows_g = RC / G;
-    double acc[TT];
+    constexpr int NA = TT >= 4 ? 1 : 4 / TT;
+    double acc[TT][2][NA];
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) acc[tt] = 0.0;
+    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+        for (int a = 0; a < NA; ++a) acc[tt][0][a] = acc[tt][1][a] = 0.0;
     for (int c = 0; c < nch; ++c) {
         const int b = c % kRClRing;
         mbar_wait(&full[b], (uint32_t)((c / kRClRing) & 1), abort_flag);
         if (active) {
             const uint8_t *wc = wring + b * chunk_bytes;
             const int rb = g * rows_g;
-#pragma unroll 4
-            for (int r = rb; r < rb + rows_g; ++r) {
-                const double wv = WR32 ? (double)reinterpret_cast<const float *>(wc)[(size_t)r * E + e]
-                                       : (double)__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(wc)[(size_t)r * E + e]);
-                const double *xr = xs + (size_t)(c * RC + r) * TT;
-                if constexpr (TT == 1) {
-                    acc[0] = fma(xr[0], wv, acc[0]);
-                } else {
+            for (int r0 = rb; r0 < rb + rows_g; r0 += NA) {
 #pragma unroll
-                    for (int tt = 0; tt < TT; tt += 2) {
-                        const double2 xv = *reinterpret_cast<const double2 *>(xr + tt);
-                        acc[tt] = fma(xv.x, wv, acc[tt]);
-                        acc[tt + 1] = fma(xv.y, wv, acc[tt + 1]);
+                for (int a = 0; a < NA; ++a) {
+                    const int r = r0 + a;
+                    if (r < rb + rows_g) {
+                        double w0, w1;
+                        if (WR32) {
+                            const uint2 f = *reinterpret_cast<const uint2 *>(wc + ((size_t)r * E + 2 * ep) * 4);
+                            w0 = f32_bits_to_f64(f.x);
+                            w1 = f32_bits_to_f64(f.y);
+                        } else {
+                            const uint32_t bb = *reinterpret_cast<const uint32_t *>(wc + ((size_t)r * E + 2 * ep) * 2);
+                            w0 = bf16_bits_to_f64(bb & 0xFFFFu);
+                            w1 = bf16_bits_to_f64(bb >> 16);
+                        }
+                        const double *xr = xs + (size_t)(c * RC + r) * TT;
+                        if constexpr (TT == 1) {
+                            acc[0][0][a] = fma(xr[0], w0, acc[0][0][a]);
+                            acc[0][1][a] = fma(xr[0], w1, acc[0][1][a]);
+                        } else {
+#pragma unroll
+                            for (int tt = 0; tt < TT; tt += 2) {
+                                const double2 xv = *reinterpret_cast<const double2 *>(xr + tt);
+                                acc[tt][0][a] = fma(xv.x, w0, acc[tt][0][a]);
+                                acc[tt][1][a] = fma(xv.x, w1, acc[tt][1][a]);
+                                acc[tt + 1][0][a] = fma(xv.y, w0, acc[tt + 1][0][a]);
+                                acc[tt + 1][1][a] = fma(xv.y, w1, acc[tt + 1][1][a]);
+                            }
+                        }
                     }
                 }
             }
@@ -364,41 +384,64 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
                       &full[b]);
         }
     }
-    // CTA sum over the row groups, in g order: red[tt][g * Ep + e]
+    // CTA sum over the row groups, in g order: red[tt][g][e]
+    if (g < G) {
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) red[tt * kRClThreads + tid] = acc[tt];
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int x2 = 0; x2 < 2; ++x2) {
+                double sum = acc[tt][x2][0];
+#pragma unroll
+                for (int a = 1; a < NA; ++a) sum += acc[tt][x2][a];
+                red[((size_t)tt * G + g) * E2 + 2 * ep + x2] = sum;
+            }
+    }
     __syncthreads();
     if (tid < E) {
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
-            double s = red[tt * kRClThreads + tid];
-            for (int gg = 1; gg < G; ++gg) s += red[tt * kRClThreads + gg * Ep + tid];
-            red[tt * kRClThreads + tid] = s;
+            double sum = red[((size_t)tt * G) * E2 + tid];
+            for (int gg = 1; gg < G; ++gg) sum += red[((size_t)tt * G + gg) * E2 + tid];
+            red[((size_t)tt * G) * E2 + tid] = sum;
         }
     }
-    cluster.sync();
     // cluster sum in rank order; token tt of the tile is finished by CTA tt % 8, warp tt / 8
     constexpr int kPer = kMaxRouterExperts / 32;
     const int warp = tid >> 5, lane = tid & 31;
     const int tt = rank + kRCl * warp;
-    if (tt < TT && t0 + tt < T) {
+    const bool fin = tt < TT && t0 + tt < T;
+    float bv[kPer];   // bias, loaded before the cluster barrier
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) bv[i] = (fin && bias && lane + 32 * i < E) ? bias[lane + 32 * i] : 0.0f;
+    cluster.sync();
+    if (fin) {
         const int t = t0 + tt;
+        const double *src[kRCl];
+#pragma unroll
+        for (int q = 0; q < kRCl; ++q) src[q] = cluster.map_shared_rank(red, q) + (size_t)tt * G * E2;
         float v[kPer];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int ee = lane + 32 * i;
-            v[i] = 0.0f;
-            if (ee < E) {
-                double parts[kRCl];
+        for (int i0 = 0; i0 < kPer; i0 += 4) {
+            // all remote partial sums of four experts per lane in flight, then added in rank order
+            double parts[4][kRCl];
 #pragma unroll
-                for (int q = 0; q < kRCl; ++q) parts[q] = cluster.map_shared_rank(red, q)[tt * kRClThreads + ee];
-                double sum = parts[0];
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int q = 1; q < kRCl; ++q) sum += parts[q];
-                float l = (float)sum;
-                if (bias) l = l + bias[ee];
-                v[i] = l;
-                if (logits) logits[(int64_t)t * E + ee] = l;
+                for (int q = 0; q < kRCl; ++q)
+                    parts[i][q] = lane + 32 * (i0 + i) < E ? src[q][lane + 32 * (i0 + i)] : 0.0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int ee = lane + 32 * (i0 + i);
+                v[i0 + i] = 0.0f;
+                if (ee < E) {
+                    double sum = parts[i][0];
+#pragma unroll
+                    for (int q = 1; q < kRCl; ++q) sum += parts[i][q];
+                    float l = (float)sum;
+                    if (bias) l = l + bv[i0 + i];
+                    v[i0 + i] = l;
+                    if (logits) logits[(int64_t)t * E + ee] = l;
+                }
             }
         }
         topk_softmax_warp(v, E, k, lane, idx + (int64_t)t * k, w + (int64_t)t * k);
@@ -417,7 +460,7 @@ static cudaError_t launch_router_cluster_t(const RouterClusterShape &sh, const v
     }
     dim3 grid(kRCl, (T + TT - 1) / TT);
     count_launch();
-    kern<<<grid, kRClThreads, sh.smem, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, sh.Ep, sh.G,
+    kern<<<grid, kRClThreads, sh.smem, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, sh.EPP, sh.G,
                                              sh.RC, sh.nch, bias, k, idx, w, logits);
     return cudaGetLastError();
 }
