@@ -427,6 +427,8 @@ moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is
                          kMaxRouterExperts, E, k);
     if (T == 0) return MOE_OK;
     if (!x || !wr || !idx || !w || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(wr)) & 15)
+        return set_error(MOE_ERR_INVALID_ARG, "x and wr must be 16-byte aligned");
     return launch_router(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, logits, ws, ws_bytes,
                          num_sms(current_device()), (cudaStream_t)stream);
 }

@@ -11,11 +11,10 @@
 //
 // Up to 256 tokens: one launch of 8-CTA clusters that split H, reduce through
 // distributed shared memory and finish with one warp per token (below).
-// Larger batches: kernel 1 (partial) - a block owns 16 tokens x all experts x
-// one slice of H, the slice count chosen so the grid fills the GPU, fp64 partial
-// sums to the workspace; kernel 2 (finish) - one warp per token adds the
-// partials in slice order, rounds, adds the bias, selects the top k with warp
-// shuffles and writes idx, w (and optionally the logits).
+// Larger batches: kernel 1 (partial) - fp64 tensor-core tiles of 64 tokens x
+// 64 experts x one slice of H, fp64 partial sums to the workspace; kernel 2
+// (finish) - one warp per token adds the partials in slice order, rounds, adds
+// the bias, selects the top k and writes idx, w (and optionally the logits).
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -23,21 +22,28 @@
 
 namespace moe {
 
-constexpr int kTT = 16;   // tokens per block
-constexpr int kHC = 16;   // H rows per shared-memory chunk
-constexpr int kRThreads = 256;
-constexpr int kMaxPairs = kTT * kMaxRouterExperts / kRThreads;   // (token, expert) pairs per thread
+// Partial-sum kernel (fp64 tensor core): a block owns 64 tokens x 64 experts x
+// one slice of H; the slice count is chosen so the grid fills the GPU a few
+// times over. fp64 x and Wr tiles of 32 rows go through shared memory (double
+// buffered); each warp accumulates a 32 x 32 (token, expert) tile with
+// mma.sync.m8n8k4.f64, whose products of bf16 / fp32 inputs are exact and
+// whose sums are fp64 in a fixed order.
+constexpr int kDT = 64;          // tokens per block
+constexpr int kDE = 64;          // experts per block
+constexpr int kDK = 32;          // H rows per shared-memory stage
+constexpr int kDThreads = 128;
+constexpr int kXS = kDK + 4;     // x tile row stride (doubles): conflict-free A fragments
+constexpr int kWS = kDE + 4;     // Wr tile row stride (doubles): conflict-free B fragments
+constexpr int kTargetBlocks = 444;   // three blocks per SM of a 148-SM B200
 
-constexpr int kTargetBlocks = 296;   // two waves of a 148-SM B200
-
-static void router_split(int T, int H, int *S, int *slice) {
-    const int tb = (T + kTT - 1) / kTT;
-    int s = (kTargetBlocks + tb - 1) / tb;
-    const int maxs = H / kHC;
+static void router_split(int T, int H, int E, int *S, int *slice) {
+    const int tiles = ((T + kDT - 1) / kDT) * ((E + kDE - 1) / kDE);
+    int s = (kTargetBlocks + tiles - 1) / tiles;
+    const int maxs = (H + kDK - 1) / kDK;
     if (s > maxs) s = maxs;
     if (s < 1) s = 1;
     int sl = (H + s - 1) / s;
-    sl = (sl + kHC - 1) / kHC * kHC;
+    sl = (sl + kDK - 1) / kDK * kDK;
     *slice = sl;
     *S = (H + sl - 1) / sl;
 }
@@ -45,92 +51,14 @@ static void router_split(int T, int H, int *S, int *slice) {
 size_t router_ws_bytes(int T, int H, int E) {
     if (T <= 0) return 0;
     int S, slice;
-    router_split(T, H, &S, &slice);
+    router_split(T, H, E, &S, &slice);
     return align_up((size_t)S * T * E * sizeof(double), 256);
 }
 
-template <bool WR32>
-__global__ void __launch_bounds__(kRThreads) router_partial_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H,
-                                                                  const void *__restrict__ wr, int E, int slice,
-                                                                  double *__restrict__ part) {
-    __shared__ double xs[kTT][kHC];
-    __shared__ double wsm[kHC][kMaxRouterExperts];
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.x * kTT;
-    const int s = blockIdx.y;
-    const int hb = s * slice;
-    const int he = min(H, hb + slice);
-    const int npairs = kTT * E;
-    double acc[kMaxPairs];
-#pragma unroll
-    for (int i = 0; i < kMaxPairs; ++i) acc[i] = 0.0;
-
-    // per-thread share of one chunk: x (kTT*kHC = 256 values, one each) and Wr (kHC*E values)
-    const int wper = (kHC * E + kRThreads - 1) / kRThreads;   // <= 16
-    float xr;
-    float wrr[kHC * kMaxRouterExperts / kRThreads];
-    auto load_chunk = [&](int h0) {
-        {
-            const int tt = tid / kHC, hh = tid % kHC;
-            const int t = t0 + tt, h = h0 + hh;
-            xr = (t < T && h < he) ? __bfloat162float(x[(int64_t)t * H + h]) : 0.0f;
-        }
-#pragma unroll
-        for (int i = 0; i < kHC * kMaxRouterExperts / kRThreads; ++i) {
-            if (i >= wper) break;
-            const int li = tid + i * kRThreads;
-            float v = 0.0f;
-            if (li < kHC * E) {
-                const int hh = li / E, e = li - hh * E;
-                const int h = h0 + hh;
-                if (h < he) {
-                    v = WR32 ? reinterpret_cast<const float *>(wr)[(int64_t)h * E + e]
-                             : __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(wr)[(int64_t)h * E + e]);
-                }
-            }
-            wrr[i] = v;
-        }
-    };
-    auto store_chunk = [&]() {
-        xs[tid / kHC][tid % kHC] = (double)xr;
-#pragma unroll
-        for (int i = 0; i < kHC * kMaxRouterExperts / kRThreads; ++i) {
-            if (i >= wper) break;
-            const int li = tid + i * kRThreads;
-            if (li < kHC * E) {
-                const int hh = li / E, e = li - hh * E;
-                wsm[hh][e] = (double)wrr[i];
-            }
-        }
-    };
-
-    if (hb < he) load_chunk(hb);
-    for (int h0 = hb; h0 < he; h0 += kHC) {
-        __syncthreads();
-        store_chunk();
-        __syncthreads();
-        if (h0 + kHC < he) load_chunk(h0 + kHC);   // next chunk in flight during the math
-#pragma unroll
-        for (int i = 0; i < kMaxPairs; ++i) {
-            const int q = tid + i * kRThreads;
-            if (q < npairs) {
-                const int tt = q / E, e = q - tt * E;
-                double a = acc[i];
-#pragma unroll
-                for (int hh = 0; hh < kHC; ++hh) a = fma(xs[tt][hh], wsm[hh][e], a);
-                acc[i] = a;
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < kMaxPairs; ++i) {
-        const int q = tid + i * kRThreads;
-        if (q < npairs) {
-            const int tt = q / E, e = q - tt * E;
-            const int t = t0 + tt;
-            if (t < T) part[((int64_t)s * T + t) * E + e] = acc[i];
-        }
-    }
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d[0]), "+d"(d[1])
+                 : "d"(a), "d"(b));
 }
 
 // Exact widening to fp64 by moving the bit fields (the exponent is rebiased by
@@ -145,6 +73,147 @@ __device__ __forceinline__ double f32_bits_to_f64(uint32_t f) {
     if ((f & 0x7F800000u) == 0) return (double)__uint_as_float(f);
     const uint32_t hi = (f & 0x80000000u) | (((f & 0x7FFFFFFFu) >> 3) + (896u << 20));
     return __hiloint2double((int)hi, (int)(f << 29));
+}
+
+template <bool WR32>
+__global__ void __launch_bounds__(kDThreads) router_dmma_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H,
+                                                               const void *__restrict__ wr, int E, int slice,
+                                                               int wvec, double *__restrict__ part) {
+    extern __shared__ __align__(16) double dsm[];
+    double *xs = dsm;                        // [2][kDT * kXS]
+    double *ws = dsm + 2 * kDT * kXS;        // [2][kDK * kWS]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * kDT, e0 = blockIdx.y * kDE, sl = blockIdx.z;
+    const int hb = sl * slice, he = min(H, hb + slice);
+    const int wt = warp >> 1, we = warp & 1;      // warp tile: tokens 32 wt.., experts 32 we..
+    const int gq = lane >> 2, cq = lane & 3;      // fragment row / column of this lane
+
+    // staging: thread -> x row (tid / 2), 16 consecutive h; Wr row (tid / 4), 16 consecutive experts
+    const int xr = tid >> 1, xh = (tid & 1) * 16;
+    const int wrow = tid >> 2, we16 = (tid & 3) * 16;
+    double xv[16], wv[16];
+    auto load = [&](int kc) {
+        const int t = t0 + xr;
+        const int h = kc + xh;
+        if (t < T && h + 16 <= he) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)t * H + h);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const uint4 u = src[q];
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    xv[q * 8 + 2 * i] = bf16_bits_to_f64(w4[i] & 0xFFFFu);
+                    xv[q * 8 + 2 * i + 1] = bf16_bits_to_f64(w4[i] >> 16);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                xv[i] = (t < T && h + i < he)
+                            ? bf16_bits_to_f64(reinterpret_cast<const uint16_t *>(x)[(int64_t)t * H + h + i])
+                            : 0.0;
+        }
+        const int kr = kc + wrow;
+        const int e = e0 + we16;
+        if (wvec && kr < he && e + 16 <= E) {   // wvec: Wr rows are a multiple of 16 bytes
+            if (WR32) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const float *>(wr) + (int64_t)kr * E + e);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 u = src[q];
+                    wv[q * 4 + 0] = f32_bits_to_f64(u.x);
+                    wv[q * 4 + 1] = f32_bits_to_f64(u.y);
+                    wv[q * 4 + 2] = f32_bits_to_f64(u.z);
+                    wv[q * 4 + 3] = f32_bits_to_f64(u.w);
+                }
+            } else {
+                const uint4 *src =
+                    reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(wr) + (int64_t)kr * E + e);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint4 u = src[q];
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        wv[q * 8 + 2 * i] = bf16_bits_to_f64(w4[i] & 0xFFFFu);
+                        wv[q * 8 + 2 * i + 1] = bf16_bits_to_f64(w4[i] >> 16);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                double v = 0.0;
+                if (kr < he && e + i < E)
+                    v = WR32 ? f32_bits_to_f64(reinterpret_cast<const uint32_t *>(wr)[(int64_t)kr * E + e + i])
+                             : bf16_bits_to_f64(reinterpret_cast<const uint16_t *>(wr)[(int64_t)kr * E + e + i]);
+                wv[i] = v;
+            }
+        }
+    };
+    auto store = [&](int b) {
+        double *xd = xs + b * kDT * kXS + xr * kXS + xh;
+        double *wd = ws + b * kDK * kWS + wrow * kWS + we16;
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            *reinterpret_cast<double2 *>(xd + i) = make_double2(xv[i], xv[i + 1]);
+            *reinterpret_cast<double2 *>(wd + i) = make_double2(wv[i], wv[i + 1]);
+        }
+    };
+
+    double acc[4][4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+
+    int b = 0;
+    if (hb < he) {
+        load(hb);
+        store(0);
+    }
+    __syncthreads();
+    for (int kc = hb; kc < he; kc += kDK) {
+        const bool more = kc + kDK < he;
+        if (more) load(kc + kDK);   // next stage in flight during the MMAs
+        const double *xa = xs + b * kDT * kXS + (32 * wt + gq) * kXS + cq;
+        const double *wb = ws + b * kDK * kWS + cq * kWS + 32 * we + gq;
+#pragma unroll
+        for (int ks = 0; ks < kDK; ks += 4) {
+            double a[4], bb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xa[i * 8 * kXS + ks];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bb[j] = wb[ks * kWS + j * 8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[i][j], a[i], bb[j]);
+        }
+        if (more) {
+            store(b ^ 1);
+            b ^= 1;
+        }
+        __syncthreads();
+    }
+    // partial sums: lane holds rows gq, columns 2 cq, 2 cq + 1 of each 8 x 8 tile
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + 32 * wt + 8 * i + gq;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + 32 * we + 8 * j + 2 * cq;
+            double *dst = part + ((int64_t)sl * T + t) * E + e;
+            if (e + 1 < E) {
+                dst[0] = acc[i][j][0];
+                dst[1] = acc[i][j][1];
+            } else if (e < E) {
+                dst[0] = acc[i][j][0];
+            }
+        }
+    }
 }
 
 // Order-preserving 32-bit key of an fp32 logit (larger logit, larger key);
@@ -489,21 +558,21 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
         return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "router_cluster launch");
     }
     int S, slice;
-    router_split(T, H, &S, &slice);
+    router_split(T, H, E, &S, &slice);
     (void)nsm;
     const size_t need = (size_t)S * T * E * sizeof(double);
     if (ws_bytes < need) return set_error(MOE_ERR_OOM, "router workspace too small (%zu < %zu)", ws_bytes, need);
     double *part = reinterpret_cast<double *>(ws);
-    dim3 grid((T + kTT - 1) / kTT, S);
+    dim3 grid((T + kDT - 1) / kDT, (E + kDE - 1) / kDE, S);
+    const int smem = (int)((2 * kDT * kXS + 2 * kDK * kWS) * sizeof(double));
+    auto kfn = wr_is_fp32 ? router_dmma_kernel<true> : router_dmma_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return set_cuda_error(e, "router smem attribute");
     count_launch();
-    if (wr_is_fp32)
-        router_partial_kernel<true><<<grid, kRThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr,
-                                                               E, slice, part);
-    else
-        router_partial_kernel<false><<<grid, kRThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H,
-                                                                wr, E, slice, part);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return set_cuda_error(e, "router_partial launch");
+    const int wvec = (E * (wr_is_fp32 ? 4 : 2)) % 16 == 0;
+    kfn<<<grid, kDThreads, smem, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, slice, wvec, part);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_cuda_error(e, "router_dmma launch");
     count_launch();
     router_finish_kernel<<<(T + 7) / 8, 256, 0, st>>>(part, S, T, E, bias, k, idx, w, logits);
     e = cudaGetLastError();

@@ -121,7 +121,8 @@ typedef struct {
  *   idx: int32 [T][k] in descending logit order, ties to the lower expert index.
  *   w: fp32 [T][k], softmax over the k selected logits. logits: nullable fp32 [T][E].
  *   ws: scratch of moe_workspace_size(T, H, ...) bytes (fp64 partial sums).
- *   Requires 1 <= k <= 16, k <= E <= 256, H % 8 == 0. T == 0 is a no-op. */
+ *   Requires 1 <= k <= 16, k <= E <= 256, H % 8 == 0, x and wr 16-byte aligned.
+ *   T == 0 is a no-op. */
 moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                           int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes,
                           moe_stream_t stream);
