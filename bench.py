@@ -351,6 +351,61 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_stack(moe, device, steps: int) -> dict:
+    """The streaming stack: 43 FP8 layers whose experts live in pinned host memory (prepacked), a
+    24 GB device LRU cache in front of them, T = 4 decode steps chained through the layers with a
+    residual, routing popularity alternating between two Zipf(1.2) permutations per layer every
+    128 steps. Reports tokens/s, the cache hit rate and the H2D bandwidth of its copies."""
+    c = synthetic.CONFIGS["stack"]
+    L_, E_, H_, k_, T_ = c["layers"], c["E"], c["H"], c["k"], c["T"][0]
+    host, shapes, routers = [], [], []
+    try:
+        for l in range(L_):
+            lay = synthetic.make_layer("stack", 0, device=device, layer=l)
+            ex = moe.Experts.from_layer(lay)
+            packed = moe.moe_prepack(ex)
+            w13 = torch.empty(packed.w13.shape, dtype=torch.uint8, pin_memory=True)
+            w2 = torch.empty(packed.w2.shape, dtype=torch.uint8, pin_memory=True)
+            w13.copy_(packed.w13)
+            w2.copy_(packed.w2)
+            host.append(moe.Experts(packed.fmt, packed.E, packed.H, packed.I, w13, w2, layout=moe.LAYOUT_TILED))
+            shapes.append(host[-1])   # with a cache only the format and sizes of the shape are read
+            g = torch.Generator().manual_seed(9000 + l)
+            perms = (torch.randperm(E_, generator=g), torch.randperm(E_, generator=g))
+            biases = [synthetic.zipf_bias(E_, c["zipf"], H_, 0, perm=pm).to(device) for pm in perms]
+            routers.append((lay.wr, biases))
+            del lay, ex, packed
+        torch.cuda.empty_cache()
+    except RuntimeError as exc:   # host memory for the pool
+        return {"unavailable": f"could not build the pinned expert pool: {exc}"[:200]}
+    cache = moe.ExpertCache(int(c["cache_bytes"]), host, device=device.index)
+    ws = torch.empty(moe.moe_workspace_size(T_, H_, c["I"], E_, k_), dtype=torch.uint8, device=device)
+    drift = c["drift_every"]
+    torch.cuda.synchronize(device)
+    t0 = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for step in range(steps):
+        x = synthetic.make_tokens(T_, H_, seed=50000 + step, device=device)
+        for l in range(L_):
+            wr, biases = routers[l]
+            out = moe.moe_layer_forward(x, wr, k_, shapes[l], bias=biases[(step // drift) % 2], cache=cache,
+                                        layer=l, ws=ws)
+            x = (x.float() + out.float()).to(torch.bfloat16)
+    e1.record()
+    torch.cuda.synchronize(device)
+    sec = e0.elapsed_time(e1) / 1e3
+    st = cache.stats()
+    cache.close()
+    refs = st["hits"] + st["misses"]
+    return {"tokens_per_s": T_ * steps / sec, "seconds": sec, "steps": steps, "layers": L_, "T": T_,
+            "cache_bytes": int(c["cache_bytes"]), "hit_rate": st["hits"] / refs if refs else None,
+            "hits": st["hits"], "misses": st["misses"], "h2d_bytes": st["bytes_h2d"],
+            "h2d_gbs": st["bytes_h2d"] / st["copy_s"] / 1e9 if st["copy_s"] > 0 else None,
+            "wall_s": time.time() - t0}
+
+
 def run_ours(args, rank, world, device):
     import expert_ffn_layer_top_b200 as moe
 
@@ -401,14 +456,16 @@ def run_ours(args, rank, world, device):
     e2e = {"value": tokens / e2e_sec, "unit": "tokens/s", "h2d_bytes_per_step": lb.T * lb.layer.H * 2,
            "d2h_bytes_per_step": lb.T * lb.layer.H * 2}
 
-    # side measurements (not the headline): other batch sizes and the prefill-shaped layer
+    # side measurements (not the headline): other batch sizes, the prefill-shaped and large layers,
+    # and the streaming stack
     if not args.quick:
-        for cfg, T in (("decode", 1), ("decode", 8), ("prefill", 4096)):
-            b = lb if (cfg == "decode" and T == 64) else LayerBench(moe, cfg, T, device,
-                                                                     nsets=NSETS if cfg == "decode" else 4)
+        for cfg, T in (("decode", 1), ("decode", 8), ("prefill", 4096), ("large", 32), ("large", 8192)):
+            nsets = NSETS if cfg == "decode" else (2 if cfg == "large" else 4)
+            b = lb if (cfg == "decode" and T == 64) else LayerBench(moe, cfg, T, device, nsets=nsets)
             b.capture()
-            s = time_steps(b.step, max(10, args.steps // 2), args.warmup, device, barrier)
-            ms_b = s / max(10, args.steps // 2) * 1e3
+            nsteps = max(10, args.steps // 2) if T < 8192 else max(10, min(args.steps // 2, 40))
+            s = time_steps(b.step, nsteps, args.warmup, device, barrier)
+            ms_b = s / nsteps * 1e3
             n_alg = [b.algorithmic_bytes(args.warmup + i) for i in range(min(8, len(b.sets)))]
             gbs = sum(n_alg) / len(n_alg) / (ms_b * 1e-3) / 1e9
             extra[f"{cfg}_T{T}"] = {"tokens_per_s": T / (ms_b * 1e-3) * world, "ms_per_layer": ms_b,
@@ -417,6 +474,7 @@ def run_ours(args, rank, world, device):
                                     "frac_bf16_peak": b.flops() / (ms_b * 1e-3) / 1e12 / bf16_tf}
             del b
             torch.cuda.empty_cache()
+        extra["stack"] = run_stack(moe, device, args.stack_steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -457,6 +515,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--stack-steps", type=int, default=512, help="decode steps of the streaming-stack run")
     ap.add_argument("--profile", default=None, help="plain launches of one workload (cfg:T, e.g. decode:64) for ncu")
     args = ap.parse_args()
     if args.warmup < 3:
