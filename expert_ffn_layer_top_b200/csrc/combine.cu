@@ -12,6 +12,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
                                                      const int32_t *__restrict__ pair_row,
                                                      const float *__restrict__ w, int k, int H,
                                                      __nv_bfloat16 *__restrict__ out) {
+    pdl_wait();
+    pdl_release();
     const int t = blockIdx.x;
     __shared__ int rows[kMaxTopK];
     __shared__ float ws[kMaxTopK];
@@ -77,12 +79,10 @@ moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair
     int threads = H / 8;
     if (threads > 256) threads = 256;
     threads = (threads + 31) / 32 * 32;
-    count_launch();
-    if (y_is_fp32)
-        combine_kernel<true><<<T, threads, 0, st>>>(y_perm, pair_row, w, k, H, reinterpret_cast<__nv_bfloat16 *>(out));
-    else
-        combine_kernel<false><<<T, threads, 0, st>>>(y_perm, pair_row, w, k, H, reinterpret_cast<__nv_bfloat16 *>(out));
-    cudaError_t e = cudaGetLastError();
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out);
+    cudaError_t e = y_is_fp32 ? launch_pdl(combine_kernel<true>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o)
+                              : launch_pdl(combine_kernel<false>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "combine launch");
 }
 

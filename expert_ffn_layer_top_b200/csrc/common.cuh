@@ -10,6 +10,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "../../include/moe.h"
 
@@ -24,6 +25,33 @@ __device__ int g_dev_error = 0;
 // returned by moe_kernel_launch_count().
 static std::atomic<unsigned long long> g_kernel_launches{0};
 inline void count_launch() { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// Programmatic dependent launch. Kernels of the layer are launched with
+// launch_pdl, so a kernel may start (and run its prologue) while its
+// predecessor in the stream is still finishing. Every such kernel calls
+// pdl_wait() before it touches anything the predecessor writes, and
+// pdl_release() only after that wait: when kernel N starts, kernel N - 1 has
+// passed its wait, so kernel N - 2 has completed and its results may be read
+// before the wait.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, then give up and flag
 

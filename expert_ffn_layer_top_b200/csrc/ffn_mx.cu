@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
+    pdl_wait();
+    pdl_release();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int e = tid; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
@@ -348,24 +350,42 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
         // =================================================== producer of pipeline w
         const int w = warp;
         if (lane == 0 && w < NP) {
+            // Weight half of a stage (FP4 codes + their scale atoms): static data.
+            auto issue_weights = [&](const MxItem &it, int st, int s) {
+                const int slot = p.expert_map ? p.expert_map[it.e] : it.e;
+                const uint8_t *wexp = p.wbase + (int64_t)slot * p.w_estride;
+                const int blk = it.m * KB + st * SUB;
+                uint64_t *fb = &sm.full[s];
+                uint8_t *sp = base + s * STAGE;
+                mbar_expect_tx(fb, TX);
+                tma_load_4d(sp, &wmap, fb, 0, 0, blk, slot);
+                bulk_load(sp + SUB * (A_BYTES + B_BYTES), wexp + (int64_t)p.m_tiles * KB * kMxCodeBytes + (int64_t)blk * 512,
+                          SUB * 512, fb);
+            };
+            // The slots start empty: the weights of this pipeline's first NSW stages go out
+            // before waiting for the kernel that writes the activations.
+            int pre = 0;
+            for (int item = blockIdx.x; item < total && pre < NSW; item += gridDim.x) {
+                const MxItem it = mx_item(sm, p, item, BN);
+                for (int st = w; st < NST && pre < NSW; st += NP, ++pre) issue_weights(it, st, w * NSW + pre);
+            }
+            pdl_wait();
+            if (w == 0) pdl_release();
             int loc = 0;   // stages this pipeline has issued
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
                 const MxItem it = mx_item(sm, p, item, BN);
-                const int slot = p.expert_map ? p.expert_map[it.e] : it.e;
-                const uint8_t *sfa = p.wbase + (int64_t)slot * p.w_estride + (int64_t)p.m_tiles * KB * kMxCodeBytes;
                 for (int st = w; st < NST; st += NP, ++loc) {
                     const int s = w * NSW + loc % NSW;
                     const uint32_t round = (uint32_t)(loc / NSW);
-                    if (!mbar_wait(&sm.empty[s], (round & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    if (loc >= pre) {
+                        if (!mbar_wait(&sm.empty[s], (round & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        issue_weights(it, st, s);
+                    }
                     uint64_t *fb = &sm.full[s];
                     uint8_t *sp = base + s * STAGE;
                     const int kb = st * SUB;
-                    const int blk = it.m * KB + kb;
-                    mbar_expect_tx(fb, TX);
-                    tma_load_4d(sp, &wmap, fb, 0, 0, blk, slot);
                     tma_load_4d(sp + SUB * A_BYTES, &bmap, fb, 0, it.row0, 0, kb);
-                    bulk_load(sp + SUB * (A_BYTES + B_BYTES), sfa + (int64_t)blk * 512, SUB * 512, fb);
                     bulk_load(sp + SUB * (A_BYTES + B_BYTES) + SUB * 512, p.sfb + ((int64_t)it.rt * KB + kb) * 512,
                               SUB * 512, fb);
                 }
@@ -564,9 +584,8 @@ static cudaError_t mx_launch_one(const CUtensorMap &wmap, const CUtensorMap &bma
     auto kfn = ffn_mx_kernel<PHASE, BN>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    count_launch();
-    kfn<<<grid, kMxThreads, smem, st>>>(wmap, bmap, p);
-    return cudaGetLastError();
+    e = launch_pdl(kfn, dim3(grid), dim3(kMxThreads), smem, st, wmap, bmap, p);
+    return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <int PHASE>
@@ -629,11 +648,10 @@ moe_status launch_mx_quant(const void *src, int gather, const int32_t *sorted_pa
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     int blocks = (P + 7) / 8;
     if (blocks > num_sms * 8) blocks = num_sms * 8;
-    count_launch();
-    mx_quant_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4 *>(src), gather, sorted_pair, k, P, K,
-                                            offsets, E, BN, reinterpret_cast<uint8_t *>(q),
-                                            reinterpret_cast<uint8_t *>(sfb));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(mx_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
+                               gather, sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(q),
+                               reinterpret_cast<uint8_t *>(sfb));
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "mx quant launch");
 }
 

@@ -174,6 +174,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
 
     const int warp = warp_id(), lane = lane_id();
     volatile int *abort_flag = &sm.abort_flag;
+    pdl_wait();   // offsets and activations come from the kernels before this one
+    if (threadIdx.x == 0) pdl_release();
 
     // ---- set-up: barriers (thread 0), TMEM (warp 1), tile prefix (warp 3)
     if (threadIdx.x == 0) {
@@ -676,9 +678,8 @@ static cudaError_t launch_one(const CUtensorMap &wmap, const CUtensorMap &bmap, 
     auto kfn = p.tiled ? ffn_tc_kernel<FMT, PHASE, BN, true> : ffn_tc_kernel<FMT, PHASE, BN, false>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    count_launch();
-    kfn<<<grid, kThreads, smem, st>>>(wmap, bmap, p);
-    return cudaGetLastError();
+    e = launch_pdl(kfn, dim3(grid), dim3(kThreads), smem, st, wmap, bmap, p);
+    return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <int FMT, int PHASE>

@@ -28,6 +28,8 @@ size_t permute_ws_bytes(int T, int k, int E) {
 __global__ void __launch_bounds__(kChunk) perm_count_kernel(const int32_t *__restrict__ idx, int P, int E,
                                                            int32_t *__restrict__ counts) {
     extern __shared__ int32_t hist[];
+    pdl_wait();
+    pdl_release();
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int p = blockIdx.x * kChunk + threadIdx.x;
@@ -46,6 +48,8 @@ __global__ void __launch_bounds__(kMaxExperts) perm_scan_kernel(const int32_t *_
                                                                int32_t *__restrict__ offsets) {
     __shared__ int32_t tot[kMaxExperts];
     __shared__ int32_t warp_sums[32];
+    pdl_wait();
+    pdl_release();
     const int e = threadIdx.x;
     int run = 0;
     if (e < E) {
@@ -90,6 +94,8 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t *__r
                                                              int32_t *__restrict__ sorted_pair,
                                                              int32_t *__restrict__ pair_row) {
     extern __shared__ int32_t wcnt[];   // [32 warps][E]
+    pdl_wait();
+    pdl_release();
     const int nw = kChunk / 32;
     for (int i = threadIdx.x; i < nw * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
@@ -125,6 +131,8 @@ __global__ void __launch_bounds__(kChunk) perm_small_kernel(const int32_t *__res
     __shared__ int32_t run[kSmallE];
     __shared__ int32_t wsum[32];
     __shared__ int32_t wcnt[kChunk / 32][kSmallE];
+    pdl_wait();
+    pdl_release();
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     for (int e = tid; e < E; e += kChunk) cnt[e] = 0;
     __syncthreads();
@@ -198,6 +206,8 @@ size_t permute_scratch_bytes(int T, int k, int E) {
 __global__ void __launch_bounds__(256) perm_gather_kernel(const uint4 *__restrict__ x, int H8, int k,
                                                          const int32_t *__restrict__ sorted_pair, int P,
                                                          uint4 *__restrict__ x_perm) {
+    pdl_wait();
+    pdl_release();
     const int64_t total = (int64_t)P * H8;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = i / H8;
@@ -217,26 +227,28 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
     }
     cudaError_t e;
     if (P <= kSmallP && E <= kSmallE) {
-        count_launch();
-        perm_small_kernel<<<1, kChunk, 0, st>>>(idx, P, E, offsets, sorted_pair, pair_row);
+        e = launch_pdl(perm_small_kernel, dim3(1), dim3(kChunk), 0, st, idx, P, E, offsets, sorted_pair, pair_row);
+        if (e != cudaSuccess) return set_cuda_error(e, "permute launch");
     } else {
         const int C = (P + kChunk - 1) / kChunk;
         const size_t half = align_up((size_t)C * E * sizeof(int32_t), 256);
         if (ws_bytes < 2 * half) return set_error(MOE_ERR_OOM, "permute workspace too small");
         int32_t *counts = reinterpret_cast<int32_t *>(ws);
         int32_t *bases = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + half);
-        count_launch();
-        perm_count_kernel<<<C, kChunk, E * sizeof(int32_t), st>>>(idx, P, E, counts);
-        count_launch();
-        perm_scan_kernel<<<1, kMaxExperts, 0, st>>>(counts, C, E, P, bases, offsets);
+        e = launch_pdl(perm_count_kernel, dim3(C), dim3(kChunk), E * sizeof(int32_t), st, idx, P, E, counts);
+        if (e == cudaSuccess)
+            e = launch_pdl(perm_scan_kernel, dim3(1), dim3(kMaxExperts), 0, st, (const int32_t *)counts, C, E, P, bases,
+                           offsets);
+        if (e != cudaSuccess) return set_cuda_error(e, "permute launch");
         const size_t sm_scatter = (size_t)(kChunk / 32) * E * sizeof(int32_t);
         if (sm_scatter > 48 * 1024) {
             e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)sm_scatter);
             if (e != cudaSuccess) return set_cuda_error(e, "scatter smem attribute");
         }
-        count_launch();
-        perm_scatter_kernel<<<C, kChunk, sm_scatter, st>>>(idx, P, E, bases, sorted_pair, pair_row);
+        e = launch_pdl(perm_scatter_kernel, dim3(C), dim3(kChunk), sm_scatter, st, idx, P, E, (const int32_t *)bases,
+                       sorted_pair, pair_row);
+        if (e != cudaSuccess) return set_cuda_error(e, "permute launch");
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "permute launch");
@@ -245,10 +257,9 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
         const int64_t total = (int64_t)P * H8;
         int blocks = (int)((total + 255) / 256);
         if (blocks > 148 * 16) blocks = 148 * 16;
-        count_launch();
-        perm_gather_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4 *>(x), H8, k, sorted_pair, P,
-                                                   reinterpret_cast<uint4 *>(x_perm));
-        e = cudaGetLastError();
+        e = launch_pdl(perm_gather_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(x), H8, k,
+                       (const int32_t *)sorted_pair, P, reinterpret_cast<uint4 *>(x_perm));
+        if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return set_cuda_error(e, "gather launch");
     }
     return MOE_OK;

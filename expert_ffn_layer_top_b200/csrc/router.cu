@@ -80,6 +80,8 @@ __global__ void __launch_bounds__(kDThreads) router_dmma_kernel(const __nv_bfloa
                                                                const void *__restrict__ wr, int E, int slice,
                                                                int wvec, double *__restrict__ part) {
     extern __shared__ __align__(16) double dsm[];
+    pdl_wait();
+    pdl_release();
     double *xs = dsm;                        // [2][kDT * kXS]
     double *ws = dsm + 2 * kDT * kXS;        // [2][kDK * kWS]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -282,6 +284,8 @@ __global__ void __launch_bounds__(256) router_finish_kernel(const double *__rest
                                                            const float *__restrict__ bias, int k,
                                                            int32_t *__restrict__ idx, float *__restrict__ w,
                                                            float *__restrict__ logits) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -386,6 +390,9 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
             bulk_load(wring + c * chunk_bytes, wsrc + c * chunk_bytes, (uint32_t)chunk_bytes, &full[c]);
         }
     }
+    // Wr is static and already on its way; x comes from the previous kernel
+    pdl_wait();
+    pdl_release();
     // x tile -> shared, as fp64 (exact), layout [h][tt]; tokens past T are zero
     for (int i = tid; i < hs * TT; i += kRClThreads) {
         const int tt = i / hs, h = i - tt * hs;
@@ -528,10 +535,9 @@ static cudaError_t launch_router_cluster_t(const RouterClusterShape &sh, const v
         if (e != cudaSuccess) return e;
     }
     dim3 grid(kRCl, (T + TT - 1) / TT);
-    count_launch();
-    kern<<<grid, kRClThreads, sh.smem, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, sh.EPP, sh.G,
-                                             sh.RC, sh.nch, bias, k, idx, w, logits);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(kern, grid, dim3(kRClThreads), sh.smem, st, reinterpret_cast<const __nv_bfloat16 *>(x),
+                               T, H, wr, E, sh.EPP, sh.G, sh.RC, sh.nch, bias, k, idx, w, logits);
+    return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <bool WR32>
@@ -568,14 +574,14 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
     auto kfn = wr_is_fp32 ? router_dmma_kernel<true> : router_dmma_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return set_cuda_error(e, "router smem attribute");
-    count_launch();
     const int wvec = (E * (wr_is_fp32 ? 4 : 2)) % 16 == 0;
-    kfn<<<grid, kDThreads, smem, st>>>(reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, slice, wvec, part);
-    e = cudaGetLastError();
+    e = launch_pdl(kfn, grid, dim3(kDThreads), smem, st, reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, slice,
+                   wvec, part);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "router_dmma launch");
-    count_launch();
-    router_finish_kernel<<<(T + 7) / 8, 256, 0, st>>>(part, S, T, E, bias, k, idx, w, logits);
-    e = cudaGetLastError();
+    e = launch_pdl(router_finish_kernel, dim3((T + 7) / 8), dim3(256), 0, st, (const double *)part, S, T, E, bias, k,
+                   idx, w, logits);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "router_finish launch");
     return MOE_OK;
 }
