@@ -209,16 +209,16 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 // Block-scaled MXFP4 path: E4M3 hi/lo planes of the permuted activations
 // [2][n][H] and of h [2][n][I], and the scale atoms of both.
 struct FfnWs {
-    size_t qx, q2, sf1, sf2, total;
+    size_t b1, b2, total;
 };
 
+// MXFP4 path: activation blobs of x (b1) and of h (b2). The other paths use
+// the region as their h buffer.
 static FfnWs ffn_ws(int n, int H, int I, int E) {
     FfnWs W;
     size_t o = 0;
-    W.qx = o; o += align_up((size_t)2 * n * H, 256);
-    W.q2 = o; o += align_up((size_t)2 * n * I, 256);
-    W.sf1 = o; o += mx_sf_bytes(n, H, E);
-    W.sf2 = o; o += mx_sf_bytes(n, I, E);
+    W.b1 = o; o += mx_blob_bytes(n, H, E);
+    W.b2 = o; o += mx_blob_bytes(n, I, E);
     W.total = o > align_up((size_t)n * I * 2, 256) ? o : align_up((size_t)n * I * 2, 256);
     return W;
 }
@@ -226,30 +226,6 @@ static FfnWs ffn_ws(int n, int H, int I, int E) {
 static size_t ffn_ws_bytes(int n_rows, int H, int I, int E) { return ffn_ws(n_rows, H, I, E).total; }
 
 static bool is_mx(const moe_experts &x) { return x.fmt == MOE_MXFP4 && x.layout == MOE_LAYOUT_TILED; }
-
-// 4D map over prepacked MXFP4 codes: (128 codes, 128 rows, K blocks of all M
-// tiles of one expert, experts or cache slots); a box is `sub` consecutive K
-// blocks. TMA spreads every 16 codes over 16 bytes.
-static moe_status mx_weight_tmap(CUtensorMap *m, const void *base, int blocks, int64_t estride, int entries,
-                                 int sub) {
-    if ((reinterpret_cast<uintptr_t>(base) & 31) || (estride & 31))
-        return set_error(MOE_ERR_UNSUPPORTED, "prepacked MXFP4 experts need 32-byte aligned bases and strides");
-    uint64_t dims[4] = {128, 128, (uint64_t)blocks, (uint64_t)entries};
-    uint64_t strides[3] = {64, (uint64_t)kMxCodeBlockBytes, (uint64_t)estride};
-    uint32_t box[4] = {128, 128, (uint32_t)sub, 1};
-    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, base, dims, strides, box,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-// 4D map over the E4M3 hi/lo planes [2][n][K] viewed as (128 bytes of a K
-// block, row, plane, K block): one box holds, for `sub` consecutive K blocks,
-// BN hi rows followed by the same BN lo rows.
-static moe_status mx_act_tmap(CUtensorMap *m, const void *base, int n, int K, int BN, int sub) {
-    uint64_t dims[4] = {128, (uint64_t)n, 2, (uint64_t)(K / 128)};
-    uint64_t strides[3] = {(uint64_t)K, (uint64_t)n * K, 128};
-    uint32_t box[4] = {128, (uint32_t)BN, 2, (uint32_t)sub};
-    return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
-}
 
 // Block-scaled MXFP4 grouped FFN. The activations are quantised first: gathered
 // from token rows x[sorted_pair[r] / k] (gather != 0) or read from x_perm.
@@ -259,15 +235,12 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     if (n_rows == 0) return MOE_OK;
     const int E = x->E, H = x->H, I = x->I;
     const Strides s = default_strides(*x);
-    const int nent = x->expert_map ? (int)(x->n_entries > 0 ? x->n_entries : E) : E;
     const int BN = choose_bn_mx(n_rows, E);
     const int nsm = num_sms(current_device());
     const FfnWs W = ffn_ws(n_rows, H, I, E);
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
-    moe_status r = launch_mx_quant(x_src, gather, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.qx, b + W.sf1,
-                                   nsm, st);
+    moe_status r = launch_mx_quant(x_src, gather, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1, nsm, st);
     if (r != MOE_OK) return r;
-    CUtensorMap wmap, bmap;
     MxParams p;
     memset(&p, 0, sizeof(p));
     p.offsets = offsets;
@@ -277,32 +250,23 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.I = I;
     p.n_rows = n_rows;
     // ---- gate/up + SwiGLU, h quantised for the down pass
-    MxPlan pl;
-    if (!mx_plan(kPhaseUp, BN, H, &pl)) return set_error(MOE_ERR_UNSUPPORTED, "H=%d: no MXFP4 pipeline plan", H);
-    if ((r = mx_weight_tmap(&wmap, x->w13, (I / 64) * (H / 128), s.w13, nent, pl.sub)) != MOE_OK) return r;
-    if ((r = mx_act_tmap(&bmap, b + W.qx, n_rows, H, BN, pl.sub)) != MOE_OK) return r;
     p.K = H;
     p.m_tiles = I / 64;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
     p.w_estride = s.w13;
-    p.sfb = b + W.sf1;
-    p.q_out = b + W.q2;
-    p.sfb_out = b + W.sf2;
-    if ((r = launch_mx_phase(kPhaseUp, BN, wmap, bmap, p, nsm, st)) != MOE_OK) return r;
+    p.bblob = b + W.b1;
+    p.bblob_out = b + W.b2;
+    if ((r = launch_mx_phase(kPhaseUp, BN, p, nsm, st)) != MOE_OK) return r;
     // ---- down projection
-    if (!mx_plan(kPhaseDown, BN, I, &pl)) return set_error(MOE_ERR_UNSUPPORTED, "I=%d: no MXFP4 pipeline plan", I);
-    if ((r = mx_weight_tmap(&wmap, x->w2, (H / 128) * (I / 128), s.w2, nent, pl.sub)) != MOE_OK) return r;
-    if ((r = mx_act_tmap(&bmap, b + W.q2, n_rows, I, BN, pl.sub)) != MOE_OK) return r;
     p.K = I;
     p.m_tiles = H / 128;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w2);
     p.w_estride = s.w2;
-    p.sfb = b + W.sf2;
-    p.q_out = nullptr;
-    p.sfb_out = nullptr;
+    p.bblob = b + W.b2;
+    p.bblob_out = nullptr;
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
-    return launch_mx_phase(kPhaseDown, BN, wmap, bmap, p, nsm, st);
+    return launch_mx_phase(kPhaseDown, BN, p, nsm, st);
 }
 
 // grouped FFN with explicit h buffer

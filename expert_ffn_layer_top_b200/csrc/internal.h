@@ -36,9 +36,15 @@ struct FfnParams {
     int64_t w_estride;          // tiled: bytes between experts
 };
 
-// Block-scaled MXFP4 path (ffn_mx.cu): weights prepacked by moe_prepack, E4M3
-// hi/lo activations with per-tile scale atoms.
-constexpr int kMxCodeBlockBytes = 128 * 64;   // prepacked MXFP4 codes of one (M tile, 128-wide K block)
+// Block-scaled MXFP4 path (ffn_mx.cu): kind::mxf4 MMAs, weights prepacked by
+// moe_prepack, activations as four E2M1 planes with per-tile scale atoms.
+constexpr int kMxStageK = 256;                   // K elements per pipeline stage
+constexpr int kMxCodeBytes = 128 * 128;          // packed codes of one (M tile, stage): 128 rows x 128 B
+constexpr int kMxABlob = kMxCodeBytes + 1024;    // + the two 512-byte scale atoms of the stage
+constexpr int kMxPlanes = 4;                     // E2M1 planes per activation value
+
+// Bytes of one activation blob (N tile of BN rows, one stage): 4 BN rows of 128 B, then two scale atoms.
+__host__ __device__ constexpr int mx_bblob_bytes(int BN) { return kMxPlanes * BN * 128 + 1024; }
 
 struct MxParams {
     const int32_t *offsets;     // [E+1]
@@ -46,17 +52,15 @@ struct MxParams {
     int E, H, I;
     int K;                      // reduction dimension of this phase (H or I)
     int m_tiles;                // I/64 (up) or H/128 (down)
-    int stages;                 // shared-memory ring depth, set by the launcher
-    int sub;                    // 128-wide K blocks per stage, set by the launcher
+    int stages;                 // shared-memory slots, set by the launcher
     int pipes;                  // independent producer/MMA pipelines, set by the launcher
     int n_rows;
-    const uint8_t *wbase;       // this phase's prepacked tensor (code blocks, then scale atoms)
+    const uint8_t *wbase;       // this phase's prepacked tensor: [m_tiles][K/256] blobs of kMxABlob bytes
     int64_t w_estride;          // bytes between experts (or cache slots)
-    const uint8_t *sfb;         // activation scale atoms [tiles][K/128][512]
+    const uint8_t *bblob;       // activation blobs [tiles][K/256][mx_bblob_bytes(BN)]
     void *out;                  // down: y [n_rows][H] (bf16 or fp32)
     int out_fp32;
-    uint8_t *q_out;             // up: E4M3 hi/lo planes of h [2][n_rows][I]
-    uint8_t *sfb_out;           // up: scale atoms of h [tiles][I/128][512]
+    uint8_t *bblob_out;         // up: blobs of h for the down pass [tiles][I/256][...]
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -76,15 +80,14 @@ moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap,
 
 int choose_bn_mx(int n_rows, int E);
 struct MxPlan {
-    int sub, pipes, stages;
+    int pipes, stages;
 };
-bool mx_plan(int phase, int BN, int K, MxPlan *pl);
+bool mx_plan(int phase, int BN, int K, int E, MxPlan *pl);
 size_t mx_tiles_ub(int n_rows, int E);
-size_t mx_sf_bytes(int n_rows, int K, int E);
-moe_status launch_mx_phase(int phase, int BN, const CUtensorMap &wmap, const CUtensorMap &bmap, MxParams p,
-                           int num_sms, cudaStream_t st);
+size_t mx_blob_bytes(int n_rows, int K, int E);
+moe_status launch_mx_phase(int phase, int BN, MxParams p, int num_sms, cudaStream_t st);
 moe_status launch_mx_quant(const void *src, int gather, const int32_t *sorted_pair, int k, int P, int K,
-                           const int32_t *offsets, int E, int BN, void *q, void *sfb, int num_sms, cudaStream_t st);
+                           const int32_t *offsets, int E, int BN, void *bblob, int num_sms, cudaStream_t st);
 
 moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           cudaStream_t st);

@@ -7,13 +7,14 @@
 //     of row r at (c*128 + r)*16), then each row's scales for that stage. The
 //     decoding FFN moves a stage with one bulk copy and its decoder threads
 //     read consecutive chunks without bank conflicts.
-//   MXFP4 (one region per expert instead of per-stage blobs): first the 8 KiB
-//     code blocks of every (M tile, stage) in order, each row after row (row r
-//     at r*64, natural K order), read by TMA boxes that spread them into the
-//     block-scaled MMA's operand layout; then the 512-byte scale atoms of every
-//     (M tile, stage) in the same order: the E8M0 scale of row r and 32-block j
-//     at byte (r % 32)*16 + (r / 32)*4 + j, the arrangement tcgen05.cp moves
-//     into TMEM. Consecutive stages are contiguous in both parts.
+//   MXFP4 (stages 256 wide): one 17 KiB blob per (M tile, stage), in that
+//     order. First the packed codes, 128 bytes per row in natural K order,
+//     with the 16-byte chunk c of row r stored at r*128 + (c ^ (r % 8))*16:
+//     the 128-byte swizzle the block-scaled MMA reads from shared memory, so
+//     one bulk copy lands the operand ready to use. Then two 512-byte scale
+//     atoms, one per 128-wide half of the stage: the E8M0 scale of row r and
+//     32-block j of the half at byte (r % 32)*16 + (r / 32)*4 + j, the
+//     arrangement tcgen05.cp moves into TMEM.
 // Values are untouched: this is a byte permutation.
 #include "common.cuh"
 #include "internal.h"
@@ -59,12 +60,15 @@ __global__ void prepack_kernel(const uint8_t *__restrict__ w, int64_t w_estride,
     uint8_t *blob = out + e * out_estride + ((int64_t)m * KB + kb) * SB;
     const uint8_t *src = w + e * w_estride + (int64_t)row * row_bytes + (int64_t)kb * RB;
     const uint8_t *ss = scale + e * s_estride + (int64_t)row * s_row_bytes + (int64_t)kb * SBY;
-    if (mx) {   // RB = 64, SBY = 4: all code blocks of the expert, then all scale atoms
-        uint8_t *ex = out + e * out_estride;
-        uint8_t *code = ex + ((int64_t)m * KB + kb) * (128 * 64) + r * 64;
-        for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4 *>(code + c * 16) = *reinterpret_cast<const uint4 *>(src + c * 16);
-        uint8_t *atom = ex + (int64_t)m_tiles * KB * (128 * 64) + ((int64_t)m * KB + kb) * 512;
+    if (mx) {   // RB = 64, SBY = 4: this thread fills half `kb % 2` of row r of blob (m, kb / 2)
+        const int half = kb & 1;
+        uint8_t *mb = out + e * out_estride + ((int64_t)m * (KB / 2) + (kb >> 1)) * kMxABlob;
+        for (int c = 0; c < 4; ++c) {
+            const int cc = half * 4 + c;   // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4 *>(mb + r * 128 + ((cc ^ (r & 7)) << 4)) =
+                *reinterpret_cast<const uint4 *>(src + c * 16);
+        }
+        uint8_t *atom = mb + kMxCodeBytes + half * 512;
         for (int j = 0; j < 4; ++j) atom[(r & 31) * 16 + (r >> 5) * 4 + j] = ss[j];
         return;
     }

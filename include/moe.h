@@ -77,11 +77,13 @@ typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3
  * TILED: produced by moe_prepack; for every (M tile, 128-wide K stage) one
  * contiguous blob holding the tile's 128 weight rows. BF16/FP8/NVFP4: codes
  * 16-byte chunk-major, then the rows' scales for that stage (one bulk copy per
- * stage). MXFP4: per expert, all 8 KiB code blocks (row after row, 64 bytes
- * per row) of every (M tile, stage), then all 512-byte scale atoms in the same
- * order, with the scale of row r and 32-block j at byte (r%32)*16 + (r/32)*4 + j;
- * this layout runs the block-scaled tensor-core path (bases and strides 32-byte
- * aligned). The values are the same; only the byte order differs. */
+ * stage). MXFP4: one 17 KiB blob per (M tile, 256-wide K stage): the tile's
+ * 128 rows of packed codes, 128 bytes per row in natural K order with the
+ * 16-byte chunk c of row r at r*128 + (c XOR (r%8))*16, then two 512-byte
+ * scale atoms (the stage's 128-wide halves) with the scale of row r and
+ * 32-block j at byte (r%32)*16 + (r/32)*4 + j; this layout runs the
+ * block-scaled FP4 tensor-core path. The values are the same; only the byte
+ * order differs. */
 typedef enum { MOE_LAYOUT_STANDARD = 0, MOE_LAYOUT_TILED = 1 } moe_layout;
 
 /* The experts of one layer.
