@@ -209,37 +209,52 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 // Block-scaled MXFP4 path: E4M3 hi/lo planes of the permuted activations
 // [2][n][H] and of h [2][n][I], and the scale atoms of both.
 struct FfnWs {
-    size_t b1, b2, total;
+    size_t h, re1, re2, b1, b2, total;
 };
 
-// MXFP4 path: activation blobs of x (b1) and of h (b2). The other paths use
-// the region as their h buffer.
+// h: bf16 [n][I] (the decoding paths' h buffer; NVFP4: h before its
+// quantisation); re1, re2: NVFP4 per-row exponent offsets of x and h; b1, b2:
+// activation blobs of x and h for the block-scaled FP4 path.
 static FfnWs ffn_ws(int n, int H, int I, int E) {
     FfnWs W;
     size_t o = 0;
+    W.h = o; o += align_up((size_t)n * I * 2, 256);
+    W.re1 = o; o += align_up((size_t)n * 4, 256);
+    W.re2 = o; o += align_up((size_t)n * 4, 256);
     W.b1 = o; o += mx_blob_bytes(n, H, E);
     W.b2 = o; o += mx_blob_bytes(n, I, E);
-    W.total = o > align_up((size_t)n * I * 2, 256) ? o : align_up((size_t)n * I * 2, 256);
+    W.total = o;
     return W;
 }
 
 static size_t ffn_ws_bytes(int n_rows, int H, int I, int E) { return ffn_ws(n_rows, H, I, E).total; }
 
-static bool is_mx(const moe_experts &x) { return x.fmt == MOE_MXFP4 && x.layout == MOE_LAYOUT_TILED; }
+// Prepacked MXFP4 experts run the block-scaled FP4 path; prepacked NVFP4 runs it
+// for token tiles of up to 16 rows (decode-sized batches) and the decoding
+// bf16 tensor-core path, which reads the same blobs, for larger ones.
+static bool use_bs(int fmt, int layout, int n_rows, int E) {
+    if (layout != MOE_LAYOUT_TILED) return false;
+    if (fmt == MOE_MXFP4) return true;
+    return fmt == MOE_NVFP4 && choose_bn_mx(n_rows, E) <= 16;
+}
+static bool is_mx(const moe_experts &x, int n_rows) { return use_bs(x.fmt, x.layout, n_rows, x.E); }
 
-// Block-scaled MXFP4 grouped FFN. The activations are quantised first: gathered
+// Block-scaled FP4 grouped FFN. The activations are quantised first: gathered
 // from token rows x[sorted_pair[r] / k] (gather != 0) or read from x_perm.
 static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sorted_pair, int k, int n_rows,
                               const int32_t *offsets, const moe_experts *x, void *y_perm, int y_is_fp32, void *ws,
                               cudaStream_t st) {
     if (n_rows == 0) return MOE_OK;
     const int E = x->E, H = x->H, I = x->I;
+    const int fmt = x->fmt == MOE_NVFP4 ? kBsNv : kBsMx;
     const Strides s = default_strides(*x);
     const int BN = choose_bn_mx(n_rows, E);
     const int nsm = num_sms(current_device());
     const FfnWs W = ffn_ws(n_rows, H, I, E);
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
-    moe_status r = launch_mx_quant(x_src, gather, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1, nsm, st);
+    int32_t *re1 = reinterpret_cast<int32_t *>(b + W.re1), *re2 = reinterpret_cast<int32_t *>(b + W.re2);
+    moe_status r = launch_mx_quant(fmt, x_src, gather ? 1 : 0, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1,
+                                   re1, nsm, st);
     if (r != MOE_OK) return r;
     MxParams p;
     memset(&p, 0, sizeof(p));
@@ -249,24 +264,34 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.H = H;
     p.I = I;
     p.n_rows = n_rows;
-    // ---- gate/up + SwiGLU, h quantised for the down pass
+    // ---- gate/up + SwiGLU; MXFP4 quantises h for the down pass in the epilogue
     p.K = H;
     p.m_tiles = I / 64;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
     p.w_estride = s.w13;
     p.bblob = b + W.b1;
+    p.rowexp = re1;
+    p.tscale = x->w13_tscale;
     p.bblob_out = b + W.b2;
-    if ((r = launch_mx_phase(kPhaseUp, BN, p, nsm, st)) != MOE_OK) return r;
+    p.hout = b + W.h;
+    if ((r = launch_mx_phase(fmt, kPhaseUp, BN, p, nsm, st)) != MOE_OK) return r;
+    if (fmt == kBsNv &&
+        (r = launch_mx_quant(fmt, b + W.h, 2, nullptr, 1, n_rows, I, offsets, E, BN, b + W.b2, re2, nsm, st)) !=
+            MOE_OK)
+        return r;
     // ---- down projection
     p.K = I;
     p.m_tiles = H / 128;
     p.wbase = reinterpret_cast<const uint8_t *>(x->w2);
     p.w_estride = s.w2;
     p.bblob = b + W.b2;
+    p.rowexp = re2;
+    p.tscale = x->w2_tscale;
     p.bblob_out = nullptr;
+    p.hout = nullptr;
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
-    return launch_mx_phase(kPhaseDown, BN, p, nsm, st);
+    return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 
 // grouped FFN with explicit h buffer
@@ -434,12 +459,12 @@ moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offset
     if (n_rows < 0) return set_error(MOE_ERR_INVALID_ARG, "n_rows < 0");
     if (n_rows == 0) return MOE_OK;
     if (!x_perm || !offsets || !y_perm || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
-    const size_t need = is_mx(*experts) ? ffn_ws_bytes(n_rows, experts->H, experts->I, experts->E)
+    const size_t need = is_mx(*experts, n_rows) ? ffn_ws_bytes(n_rows, experts->H, experts->I, experts->E)
                                         : align_up((size_t)n_rows * experts->I * 2, 256);
     if (ws_bytes < need) return set_error(MOE_ERR_OOM, "FFN workspace too small (%zu < %zu)", ws_bytes, need);
     if ((reinterpret_cast<uintptr_t>(x_perm) | reinterpret_cast<uintptr_t>(ws)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "x_perm and ws must be 16-byte aligned");
-    if (is_mx(*experts))
+    if (is_mx(*experts, n_rows))
         return mx_ffn_impl(x_perm, 0, nullptr, 1, n_rows, offsets, experts, y_perm, y_is_fp32, ws,
                            (cudaStream_t)stream);
     return grouped_ffn_impl(x_perm, n_rows, offsets, experts, y_perm, y_is_fp32, ws, (cudaStream_t)stream);
@@ -514,9 +539,9 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     moe_status r = moe_route_topk(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router,
                                   L.idx - L.router, stream);
     if (r != MOE_OK) return r;
-    // The block-scaled MXFP4 path gathers the token rows itself while quantising them.
+    // The block-scaled FP4 path gathers the token rows itself while quantising them.
     const int layout = cache ? cache_layout(cache) : experts->layout;
-    const bool mx = experts->fmt == MOE_MXFP4 && layout == MOE_LAYOUT_TILED;
+    const bool mx = use_bs(experts->fmt, layout, T * k, E);
     r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, mx ? nullptr : b + L.x_perm, b + L.perm,
                     L.x_perm - L.perm, stream);
     if (r != MOE_OK) return r;
@@ -526,7 +551,7 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
         if (r != MOE_OK) return r;
         if ((r = check_experts(&view)) != MOE_OK) return r;
     }
-    if (is_mx(view) != mx) return set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
+    if (is_mx(view, T * k) != mx) return set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
     if (mx)
         r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
     else

@@ -1,6 +1,8 @@
-// Grouped SwiGLU expert FFN for MXFP4 experts on the block-scaled FP4 tensor
-// core path: tcgen05.mma kind::mxf4 (E2M1 times E2M1, one E8M0 scale per 32 K
-// elements on both sides, fp32 accumulation in TMEM, K = 64 per instruction).
+// Grouped SwiGLU expert FFN for FP4 experts on the block-scaled tensor core
+// path, fp32 accumulation in TMEM, K = 64 per instruction:
+//   MXFP4: tcgen05.mma kind::mxf4, one E8M0 scale per 32 K elements;
+//   NVFP4: tcgen05.mma kind::mxf4nvf4 scale_vec::4X, one E4M3 scale per 16 K
+//          elements, and the per-expert fp32 tensor scale in the epilogue.
 // Both operands stay packed, two codes per byte, from HBM to the tensor core.
 //
 // Activations: a bf16 value x of a 32-block whose largest magnitude has binary
@@ -11,17 +13,23 @@
 // four planes are within 2^(e - 11), about 2^-11 of the block maximum, of x.
 // The planes of a token are four rows of the B operand (plane p of token n is
 // row p BN + n), each with its own scale; the epilogue adds the four columns.
+// NVFP4 scales are E4M3, which hold the powers of two 2^-9..2^8 only: a token
+// row with largest magnitude 2^E stores every plane scale multiplied by
+// 2^(3p + C), C = 9 - E (so the largest block lands on 2^8), and the epilogue
+// multiplies column (p, n) by 2^-(3p + C); blocks more than 2^17 below the row
+// maximum keep the smallest scale and lose only digits below 2^-17 of it.
 //
 // Work item: an N tile of BN rows of one expert x one M tile of 128 weight rows
 // (UP: 64 gate rows and the matching 64 up rows; DOWN: 128 rows). A stage is a
 // 256-wide K slice and each operand of a stage arrives by one bulk copy:
 //   weights, prepacked: 128 rows x 128 bytes, the 16-byte chunk c of row r at
 //     r*128 + (c ^ (r % 8))*16 (the 128-byte swizzle of the MMA descriptor),
-//     then the scale atoms of the stage's two 128-wide halves;
-//   activations, written by the quantiser (and, for DOWN, by the UP epilogue):
-//     N = 4 BN rows in the same swizzled form, then their two scale atoms.
+//     then the scale atoms of the stage (MXFP4: two, one per 128-wide half;
+//     NVFP4: four, one per 64-wide quarter);
+//   activations, written by the quantiser (MXFP4 DOWN: by the UP epilogue):
+//     N = 4 BN rows in the same swizzled form, then their scale atoms.
 // A scale atom is 512 bytes: byte (r % 32) * 16 + (r / 32) * 4 + j holds the
-// scale of operand row r and 32-block j of the half; tcgen05.cp 32x128b.warpx4
+// scale of operand row r and scale block j of its K range; tcgen05.cp 32x128b.warpx4
 // puts atom row l into TMEM lanes l, l+32, l+64, l+96 (4 columns), where the
 // MMA reads the scale of row r: lane r, column r / 32, byte j.
 //
@@ -57,6 +65,19 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bd
         : "memory");
 }
 
+// The same with kind::mxf4nvf4: four E4M3 scales per row and instruction
+// (the whole 32-bit scale column).
+__device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+            "r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 // Shared-memory descriptor of a scale atom: no swizzle, K-major, core matrices
 // of 8 rows x 16 bytes stacked 128 bytes apart.
 __device__ __forceinline__ uint64_t sf_atom_desc(uint32_t saddr) {
@@ -70,6 +91,17 @@ __device__ __forceinline__ uint64_t sf_atom_desc(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_mxf4(int N, uint32_t id) {
     return (id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) |
            (id << 29);
+}
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: A and B E2M1, E4M3
+// scales, both K-major, M = 128, K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (0u << 23) | ((128u >> 4) << 24);
+}
+
+// E4M3 byte of 2^k, -9 <= k <= 8 (k < -6: subnormal).
+__device__ __forceinline__ uint8_t e4m3_pow2(int k) {
+    return k >= -6 ? (uint8_t)((k + 7) << 3) : (uint8_t)(1u << (k + 9));
 }
 
 __device__ __forceinline__ uint32_t atom_offset(int row, int j) { return (row & 31) * 16 + (row >> 5) * 4 + j; }
@@ -163,13 +195,65 @@ __device__ __forceinline__ uint4 deinterleave8(uint4 o) {
     return v;
 }
 
-// One warp per (permuted row r, 256-wide stage st), grid-stride; each lane
-// takes 8 consecutive elements. The row is x[sorted_pair[r] / k] (gather != 0,
-// natural order) or x_perm[r] (operand order). Its four planes go to rows
-// p BN + n (n = (r - offsets[e]) % BN) of the activation blob (tile, st) of its
-// N tile, tile = tile_start[e] + (r - offsets[e]) / BN; the plane scales go
-// into that blob's scale atoms.
-__global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__ src, int gather,
+// s_off[0..E] = offsets; s_tile[e] = sum over e' < e of ceil(n_e' / BN). 256 threads.
+__device__ __forceinline__ void quant_tile_prefix(const int32_t *__restrict__ offsets, int E, int BN, int *s_off,
+                                                  int *s_tile, int *s_wsum) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e <= E; e += blockDim.x) s_off[e] = offsets[e];
+    __syncthreads();
+    int cnt[4], run = 0;   // 4 experts per thread
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = tid * 4 + i;
+        cnt[i] = e < E ? (s_off[e + 1] - s_off[e] + BN - 1) / BN : 0;
+        run += cnt[i];
+    }
+    int incl = run;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int base = incl - run;
+    for (int w = 0; w < warp; ++w) base += s_wsum[w];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = tid * 4 + i;
+        if (e <= E) s_tile[e] = base;
+        base += cnt[i];
+    }
+    __syncthreads();
+}
+
+// Expert e with s_off[e] <= r < s_off[e + 1].
+__device__ __forceinline__ int expert_of_row(const int *s_off, int E, int r) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ void bf16x8_to_float(uint4 u, float (&v)[8]) {
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[h]));
+        v[2 * h] = f.x;
+        v[2 * h + 1] = f.y;
+    }
+}
+
+// MXFP4 activations. One warp per (permuted row r, 256-wide stage st),
+// grid-stride; each lane takes 8 consecutive elements. The row is x_perm[r]
+// (mode 0, operand order) or x[sorted_pair[r] / k] (mode 1, natural order).
+// Its four planes go to rows p BN + n (n = (r - offsets[e]) % BN) of the
+// activation blob (tile, st) of its N tile, tile = tile_start[e] + (r -
+// offsets[e]) / BN; the plane scales go into that blob's scale atoms.
+__global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
                                                        uint8_t *__restrict__ bblob) {
@@ -178,60 +262,23 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
     __shared__ int s_wsum[8];
     pdl_wait();
     pdl_release();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int e = tid; e <= E; e += blockDim.x) s_off[e] = offsets[e];
-    __syncthreads();
-    // tile prefix: s_tile[e] = sum over e' < e of ceil(n_e' / BN), 256 threads x 4 experts
-    {
-        int cnt[4], run = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = tid * 4 + i;
-            cnt[i] = e < E ? (s_off[e + 1] - s_off[e] + BN - 1) / BN : 0;
-            run += cnt[i];
-        }
-        int incl = run;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += v;
-        }
-        if (lane == 31) s_wsum[warp] = incl;
-        __syncthreads();
-        int base = incl - run;
-        for (int w = 0; w < warp; ++w) base += s_wsum[w];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = tid * 4 + i;
-            if (e <= E) s_tile[e] = base;
-            base += cnt[i];
-        }
-    }
-    __syncthreads();
-    const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = mx_bblob_bytes(BN);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
+    const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsMx, BN);
     const int64_t units = (int64_t)P * KST;
     const int64_t nw = (int64_t)gridDim.x * 8;
     for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += nw) {
         const int r = (int)(u / KST), st = (int)(u - (int64_t)r * KST);
-        int lo = 0, hi = E - 1;   // expert with s_off[e] <= r < s_off[e + 1]
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_off[mid] <= r) lo = mid; else hi = mid - 1;
-        }
-        const int rel = r - s_off[lo];
-        const int tile = s_tile[lo] + rel / BN, n = rel % BN;
-        uint4 uv = src[(int64_t)(gather ? sorted_pair[r] / k : r) * K8 + st * 32 + lane];
-        if (!gather) uv = deinterleave8(uv);
-        const uint32_t w4[4] = {uv.x, uv.y, uv.z, uv.w};
+        const int e = expert_of_row(s_off, E, r);
+        const int rel = r - s_off[e];
+        const int tile = s_tile[e] + rel / BN, n = rel % BN;
+        uint4 uv = src[(int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8 + st * 32 + lane];
+        if (mode == 0) uv = deinterleave8(uv);
         float v[8];
+        bf16x8_to_float(uv, v);
         float amax = 0.0f;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[h]));
-            v[2 * h] = f.x;
-            v[2 * h + 1] = f.y;
-            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
         // 4 consecutive lanes hold one 32-block
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -245,6 +292,82 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
             const int R = pl * BN + n;
             *reinterpret_cast<uint32_t *>(blob + sw128_chunk(R, c16) + (lane & 3) * 4) = pw[pl];
             if ((lane & 3) == 0) blob[NROW * 128 + (c16 >> 2) * 512 + atom_offset(R, c16 & 3)] = (uint8_t)(s - 3 * pl);
+        }
+    }
+}
+
+// NVFP4 activations. One warp per permuted row r (grid-stride): the row is
+// x_perm[r] (mode 0), x[sorted_pair[r] / k] (mode 1) or src[r] (mode 2, natural
+// order). A first pass finds the row maximum 2^E and the offset C = 9 - E
+// (rowexp[r]); then every 16-block with maximum exponent e gets the E4M3 scale
+// 2^min(8, max(-9, e - 1 + C)) for all four planes, plane p carrying the unit
+// 2^(scale exponent - 3p - C). Rows and atoms as in mx_quant_kernel.
+__global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__ src, int mode,
+                                                       const int32_t *__restrict__ sorted_pair, int k, int P, int K,
+                                                       const int32_t *__restrict__ offsets, int E, int BN,
+                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp) {
+    __shared__ int s_off[kMaxExperts + 1];
+    __shared__ int s_tile[kMaxExperts + 1];
+    __shared__ int s_wsum[8];
+    pdl_wait();
+    pdl_release();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
+    const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsNv, BN);
+    for (int r = blockIdx.x * 8 + warp; r < P; r += gridDim.x * 8) {
+        const int e = expert_of_row(s_off, E, r);
+        const int rel = r - s_off[e];
+        const int tile = s_tile[e] + rel / BN, n = rel % BN;
+        const uint4 *srow = src + (int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8;
+        // pass 1: row maximum (order does not matter)
+        float amax = 0.0f;
+        for (int c = lane; c < K8; c += 32) {
+            float v[8];
+            bf16x8_to_float(__ldcg(srow + c), v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        }
+        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+        int Er = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 0;
+        Er = Er < -90 ? -90 : Er;
+        const int C = 9 - Er;
+        if (lane == 0) rowexp[r] = C;
+        // pass 2: planes, 8 elements per lane, 2 lanes per 16-block
+        for (int c = lane; c < K8; c += 32) {
+            uint4 uv = __ldcg(srow + c);
+            if (mode == 0) uv = deinterleave8(uv);
+            float v[8];
+            bf16x8_to_float(uv, v);
+            float bmax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+            bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+            int ks = bmax > 0.0f ? (int)((__float_as_uint(bmax) >> 23) & 0xFF) - 128 + C : -9;
+            ks = ks < -9 ? -9 : (ks > 8 ? 8 : ks);
+            uint32_t pw[kMxPlanes];
+            float rr[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rr[i] = v[i];
+#pragma unroll
+            for (int pl = 0; pl < kMxPlanes; ++pl) {
+                const int uexp = ks - 3 * pl - C;   // plane unit 2^uexp, |uexp| <= 126
+                const float inv = exp2_neg_biased(uexp + 127), unit = exp2_biased(uexp + 127);
+                float t[8], q[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t[i] = rr[i] * inv;
+                pw[pl] = e2m1x8(t, q);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) rr[i] = fmaf(-q[i], unit, rr[i]);
+            }
+            const int st = c >> 5, cc = c & 31, c16 = cc >> 2, b16 = cc >> 1;
+            uint8_t *blob = bblob + ((int64_t)tile * KST + st) * BB;
+            const uint8_t sb = e4m3_pow2(ks);
+#pragma unroll
+            for (int pl = 0; pl < kMxPlanes; ++pl) {
+                const int R = pl * BN + n;
+                *reinterpret_cast<uint32_t *>(blob + sw128_chunk(R, c16) + (cc & 3) * 4) = pw[pl];
+                if ((cc & 1) == 0) blob[NROW * 128 + (b16 >> 2) * 512 + atom_offset(R, b16 & 3)] = sb;
+            }
         }
     }
 }
@@ -296,22 +419,25 @@ __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int
 // parity wait on a slot barrier is exactly one phase after the previous one.
 //   warps 0-3   producers: per stage one bulk copy of the weight blob and one
 //               of the activation blob. Warp 2 also builds the tile prefix.
-//   warps 12-15 MMA issuers (warp 12 owns TMEM): per stage four tcgen05.cp of
-//               scale atoms, four kind::mxf4 MMAs of K = 64, one commit.
+//   warps 12-15 MMA issuers (warp 12 owns TMEM): per stage one tcgen05.cp per
+//               scale atom, four MMAs of K = 64, one commit.
 //   warps 4-7   epilogue of even items (accumulator buffer 0);
 //   warps 8-11  epilogue of odd items (buffer 1). The epilogue adds the NP
 //               pipelines' accumulators and the four planes' columns.
 // TMEM columns: accumulator (buffer a, pipeline w) at (a NW + w) N; from 2 NW N
-// on, 32 scale columns per pipeline (two rotating groups of 16: weight atoms at
-// +0 and +4, activation atoms at +8 and +12).
-template <int PHASE, int BN>
+// on, 16 NA scale columns per pipeline (two rotating groups of 8 NA: the NA
+// weight atoms, then the NA activation atoms, 4 columns each).
+template <int FMT, int PHASE, int BN>
 __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_constant__ MxParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     constexpr int N = kMxPlanes * BN;                       // MMA N: the planes' rows
     constexpr int NW = N <= 32 ? 4 : (N <= 64 ? 2 : 1);    // pipelines TMEM has room for
-    constexpr int BBLOB = mx_bblob_bytes(BN);
-    constexpr int STAGE = kMxABlob + BBLOB;                 // a multiple of 1024
+    constexpr int NA = bs_atoms(FMT);                       // scale atoms per operand and stage
+    constexpr int ABLOB = bs_ablob_bytes(FMT);
+    constexpr int BBLOB = bs_bblob_bytes(FMT, BN);
+    constexpr int STAGE = ABLOB + BBLOB;                    // a multiple of 1024
     constexpr uint32_t SFCOL = 2 * NW * N;
+    static_assert(SFCOL + NW * 16 * NA <= 512, "TMEM columns");
     const int NP = p.pipes;                                 // divides the stages per item, <= NW
     const int NSW = p.stages / NP;                          // slots per pipeline
 
@@ -389,8 +515,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                 uint64_t *fb = &sm.full[s];
                 mbar_expect_tx(fb, (uint32_t)STAGE);
                 bulk_load(base + s * STAGE,
-                          p.wbase + (int64_t)it.slot * p.w_estride + ((int64_t)it.m * KST + st) * kMxABlob,
-                          kMxABlob, fb);
+                          p.wbase + (int64_t)it.slot * p.w_estride + ((int64_t)it.m * KST + st) * ABLOB, ABLOB,
+                          fb);
             };
             // The slots start empty: the weights of this pipeline's first NSW stages go out
             // before waiting for the kernel that writes the activations.
@@ -412,7 +538,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                         if (!mbar_wait(&sm.empty[s], (round & 1) ^ 1, abort_flag)) { ok = false; break; }
                         issue_weights(it, st, s);
                     }
-                    bulk_load(base + s * STAGE + kMxABlob, p.bblob + ((int64_t)it.rt * KST + st) * BBLOB, BBLOB,
+                    bulk_load(base + s * STAGE + ABLOB, p.bblob + ((int64_t)it.rt * KST + st) * BBLOB, BBLOB,
                               &sm.full[s]);
                 }
             }
@@ -442,18 +568,25 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                     if (!mbar_wait(&sm.full[s], (uint32_t)((loc / NSW) & 1), abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sp = base_u32 + s * STAGE;
-                    const uint32_t sfc = tmem + SFCOL + 32 * w + 16 * sc;   // this stage's scale columns
-                    tmem_cp_atom(sfc, sf_atom_desc(sp + kMxCodeBytes));
-                    tmem_cp_atom(sfc + 4, sf_atom_desc(sp + kMxCodeBytes + 512));
-                    tmem_cp_atom(sfc + 8, sf_atom_desc(sp + kMxABlob + N * 128));
-                    tmem_cp_atom(sfc + 12, sf_atom_desc(sp + kMxABlob + N * 128 + 512));
+                    const uint32_t sfa = tmem + SFCOL + 16 * NA * w + 8 * NA * sc;   // this stage's scales
+                    const uint32_t sfb = sfa + 4 * NA;
+#pragma unroll
+                    for (int a = 0; a < NA; ++a) {
+                        tmem_cp_atom(sfa + 4 * a, sf_atom_desc(sp + kMxCodeBytes + 512 * a));
+                        tmem_cp_atom(sfb + 4 * a, sf_atom_desc(sp + ABLOB + N * 128 + 512 * a));
+                    }
                     const uint64_t adesc = smem_desc_sw128(sp);
-                    const uint64_t bdesc = smem_desc_sw128(sp + kMxABlob);
+                    const uint64_t bdesc = smem_desc_sw128(sp + ABLOB);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {   // K = 64 each: 32 bytes further along the row
-                        const uint32_t id = (uint32_t)(i & 1) * 2, h = (uint32_t)(i >> 1) * 4;
-                        mma_mxf4(d, adesc + (uint64_t)(2 * i), bdesc + (uint64_t)(2 * i), idesc_mxf4(N, id),
-                                 (sfc + h) | (id << 30), (sfc + 8 + h) | (id << 30), (k | i) != 0);
+                        if constexpr (FMT == kBsMx) {   // two 32-blocks: bytes id, id + 1 of atom i / 2
+                            const uint32_t id = (uint32_t)(i & 1) * 2, h = (uint32_t)(i >> 1) * 4;
+                            mma_mxf4(d, adesc + (uint64_t)(2 * i), bdesc + (uint64_t)(2 * i), idesc_mxf4(N, id),
+                                     (sfa + h) | (id << 30), (sfb + h) | (id << 30), (k | i) != 0);
+                        } else {                        // four 16-blocks: the whole column of atom i
+                            mma_nvf4(d, adesc + (uint64_t)(2 * i), bdesc + (uint64_t)(2 * i), idesc_nvf4(N),
+                                     sfa + 4 * i, sfb + 4 * i, (k | i) != 0);
+                        }
                     }
                     sc ^= 1;
                     mma_commit(&sm.empty[s]);
@@ -484,10 +617,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
             constexpr int HCH = CH / 2;             // UP: tokens per warp of a gate/up pair
             for (int c0 = 0; c0 < BN && ok; c0 += CH, ++xc) {
-                // sum over the pipelines and the four planes for tokens c0..c0+CH-1
+                // sum over the pipelines and the four planes for tokens c0..c0+CH-1; the
+                // NVFP4 planes carry the extra factor 2^(3p) in their scales
                 float val[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) val[j] = 0.0f;
+                constexpr float kPw[kMxPlanes] = {1.0f, FMT == kBsNv ? 0.125f : 1.0f, FMT == kBsNv ? 0.015625f : 1.0f,
+                                                  FMT == kBsNv ? 0.001953125f : 1.0f};
                 if constexpr (BN <= 8) {
                     for (int w = 0; w < NP; ++w) {   // all N <= 32 columns of pipeline w
                         uint32_t v0[16], v1[16];
@@ -499,7 +635,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
 #pragma unroll
                             for (int pl = 0; pl < kMxPlanes; ++pl) {
                                 const int col = pl * BN + j;
-                                val[j] += __uint_as_float(col < 16 ? v0[col & 15] : v1[col & 15]);
+                                val[j] = fmaf(__uint_as_float(col < 16 ? v0[col & 15] : v1[col & 15]), kPw[pl], val[j]);
                             }
                         }
                     }
@@ -512,7 +648,15 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
 #pragma unroll
                         for (int pl = 0; pl < kMxPlanes; ++pl)
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) val[j] += __uint_as_float(v[pl][j]);
+                            for (int j = 0; j < 16; ++j) val[j] = fmaf(__uint_as_float(v[pl][j]), kPw[pl], val[j]);
+                    }
+                }
+                if constexpr (FMT == kBsNv) {   // 2^-C of each token row, times the expert's tensor scale
+                    const float ts = p.tscale[it.e];
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) {
+                        const int C = c0 + j < it.nvalid ? __ldcg(p.rowexp + it.row0 + c0 + j) : 0;
+                        val[j] *= exp2_neg_biased(C + 127) * ts;
                     }
                 }
                 if (PHASE == kPhaseDown) {
@@ -547,6 +691,18 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                     // channel ch = 64 m + 32 pr + lane: this warp holds one 32-block of h,
                     // which is one 16-byte chunk of a row of the down pass's activation blob
                     const int ch = it.m * 64 + pr * 32 + lane;
+                    if constexpr (FMT == kBsNv) {   // h in bf16; the NVFP4 quantiser makes its planes
+#pragma unroll
+                        for (int j = 0; j < HCH; ++j) {
+                            const float g = gate ? val[j] : other[j];
+                            const float uu = gate ? other[j] : val[HCH + j];
+                            const int tok = c0 + t0 + j;
+                            if (tok < it.nvalid)
+                                reinterpret_cast<__nv_bfloat16 *>(p.hout)[(int64_t)(it.row0 + tok) * p.I + ch] =
+                                    __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * uu);
+                        }
+                        continue;
+                    }
                     const int c16 = (ch >> 5) & 7;   // 32-block within the 256-wide stage
                     uint8_t *blob = p.bblob_out + ((int64_t)it.rt * (p.I / kMxStageK) + (ch >> 8)) * BBLOB;
 #pragma unroll
@@ -608,44 +764,46 @@ size_t mx_tiles_ub(int n_rows, int E) {
     return (size_t)(n_rows + BN - 1) / BN + (size_t)E;
 }
 
+// Activation blob bytes of n_rows rows and reduction K, sized for NVFP4 (the
+// larger of the two formats' blobs).
 size_t mx_blob_bytes(int n_rows, int K, int E) {
-    return align_up(mx_tiles_ub(n_rows, E) * (K / kMxStageK) * mx_bblob_bytes(choose_bn_mx(n_rows, E)), 256);
+    return align_up(mx_tiles_ub(n_rows, E) * (K / kMxStageK) * bs_bblob_bytes(kBsNv, choose_bn_mx(n_rows, E)), 256);
 }
 
-static size_t mx_smem_bytes(int phase, int BN, int stages, int E) {
-    const size_t stage = (size_t)kMxABlob + mx_bblob_bytes(BN);
+static size_t mx_smem_bytes(int fmt, int phase, int BN, int stages, int E) {
+    const size_t stage = (size_t)bs_ablob_bytes(fmt) + bs_bblob_bytes(fmt, BN);
     return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 128 * kMxXch * 4 : 0) + sizeof(MxSmem) +
            (size_t)(3 * E + 2) * sizeof(int);
 }
 
-template <int PHASE, int BN>
+template <int FMT, int PHASE, int BN>
 static cudaError_t mx_launch_one(const MxParams &p, int grid, size_t smem, cudaStream_t st) {
-    auto kfn = ffn_mx_kernel<PHASE, BN>;
+    auto kfn = ffn_mx_kernel<FMT, PHASE, BN>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kfn, dim3(grid), dim3(kMxThreads), smem, st, p);
     return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
-template <int PHASE>
+template <int FMT, int PHASE>
 static cudaError_t mx_launch_bn(int BN, const MxParams &p, int grid, size_t smem, cudaStream_t st) {
     switch (BN) {
-        case 4: return mx_launch_one<PHASE, 4>(p, grid, smem, st);
-        case 8: return mx_launch_one<PHASE, 8>(p, grid, smem, st);
-        case 16: return mx_launch_one<PHASE, 16>(p, grid, smem, st);
-        default: return mx_launch_one<PHASE, 32>(p, grid, smem, st);
+        case 4: return mx_launch_one<FMT, PHASE, 4>(p, grid, smem, st);
+        case 8: return mx_launch_one<FMT, PHASE, 8>(p, grid, smem, st);
+        case 16: return mx_launch_one<FMT, PHASE, 16>(p, grid, smem, st);
+        default: return mx_launch_one<FMT, PHASE, 32>(p, grid, smem, st);
     }
 }
 
 // Pipelines and ring depth of one phase: as many pipelines as divide the
 // stages of an item and fit TMEM (4 for N <= 32, 2 for N = 64, else 1), with
 // at least two slots each in the shared memory of one CTA. False if none fits.
-bool mx_plan(int phase, int BN, int K, int E, MxPlan *pl) {
+bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl) {
     const int KST = K / kMxStageK;
     const int N = kMxPlanes * BN;
     const int nw = N <= 32 ? 4 : (N <= 64 ? 2 : 1);
     int fit = kMxMaxStages;
-    while (fit > 0 && mx_smem_bytes(phase, BN, fit, E) > (size_t)kMxSmemCap) --fit;
+    while (fit > 0 && mx_smem_bytes(fmt, phase, BN, fit, E) > (size_t)kMxSmemCap) --fit;
     for (int np = nw < KST ? nw : KST; np >= 1; --np) {
         if (KST % np) continue;
         const int nsw = fit / np;
@@ -657,34 +815,48 @@ bool mx_plan(int phase, int BN, int K, int E, MxPlan *pl) {
     return false;
 }
 
-moe_status launch_mx_phase(int phase, int BN, MxParams p, int num_sms, cudaStream_t st) {
+moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st) {
     if (p.K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", p.K, kMxStageK);
     MxPlan pl;
-    if (!mx_plan(phase, BN, p.K, p.E, &pl))
-        return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no pipeline plan for MXFP4", p.K);
+    if (!mx_plan(fmt, phase, BN, p.K, p.E, &pl))
+        return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no pipeline plan for the block-scaled FP4 path", p.K);
     p.pipes = pl.pipes;
     p.stages = pl.stages;
-    size_t smem = mx_smem_bytes(phase, BN, pl.stages, p.E);
+    size_t smem = mx_smem_bytes(fmt, phase, BN, pl.stages, p.E);
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: it allocates all 512 TMEM columns
     const int64_t items_ub = ((int64_t)p.n_rows / BN + p.E) * p.m_tiles;
     const int grid = (int)(items_ub < num_sms ? (items_ub > 0 ? items_ub : 1) : num_sms);
-    cudaError_t e = phase == kPhaseUp ? mx_launch_bn<kPhaseUp>(BN, p, grid, smem, st)
-                                      : mx_launch_bn<kPhaseDown>(BN, p, grid, smem, st);
-    if (e != cudaSuccess) return set_cuda_error(e, "mx ffn kernel launch");
+    cudaError_t e;
+    if (fmt == kBsNv)
+        e = phase == kPhaseUp ? mx_launch_bn<kBsNv, kPhaseUp>(BN, p, grid, smem, st)
+                              : mx_launch_bn<kBsNv, kPhaseDown>(BN, p, grid, smem, st);
+    else
+        e = phase == kPhaseUp ? mx_launch_bn<kBsMx, kPhaseUp>(BN, p, grid, smem, st)
+                              : mx_launch_bn<kBsMx, kPhaseDown>(BN, p, grid, smem, st);
+    if (e != cudaSuccess) return set_cuda_error(e, "block-scaled ffn kernel launch");
     return MOE_OK;
 }
 
-moe_status launch_mx_quant(const void *src, int gather, const int32_t *sorted_pair, int k, int P, int K,
-                           const int32_t *offsets, int E, int BN, void *bblob, int num_sms, cudaStream_t st) {
+moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
+                           const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
+                           cudaStream_t st) {
     if (P == 0) return MOE_OK;
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
-    const int64_t units = (int64_t)P * (K / kMxStageK);
-    int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
-    cudaError_t e = launch_pdl(mx_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
-                               gather, sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob));
+    cudaError_t e;
+    if (fmt == kBsNv) {   // one warp per row
+        const int blocks = (P + 7) / 8 < num_sms * 8 ? (P + 7) / 8 : num_sms * 8;
+        e = launch_pdl(nv_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp);
+    } else {              // one warp per (row, stage)
+        if (mode == 2) return set_error(MOE_ERR_UNSUPPORTED, "MXFP4 quantiser mode 2");
+        const int64_t units = (int64_t)P * (K / kMxStageK);
+        const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
+        e = launch_pdl(mx_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob));
+    }
     if (e == cudaSuccess) e = cudaGetLastError();
-    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "mx quant launch");
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "block-scaled quantiser launch");
 }
 
 }  // namespace moe

@@ -146,6 +146,9 @@ __device__ __forceinline__ ItemInfo decode_item(const FfnSmem &sm, const FfnPara
 // TILED: the weights were prepacked by moe_prepack into one contiguous blob per
 // (M tile, K stage) - 128 rows of codes, 16-byte chunk-major, followed by the
 // rows' scales for that stage - and each stage arrives with one bulk copy.
+// Prepacked NVFP4 has the block-scaled path's blobs instead (one per 256-wide
+// stage: 128-byte rows of codes in the 128-byte swizzle, then four scale
+// atoms); a ring slot holds one such blob and serves two 128-wide stages.
 // Otherwise the codes come from the row-major tensor through a 3D TMA box and
 // the scales through one bulk copy per tile.
 template <int FMT, int PHASE, int BN, bool TILED>
@@ -155,7 +158,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
     constexpr int RB = RawFmt<FMT>::kRowBytes;
     constexpr int SBY = RawFmt<FMT>::kScaleBytes;
     constexpr int RAWB = 128 * RB;                          // code bytes per stage
-    constexpr int SB = RAWB + (TILED ? 128 * SBY : 0);      // smem bytes per stage (codes [+ scales])
+    constexpr bool NVB = TILED && FMT == MOE_NVFP4;         // block-scaled blob layout
+    constexpr int KPS = NVB ? 2 : 1;                        // 128-wide stages per ring slot
+    constexpr int SB = KPS * (RAWB + (TILED ? 128 * SBY : 0));   // smem bytes per slot (codes [+ scales])
     constexpr int BSTAGE = BN * 256;            // activation bytes per stage (two 64-column atoms)
     constexpr int BGROUP = kG * BSTAGE;         // activation bytes per group
 
@@ -260,14 +265,14 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     bulk_load(dst + 64 * p.s_rowbytes, sbase + (int64_t)rowB * p.s_rowbytes, 64 * p.s_rowbytes,
                               &sm.scfull[sb]);
                 }
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = 0; kb < KB; kb += KPS) {
                     if (!mbar_wait(&sm.rempty[s], ph ^ 1, abort_flag)) { ok = false; break; }
                     uint64_t *fb = &sm.rfull[s];
                     mbar_expect_tx(fb, SB);
                     uint8_t *raw = rawst + s * SB;
                     if (TILED) {
                         const uint8_t *src = p.wbase + (int64_t)slot * p.w_estride +
-                                             ((int64_t)it.m * KB + kb) * SB;
+                                             ((int64_t)it.m * (KB / KPS) + kb / KPS) * SB;
                         bulk_load(raw, src, SB, fb);
                     } else if (FMT == MOE_BF16) {
                         // two 64-column boxes per 64-row half
@@ -466,13 +471,15 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                     }
                     ++gstart;
                 }
-                if (!mbar_wait(&sm.rfull[s], ph, abort_flag)) { ok = false; break; }
+                if (kb % KPS == 0 && !mbar_wait(&sm.rfull[s], ph, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint8_t *raw = rawst + s * SB;
+                const int hk = kb & (KPS - 1);   // NVB: 128-wide half of the blob
                 // 16-byte chunk c of this thread's row, and its scales for this stage
                 auto chunk = [&](int c) -> uint4 {
                     const uint8_t *a;
-                    if (TILED) a = raw + ((c * 128 + m) << 4);
+                    if (NVB) a = raw + m * 128 + (((hk * 4 + c) ^ (m & 7)) << 4);
+                    else if (TILED) a = raw + ((c * 128 + m) << 4);
                     else if (FMT == MOE_MXFP4 || FMT == MOE_NVFP4) a = raw + rh * (RAWB / 2) + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4);
                     else if (FMT == MOE_FP8_E4M3_K128) a = raw + rh * (RAWB / 2) + rr * 128 + ((c ^ (rr & 7)) << 4);
                     else a = raw + (rh * 2 + (c >> 3)) * 8192 + rr * 128 + (((c & 7) ^ (rr & 7)) << 4);
@@ -500,7 +507,12 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                             for (int j = 0; j < 16; ++j) o[j] = bmul2(o[j], f2);
                         }
                     } else {
-                        const uint32_t sc2 = *reinterpret_cast<const uint16_t *>(scs + 2 * sub);   // two blocks of 16
+                        // two blocks of 16; NVB: blocks 2 sub, 2 sub + 1 of half hk sit in atom
+                        // 2 hk + sub / 2 at scale positions 2 (sub % 2), + 1 of row m
+                        const uint8_t *s2 = NVB ? raw + 128 * 128 + (2 * hk + (sub >> 1)) * 512 + (m & 31) * 16 +
+                                                      (m >> 5) * 4 + 2 * (sub & 1)
+                                                : scs + 2 * sub;
+                        const uint32_t sc2 = *reinterpret_cast<const uint16_t *>(s2);
                         uint32_t f[2];
 #pragma unroll
                         for (int b = 0; b < 2; ++b) {
@@ -556,9 +568,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ 
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&sm.adec[sa]);
-                    mbar_arrive(&sm.rempty[s]);   // codes read: the slot can be refilled
+                    if (hk == KPS - 1) mbar_arrive(&sm.rempty[s]);   // codes read: the slot can be refilled
                 }
-                if (++s == nr) { s = 0; ph ^= 1; }
+                if (hk == KPS - 1 && ++s == nr) { s = 0; ph ^= 1; }
                 if (++sa == na) sa = 0;
             }
             if (!ok) break;
@@ -665,7 +677,8 @@ static size_t ffn_smem_bytes(int fmt, int phase, int BN, int stages, int bgroups
     const int rb = stage_code_bytes(fmt);
     size_t b = 1024;                                     // alignment slack
     b += (size_t)bgroups * kG * BN * 256;
-    b += (size_t)stages * 128 * (rb + (tiled ? stage_scale_bytes(fmt) : 0));
+    const int kps = tiled && fmt == MOE_NVFP4 ? 2 : 1;   // prepacked NVFP4: one 256-wide blob per slot
+    b += (size_t)stages * kps * 128 * (rb + (tiled ? stage_scale_bytes(fmt) : 0));
     if (!tiled) b += 2 * (size_t)((128 * s_rowbytes + 15) & ~15);
     if (phase == kPhaseUp) b += 64 * kXchStride * 4;
     b += sizeof(FfnSmem);

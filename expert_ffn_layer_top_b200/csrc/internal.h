@@ -36,15 +36,20 @@ struct FfnParams {
     int64_t w_estride;          // tiled: bytes between experts
 };
 
-// Block-scaled MXFP4 path (ffn_mx.cu): kind::mxf4 MMAs, weights prepacked by
-// moe_prepack, activations as four E2M1 planes with per-tile scale atoms.
+// Block-scaled FP4 path (ffn_mx.cu) for MXFP4 (kind::mxf4, E8M0 scales per 32)
+// and NVFP4 (kind::mxf4nvf4, E4M3 scales per 16) experts prepacked by
+// moe_prepack; activations as four E2M1 planes with per-tile scale atoms.
+constexpr int kBsMx = 0, kBsNv = 1;              // formats of the path
 constexpr int kMxStageK = 256;                   // K elements per pipeline stage
 constexpr int kMxCodeBytes = 128 * 128;          // packed codes of one (M tile, stage): 128 rows x 128 B
-constexpr int kMxABlob = kMxCodeBytes + 1024;    // + the two 512-byte scale atoms of the stage
 constexpr int kMxPlanes = 4;                     // E2M1 planes per activation value
 
-// Bytes of one activation blob (N tile of BN rows, one stage): 4 BN rows of 128 B, then two scale atoms.
-__host__ __device__ constexpr int mx_bblob_bytes(int BN) { return kMxPlanes * BN * 128 + 1024; }
+// 512-byte scale atoms per operand and stage (each covers 4 scales per row).
+__host__ __device__ constexpr int bs_atoms(int f) { return f == kBsNv ? 4 : 2; }
+// Bytes of one weight blob (M tile, stage): codes, then the scale atoms.
+__host__ __device__ constexpr int bs_ablob_bytes(int f) { return kMxCodeBytes + 512 * bs_atoms(f); }
+// Bytes of one activation blob (N tile of BN rows, stage): 4 BN rows of 128 B, then the scale atoms.
+__host__ __device__ constexpr int bs_bblob_bytes(int f, int BN) { return kMxPlanes * BN * 128 + 512 * bs_atoms(f); }
 
 struct MxParams {
     const int32_t *offsets;     // [E+1]
@@ -55,12 +60,15 @@ struct MxParams {
     int stages;                 // shared-memory slots, set by the launcher
     int pipes;                  // independent producer/MMA pipelines, set by the launcher
     int n_rows;
-    const uint8_t *wbase;       // this phase's prepacked tensor: [m_tiles][K/256] blobs of kMxABlob bytes
+    const uint8_t *wbase;       // this phase's prepacked tensor: [m_tiles][K/256] weight blobs
     int64_t w_estride;          // bytes between experts (or cache slots)
-    const uint8_t *bblob;       // activation blobs [tiles][K/256][mx_bblob_bytes(BN)]
+    const uint8_t *bblob;       // activation blobs [tiles][K/256]
+    const int32_t *rowexp;      // NVFP4: per-row exponent offset of the activation planes [n_rows]
+    const float *tscale;        // NVFP4: per-expert tensor scale of this phase's weights [E]
     void *out;                  // down: y [n_rows][H] (bf16 or fp32)
     int out_fp32;
-    uint8_t *bblob_out;         // up: blobs of h for the down pass [tiles][I/256][...]
+    uint8_t *bblob_out;         // MXFP4 up: blobs of h for the down pass [tiles][I/256]
+    void *hout;                 // NVFP4 up: h bf16 [n_rows][I]
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -82,12 +90,15 @@ int choose_bn_mx(int n_rows, int E);
 struct MxPlan {
     int pipes, stages;
 };
-bool mx_plan(int phase, int BN, int K, int E, MxPlan *pl);
+bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl);
 size_t mx_tiles_ub(int n_rows, int E);
 size_t mx_blob_bytes(int n_rows, int K, int E);
-moe_status launch_mx_phase(int phase, int BN, MxParams p, int num_sms, cudaStream_t st);
-moe_status launch_mx_quant(const void *src, int gather, const int32_t *sorted_pair, int k, int P, int K,
-                           const int32_t *offsets, int E, int BN, void *bblob, int num_sms, cudaStream_t st);
+moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st);
+// src rows: mode 0 x_perm[r] (operand order), 1 x[sorted_pair[r] / k] (natural
+// order), 2 src[r] (natural order; NVFP4 only). rowexp: NVFP4 only.
+moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
+                           const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
+                           cudaStream_t st);
 
 moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           cudaStream_t st);

@@ -3,18 +3,20 @@
 // For every expert, M tile and 128-wide K stage the tiled layout holds one
 // contiguous blob with the 128 weight rows of the tile (gate/up: 64 gate rows
 // then the 64 matching up rows; down: 128 consecutive rows):
-//   BF16, FP8, NVFP4: the codes as 16-byte chunks in chunk-major order (chunk c
-//     of row r at (c*128 + r)*16), then each row's scales for that stage. The
+//   BF16, FP8: the codes as 16-byte chunks in chunk-major order (chunk c of
+//     row r at (c*128 + r)*16), then each row's scales for that stage. The
 //     decoding FFN moves a stage with one bulk copy and its decoder threads
 //     read consecutive chunks without bank conflicts.
-//   MXFP4 (stages 256 wide): one 17 KiB blob per (M tile, stage), in that
+//   MXFP4, NVFP4 (stages 256 wide): one blob per (M tile, stage), in that
 //     order. First the packed codes, 128 bytes per row in natural K order,
 //     with the 16-byte chunk c of row r stored at r*128 + (c ^ (r % 8))*16:
 //     the 128-byte swizzle the block-scaled MMA reads from shared memory, so
-//     one bulk copy lands the operand ready to use. Then two 512-byte scale
-//     atoms, one per 128-wide half of the stage: the E8M0 scale of row r and
-//     32-block j of the half at byte (r % 32)*16 + (r / 32)*4 + j, the
-//     arrangement tcgen05.cp moves into TMEM.
+//     one bulk copy lands the operand ready to use. Then the 512-byte scale
+//     atoms: the scale of row r and scale block j of the atom's K range at
+//     byte (r % 32)*16 + (r / 32)*4 + j, the arrangement tcgen05.cp moves into
+//     TMEM. MXFP4: two atoms (E8M0 per 32, one atom per 128-wide half), a
+//     17 KiB blob; NVFP4: four atoms (E4M3 per 16, one per 64-wide quarter),
+//     an 18 KiB blob.
 // Values are untouched: this is a byte permutation.
 #include "common.cuh"
 #include "internal.h"
@@ -60,16 +62,19 @@ __global__ void prepack_kernel(const uint8_t *__restrict__ w, int64_t w_estride,
     uint8_t *blob = out + e * out_estride + ((int64_t)m * KB + kb) * SB;
     const uint8_t *src = w + e * w_estride + (int64_t)row * row_bytes + (int64_t)kb * RB;
     const uint8_t *ss = scale + e * s_estride + (int64_t)row * s_row_bytes + (int64_t)kb * SBY;
-    if (mx) {   // RB = 64, SBY = 4: this thread fills half `kb % 2` of row r of blob (m, kb / 2)
+    if (mx) {   // FP4, RB = 64: this thread fills half `kb % 2` of row r of blob (m, kb / 2)
         const int half = kb & 1;
-        uint8_t *mb = out + e * out_estride + ((int64_t)m * (KB / 2) + (kb >> 1)) * kMxABlob;
+        const int blob = kMxCodeBytes + 2 * 128 * SBY;   // SBY = 4 (MXFP4) or 8 (NVFP4) scales per half
+        uint8_t *mb = out + e * out_estride + ((int64_t)m * (KB / 2) + (kb >> 1)) * blob;
         for (int c = 0; c < 4; ++c) {
             const int cc = half * 4 + c;   // 16-byte chunk of the 128-byte row
             *reinterpret_cast<uint4 *>(mb + r * 128 + ((cc ^ (r & 7)) << 4)) =
                 *reinterpret_cast<const uint4 *>(src + c * 16);
         }
-        uint8_t *atom = mb + kMxCodeBytes + half * 512;
-        for (int j = 0; j < 4; ++j) atom[(r & 31) * 16 + (r >> 5) * 4 + j] = ss[j];
+        for (int i = 0; i < SBY; ++i) {   // scale i of the half: atom half * SBY/4 + i/4, block i % 4
+            uint8_t *atom = mb + kMxCodeBytes + (half * (SBY / 4) + i / 4) * 512;
+            atom[(r & 31) * 16 + (r >> 5) * 4 + (i & 3)] = ss[i];
+        }
         return;
     }
     for (int c = 0; c < RB / 16; ++c)
@@ -97,7 +102,7 @@ moe_status launch_prepack(const moe_experts &in, int which, void *out, int64_t o
     const int blocks = (int)((total + 255) / 256);
     count_launch();
     prepack_kernel<<<blocks, 256, 0, st>>>(w, w_es, s, s_es, in.E, in.I, K, which, mt, KB, RB, SBY, row_bytes,
-                                           s_row_bytes, in.fmt == MOE_MXFP4, reinterpret_cast<uint8_t *>(out),
+                                           s_row_bytes, in.fmt == MOE_MXFP4 || in.fmt == MOE_NVFP4, reinterpret_cast<uint8_t *>(out),
                                            out_estride);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "prepack launch");

@@ -154,17 +154,22 @@ def test_combine_parity(moe, y_fp32):
 
 
 FFN_CASES = [(fmt, T, tiled) for fmt in ("bf16", "fp8", "mxfp4", "nvfp4") for T in (40, 100, 200, 600)
-             for tiled in (False, True)] + [("mxfp4", 24, True), ("mxfp4", 9, True)]
+             for tiled in (False, True)] + [(f, T, True) for f in ("mxfp4", "nvfp4") for T in (24, 9, 3)]
 
 
 @pytest.mark.parametrize("fmt,T,tiled", FFN_CASES)
 def test_grouped_ffn_parity(moe, fmt, T, tiled):
     """T = 40/100/200/600 with E = 8, k = 2 exercises token tiles of 16/32/64/128,
     on row-major weights and on weights prepacked into the tiled layout.
-    Prepacked MXFP4 runs the block-scaled path (token tiles of 8/16/32/64; T = 9
-    and 24 give tiles of 8 with ragged tails), whose h never exists in bf16:
-    there the down-projection output is compared."""
+    Prepacked MXFP4 runs the block-scaled FP4 path (token tiles of 4/8/16/32;
+    T = 3, 9 and 24 give ragged tails), and so does prepacked NVFP4 while the
+    mean rows per expert (2T / 8 here) is at most 16; larger NVFP4 batches take
+    the decoding path, reading the same prepacked blobs. The block-scaled MXFP4
+    h never exists in bf16, so there the down-projection output is compared;
+    the block-scaled NVFP4 h is written in bf16, natural column order, at the
+    start of the workspace."""
     mx = fmt == "mxfp4" and tiled
+    nv_bs = fmt == "nvfp4" and tiled and -(-2 * T // 8) <= 16
     cfg = dict(H=256, E=8, k=2, I=256, fmt=fmt, wr_fp32=False)
     L = synthetic.make_layer(cfg, seed=7)
     x = synthetic.make_tokens(T, 256, seed=7)
@@ -179,6 +184,12 @@ def test_grouped_ffn_parity(moe, fmt, T, tiled):
     if mx:
         y = moe.moe_grouped_ffn(xp, off, ex)
         torch.cuda.synchronize()
+    elif nv_bs:
+        ws = torch.empty(moe.moe_workspace_size(T * 2, 256, 256, 8, 1, False), dtype=torch.uint8, device="cuda")
+        y = moe.moe_grouped_ffn(xp, off, ex, ws=ws)
+        torch.cuda.synchronize()
+        h = ws[: T * 2 * 256 * 2].view(torch.bfloat16).view(T * 2, 256)
+        assert rel_err(h.float().cpu().numpy(), h_o) < TOL, "gate/up + SwiGLU"
     else:
         ws = torch.empty(T * 2 * 256 * 2 + 256, dtype=torch.uint8, device="cuda")
         y = moe.moe_grouped_ffn(xp, off, ex, ws=ws)
