@@ -751,9 +751,12 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ host side
 
+// Token tile of the block-scaled path from the mean rows per expert. The
+// smallest tile is 8, not 4: with skewed routing a few experts take many rows,
+// and every extra tile of an expert passes its weights through the SM again,
+// while a half-empty tile of 8 costs only activation bytes.
 int choose_bn_mx(int n_rows, int E) {
     const int avg = (n_rows + E - 1) / (E > 0 ? E : 1);
-    if (avg <= 2) return 4;
     if (avg <= 8) return 8;
     if (avg <= 16) return 16;
     return 32;
@@ -788,7 +791,6 @@ static cudaError_t mx_launch_one(const MxParams &p, int grid, size_t smem, cudaS
 template <int FMT, int PHASE>
 static cudaError_t mx_launch_bn(int BN, const MxParams &p, int grid, size_t smem, cudaStream_t st) {
     switch (BN) {
-        case 4: return mx_launch_one<FMT, PHASE, 4>(p, grid, smem, st);
         case 8: return mx_launch_one<FMT, PHASE, 8>(p, grid, smem, st);
         case 16: return mx_launch_one<FMT, PHASE, 16>(p, grid, smem, st);
         default: return mx_launch_one<FMT, PHASE, 32>(p, grid, smem, st);

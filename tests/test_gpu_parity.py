@@ -161,7 +161,7 @@ FFN_CASES = [(fmt, T, tiled) for fmt in ("bf16", "fp8", "mxfp4", "nvfp4") for T 
 def test_grouped_ffn_parity(moe, fmt, T, tiled):
     """T = 40/100/200/600 with E = 8, k = 2 exercises token tiles of 16/32/64/128,
     on row-major weights and on weights prepacked into the tiled layout.
-    Prepacked MXFP4 runs the block-scaled FP4 path (token tiles of 4/8/16/32;
+    Prepacked MXFP4 runs the block-scaled FP4 path (token tiles of 8/16/32;
     T = 3, 9 and 24 give ragged tails), and so does prepacked NVFP4 while the
     mean rows per expert (2T / 8 here) is at most 16; larger NVFP4 batches take
     the decoding path, reading the same prepacked blobs. The block-scaled MXFP4
