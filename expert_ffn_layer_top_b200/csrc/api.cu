@@ -536,15 +536,31 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     int32_t *offsets = reinterpret_cast<int32_t *>(b + L.offsets);
     int32_t *sorted = reinterpret_cast<int32_t *>(b + L.sorted);
     int32_t *prow = reinterpret_cast<int32_t *>(b + L.pair_row);
-    moe_status r = moe_route_topk(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router,
-                                  L.idx - L.router, stream);
-    if (r != MOE_OK) return r;
-    // The block-scaled FP4 path gathers the token rows itself while quantising them.
+    // The block-scaled FP4 path gathers the token rows itself while quantising them, so
+    // it needs no x_perm, and for small batches the router kernel also permutes.
     const int layout = cache ? cache_layout(cache) : experts->layout;
     const bool mx = use_bs(experts->fmt, layout, T * k, E);
-    r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, mx ? nullptr : b + L.x_perm, b + L.perm,
-                    L.x_perm - L.perm, stream);
+    moe_status r;
+    int fused = 0;
+    if (mx) {
+        if (H % 8 || E < 1 || E > kMaxRouterExperts || k < 1 || k > kMaxTopK || k > E)
+            return set_error(MOE_ERR_UNSUPPORTED, "router needs 1<=k<=%d, k<=E<=%d (E=%d k=%d)", kMaxTopK,
+                             kMaxRouterExperts, E, k);
+        if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(wr)) & 15)
+            return set_error(MOE_ERR_INVALID_ARG, "x and wr must be 16-byte aligned");
+        const RouterFuse fz{offsets, sorted, prow, nullptr};
+        r = launch_router(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router, L.idx - L.router,
+                          num_sms(current_device()), st, &fz, &fused);
+    } else {
+        r = moe_route_topk(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router, L.idx - L.router,
+                           stream);
+    }
     if (r != MOE_OK) return r;
+    if (!fused) {
+        r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, mx ? nullptr : b + L.x_perm, b + L.perm,
+                        L.x_perm - L.perm, stream);
+        if (r != MOE_OK) return r;
+    }
     moe_experts view = *experts;
     if (cache) {
         r = cache_resolve_and_map(cache, layer, idx, T, k, experts, &view, st);

@@ -36,6 +36,26 @@ inline void count_launch() { g_kernel_launches.fetch_add(1, std::memory_order_re
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) only when a launch needs
+// more than the kernel was last given on this device: the call costs
+// microseconds of host time on every launch otherwise.
+template <auto KERN>
+inline cudaError_t ensure_max_smem(int bytes) {
+    constexpr int kDevs = 64;
+    static std::atomic<int> given[kDevs];   // zero-initialised (static storage)
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kDevs && given[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kDevs) {
+        int cur = given[dev].load(std::memory_order_relaxed);
+        while (cur < bytes && !given[dev].compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+        }
+    }
+    return e;
+}
+
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                               Args &&...args) {

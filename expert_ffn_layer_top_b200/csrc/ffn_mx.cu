@@ -782,7 +782,7 @@ static size_t mx_smem_bytes(int fmt, int phase, int BN, int stages, int E) {
 template <int FMT, int PHASE, int BN>
 static cudaError_t mx_launch_one(const MxParams &p, int grid, size_t smem, cudaStream_t st) {
     auto kfn = ffn_mx_kernel<FMT, PHASE, BN>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_max_smem<ffn_mx_kernel<FMT, PHASE, BN>>((int)smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kfn, dim3(grid), dim3(kMxThreads), smem, st, p);
     return e == cudaSuccess ? cudaGetLastError() : e;

@@ -689,7 +689,8 @@ template <int FMT, int PHASE, int BN>
 static cudaError_t launch_one(const CUtensorMap &wmap, const CUtensorMap &bmap, const FfnParams &p, int grid,
                               size_t smem, cudaStream_t st) {
     auto kfn = p.tiled ? ffn_tc_kernel<FMT, PHASE, BN, true> : ffn_tc_kernel<FMT, PHASE, BN, false>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = p.tiled ? ensure_max_smem<ffn_tc_kernel<FMT, PHASE, BN, true>>((int)smem)
+                            : ensure_max_smem<ffn_tc_kernel<FMT, PHASE, BN, false>>((int)smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kfn, dim3(grid), dim3(kThreads), smem, st, wmap, bmap, p);
     return e == cudaSuccess ? cudaGetLastError() : e;

@@ -105,9 +105,16 @@ moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscal
 
 // router (router.cu)
 size_t router_ws_bytes(int T, int H, int E);
+// Outputs of the permutation for a router launch that also permutes (the
+// layer forward); the launcher fills in the ticket counter.
+struct RouterFuse {
+    int32_t *offsets, *sorted_pair, *pair_row;
+    unsigned int *ticket;
+};
+// fuse may be null; *fused (if given) tells whether the permutation was done.
 moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                          int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes, int nsm,
-                         cudaStream_t st);
+                         cudaStream_t st, const RouterFuse *fuse = nullptr, int *fused = nullptr);
 
 // permutation (permute.cu)
 size_t permute_ws_bytes(int T, int k, int E);

@@ -14,6 +14,7 @@
 //             8-column groups stored in the operand order 0,4,1,5,2,6,3,7
 #include "common.cuh"
 #include "internal.h"
+#include "permute_small.cuh"
 
 namespace moe {
 
@@ -117,81 +118,15 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t *__r
 }
 
 // Small batches (P <= kSmallP, E <= kSmallE): the whole counting sort in one
-// block - histogram, scan, then the chunks of 1024 pairs in order, each pair
-// placed at its expert's running position + its rank among equal experts of
-// earlier warps of the chunk + its rank inside its warp.
-constexpr int kSmallP = 8192;
-constexpr int kSmallE = 256;
-
+// block of kChunk threads (permute_small.cuh).
 __global__ void __launch_bounds__(kChunk) perm_small_kernel(const int32_t *__restrict__ idx, int P, int E,
                                                            int32_t *__restrict__ offsets,
                                                            int32_t *__restrict__ sorted_pair,
                                                            int32_t *__restrict__ pair_row) {
-    __shared__ int32_t cnt[kSmallE];
-    __shared__ int32_t run[kSmallE];
-    __shared__ int32_t wsum[32];
-    __shared__ int32_t wcnt[kChunk / 32][kSmallE];
+    __shared__ SmallPermuteSmem<kChunk> sm;
     pdl_wait();
     pdl_release();
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    for (int e = tid; e < E; e += kChunk) cnt[e] = 0;
-    __syncthreads();
-    for (int p = tid; p < P; p += kChunk) {
-        const int e = idx[p];
-        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
-        else flag_error(2);
-    }
-    __syncthreads();
-    // exclusive scan over experts (E <= 256: the first 8 warps hold one expert per lane)
-    int c = (tid < E) ? cnt[tid] : 0;
-    int incl = c;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += v;
-    }
-    if (lane == 31) wsum[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int s = wsum[lane];
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, s, d);
-            if (lane >= d) s += v;
-        }
-        wsum[lane] = s;   // inclusive over warps
-    }
-    __syncthreads();
-    if (tid < E) {
-        const int excl = incl - c + (wid > 0 ? wsum[wid - 1] : 0);
-        offsets[tid] = excl;
-        run[tid] = excl;
-    }
-    if (tid == 0) offsets[E] = P;
-    for (int c0 = 0; c0 < P; c0 += kChunk) {
-        for (int i = tid; i < (kChunk / 32) * E; i += kChunk) (&wcnt[0][0])[(i / E) * kSmallE + (i % E)] = 0;
-        __syncthreads();
-        const int p = c0 + tid;
-        int e = (p < P) ? idx[p] : -1 - lane;
-        if (p < P && (e < 0 || e >= E)) e = -1 - lane;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank_w = __popc(peers & ((1u << lane) - 1u));
-        if (e >= 0 && rank_w == 0) wcnt[wid][e] = __popc(peers);
-        __syncthreads();
-        if (e >= 0) {
-            int rank = run[e] + rank_w;
-            for (int w2 = 0; w2 < wid; ++w2) rank += wcnt[w2][e];
-            sorted_pair[rank] = p;
-            pair_row[p] = rank;
-        }
-        __syncthreads();
-        for (int ee = tid; ee < E; ee += kChunk) {
-            int add = 0;
-            for (int w2 = 0; w2 < kChunk / 32; ++w2) add += wcnt[w2][ee];
-            run[ee] += add;
-        }
-        __syncthreads();
-    }
+    small_permute<kChunk>(idx, P, E, offsets, sorted_pair, pair_row, sm);
 }
 
 // Workspace bytes launch_permute actually uses for these sizes: none on the

@@ -18,7 +18,10 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include <mutex>
+
 #include "internal.h"
+#include "permute_small.cuh"
 
 namespace moe {
 
@@ -315,6 +318,11 @@ __global__ void __launch_bounds__(256) router_finish_kernel(const double *__rest
 // chunk. The G parts are added in g order inside the CTA, then the 8 CTA sums in
 // rank order through distributed shared memory, so the result is one fixed
 // fp64 summation order. One warp per token rounds, biases and selects the top k.
+//
+// With fz.ticket set (the layer forward), the routing and the permutation run
+// in this one kernel: every cluster publishes its tokens' top-k and takes a
+// ticket, and the cluster that takes the last ticket sorts all T k pairs by
+// expert (small_permute). No cluster waits on another.
 constexpr int kRCl = 8;              // CTAs per cluster (H slices)
 constexpr int kRClThreads = 256;
 constexpr int kRClChunkMax = 24576;  // bytes of Wr per ring chunk
@@ -355,11 +363,18 @@ static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClus
     return sh->smem <= 200 * 1024;
 }
 
+// Ticket counters of the fused routing + permutation, one per stream (see
+// route_ticket): zero when the module loads, and every fused launch leaves its
+// counter at zero again (the last cluster resets it), so a launch counts from 0.
+constexpr int kTicketSlots = 256;
+__device__ unsigned int g_route_ticket[kTicketSlots];
+
 template <bool WR32, int TT>
 __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     router_cluster_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H, const void *__restrict__ wr, int E,
                           int EPP, int G, int RC, int nch, const float *__restrict__ bias, int k,
-                          int32_t *__restrict__ idx, float *__restrict__ w, float *__restrict__ logits) {
+                          int32_t *__restrict__ idx, float *__restrict__ w, float *__restrict__ logits,
+                          RouterFuse fz) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     constexpr int eb = WR32 ? 4 : 2;
@@ -521,47 +536,99 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
             }
         }
         topk_softmax_warp(v, E, k, lane, idx + (int64_t)t * k, w + (int64_t)t * k);
+        if (fz.ticket) __threadfence();   // the top-k is visible before this cluster's ticket
     }
     cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
+    if (fz.ticket && rank == 0) {
+        __shared__ int s_last;
+        if (tid == 0) {
+            s_last = atomicAdd(fz.ticket, 1u) + 1u == gridDim.y;
+            if (s_last) __threadfence();
+        }
+        __syncthreads();
+        if (s_last) {   // the ring and the sums are no longer needed: their space is the scratch
+            auto &ps = *reinterpret_cast<SmallPermuteSmem<kRClThreads> *>(rsm + 64);
+            small_permute<kRClThreads>(idx, T * k, E, fz.offsets, fz.sorted_pair, fz.pair_row, ps);
+            if (tid == 0) atomicExch(fz.ticket, 0u);   // ready for the next launch on this counter
+        }
+    }
 }
 
 template <bool WR32, int TT>
 static cudaError_t launch_router_cluster_t(const RouterClusterShape &sh, const void *x, int T, int H, const void *wr,
                                            int E, const float *bias, int k, int32_t *idx, float *w, float *logits,
-                                           cudaStream_t st) {
+                                           const RouterFuse &fz, cudaStream_t st) {
     auto kern = router_cluster_kernel<WR32, TT>;
-    if (sh.smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh.smem);
+    size_t smem = sh.smem;
+    if (fz.ticket && smem < 64 + sizeof(SmallPermuteSmem<kRClThreads>)) smem = 64 + sizeof(SmallPermuteSmem<kRClThreads>);
+    if (smem > 48 * 1024) {
+        cudaError_t e = ensure_max_smem<router_cluster_kernel<WR32, TT>>((int)smem);
         if (e != cudaSuccess) return e;
     }
     dim3 grid(kRCl, (T + TT - 1) / TT);
-    cudaError_t e = launch_pdl(kern, grid, dim3(kRClThreads), sh.smem, st, reinterpret_cast<const __nv_bfloat16 *>(x),
-                               T, H, wr, E, sh.EPP, sh.G, sh.RC, sh.nch, bias, k, idx, w, logits);
+    cudaError_t e = launch_pdl(kern, grid, dim3(kRClThreads), smem, st, reinterpret_cast<const __nv_bfloat16 *>(x),
+                               T, H, wr, E, sh.EPP, sh.G, sh.RC, sh.nch, bias, k, idx, w, logits, fz);
     return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <bool WR32>
 static cudaError_t launch_router_cluster(const RouterClusterShape &sh, const void *x, int T, int H, const void *wr,
                                          int E, const float *bias, int k, int32_t *idx, float *w, float *logits,
-                                         cudaStream_t st) {
+                                         const RouterFuse &fz, cudaStream_t st) {
     switch (sh.TT) {
-    case 1: return launch_router_cluster_t<WR32, 1>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
-    case 2: return launch_router_cluster_t<WR32, 2>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
-    case 4: return launch_router_cluster_t<WR32, 4>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
-    case 8: return launch_router_cluster_t<WR32, 8>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
-    default: return launch_router_cluster_t<WR32, 16>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
+    case 1: return launch_router_cluster_t<WR32, 1>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
+    case 2: return launch_router_cluster_t<WR32, 2>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
+    case 4: return launch_router_cluster_t<WR32, 4>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
+    case 8: return launch_router_cluster_t<WR32, 8>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
+    default: return launch_router_cluster_t<WR32, 16>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
     }
+}
+
+// The ticket counter of (device, stream): launches on one stream run in order, so
+// one counter per stream is never shared by two launches at once. Slots are
+// handed out per (device, stream) on first use; a device holds kTicketSlots of
+// them (after that many streams, slots are reused round-robin). Null if the
+// counters cannot be found, and the caller permutes in its own launch.
+static unsigned int *route_ticket(cudaStream_t st) {
+    struct Slot { int dev; cudaStream_t st; int idx; };
+    static std::mutex mu;
+    static Slot slots[64 * kTicketSlots];
+    static int nslots = 0, next_idx[64] = {};
+    static unsigned int *base[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!base[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_ticket) != cudaSuccess) return nullptr;
+        base[dev] = reinterpret_cast<unsigned int *>(p);
+    }
+    for (int i = 0; i < nslots; ++i)
+        if (slots[i].dev == dev && slots[i].st == st) return base[dev] + slots[i].idx;
+    const int idx = next_idx[dev]++ % kTicketSlots;
+    if (nslots < 64 * kTicketSlots) slots[nslots++] = Slot{dev, st, idx};
+    return base[dev] + idx;
 }
 
 moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                          int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes, int nsm,
-                         cudaStream_t st) {
+                         cudaStream_t st, const RouterFuse *fuse, int *fused) {
+    if (fused) *fused = 0;
     if (T == 0) return MOE_OK;
     RouterClusterShape sh;
     if (router_cluster_shape(T, H, E, wr_is_fp32, &sh) && (reinterpret_cast<uintptr_t>(wr) & 15) == 0) {
-        cudaError_t e = wr_is_fp32 ? launch_router_cluster<true>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st)
-                                   : launch_router_cluster<false>(sh, x, T, H, wr, E, bias, k, idx, w, logits, st);
-        return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "router_cluster launch");
+        // the permutation joins this kernel when asked for and small enough for one block
+        RouterFuse fz{};
+        if (fuse && (int64_t)T * k <= kSmallP && E <= kSmallE) {
+            fz = *fuse;
+            fz.ticket = route_ticket(st);
+        }
+        cudaError_t e = wr_is_fp32
+                            ? launch_router_cluster<true>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st)
+                            : launch_router_cluster<false>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
+        if (e != cudaSuccess) return set_cuda_error(e, "router_cluster launch");
+        if (fused) *fused = fz.ticket != nullptr;
+        return MOE_OK;
     }
     int S, slice;
     router_split(T, H, E, &S, &slice);
@@ -572,7 +639,8 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
     dim3 grid((T + kDT - 1) / kDT, (E + kDE - 1) / kDE, S);
     const int smem = (int)((2 * kDT * kXS + 2 * kDK * kWS) * sizeof(double));
     auto kfn = wr_is_fp32 ? router_dmma_kernel<true> : router_dmma_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = wr_is_fp32 ? ensure_max_smem<router_dmma_kernel<true>>(smem)
+                               : ensure_max_smem<router_dmma_kernel<false>>(smem);
     if (e != cudaSuccess) return set_cuda_error(e, "router smem attribute");
     const int wvec = (E * (wr_is_fp32 ? 4 : 2)) % 16 == 0;
     e = launch_pdl(kfn, grid, dim3(kDThreads), smem, st, reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, slice,

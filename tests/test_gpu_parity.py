@@ -263,6 +263,37 @@ def test_layer_decode_mxfp4(moe, decode_layer, T):
     _layer_check(moe, decode_layer, x)
 
 
+def test_layer_fused_routing_and_permutation(moe, decode_layer):
+    """On the block-scaled path a small batch routes and permutes in one router
+    launch (the last cluster to finish sorts the pairs by expert), so a layer
+    call is 5 kernels. CUDA-graph replays reuse one launch's arguments, the
+    ticket epoch included; each replay must give the eager result."""
+    L = decode_layer.to("cuda")
+    ex = moe.moe_prepack(moe.Experts.from_layer(L))
+    T = 64
+    x = synthetic.make_tokens(T, L.H, seed=77).cuda()
+    ws = torch.empty(moe.moe_workspace_size(T, L.H, L.I, L.E, L.k), dtype=torch.uint8, device="cuda")
+    out = torch.empty(T, L.H, dtype=torch.bfloat16, device="cuda")
+    n0 = moe.moe_kernel_launch_count()
+    ref = moe.moe_layer_forward(x, L.wr, L.k, ex, bias=L.bias, ws=ws, out=out).clone()
+    assert moe.moe_kernel_launch_count() - n0 == 5
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        moe.moe_layer_forward(x, L.wr, L.k, ex, bias=L.bias, ws=ws, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_layer_forward(x, L.wr, L.k, ex, bias=L.bias, ws=ws, out=out)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    assert moe.moe_device_error() == 0
+
+
 def test_layer_decode_mxfp4_standard_layout(moe, decode_layer):
     x = synthetic.make_tokens(64, 2048, seed=9)
     _layer_check(moe, decode_layer, x, tiled=False)
