@@ -331,7 +331,7 @@ constexpr int kTokenKernelMaxT = 256;
 
 struct RouterClusterShape {
     int TT;      // tokens per cluster tile (1, 2, 4, 8 or 16)
-    int EPP;     // expert pairs per row group, rounded up to a warp
+    int EPP;     // threads per row group: E / 4 experts each, rounded up to a warp
     int G;       // row groups per chunk (kRClThreads / EPP)
     int hs;      // rows per CTA (H / 8)
     int RC;      // rows per chunk
@@ -340,10 +340,10 @@ struct RouterClusterShape {
 };
 
 static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClusterShape *sh) {
-    if (T > kTokenKernelMaxT || H % kRCl || E % 2) return false;
+    if (T > kTokenKernelMaxT || H % kRCl || E % 4) return false;
     const int eb = wr_is_fp32 ? 4 : 2;
     if ((E * eb) % 16) return false;
-    sh->EPP = (E / 2 + 31) / 32 * 32;
+    sh->EPP = (E / 4 + 31) / 32 * 32;
     sh->G = kRClThreads / sh->EPP;
     sh->hs = H / kRCl;
     int TT = 1;
@@ -353,12 +353,12 @@ static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClus
     if (rc > sh->hs) rc = sh->hs;
     int p = 1;
     while (p * 2 <= rc) p *= 2;
-    while (p >= sh->G && (sh->hs % p || p % sh->G)) p /= 2;
-    if (p < sh->G || p < 1) return false;
+    while (p >= 4 * sh->G && (sh->hs % p || p % (4 * sh->G))) p /= 2;   // 4 rows per thread and step
+    if (p < 4 * sh->G) return false;
     sh->RC = p;
     sh->nch = sh->hs / p;
     const size_t ring = (size_t)kRClRing * p * E * eb;
-    const size_t red = (size_t)TT * sh->G * 2 * sh->EPP * sizeof(double);
+    const size_t red = (size_t)TT * sh->G * 4 * sh->EPP * sizeof(double);
     sh->smem = 64 + (ring > red ? ring : red) + (size_t)sh->hs * TT * sizeof(double);
     return sh->smem <= 200 * 1024;
 }
@@ -384,7 +384,7 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     const int hs = H / kRCl;
     const size_t chunk_bytes = (size_t)RC * E * eb;
     const size_t ring = (size_t)kRClRing * chunk_bytes;
-    const int E2 = 2 * EPP;                                        // expert slots per row group
+    const int E2 = 4 * EPP;                                        // expert slots per row group
     const size_t red_bytes = (size_t)TT * G * E2 * sizeof(double);
     uint8_t *wring = rsm + 64;
     double *red = reinterpret_cast<double *>(rsm + 64);              // aliases the ring after the loop
@@ -417,53 +417,56 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     }
     __syncthreads();
 
-    // thread (g, ep) owns experts 2 ep and 2 ep + 1 for every token of the tile over
-    // rows [g rows_g, (g + 1) rows_g) of each chunk; NA independent fp64 sums per
-    // (token, expert) keep at least 8 FMA chains in flight, added in order at the end
+    // thread (g, ep) owns experts 4 ep .. 4 ep + 3 for every token of the tile over
+    // rows [g rows_g, (g + 1) rows_g) of each chunk (a row group is whole warps, so
+    // a warp reads one row of x at a time: a broadcast). Four rows' weights are
+    // loaded before their FMAs; NA independent fp64 sums per (token, expert) keep
+    // at least 8 chains in flight, added in order at the end.
     const int ep = tid % EPP, g = tid / EPP;
-    const bool active = g < G && 2 * ep < E;
-    const int rows_g = RC / G;
-    constexpr int NA = TT >= 4 ? 1 : 4 / TT;
-    double acc[TT][2][NA];
+    const bool active = g < G && 4 * ep < E;
+    const int rows_g = RC / G;   // a multiple of 4
+    constexpr int NA = TT >= 2 ? 1 : 2;
+    double acc[TT][4][NA];
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-        for (int a = 0; a < NA; ++a) acc[tt][0][a] = acc[tt][1][a] = 0.0;
+        for (int e4 = 0; e4 < 4; ++e4)
+#pragma unroll
+            for (int a = 0; a < NA; ++a) acc[tt][e4][a] = 0.0;
     for (int c = 0; c < nch; ++c) {
         const int b = c % kRClRing;
         mbar_wait(&full[b], (uint32_t)((c / kRClRing) & 1), abort_flag);
         if (active) {
-            const uint8_t *wc = wring + b * chunk_bytes;
+            const uint8_t *wc = wring + b * chunk_bytes + (size_t)4 * ep * eb;
             const int rb = g * rows_g;
-            for (int r0 = rb; r0 < rb + rows_g; r0 += NA) {
+            for (int r0 = rb; r0 < rb + rows_g; r0 += 4) {
+                double wv[4][4];
 #pragma unroll
-                for (int a = 0; a < NA; ++a) {
-                    const int r = r0 + a;
-                    if (r < rb + rows_g) {
-                        double w0, w1;
-                        if (WR32) {
-                            const uint2 f = *reinterpret_cast<const uint2 *>(wc + ((size_t)r * E + 2 * ep) * 4);
-                            w0 = f32_bits_to_f64(f.x);
-                            w1 = f32_bits_to_f64(f.y);
-                        } else {
-                            const uint32_t bb = *reinterpret_cast<const uint32_t *>(wc + ((size_t)r * E + 2 * ep) * 2);
-                            w0 = bf16_bits_to_f64(bb & 0xFFFFu);
-                            w1 = bf16_bits_to_f64(bb >> 16);
-                        }
-                        const double *xr = xs + (size_t)(c * RC + r) * TT;
-                        if constexpr (TT == 1) {
-                            acc[0][0][a] = fma(xr[0], w0, acc[0][0][a]);
-                            acc[0][1][a] = fma(xr[0], w1, acc[0][1][a]);
-                        } else {
+                for (int i = 0; i < 4; ++i) {
+                    const uint8_t *src = wc + (size_t)(r0 + i) * E * eb;
+                    if (WR32) {
+                        const uint4 f = *reinterpret_cast<const uint4 *>(src);
+                        wv[i][0] = f32_bits_to_f64(f.x);
+                        wv[i][1] = f32_bits_to_f64(f.y);
+                        wv[i][2] = f32_bits_to_f64(f.z);
+                        wv[i][3] = f32_bits_to_f64(f.w);
+                    } else {
+                        const uint2 bb = *reinterpret_cast<const uint2 *>(src);
+                        wv[i][0] = bf16_bits_to_f64(bb.x & 0xFFFFu);
+                        wv[i][1] = bf16_bits_to_f64(bb.x >> 16);
+                        wv[i][2] = bf16_bits_to_f64(bb.y & 0xFFFFu);
+                        wv[i][3] = bf16_bits_to_f64(bb.y >> 16);
+                    }
+                }
 #pragma unroll
-                            for (int tt = 0; tt < TT; tt += 2) {
-                                const double2 xv = *reinterpret_cast<const double2 *>(xr + tt);
-                                acc[tt][0][a] = fma(xv.x, w0, acc[tt][0][a]);
-                                acc[tt][1][a] = fma(xv.x, w1, acc[tt][1][a]);
-                                acc[tt + 1][0][a] = fma(xv.y, w0, acc[tt + 1][0][a]);
-                                acc[tt + 1][1][a] = fma(xv.y, w1, acc[tt + 1][1][a]);
-                            }
-                        }
+                for (int i = 0; i < 4; ++i) {
+                    const double *xr = xs + (size_t)(c * RC + r0 + i) * TT;
+                    const int a = i % NA;
+#pragma unroll
+                    for (int tt = 0; tt < TT; ++tt) {
+                        const double xv = xr[tt];
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) acc[tt][e4][a] = fma(xv, wv[i][e4], acc[tt][e4][a]);
                     }
                 }
             }
@@ -480,11 +483,11 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
-            for (int x2 = 0; x2 < 2; ++x2) {
-                double sum = acc[tt][x2][0];
+            for (int e4 = 0; e4 < 4; ++e4) {
+                double sum = acc[tt][e4][0];
 #pragma unroll
-                for (int a = 1; a < NA; ++a) sum += acc[tt][x2][a];
-                red[((size_t)tt * G + g) * E2 + 2 * ep + x2] = sum;
+                for (int a = 1; a < NA; ++a) sum += acc[tt][e4][a];
+                red[((size_t)tt * G + g) * E2 + 4 * ep + e4] = sum;
             }
     }
     __syncthreads();
