@@ -5,7 +5,7 @@ Source: winzheng.com "FreeToken ... 753B local inference MoE", section
 high-frequency experts, with weight movement overlapped with compute); the
 aimodeling.com English page, section "Three Engineering Cores" (the same LRU
 cache plus double-buffered streaming). The pages name the policy only ("LRU");
-the rules below are this build's reading, written so that the hit/miss trace
+the rules below are the reading taken here, written so that the hit/miss trace
 and the final table are fully determined:
 
 * S slots, all free at start. A miss takes the lowest-index free slot.
