@@ -298,6 +298,9 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
 static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *x,
                                    void *y_perm, int y_is_fp32, void *h, cudaStream_t st) {
     if (n_rows == 0) return MOE_OK;
+    // prepacked MXFP4 has only the block-scaled path's blobs (use_bs always takes it)
+    if (x->fmt == MOE_MXFP4 && x->layout == MOE_LAYOUT_TILED)
+        return set_error(MOE_ERR_UNSUPPORTED, "prepacked MXFP4 runs on the block-scaled path only");
     const Strides s = default_strides(*x);
     const int nent = x->expert_map ? (int)(x->n_entries > 0 ? x->n_entries : x->E) : x->E;
     const int BN = choose_bn(n_rows, x->E);
