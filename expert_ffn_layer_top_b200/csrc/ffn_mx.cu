@@ -377,8 +377,9 @@ __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__
 struct MxSmem {
     uint64_t full[kMxMaxStages];
     uint64_t empty[kMxMaxStages];
-    uint64_t accfull[2];      // every pipeline's MMA warp commits
-    uint64_t accempty[2];     // the epilogue group of that buffer (128 threads)
+    uint64_t accfull[8];      // stage-parallel: [buffer], every pipeline's MMA warp commits;
+                              // item-parallel: [2 pipeline + buffer], that pipeline's MMA warp
+    uint64_t accempty[8];     // the epilogue group that read the buffer (128 threads)
     uint64_t mmadone[4];
     uint64_t xfull[2], xempty[2];   // gate/up exchange, per epilogue group
     uint32_t tmem_base;
@@ -450,15 +451,24 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
     volatile int *abort_flag = &sm.abort_flag;
 
     const int KST = p.K / kMxStageK;   // stages per item
-    const int PER = KST / NP;          // stages per item and pipeline
+    // Stage-parallel: pipeline w takes stages w, w + NP, ... of every item, and the
+    // epilogue adds the pipelines' accumulators. Item-parallel (p.itempar): pipeline
+    // w takes every stage of the CTA's items w, w + NP, ..., each in its own
+    // accumulators, so its MMA warp meets an item boundary once per item.
+    const bool IP = p.itempar != 0;
+    const int j0 = IP ? (warp & 3) : 0, dj = IP ? NP : 1;   // the pipeline's items (w = warp & 3)
+    const int st0 = IP ? 0 : (warp & 3), dst = IP ? 1 : NP;  // its stages of an item
+    const int PER = IP ? KST : KST / NP;                     // stages per item and pipeline
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMxMaxStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&sm.accfull[a], NP);
+        for (int a = 0; a < 8; ++a) {
+            mbar_init(&sm.accfull[a], IP ? 1 : NP);
             mbar_init(&sm.accempty[a], 128);
+        }
+        for (int a = 0; a < 2; ++a) {
             mbar_init(&sm.xfull[a], 128);
             mbar_init(&sm.xempty[a], 128);
         }
@@ -521,17 +531,17 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             // The slots start empty: the weights of this pipeline's first NSW stages go out
             // before waiting for the kernel that writes the activations.
             int pre = 0;
-            for (int item = blockIdx.x; item < total && pre < NSW; item += gridDim.x) {
+            for (int item = blockIdx.x + j0 * gridDim.x; item < total && pre < NSW; item += dj * gridDim.x) {
                 const MxItem it = mx_item(tab, p, item, BN);
-                for (int st = w; st < KST && pre < NSW; st += NP, ++pre) issue_weights(it, st, w * NSW + pre);
+                for (int st = st0; st < KST && pre < NSW; st += dst, ++pre) issue_weights(it, st, w * NSW + pre);
             }
             pdl_wait();
             if (w == 0) pdl_release();
             int loc = 0;   // stages this pipeline has issued
             bool ok = true;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            for (int item = blockIdx.x + j0 * gridDim.x; item < total && ok; item += dj * gridDim.x) {
                 const MxItem it = mx_item(tab, p, item, BN);
-                for (int st = w; st < KST; st += NP, ++loc) {
+                for (int st = st0; st < KST; st += dst, ++loc) {
                     const int s = w * NSW + loc % NSW;
                     const uint32_t round = (uint32_t)(loc / NSW);
                     if (loc >= pre) {
@@ -558,9 +568,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             int loc = 0, lt = 0, sc = 0;
             bool ok = true;
             const uint32_t base_u32 = smem_u32(base);
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
-                const int a = lt & 1;
-                if (!mbar_wait(&sm.accempty[a], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            for (int item = blockIdx.x + j0 * gridDim.x; item < total && ok; item += dj * gridDim.x, ++lt) {
+                const int a = lt & 1, bi = IP ? 2 * w + a : a;   // lt: this pipeline's items so far
+                if (!mbar_wait(&sm.accempty[bi], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)((a * NW + w) * N);
                 for (int k = 0; k < PER; ++k, ++loc) {
@@ -592,7 +602,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                     mma_commit(&sm.empty[s]);
                 }
                 if (!ok) break;
-                mma_commit(&sm.accfull[a]);
+                mma_commit(&sm.accfull[bi]);
             }
             mma_commit(&sm.mmadone[w]);
             const uint64_t t0 = globaltimer();
@@ -610,8 +620,11 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         bool ok = true;
         for (int item = blockIdx.x + grp * gridDim.x; item < total && ok; item += 2 * gridDim.x, lt += 2) {
             const MxItem it = mx_item(tab, p, item, BN);
-            const int a = grp;
-            if (!mbar_wait(&sm.accfull[a], (lt >> 1) & 1, abort_flag)) break;
+            // lt: the item's index in this CTA. Item-parallel: pipeline lt % NP, its item lt / NP.
+            const int wi = IP ? lt % NP : 0, li = IP ? lt / NP : lt;
+            const int a = li & 1, bi = IP ? 2 * wi + a : a;
+            const int wlo = IP ? wi : 0, whi = IP ? wi + 1 : NP;   // accumulators to add
+            if (!mbar_wait(&sm.accfull[bi], (li >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NW * N);
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
@@ -625,7 +638,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                 constexpr float kPw[kMxPlanes] = {1.0f, FMT == kBsNv ? 0.125f : 1.0f, FMT == kBsNv ? 0.015625f : 1.0f,
                                                   FMT == kBsNv ? 0.001953125f : 1.0f};
                 if constexpr (BN <= 8) {
-                    for (int w = 0; w < NP; ++w) {   // all N <= 32 columns of pipeline w
+                    for (int w = wlo; w < whi; ++w) {   // all N <= 32 columns of pipeline w
                         uint32_t v0[16], v1[16];
                         tmem_ld16(acc0 + w * N, v0);
                         if constexpr (N > 16) tmem_ld16(acc0 + w * N + 16, v1);
@@ -640,7 +653,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                         }
                     }
                 } else {
-                    for (int w = 0; w < NP; ++w) {
+                    for (int w = wlo; w < whi; ++w) {
                         uint32_t v[kMxPlanes][16];
 #pragma unroll
                         for (int pl = 0; pl < kMxPlanes; ++pl) tmem_ld16(acc0 + w * N + pl * BN + c0, v[pl]);
@@ -739,7 +752,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             }
             if (!ok) break;
             tc_fence_before();
-            mbar_arrive(&sm.accempty[a]);
+            mbar_arrive(&sm.accempty[bi]);
         }
     }
 
@@ -800,6 +813,8 @@ static cudaError_t mx_launch_bn(int BN, const MxParams &p, int grid, size_t smem
 // Pipelines and ring depth of one phase: as many pipelines as divide the
 // stages of an item and fit TMEM (4 for N <= 32, 2 for N = 64, else 1), with
 // at least two slots each in the shared memory of one CTA. False if none fits.
+// When that leaves one stage per item and pipeline, every stage would be an
+// item boundary for its MMA warp: the pipelines take whole items instead.
 bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl) {
     const int KST = K / kMxStageK;
     const int N = kMxPlanes * BN;
@@ -812,6 +827,7 @@ bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl) {
         if (nsw < 2) continue;
         pl->pipes = np;
         pl->stages = np * nsw;
+        pl->itempar = np > 1 && KST / np == 1;
         return true;
     }
     return false;
@@ -824,6 +840,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
         return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no pipeline plan for the block-scaled FP4 path", p.K);
     p.pipes = pl.pipes;
     p.stages = pl.stages;
+    p.itempar = pl.itempar;
     size_t smem = mx_smem_bytes(fmt, phase, BN, pl.stages, p.E);
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: it allocates all 512 TMEM columns
     const int64_t items_ub = ((int64_t)p.n_rows / BN + p.E) * p.m_tiles;

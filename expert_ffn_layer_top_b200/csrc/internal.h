@@ -59,6 +59,7 @@ struct MxParams {
     int m_tiles;                // I/64 (up) or H/128 (down)
     int stages;                 // shared-memory slots, set by the launcher
     int pipes;                  // independent producer/MMA pipelines, set by the launcher
+    int itempar;                // pipelines take whole items (else stages of every item), set by the launcher
     int n_rows;
     const uint8_t *wbase;       // this phase's prepacked tensor: [m_tiles][K/256] weight blobs
     int64_t w_estride;          // bytes between experts (or cache slots)
@@ -88,7 +89,7 @@ moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap,
 
 int choose_bn_mx(int n_rows, int E);
 struct MxPlan {
-    int pipes, stages;
+    int pipes, stages, itempar;
 };
 bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl);
 size_t mx_tiles_ub(int n_rows, int E);

@@ -202,6 +202,26 @@ def test_grouped_ffn_parity(moe, fmt, T, tiled):
     assert moe.moe_device_error() == 0
 
 
+@pytest.mark.parametrize("fmt,T", [("mxfp4", 40), ("mxfp4", 9), ("nvfp4", 40)])
+def test_grouped_ffn_item_parallel_down(moe, fmt, T):
+    """I = 768 gives the down projection 3 stages of 256 per item on 3 pipelines;
+    there the pipelines take whole items (item-parallel) and the epilogue reads
+    one pipeline's accumulators per item."""
+    cfg = dict(H=256, E=8, k=2, I=768, fmt=fmt, wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=11)
+    x = synthetic.make_tokens(T, 256, seed=11)
+    idx = _rand_idx(T, 2, 8, T)
+    off_o, sp_o, pr_o = oracle.permute(idx, 8)
+    y_o = oracle.ffn(x, L, off_o, sp_o, 2)
+    ex = moe.moe_prepack(moe.Experts.from_layer(L.to("cuda")))
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), 8, x.cuda())
+    y = moe.moe_grouped_ffn(xp, off, ex)
+    torch.cuda.synchronize()
+    err = rel_err(bf16_np(y), y_o)
+    assert err < TOL, f"down projection: error {err:.3e}"
+    assert moe.moe_device_error() == 0
+
+
 def test_grouped_ffn_fp32_output(moe):
     cfg = dict(H=256, E=8, k=2, I=256, fmt="nvfp4", wr_fp32=False)
     L = synthetic.make_layer(cfg, seed=8)
