@@ -296,10 +296,11 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
     }
 }
 
-// NVFP4 activations. One warp per permuted row r (grid-stride): the row is
-// x_perm[r] (mode 0), x[sorted_pair[r] / k] (mode 1) or src[r] (mode 2, natural
-// order). A first pass finds the row maximum 2^E and the offset C = 9 - E
-// (rowexp[r]); then every 16-block with maximum exponent e gets the E4M3 scale
+// NVFP4 activations. One block per permuted row r (grid-stride), each thread
+// 8 consecutive elements at a time: the row is x_perm[r] (mode 0),
+// x[sorted_pair[r] / k] (mode 1) or src[r] (mode 2, natural order). A first
+// pass finds the row maximum 2^E and the offset C = 9 - E (rowexp[r]); then
+// every 16-block with maximum exponent e gets the E4M3 scale
 // 2^min(8, max(-9, e - 1 + C)) for all four planes, plane p carrying the unit
 // 2^(scale exponent - 3p - C). Rows and atoms as in mx_quant_kernel.
 __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__ src, int mode,
@@ -309,31 +310,39 @@ __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
+    __shared__ uint32_t s_max[8];
     pdl_wait();
     pdl_release();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsNv, BN);
-    for (int r = blockIdx.x * 8 + warp; r < P; r += gridDim.x * 8) {
+    for (int r = blockIdx.x; r < P; r += gridDim.x) {
         const int e = expert_of_row(s_off, E, r);
         const int rel = r - s_off[e];
         const int tile = s_tile[e] + rel / BN, n = rel % BN;
         const uint4 *srow = src + (int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8;
-        // pass 1: row maximum (order does not matter)
+        // pass 1: row maximum (order does not matter): warps, then the block
         float amax = 0.0f;
-        for (int c = lane; c < K8; c += 32) {
+        for (int c = tid; c < K8; c += 256) {
             float v[8];
             bf16x8_to_float(__ldcg(srow + c), v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
         }
-        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+        const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+        if (lane == 0) s_max[warp] = wmax;
+        __syncthreads();
+        uint32_t bmax_bits = s_max[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) bmax_bits = max(bmax_bits, s_max[i]);
+        __syncthreads();   // s_max is rewritten for the next row
+        amax = __uint_as_float(bmax_bits);
         int Er = amax > 0.0f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 0;
         Er = Er < -90 ? -90 : Er;
         const int C = 9 - Er;
-        if (lane == 0) rowexp[r] = C;
-        // pass 2: planes, 8 elements per lane, 2 lanes per 16-block
-        for (int c = lane; c < K8; c += 32) {
+        if (tid == 0) rowexp[r] = C;
+        // pass 2: planes, 8 elements per thread, 2 neighbouring lanes per 16-block
+        for (int c = tid; c < K8; c += 256) {
             uint4 uv = __ldcg(srow + c);
             if (mode == 0) uv = deinterleave8(uv);
             float v[8];
@@ -863,8 +872,8 @@ moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *so
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
     cudaError_t e;
-    if (fmt == kBsNv) {   // one warp per row
-        const int blocks = (P + 7) / 8 < num_sms * 8 ? (P + 7) / 8 : num_sms * 8;
+    if (fmt == kBsNv) {   // one block per row
+        const int blocks = P < num_sms * 8 ? P : num_sms * 8;
         e = launch_pdl(nv_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
                        sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp);
     } else {              // one warp per (row, stage)
