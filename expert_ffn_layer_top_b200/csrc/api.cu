@@ -206,8 +206,9 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 }
 
 // Scratch of the grouped FFN. Decoding path: h, bf16 [n][I] at offset 0.
-// Block-scaled MXFP4 path: E4M3 hi/lo planes of the permuted activations
-// [2][n][H] and of h [2][n][I], and the scale atoms of both.
+// Block-scaled FP4 path: the activation blobs (four E2M1 planes and their scale
+// atoms) of x and of h; NVFP4 also keeps h in bf16 at offset 0 and the per-row
+// exponent offsets of x and h.
 struct FfnWs {
     size_t h, re1, re2, b1, b2, total;
 };

@@ -170,9 +170,13 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
  *   x_perm: bf16 [n_rows][H] in the interleaved layout written by moe_permute.
  *   y_perm: [n_rows][H], natural column order.
  *   ws: scratch; moe_workspace_size(n_rows, H, I, E, 1, y_is_fp32) bytes
- *   always suffice. Row-major or BF16/FP8/NVFP4 experts keep h there
- *   ([n_rows][I] bf16, operand column order); prepacked MXFP4 experts keep the
- *   E4M3 hi/lo split of x_perm and of h (bf16-exact) and their scale atoms.
+ *   always suffice. The decoding path (row-major experts, BF16, FP8, and
+ *   prepacked NVFP4 with more than 16 rows per expert on average) keeps h there
+ *   ([n_rows][I] bf16, operand column order). The block-scaled FP4 path
+ *   (prepacked MXFP4; prepacked NVFP4 up to 16 rows per expert) keeps x_perm and
+ *   h as four E2M1 planes each, within 2^-11 of each 32-block's (16-block's)
+ *   maximum, with their scale atoms; for NVFP4 also h in bf16 [n_rows][I],
+ *   natural column order, at the start of ws.
  *   Requires H % 256 == 0, I % 256 == 0, E <= 1024. n_rows == 0 is a no-op. */
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
                            void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
