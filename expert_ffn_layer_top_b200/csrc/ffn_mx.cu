@@ -421,19 +421,21 @@ __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int
     return it;
 }
 
-// Warp roles (512 threads, one CTA per SM, persistent over items). The K
-// stages of an item are dealt round-robin to NP independent pipelines: pipeline
-// w (producer warp w, MMA warp 12 + w, its own ring of slots and its own
-// accumulators) handles stages w, w + NP, ... of every item, in order. One
-// producer fills and one issuer drains each slot, both in order, so every
-// parity wait on a slot barrier is exactly one phase after the previous one.
+// Warp roles (512 threads, one CTA per SM, persistent over items). NP
+// independent pipelines: pipeline w is producer warp w, MMA warp 12 + w, its own
+// ring of slots and its own double-buffered accumulators. It handles either
+// stages w, w + NP, ... of every item (stage-parallel) or every stage of items
+// w, w + NP, ... of the CTA (item-parallel, p.itempar), in order. One producer
+// fills and one issuer drains each slot, both in order, so every parity wait on
+// a slot barrier is exactly one phase after the previous one.
 //   warps 0-3   producers: per stage one bulk copy of the weight blob and one
 //               of the activation blob. Warp 2 also builds the tile prefix.
 //   warps 12-15 MMA issuers (warp 12 owns TMEM): per stage one tcgen05.cp per
 //               scale atom, four MMAs of K = 64, one commit.
-//   warps 4-7   epilogue of even items (accumulator buffer 0);
-//   warps 8-11  epilogue of odd items (buffer 1). The epilogue adds the NP
-//               pipelines' accumulators and the four planes' columns.
+//   warps 4-7   epilogue of the CTA's even items;
+//   warps 8-11  epilogue of its odd items. The epilogue adds the accumulators
+//               of the pipelines that worked on the item (all NP, or the one
+//               owner) and the four planes' columns.
 // TMEM columns: accumulator (buffer a, pipeline w) at (a NW + w) N; from 2 NW N
 // on, 16 NA scale columns per pipeline (two rotating groups of 8 NA: the NA
 // weight atoms, then the NA activation atoms, 4 columns each).
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
     constexpr int STAGE = ABLOB + BBLOB;                    // a multiple of 1024
     constexpr uint32_t SFCOL = 2 * NW * N;
     static_assert(SFCOL + NW * 16 * NA <= 512, "TMEM columns");
-    const int NP = p.pipes;                                 // divides the stages per item, <= NW
+    const int NP = p.pipes;                                 // <= NW; stage-parallel: divides the stages per item
     const int NSW = p.stages / NP;                          // slots per pipeline
 
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
