@@ -37,39 +37,43 @@ def build(force: bool = False) -> str:
     return _SO
 
 
+def _bind(path: str):
+    """Load a build of oracle.c and declare its entry points."""
+    L = C.CDLL(path)
+    P = C.c_void_p
+    i = C.c_int
+    f = C.c_float
+    L.oracle_e2m1.restype = C.c_double
+    L.oracle_e2m1.argtypes = [i]
+    L.oracle_e8m0.restype = C.c_double
+    L.oracle_e8m0.argtypes = [i]
+    L.oracle_e4m3.restype = C.c_double
+    L.oracle_e4m3.argtypes = [i]
+    L.oracle_bf16_round.restype = C.c_double
+    L.oracle_bf16_round.argtypes = [C.c_double]
+    L.oracle_dequant.restype = i
+    L.oracle_dequant.argtypes = [i, i, i, P, P, f, P]
+    L.oracle_route.restype = None
+    L.oracle_route.argtypes = [P, i, i, P, i, P, i, i, P, P, P]
+    L.oracle_permute.restype = None
+    L.oracle_permute.argtypes = [P, i, i, i, P, P, P]
+    L.oracle_ffn.restype = i
+    L.oracle_ffn.argtypes = [P, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
+    L.oracle_combine.restype = None
+    L.oracle_combine.argtypes = [P, P, P, i, i, i, P]
+    L.oracle_layer.restype = i
+    L.oracle_layer.argtypes = [P, i, i, P, i, P, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P, P]
+    L.oracle_token_rows.restype = i
+    L.oracle_token_rows.argtypes = [P, i, i, i, i, P, P, P, P, P, P, P, P, P, i, P]
+    L.oracle_threads.restype = i
+    L.oracle_threads.argtypes = []
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = C.CDLL(_SO)
-        P = C.c_void_p
-        i = C.c_int
-        f = C.c_float
-        L.oracle_e2m1.restype = C.c_double
-        L.oracle_e2m1.argtypes = [i]
-        L.oracle_e8m0.restype = C.c_double
-        L.oracle_e8m0.argtypes = [i]
-        L.oracle_e4m3.restype = C.c_double
-        L.oracle_e4m3.argtypes = [i]
-        L.oracle_bf16_round.restype = C.c_double
-        L.oracle_bf16_round.argtypes = [C.c_double]
-        L.oracle_dequant.restype = i
-        L.oracle_dequant.argtypes = [i, i, i, P, P, f, P]
-        L.oracle_route.restype = None
-        L.oracle_route.argtypes = [P, i, i, P, i, P, i, i, P, P, P]
-        L.oracle_permute.restype = None
-        L.oracle_permute.argtypes = [P, i, i, i, P, P, P]
-        L.oracle_ffn.restype = i
-        L.oracle_ffn.argtypes = [P, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
-        L.oracle_combine.restype = None
-        L.oracle_combine.argtypes = [P, P, P, i, i, i, P]
-        L.oracle_layer.restype = i
-        L.oracle_layer.argtypes = [P, i, i, P, i, P, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P, P]
-        L.oracle_token_rows.restype = i
-        L.oracle_token_rows.argtypes = [P, i, i, i, i, P, P, P, P, P, P, P, P, P, i, P]
-        L.oracle_threads.restype = i
-        L.oracle_threads.argtypes = []
-        _lib = L
+        _lib = _bind(build())
     return _lib
 
 

@@ -304,6 +304,18 @@ def test_lru_hand_worked_trace():
         assert (s.hits, s.misses) == tuple(int(v) for v in counts.split())
 
 
+def test_lru_ids_resolved_once_in_ascending_order():
+    """Hand-worked: 4 free slots, one call asking for 5, 2, 7, 2. The ids are
+    taken once each in ascending order, so 2, 5, 7 land in slots 0, 1, 2 and
+    the call counts three misses. A second call asking for 6, 5 with slot 3
+    free: 5 hits, 6 takes slot 3."""
+    s = LruSim(4, 1, 8, 1)
+    assert s.resolve(0, [5, 2, 7, 2]) == [(2, 0), (5, 1), (7, 2)]
+    assert (s.hits, s.misses, s.loads) == (0, 3, 3)
+    assert s.resolve(0, [6, 5]) == [(6, 3)]
+    assert (s.hits, s.misses, s.loads) == (1, 4, 4)
+
+
 def test_lru_single_request_calls_equal_textbook_lru():
     """With one id per call the protection rule only shields the MRU slot,
     which textbook LRU never evicts: the two must agree exactly."""

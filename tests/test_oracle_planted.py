@@ -1,0 +1,136 @@
+"""Planted mistakes in the oracle, caught by its pins. CPU only.
+
+Each case edits one plausible error into a copy of the oracle (a wrong
+exponent bias, a swapped nibble, a dropped term, a wrong sign or index, a
+transposed operand, a broken cache rule), builds or loads that copy, and runs
+every pin of test_oracle.py against it. At least one pin must fail. The copies
+live under _build/planted; the oracle itself is never modified. Every planted
+edit keeps all memory accesses inside the buffers the pins pass in.
+"""
+import os
+import subprocess
+import sys
+import types
+
+import pytest
+
+import oracle
+import test_oracle as pins
+from conftest import ROOT
+
+_DIR = os.path.join(ROOT, "_build", "planted")
+
+# (name, exact text in oracle.c, replacement). The text must occur once.
+C_PLANTS = [
+    ("e2m1_exponent_bias", "ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)"),
+    ("e2m1_subnormal_step", "(e == 0) ? 0.5 * m", "(e == 0) ? 1.0 * m"),
+    ("e8m0_bias", "ldexp(1.0, code - 127)", "ldexp(1.0, code - 128)"),
+    ("e4m3_exponent_bias", "ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    ("e4m3_subnormal_exponent", "ldexp(m / 8.0, -6)", "ldexp(m / 8.0, -7)"),
+    ("e4m3_no_nan", "if (e == 15 && m == 7) return NAN;", ""),
+    ("fp4_nibble_order", "(c & 1) ? (byte >> 4) : (byte & 15)", "(c & 1) ? (byte & 15) : (byte >> 4)"),
+    ("mxfp4_scale_block_64", "(size_t)r * (K / 32) + c / 32]", "(size_t)r * (K / 32) + c / 64]"),
+    ("mxfp4_scale_row_dropped", "(size_t)r * (K / 32) + c / 32]", "c / 32]"),
+    ("nvfp4_tensor_scale_dropped", "v = (q * s) * tscale;", "v = q * s;"),
+    ("nvfp4_scale_block_32", "(size_t)r * (K / 16) + c / 16]", "(size_t)r * (K / 16) + c / 32]"),
+    ("fp8_scale_row_dropped", "(size_t)r * (K / 128) + c / 128]", "c / 128]"),
+    ("bf16_round_half_up", "u += 0x7fffu + lsb;", "u += 0x7fffu;"),
+    ("bf16_truncate", "u += 0x7fffu + lsb;", "u += 0;"),
+    ("router_fp32_sum", "double acc = 0.0;\n            for (int h = 0; h < H; ++h) {",
+     "float acc = 0.0f;\n            for (int h = 0; h < H; ++h) {"),
+    ("router_bias_before_rounding", "float lf = (float)acc;\n            if (bias) lf = lf + bias[e];",
+     "float lf = (float)(bias ? acc + bias[e] : acc);"),
+    ("router_weight_transposed", "((const float *)wr)[(size_t)h * E + e]", "((const float *)wr)[(size_t)e * H + h]"),
+    ("topk_ties_to_higher_index", "if (best < 0 || l[e] > l[best]) best = e;",
+     "if (best < 0 || l[e] >= l[best]) best = e;"),
+    ("topk_ascending", "if (best < 0 || l[e] > l[best]) best = e;", "if (best < 0 || l[e] < l[best]) best = e;"),
+    ("gating_sign", "w[(size_t)t * k + j] = expf(l[order[j]] - l0) / z;",
+     "w[(size_t)t * k + j] = expf(l0 - l[order[j]]) / z;"),
+    ("gating_not_normalised", "w[(size_t)t * k + j] = expf(l[order[j]] - l0) / z;",
+     "w[(size_t)t * k + j] = expf(l[order[j]] - l0);"),
+    ("permutation_descending_within_expert", "int r = offsets[e] + fill[e]++;",
+     "int r = offsets[e + 1] - 1 - fill[e]++;"),
+    ("silu_sign", "return z / (1.0f + expf(-z));", "return z / (1.0f + expf(z));"),
+    ("silu_dropped", "float hv = bf16_to_f32(f32_to_bf16(silu(g) * u));",
+     "float hv = bf16_to_f32(f32_to_bf16(g * u));"),
+    ("gate_up_swapped", "*wg = w13f + (size_t)i * H, *wu = w13f + (size_t)(I + i) * H;",
+     "*wu = w13f + (size_t)i * H, *wg = w13f + (size_t)(I + i) * H;"),
+    ("h_not_rounded_to_bf16", "float hv = bf16_to_f32(f32_to_bf16(silu(g) * u));", "float hv = silu(g) * u;"),
+    ("down_projection_transposed", "for (int i = 0; i < I; ++i) acc += hbuf[i] * w2r[i];",
+     "for (int i = 0; i < I; ++i) acc += hbuf[i] * w2f[(size_t)i * H + j];"),
+    ("token_of_row_modulo", "tok[r] = sorted_pair[offsets[e] + r] / k;", "tok[r] = sorted_pair[offsets[e] + r] % k;"),
+    ("expert_stride_of_w2_used_for_w13",
+     "\n        bad |= oracle_dequant(fmt, 2 * I, H, (const char *)w13 + e * b13,",
+     "\n        bad |= oracle_dequant(fmt, 2 * I, H, (const char *)w13 + e * b2,"),
+    ("combine_first_gate_only", "acc += w[(size_t)t * k + j] * y_perm[(size_t)r * H + c];",
+     "acc += w[(size_t)t * k] * y_perm[(size_t)r * H + c];"),
+    ("combine_skips_pair_row", "int r = pair_row[(size_t)t * k + j];", "int r = t * k + j;"),
+]
+
+# (name, exact text in lru.py, replacement).
+LRU_PLANTS = [
+    ("evicts_most_recent", "s = min(cand, key=lambda i: (self.stamp[i], i))",
+     "s = max(cand, key=lambda i: (self.stamp[i], i))"),
+    ("previous_call_unprotected", "if self.ref_call[i] < c - 1]", "if self.ref_call[i] < c]"),
+    ("highest_free_slot", "s = free[0]", "s = free[-1]"),
+    ("ids_in_request_order", "ids = sorted(set(int(i) for i in ids))", "ids = list(dict.fromkeys(int(i) for i in ids))"),
+    ("prefetch_counts_hits", "        if count:\n", "        if True:\n"),
+    ("failed_call_not_rolled_back",
+     "                        (self.owner, self.stamp, self.ref_call, self.slot_of, self.clock) = snapshot\n", ""),
+    ("hit_not_refreshed", "                hits += 1\n", "                hits += 1\n                continue\n"),
+]
+
+PARAMS = {"test_permutation_is_stable_counting_sort": [(16, 2, 8), (64, 8, 128)]}
+
+
+def _pins():
+    out = []
+    for name in sorted(dir(pins)):
+        if name.startswith("test_"):
+            fn = getattr(pins, name)
+            for args in PARAMS.get(name, [()]):
+                out.append((name, fn, args))
+    return out
+
+
+def _failing_pins():
+    failed = []
+    for name, fn, args in _pins():
+        try:
+            fn(*args)
+        except (Exception, pytest.fail.Exception):
+            failed.append(name)
+    return failed
+
+
+def _plant(text, old, new):
+    assert text.count(old) == 1, f"planting text occurs {text.count(old)} times: {old!r}"
+    return text.replace(old, new)
+
+
+def test_unplanted_oracle_passes_every_pin():
+    assert _failing_pins() == []
+
+
+@pytest.mark.parametrize("name,old,new", C_PLANTS, ids=[p[0] for p in C_PLANTS])
+def test_planted_c_mistake_is_caught(name, old, new, monkeypatch):
+    os.makedirs(_DIR, exist_ok=True)
+    src = _plant(open(oracle._SRC).read(), old, new)
+    c = os.path.join(_DIR, f"{name}.c")
+    so = os.path.join(_DIR, f"{name}.{os.getpid()}.so")
+    with open(c, "w") as f:
+        f.write(src)
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", c, "-o", so, "-lm"])
+    monkeypatch.setattr(oracle, "_lib", oracle._bind(so))
+    assert _failing_pins(), f"no pin fails with '{name}' planted"
+
+
+@pytest.mark.parametrize("name,old,new", LRU_PLANTS, ids=[p[0] for p in LRU_PLANTS])
+def test_planted_lru_mistake_is_caught(name, old, new, monkeypatch):
+    path = os.path.join(os.path.dirname(oracle.__file__), "lru.py")
+    mod = types.ModuleType(f"planted_lru_{name}")
+    exec(compile(_plant(open(path).read(), old, new), path, "exec"), mod.__dict__)
+    sys.modules.pop(mod.__name__, None)
+    monkeypatch.setattr(pins, "LruSim", mod.LruSim)
+    monkeypatch.setattr(pins, "CacheFull", mod.CacheFull)
+    assert _failing_pins(), f"no pin fails with '{name}' planted"
