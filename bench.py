@@ -440,14 +440,15 @@ def run_ours(args, rank, world, device):
                 "peak_kind": peak_kind, "layer_achieved_gbs": layer_gbs}
 
     # end to end through the C ABI with host buffers: every step copies its x in from pinned host memory and
-    # its output back to pinned host memory. As in a serving loop, the copies run on a second stream with
-    # double buffers, so step i+1's input and step i-1's output move while step i computes; the timed
-    # region ends when the last output has reached the host.
+    # its output back to pinned host memory. As in a serving loop, the copies run on two more streams (one
+    # per direction, so neither queues behind the other) with double buffers: step i+1's input and step
+    # i-1's output move while step i computes. The timed region ends when the last output has reached the
+    # host.
     xh = [x.cpu().pin_memory() for x in lb.xs]
     oh = [torch.empty(lb.T, lb.layer.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     xd = [torch.empty_like(lb.xs[0]) for _ in range(2)]
     od = [torch.empty_like(lb.out) for _ in range(2)]
-    io = torch.cuda.Stream(device)
+    h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
     cs = torch.cuda.current_stream(device)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -458,19 +459,19 @@ def run_ours(args, rank, world, device):
 
     def e2e_step(i):
         j, b = i % NSETS, i & 1
-        with torch.cuda.stream(io):
-            io.wait_event(ev_done[b])          # the layer that last read xd[b] has finished
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(ev_done[b])         # the layer that last read xd[b] has finished
             xd[b].copy_(xh[j], non_blocking=True)
-            ev_in[b].record(io)
+            ev_in[b].record(h2d)
         cs.wait_event(ev_in[b])
         cs.wait_event(ev_out[b])               # od[b]'s previous contents have reached the host
         s = lb.sets[j]
         moe.moe_layer_forward(xd[b], s.wr, lb.k, lb.experts[j], bias=s.bias, ws=lb.ws, out=od[b])
         ev_done[b].record(cs)
-        with torch.cuda.stream(io):
-            io.wait_event(ev_done[b])
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_done[b])
             oh[b].copy_(od[b], non_blocking=True)
-            ev_out[b].record(io)
+            ev_out[b].record(d2h)
 
     def e2e_steps(K: int, W: int):
         for i in range(W):
@@ -482,7 +483,7 @@ def run_ours(args, rank, world, device):
         e0.record(cs)
         for i in range(K):
             e2e_step(W + i)
-        cs.wait_stream(io)                     # the last output copy is inside the timed region
+        cs.wait_stream(d2h)                    # the last output copy is inside the timed region
         e1.record(cs)
         torch.cuda.synchronize(device)
         if barrier:
