@@ -493,7 +493,9 @@ def run_ours(args, rank, world, device):
     e2e_sec = e2e_steps(args.steps, args.warmup)
     e2e_sec = max_over_ranks(e2e_sec, world, device)
     e2e = {"value": tokens / e2e_sec, "unit": "tokens/s", "h2d_bytes_per_step": lb.T * lb.layer.H * 2,
-           "d2h_bytes_per_step": lb.T * lb.layer.H * 2}
+           "d2h_bytes_per_step": lb.T * lb.layer.H * 2,
+           "how": "eager moe_layer_forward calls; each step's H2D and D2H copies on their own streams, "
+                  "double-buffered, overlapping the layers"}
 
     # side measurements (not the headline): other batch sizes, the prefill-shaped and large layers,
     # and the streaming stack
