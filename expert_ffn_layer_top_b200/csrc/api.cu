@@ -523,6 +523,8 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     const int E = experts->E, H = experts->H, I = experts->I;
     if (T < 0) return set_error(MOE_ERR_INVALID_ARG, "T < 0");
     if (T == 0) return MOE_OK;
+    if (k < 1 || k > kMaxTopK || k > E)
+        return set_error(MOE_ERR_INVALID_ARG, "k=%d outside 1..min(%d, E=%d)", k, kMaxTopK, E);
     if (!cache) {
         moe_status r = check_experts(experts);
         if (r != MOE_OK) return r;

@@ -196,7 +196,10 @@ moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_ro
 moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           moe_stream_t stream);
 
-/* Bytes of one expert's prepacked w13 (which = 0) or w2 (which = 1). */
+/* Bytes of one expert's prepacked w13 (which = 0) or w2 (which = 1): equal to
+ * its standard layout's code and scale bytes, since prepacking only reorders
+ * bytes. Host-only; 0 for an unknown format, H or I not a positive multiple of
+ * 256, or `which` other than 0 and 1. */
 size_t moe_prepacked_expert_bytes(int fmt, int H, int I, int which);
 
 /* Rewrite a layer's experts from MOE_LAYOUT_STANDARD into MOE_LAYOUT_TILED
@@ -215,7 +218,13 @@ struct expert_cache;
  *     missing experts are streamed from the cache's pinned host pool first
  *     (one host synchronisation per call to read the miss list).
  *   idx_out, w_out: nullable copies of the routing.
- *   y_is_fp32: keep the expert outputs in fp32 before the combine. */
+ *   y_is_fp32: keep the expert outputs in fp32 before the combine.
+ * T == 0 is a no-op. Errors: INVALID_ARG for NULL experts, x, wr, out or ws,
+ * T < 0, k outside 1..min(16, E), x or wr not 16-byte aligned, or ws not
+ * 256-byte aligned; UNSUPPORTED for a shape or format outside the kernels (as
+ * for moe_grouped_ffn; the router takes E <= 256); OOM when ws_bytes is below
+ * moe_workspace_size(); CACHE_FULL when the cache cannot hold the layer's
+ * experts, with the table left unchanged. */
 moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp32, const float *bias, int k,
                              const moe_experts *experts, struct expert_cache *cache, int layer, int y_is_fp32,
                              void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
