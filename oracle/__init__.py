@@ -6,8 +6,9 @@ and shares no code with it. The arithmetic lives in ``oracle.c`` (plain C,
 fp32 with fp64 router sums); this module builds it with gcc and wraps it with
 ctypes and numpy. ``lru.py`` simulates the expert cache policy.
 
-parity unpinned against the pages: they print no layer-level values; the
-tests pin every function to closed forms, library routines and brute force.
+The pages print no layer-level values, so the tests pin every function to
+hand-worked fixtures, library routines, closed forms, invariants and brute
+force instead, and check that planted mistakes are caught.
 """
 from __future__ import annotations
 

@@ -30,9 +30,13 @@
  *   FP8   = E4M3 * fp32 (one scale per row and 128 elements along K).
  *   READING: two E2M1 codes per byte, the low nibble holds the lower K index.
  *
- * parity unpinned against the pages themselves: the pages print no layer-level
- * values. Each function is pinned by the tests to closed forms, library
- * routines and brute force instead.
+ * Pins: the pages print no layer-level values to compare against, so every
+ * function here is pinned by the tests to something other than itself: hand
+ * worked fixtures (E2M1 table, an MXFP4 row), library decoders (torch float8
+ * E4M3 / E8M0, bf16 rounding), closed forms (fp64 matmul rounded once, the
+ * softmax ratios, a dense SwiGLU MLP at k = E = 1), invariants (a stable
+ * counting sort, power-of-two scale steps) and fp64 brute force per token.
+ * Planted mistakes in a copy of this file are each caught by one of them.
  */
 #include <math.h>
 #include <stdint.h>
