@@ -316,6 +316,24 @@ def test_lru_ids_resolved_once_in_ascending_order():
     assert (s.hits, s.misses, s.loads) == (1, 4, 4)
 
 
+def test_lru_evict_hand_worked():
+    """Hand-worked: 4 slots, 2 layers of 8 experts. Freed slots are taken
+    again lowest first; evict(layer, ids) frees only those experts of that
+    layer, evict(layer) all of the layer, evict() everything."""
+    s = LruSim(4, 2, 8, 1)
+    assert s.resolve(0, [1, 2]) == [(1, 0), (2, 1)]
+    assert s.resolve(1, [3]) == [(3, 2)]
+    s.evict(0, [2])
+    assert s.table()[0 * 8 + 2] == -1 and s.table()[0 * 8 + 1] == 0 and s.table()[1 * 8 + 3] == 2
+    assert s.resolve(1, [5, 6]) == [(5, 1), (6, 3)]
+    s.evict(1)
+    assert [v for v in s.table() if v >= 0] == [0]          # only layer 0 expert 1, in slot 0
+    assert s.resolve(0, [7]) == [(7, 1)]
+    s.evict()
+    assert all(v == -1 for v in s.table())
+    assert s.resolve(1, [0]) == [(0, 0)]
+
+
 def test_lru_single_request_calls_equal_textbook_lru():
     """With one id per call the protection rule only shields the MRU slot,
     which textbook LRU never evicts: the two must agree exactly."""

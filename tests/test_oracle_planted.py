@@ -78,6 +78,8 @@ LRU_PLANTS = [
     ("failed_call_not_rolled_back",
      "                        (self.owner, self.stamp, self.ref_call, self.slot_of, self.clock) = snapshot\n", ""),
     ("hit_not_refreshed", "                hits += 1\n", "                hits += 1\n                continue\n"),
+    ("evict_ignores_layer", "            if layer >= 0 and o[0] != layer:\n                continue\n", ""),
+    ("evict_ignores_ids", "            if ids is not None and o[1] not in set(ids):\n                continue\n", ""),
 ]
 
 PARAMS = {"test_permutation_is_stable_counting_sort": [(16, 2, 8), (64, 8, 128)]}
