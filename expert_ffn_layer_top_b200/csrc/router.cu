@@ -608,8 +608,12 @@ static unsigned int *route_ticket(cudaStream_t st) {
     }
     for (int i = 0; i < nslots; ++i)
         if (slots[i].dev == dev && slots[i].st == st) return base[dev] + slots[i].idx;
-    const int idx = next_idx[dev]++ % kTicketSlots;
-    if (nslots < 64 * kTicketSlots) slots[nslots++] = Slot{dev, st, idx};
+    // Every stream keeps its own counter: two streams sharing one could interleave
+    // their tickets. Past kTicketSlots streams on a device, calls take the unfused
+    // path (a separate permutation launch).
+    if (next_idx[dev] >= kTicketSlots) return nullptr;
+    const int idx = next_idx[dev]++;
+    slots[nslots++] = Slot{dev, st, idx};
     return base[dev] + idx;
 }
 
