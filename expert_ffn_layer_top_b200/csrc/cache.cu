@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "lru_table.cuh"
 
 struct expert_cache {
     int device = 0, n_layers = 0, E = 0, H = 0, I = 0, fmt = 0, layout = 0;
@@ -61,101 +62,6 @@ struct expert_cache {
 
 namespace moe {
 
-enum { ST_HEAD = 0, ST_TAIL, ST_CALLS, ST_FREE, ST_HINT, ST_LASTN, ST_N };
-constexpr int kNone = -1;
-constexpr int kNeverRef = -(1 << 30);
-
-struct LruTable {
-    int32_t *slot_of, *owner, *prev, *next, *ref;
-    uint32_t *freeb, *last;
-    int32_t *st;
-    unsigned long long *counts;
-    int S, E, L;
-};
-
-__device__ void lru_unlink(LruTable &t, int s) {
-    const int p = t.prev[s], n = t.next[s];
-    if (p != kNone) t.next[p] = n; else t.st[ST_HEAD] = n;
-    if (n != kNone) t.prev[n] = p; else t.st[ST_TAIL] = p;
-    t.prev[s] = t.next[s] = kNone;
-}
-
-__device__ void lru_append(LruTable &t, int s) {
-    const int tl = t.st[ST_TAIL];
-    t.prev[s] = tl;
-    t.next[s] = kNone;
-    if (tl != kNone) t.next[tl] = s; else t.st[ST_HEAD] = s;
-    t.st[ST_TAIL] = s;
-}
-
-__device__ int lru_pop_free(LruTable &t) {
-    const int words = (t.S + 31) / 32;
-    for (int w = t.st[ST_HINT]; w < words; ++w) {
-        const uint32_t v = t.freeb[w];
-        if (v) {
-            const int b = __ffs(v) - 1;
-            t.freeb[w] = v & ~(1u << b);
-            t.st[ST_HINT] = w;
-            t.st[ST_FREE] -= 1;
-            return w * 32 + b;
-        }
-    }
-    return kNone;
-}
-
-// One call (resolve or prefetch) of `layer` with the request bitmap `req`.
-// Writes (e, slot) loads to out[0..2n). Returns the number of loads, or -1 (cache full).
-__device__ int lru_call(LruTable &t, int layer, const uint32_t *req, bool counted, int32_t *out) {
-    const int c = t.st[ST_CALLS];
-    const int words = (t.E + 31) / 32;
-    int misses = 0, newprot = 0;
-    for (int w = 0; w < words; ++w)
-        for (uint32_t v = req[w]; v; v &= v - 1) {
-            const int e = w * 32 + __ffs(v) - 1;
-            const int s = t.slot_of[layer * t.E + e];
-            if (s < 0) ++misses;
-            else if (t.ref[s] < c - 1) ++newprot;
-        }
-    const int occupied = t.S - t.st[ST_FREE];
-    const int evictable = occupied - t.st[ST_LASTN] - newprot;
-    if (misses > t.st[ST_FREE] + evictable) return -1;
-    int nl = 0, nref = 0, hits = 0;
-    for (int w = 0; w < words; ++w)
-        for (uint32_t v = req[w]; v; v &= v - 1) {
-            const int e = w * 32 + __ffs(v) - 1;
-            const int key = layer * t.E + e;
-            int s = t.slot_of[key];
-            if (s >= 0) {
-                ++hits;
-                lru_unlink(t, s);
-            } else {
-                s = lru_pop_free(t);
-                if (s == kNone) {
-                    s = t.st[ST_HEAD];
-                    while (s != kNone && t.ref[s] >= c - 1) s = t.next[s];
-                    if (s == kNone) { flag_error(2); return -1; }   // excluded by the count above
-                    lru_unlink(t, s);
-                    t.slot_of[t.owner[s]] = kNone;
-                }
-                t.owner[s] = key;
-                t.slot_of[key] = s;
-                out[2 * nl] = e;
-                out[2 * nl + 1] = s;
-                ++nl;
-            }
-            lru_append(t, s);
-            t.ref[s] = c;
-            ++nref;
-        }
-    t.st[ST_CALLS] = c + 1;
-    t.st[ST_LASTN] = nref;
-    if (counted) {
-        t.counts[0] += hits;
-        t.counts[1] += nl;
-    }
-    return nl;
-}
-
 // mode 0: resolve `layer` from idx[P] (+ prefetch layer+1's prediction if prefetch_next)
 // mode 1: prefetch `layer` with the explicit ids in io (count io[0], ids io[1..])
 // Output in io: [0] status (0 ok, 6 cache full), [1] n resolve loads, [2] n prefetch loads
@@ -183,77 +89,14 @@ __global__ void __launch_bounds__(32) lru_kernel(LruTable t, int layer, const in
     }
     __syncwarp();
     if (lane != 0) return;
-    int32_t *pairs = io + 3;
-    const int na = lru_call(t, layer, req, mode == 0, pairs);
-    if (na < 0) {
-        io[0] = MOE_ERR_CACHE_FULL;
-        io[1] = 0;
-        io[2] = -1;
-        return;
-    }
-    io[0] = 0;
-    io[1] = na;
-    io[2] = -1;
-    if (mode == 0) {
-        for (int w = 0; w < words; ++w) t.last[layer * words + w] = req[w];
-        if (prefetch_next && layer + 1 < t.L) {
-            const int nb = lru_call(t, layer + 1, t.last + (layer + 1) * words, false, pairs + 2 * na);
-            io[2] = nb;   // -1 when the prediction does not fit: skipped, not an error
-        }
-    }
+    lru_run(t, layer, req, mode, prefetch_next, io);
 }
 
-__global__ void lru_init_kernel(LruTable t) {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < t.L * t.E) t.slot_of[i] = kNone;
-    if (i < t.S) {
-        t.owner[i] = kNone;
-        t.prev[i] = t.next[i] = kNone;
-        t.ref[i] = kNeverRef;
-    }
-    const int words = (t.S + 31) / 32;
-    if (i < words) {
-        const int rem = t.S - i * 32;
-        t.freeb[i] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-    }
-    const int lw = (t.E + 31) / 32;
-    if (i < t.L * lw) t.last[i] = 0;
-    if (i == 0) {
-        t.st[ST_HEAD] = t.st[ST_TAIL] = kNone;
-        t.st[ST_CALLS] = 0;
-        t.st[ST_FREE] = t.S;
-        t.st[ST_HINT] = 0;
-        t.st[ST_LASTN] = 0;
-        t.counts[0] = t.counts[1] = 0;
-    }
-}
+__global__ void lru_init_kernel(LruTable t) { lru_init_one(t, blockIdx.x * blockDim.x + threadIdx.x); }
 
-// Free slots matching (layer, ids). ids in io[1..io[0]] (io[0] = -1: all of the layer).
+// Free slots matching (layer, ids) (see lru_evict).
 __global__ void lru_evict_kernel(LruTable t, int layer, const int32_t *io) {
-    if (threadIdx.x != 0) return;
-    const int n = io[0];
-    for (int s = 0; s < t.S; ++s) {
-        const int key = t.owner[s];
-        if (key < 0) continue;
-        const int l = key / t.E, e = key % t.E;
-        if (layer >= 0 && l != layer) continue;
-        if (layer >= 0 && n >= 0) {
-            bool m = false;
-            for (int i = 0; i < n; ++i) m |= io[1 + i] == e;
-            if (!m) continue;
-        }
-        lru_unlink(t, s);
-        t.slot_of[key] = kNone;
-        t.owner[s] = kNone;
-        t.ref[s] = kNeverRef;
-        t.freeb[s >> 5] |= 1u << (s & 31);
-        t.st[ST_FREE] += 1;
-        if ((s >> 5) < t.st[ST_HINT]) t.st[ST_HINT] = s >> 5;
-    }
-    int nref = 0;
-    const int c = t.st[ST_CALLS];
-    for (int s = 0; s < t.S; ++s) nref += t.ref[s] == c - 1;
-    t.st[ST_LASTN] = nref;
+    if (threadIdx.x == 0) lru_evict(t, layer, io);
 }
 
 static LruTable table_of(expert_cache *c) {
