@@ -224,7 +224,8 @@ moe_status expert_cache_init(struct expert_cache **out, size_t capacity_bytes, i
     if (!out || !host_layers || n_layers <= 0) return set_error(MOE_ERR_INVALID_ARG, "bad cache arguments");
     *out = nullptr;
     const moe_experts &l0 = host_layers[0];
-    if (l0.fmt < MOE_BF16 || l0.fmt > MOE_NVFP4 || l0.E <= 0 || l0.E > kMaxExperts || l0.H % 256 || l0.I % 256)
+    if (l0.fmt < MOE_BF16 || l0.fmt > MOE_NVFP4 || l0.E <= 0 || l0.E > kMaxExperts || l0.H <= 0 || l0.I <= 0 ||
+        l0.H % 256 || l0.I % 256)
         return set_error(MOE_ERR_UNSUPPORTED, "unsupported layer shape for the cache");
     for (int l = 1; l < n_layers; ++l) {
         const moe_experts &x = host_layers[l];
@@ -263,8 +264,9 @@ moe_status expert_cache_init(struct expert_cache **out, size_t capacity_bytes, i
     c->slot_bytes = o;
     const size_t S = capacity_bytes / c->slot_bytes;
     if (S < 1) {
+        const size_t need = c->slot_bytes;
         delete c;
-        return set_error(MOE_ERR_CACHE_FULL, "capacity below one expert (%zu bytes)", c->slot_bytes);
+        return set_error(MOE_ERR_CACHE_FULL, "capacity below one expert (%zu bytes)", need);
     }
     c->n_slots = (int)S;
     const int L = n_layers, E = c->E, lw = (E + 31) / 32;

@@ -74,16 +74,21 @@ typedef enum {
 typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3 } moe_wfmt;
 
 /* Memory layout of the expert codes. STANDARD: row-major as described above.
- * TILED: produced by moe_prepack; for every (M tile, 128-wide K stage) one
- * contiguous blob holding the tile's 128 weight rows. BF16/FP8/NVFP4: codes
- * 16-byte chunk-major, then the rows' scales for that stage (one bulk copy per
- * stage). MXFP4: one 17 KiB blob per (M tile, 256-wide K stage): the tile's
- * 128 rows of packed codes, 128 bytes per row in natural K order with the
- * 16-byte chunk c of row r at r*128 + (c XOR (r%8))*16, then two 512-byte
- * scale atoms (the stage's 128-wide halves) with the scale of row r and
- * 32-block j at byte (r%32)*16 + (r/32)*4 + j; this layout runs the
- * block-scaled FP4 tensor-core path. The values are the same; only the byte
- * order differs. */
+ * TILED: produced by moe_prepack. The values are the same and so is the byte
+ * count (codes plus scales); only the byte order differs. Weight rows form M
+ * tiles of 128 (w13: 64 gate rows and the 64 matching up rows; w2: 128
+ * consecutive rows), and every (M tile, K stage) is one contiguous blob, so
+ * one bulk copy moves a stage. Blobs are ordered by M tile, then stage.
+ *   BF16, FP8 (stages 128 wide): the codes as 16-byte chunks, chunk c of row r
+ *     at (c*128 + r)*16, then each row's scales for the stage (FP8: one fp32).
+ *   MXFP4, NVFP4 (stages 256 wide): 128 rows of packed codes, 128 bytes per
+ *     row in natural K order, the 16-byte chunk c of row r at
+ *     r*128 + (c XOR (r%8))*16; then 512-byte scale atoms, the scale of row r
+ *     and block j of the atom's K range at byte (r%32)*16 + (r/32)*4 + j.
+ *     MXFP4: two atoms (E8M0 per 32, one per 128-wide half), 17 KiB per blob.
+ *     NVFP4: four atoms (E4M3 per 16, one per 64-wide quarter), 18 KiB.
+ * Prepacked MXFP4 runs the block-scaled FP4 tensor-core path; prepacked NVFP4
+ * runs it for up to 16 rows per expert on average, else the decoding path. */
 typedef enum { MOE_LAYOUT_STANDARD = 0, MOE_LAYOUT_TILED = 1 } moe_layout;
 
 /* The experts of one layer.
@@ -124,7 +129,9 @@ typedef struct {
  *   w: fp32 [T][k], softmax over the k selected logits. logits: nullable fp32 [T][E].
  *   ws: scratch of moe_workspace_size(T, H, ...) bytes (fp64 partial sums).
  *   Requires 1 <= k <= 16, k <= E <= 256, H % 8 == 0, x and wr 16-byte aligned.
- *   T == 0 is a no-op. */
+ *   T == 0 is a no-op. Errors: INVALID_ARG for T < 0, H not a positive multiple
+ *   of 8, NULL x, wr, idx, w or ws, or x or wr misaligned; UNSUPPORTED for k or
+ *   E outside the limits; OOM when ws_bytes is below what the call needs. */
 moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                           int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes,
                           moe_stream_t stream);
@@ -136,7 +143,11 @@ moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is
  *   x_perm (nullable): bf16 [T*k][H], row r = x[sorted_pair[r] / k], with the
  *     columns of every aligned group of 8 stored in the order 0,4,1,5,2,6,3,7
  *     (the operand layout of moe_grouped_ffn).
- *   Bit-exact and deterministic. Requires H % 8 == 0. */
+ *   Bit-exact and deterministic. Requires H % 8 == 0.
+ *   Errors: INVALID_ARG for T < 0, k outside 1..16, E outside 1..1024, NULL
+ *   offsets, NULL idx, sorted_pair, pair_row or ws when T > 0, x_perm without x,
+ *   H not a positive multiple of 8 or x or x_perm not 16-byte aligned when x_perm
+ *   is given; OOM when ws_bytes is below what the call needs. */
 moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
                        int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
@@ -177,13 +188,19 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
  *   h as four E2M1 planes each, within 2^-11 of each 32-block's (16-block's)
  *   maximum, with their scale atoms; for NVFP4 also h in bf16 [n_rows][I],
  *   natural column order, at the start of ws.
- *   Requires H % 256 == 0, I % 256 == 0, E <= 1024. n_rows == 0 is a no-op. */
+ *   Requires H % 256 == 0, I % 256 == 0, E <= 1024. n_rows == 0 is a no-op.
+ *   Errors: UNSUPPORTED for an unknown format, E outside 1..1024, or H or I not
+ *   positive multiples of 256; INVALID_ARG for NULL pointers, an unknown layout,
+ *   missing scale planes or NVFP4 tensor scales, arrays or strides not 16-byte
+ *   aligned, or n_rows < 0; OOM when ws_bytes is below what the call needs. */
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
                            void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Gate-weighted combine: out[t] = sum_{j<k} w[t,j] * y_perm[pair_row[t*k+j]],
  * accumulated in fp32 in order of j, rounded to bf16.
- *   y_perm: [T*k][H] bf16 or fp32 (y_is_fp32); out: bf16 [T][H]. H % 8 == 0. */
+ *   y_perm: [T*k][H] bf16 or fp32 (y_is_fp32); out: bf16 [T][H]. H % 8 == 0.
+ *   T == 0 is a no-op. Errors: INVALID_ARG for T < 0, k outside 1..16, H not a
+ *   positive multiple of 8, NULL pointers, or y_perm or out not 16-byte aligned. */
 moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
                        int H, void *out, moe_stream_t stream);
 
@@ -192,7 +209,10 @@ moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_ro
  * applies to its weight tiles. Exact for BF16 and MXFP4 (within bf16 range);
  * NVFP4 ((E2M1 * E4M3) * tscale) and FP8 (E4M3 * fp32 scale) are rounded to
  * bf16. w/scale as in moe_experts for a single expert; tscale: host value
- * (NVFP4 only). K must be a multiple of the format's block (128/32/16/8). */
+ * (NVFP4 only). K must be a multiple of the format's block (128/32/16/8).
+ * rows == 0 is a no-op. Errors: UNSUPPORTED for an unknown format; INVALID_ARG
+ * for rows < 0, K not a positive multiple of the block, NULL pointers (scale
+ * may be NULL for BF16), or w or out not 16-byte aligned. */
 moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           moe_stream_t stream);
 
@@ -207,7 +227,9 @@ size_t moe_prepacked_expert_bytes(int fmt, int H, int I, int which);
  *   in: standard-layout experts (device pointers; expert_map must be NULL).
  *   out_w13, out_w2: device buffers of E * moe_prepacked_expert_bytes(...) bytes,
  *   16-byte aligned. The result is used through a moe_experts with
- *   layout = MOE_LAYOUT_TILED, w13 = out_w13, w2 = out_w2 (tscales unchanged). */
+ *   layout = MOE_LAYOUT_TILED, w13 = out_w13, w2 = out_w2 (tscales unchanged).
+ *   Errors: those of moe_grouped_ffn's expert checks; INVALID_ARG for a tiled
+ *   input, an expert_map, or NULL or misaligned outputs. */
 moe_status moe_prepack(const moe_experts *in, void *out_w13, void *out_w2, moe_stream_t stream);
 
 struct expert_cache;
@@ -249,18 +271,25 @@ size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32);
 /* host_layers: host array [n_layers] of layer descriptions whose code/scale
  * pointers are host pointers into page-locked (pinned) memory; all layers
  * share fmt, E, H, I. The library allocates the slot pool, the table, a copy
- * stream and events on `device`. The library keeps the pointers, not copies. */
+ * stream and events on `device`. The library keeps the pointers, not copies.
+ * Errors: INVALID_ARG for NULL arguments, n_layers <= 0, or layers that differ
+ * in format, shape or layout; UNSUPPORTED for a shape the grouped FFN rejects;
+ * CACHE_FULL when capacity_bytes holds less than one expert; OOM or CUDA when
+ * an allocation or copy fails. */
 moe_status expert_cache_init(struct expert_cache **cache, size_t capacity_bytes, int n_layers,
                              const moe_experts *host_layers, int device);
 
 /* Load the listed experts of `layer` (host array ids[n]) ahead of use, on the
  * copy stream, without counting hits or misses. Synchronises with `stream`
- * once to read back the loads the table update decided. */
+ * once to read back the loads the table update decided. n == 0 is a no-op.
+ * Errors: INVALID_ARG for a bad layer, n outside 0..E or NULL ids; CACHE_FULL
+ * when the experts do not fit, with the table left unchanged. */
 moe_status expert_cache_prefetch(struct expert_cache *cache, int layer, const int32_t *ids, int n,
                                  moe_stream_t stream);
 
 /* Free slots: layer -1 = every slot; n -1 = all experts of `layer`; else the
- * n listed experts (host array). Synchronous. */
+ * n listed experts (host array). Synchronous. Errors: INVALID_ARG for a layer
+ * outside -1..n_layers-1, n > E, or NULL ids with n > 0. */
 moe_status expert_cache_evict(struct expert_cache *cache, int layer, const int32_t *ids, int n);
 
 /* Counters since init: hits and misses of layer-forward calls, bytes copied

@@ -8,6 +8,8 @@ library's host-side checks, so no kernel is launched. The module runs only
 where no CUDA device is visible, so that even a missing check could not reach
 a device with those pointers; on a GPU the parity suite has its own
 bad-argument test through real tensors."""
+import ctypes
+
 import pytest
 import torch
 
@@ -106,6 +108,33 @@ def test_layer_forward_checks():
     assert f(exw, ptr=fake, ws_bytes=256) == OOM
     need = moe.moe_workspace_size(4, 256, 512, 8, 2)
     assert f"< {need}" in _err()
+
+
+def test_cache_init_checks_the_layers_first():
+    L = moe.lib()
+    h = ctypes.c_void_p()
+
+    def init(layers, cap=1 << 30, out=True):
+        arr = (_Experts * max(len(layers), 1))(*layers)
+        return L.expert_cache_init(ctypes.byref(h) if out else None, cap, len(layers), arr, 0)
+
+    assert init([_experts()], out=False) == INVALID_ARG
+    assert init([]) == INVALID_ARG
+    for bad in (_experts(H=0), _experts(I=0), _experts(H=-256), _experts(H=200), _experts(E=0), _experts(E=1025),
+                _experts(fmt=7)):
+        assert init([bad]) == UNSUPPORTED
+    assert init([_experts(), _experts(I=256)]) == INVALID_ARG      # layers differ in shape
+    assert init([_experts(), _experts(fmt="fp8")]) == INVALID_ARG  # ... in format
+    assert not h.value                                              # nothing was created
+
+
+def test_cache_calls_reject_a_null_cache():
+    L = moe.lib()
+    assert L.expert_cache_prefetch(None, 0, None, 0, None) == INVALID_ARG
+    assert L.expert_cache_evict(None, -1, None, -1) == INVALID_ARG
+    assert L.expert_cache_stats(None, None, None, None, None) == INVALID_ARG
+    assert L.expert_cache_slot_of(None, 0, 0, None) == INVALID_ARG
+    assert L.expert_cache_destroy(None) == OK
 
 
 def test_workspace_size_is_monotone_and_rejects_bad_sizes():
