@@ -118,6 +118,9 @@ moe_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const voi
 
 // ------------------------------------------------------------------ helpers
 
+// True when p (possibly NULL) is not a multiple of `align` bytes.
+static bool misaligned(const void *p, uintptr_t align) { return (reinterpret_cast<uintptr_t>(p) & (align - 1)) != 0; }
+
 static int elem_bytes_x2(int fmt) {   // bytes per element, times 2
     return fmt == MOE_BF16 ? 4 : fmt == MOE_FP8_E4M3_K128 ? 2 : 1;
 }
@@ -161,6 +164,8 @@ static moe_status check_experts(const moe_experts *x) {
     if (x->layout == MOE_LAYOUT_STANDARD)
         a |= reinterpret_cast<uintptr_t>(x->w13_scale) | reinterpret_cast<uintptr_t>(x->w2_scale);
     if (a & 15) return set_error(MOE_ERR_INVALID_ARG, "expert arrays not 16-byte aligned");
+    if (misaligned(x->w13_tscale, 4) || misaligned(x->w2_tscale, 4) || misaligned(x->expert_map, 4))
+        return set_error(MOE_ERR_INVALID_ARG, "tensor scales and expert_map must be 4-byte aligned");
     return MOE_OK;
 }
 
@@ -422,6 +427,8 @@ moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is
     if (!x || !wr || !idx || !w || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(wr)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "x and wr must be 16-byte aligned");
+    if (misaligned(idx, 4) || misaligned(w, 4) || misaligned(logits, 4) || misaligned(bias, 4) || misaligned(ws, 16))
+        return set_error(MOE_ERR_INVALID_ARG, "idx, w, logits and bias must be 4-byte aligned, ws 16-byte aligned");
     return launch_router(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, logits, ws, ws_bytes,
                          num_sms(current_device()), (cudaStream_t)stream);
 }
@@ -437,6 +444,9 @@ moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, i
     if (x_perm && (H <= 0 || H % 8)) return set_error(MOE_ERR_INVALID_ARG, "H must be a positive multiple of 8");
     if (x_perm && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(x_perm)) & 15))
         return set_error(MOE_ERR_INVALID_ARG, "x and x_perm must be 16-byte aligned");
+    if (misaligned(idx, 4) || misaligned(offsets, 4) || misaligned(sorted_pair, 4) || misaligned(pair_row, 4) ||
+        misaligned(ws, 16))
+        return set_error(MOE_ERR_INVALID_ARG, "int32 arrays must be 4-byte aligned, ws 16-byte aligned");
     return launch_permute(idx, T, k, E, x, H, offsets, sorted_pair, pair_row, x_perm, ws, ws_bytes,
                           (cudaStream_t)stream);
 }
@@ -468,6 +478,8 @@ moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offset
     if (ws_bytes < need) return set_error(MOE_ERR_OOM, "FFN workspace too small (%zu < %zu)", ws_bytes, need);
     if ((reinterpret_cast<uintptr_t>(x_perm) | reinterpret_cast<uintptr_t>(ws)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "x_perm and ws must be 16-byte aligned");
+    if (misaligned(y_perm, 16) || misaligned(offsets, 4))
+        return set_error(MOE_ERR_INVALID_ARG, "y_perm must be 16-byte aligned, offsets 4-byte aligned");
     if (is_mx(*experts, n_rows))
         return mx_ffn_impl(x_perm, 0, nullptr, 1, n_rows, offsets, experts, y_perm, y_is_fp32, ws,
                            (cudaStream_t)stream);
@@ -481,6 +493,8 @@ moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscal
     if (rows < 0 || K <= 0 || K % kq) return set_error(MOE_ERR_INVALID_ARG, "K=%d must be a multiple of %d", K, kq);
     if (rows == 0) return MOE_OK;
     if (!w || !out || (fmt != MOE_BF16 && !scale)) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (fmt == MOE_FP8_E4M3_K128 && misaligned(scale, 4))
+        return set_error(MOE_ERR_INVALID_ARG, "FP8 scales must be 4-byte aligned");
     if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(out)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "w and out must be 16-byte aligned");
     return launch_dequant(fmt, w, scale, tscale, rows, K, out, (cudaStream_t)stream);
@@ -512,6 +526,8 @@ moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_ro
     if (!y_perm || !pair_row || !w || !out) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
     if ((reinterpret_cast<uintptr_t>(y_perm) | reinterpret_cast<uintptr_t>(out)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "y_perm and out must be 16-byte aligned");
+    if (misaligned(pair_row, 4) || misaligned(w, 4))
+        return set_error(MOE_ERR_INVALID_ARG, "pair_row and w must be 4-byte aligned");
     return launch_combine(y_perm, y_is_fp32, pair_row, w, T, k, H, out, (cudaStream_t)stream);
 }
 
@@ -532,6 +548,8 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
         return set_error(MOE_ERR_UNSUPPORTED, "bad layer shape");
     }
     if (!x || !wr || !out || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (misaligned(bias, 4) || misaligned(idx_out, 4) || misaligned(w_out, 4) || misaligned(out, 16))
+        return set_error(MOE_ERR_INVALID_ARG, "bias, idx_out and w_out must be 4-byte aligned, out 16-byte aligned");
     const LayerWs L = layer_ws(T, H, I, E, k, y_is_fp32);
     if (ws_bytes < L.total) return set_error(MOE_ERR_OOM, "workspace %zu < %zu bytes", ws_bytes, L.total);
     if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOE_ERR_INVALID_ARG, "ws must be 256-byte aligned");

@@ -130,8 +130,9 @@ typedef struct {
  *   ws: scratch of moe_workspace_size(T, H, ...) bytes (fp64 partial sums).
  *   Requires 1 <= k <= 16, k <= E <= 256, H % 8 == 0, x and wr 16-byte aligned.
  *   T == 0 is a no-op. Errors: INVALID_ARG for T < 0, H not a positive multiple
- *   of 8, NULL x, wr, idx, w or ws, or x or wr misaligned; UNSUPPORTED for k or
- *   E outside the limits; OOM when ws_bytes is below what the call needs. */
+ *   of 8, NULL x, wr, idx, w or ws, x, wr or ws not 16-byte aligned, or idx, w,
+ *   logits or bias not 4-byte aligned; UNSUPPORTED for k or E outside the
+ *   limits; OOM when ws_bytes is below what the call needs. */
 moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                           int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes,
                           moe_stream_t stream);
@@ -147,7 +148,8 @@ moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is
  *   Errors: INVALID_ARG for T < 0, k outside 1..16, E outside 1..1024, NULL
  *   offsets, NULL idx, sorted_pair, pair_row or ws when T > 0, x_perm without x,
  *   H not a positive multiple of 8 or x or x_perm not 16-byte aligned when x_perm
- *   is given; OOM when ws_bytes is below what the call needs. */
+ *   is given, int32 arrays not 4-byte aligned, or ws not 16-byte aligned; OOM
+ *   when ws_bytes is below what the call needs. */
 moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
                        int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
@@ -191,8 +193,10 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
  *   Requires H % 256 == 0, I % 256 == 0, E <= 1024. n_rows == 0 is a no-op.
  *   Errors: UNSUPPORTED for an unknown format, E outside 1..1024, or H or I not
  *   positive multiples of 256; INVALID_ARG for NULL pointers, an unknown layout,
- *   missing scale planes or NVFP4 tensor scales, arrays or strides not 16-byte
- *   aligned, or n_rows < 0; OOM when ws_bytes is below what the call needs. */
+ *   missing scale planes or NVFP4 tensor scales, codes, scales, strides, x_perm,
+ *   y_perm or ws not 16-byte aligned, tensor scales, expert_map or offsets not
+ *   4-byte aligned, or n_rows < 0; OOM when ws_bytes is below what the call
+ *   needs. */
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
                            void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -200,7 +204,8 @@ moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offset
  * accumulated in fp32 in order of j, rounded to bf16.
  *   y_perm: [T*k][H] bf16 or fp32 (y_is_fp32); out: bf16 [T][H]. H % 8 == 0.
  *   T == 0 is a no-op. Errors: INVALID_ARG for T < 0, k outside 1..16, H not a
- *   positive multiple of 8, NULL pointers, or y_perm or out not 16-byte aligned. */
+ *   positive multiple of 8, NULL pointers, y_perm or out not 16-byte aligned, or
+ *   pair_row or w not 4-byte aligned. */
 moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
                        int H, void *out, moe_stream_t stream);
 
@@ -212,7 +217,8 @@ moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_ro
  * (NVFP4 only). K must be a multiple of the format's block (128/32/16/8).
  * rows == 0 is a no-op. Errors: UNSUPPORTED for an unknown format; INVALID_ARG
  * for rows < 0, K not a positive multiple of the block, NULL pointers (scale
- * may be NULL for BF16), or w or out not 16-byte aligned. */
+ * may be NULL for BF16), w or out not 16-byte aligned, or FP8 scales not
+ * 4-byte aligned. */
 moe_status moe_dequantize(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           moe_stream_t stream);
 
@@ -242,8 +248,8 @@ struct expert_cache;
  *   idx_out, w_out: nullable copies of the routing.
  *   y_is_fp32: keep the expert outputs in fp32 before the combine.
  * T == 0 is a no-op. Errors: INVALID_ARG for NULL experts, x, wr, out or ws,
- * T < 0, k outside 1..min(16, E), x or wr not 16-byte aligned, or ws not
- * 256-byte aligned; UNSUPPORTED for a shape or format outside the kernels (as
+ * T < 0, k outside 1..min(16, E), x, wr or out not 16-byte aligned, bias,
+ * idx_out or w_out not 4-byte aligned, or ws not 256-byte aligned; UNSUPPORTED for a shape or format outside the kernels (as
  * for moe_grouped_ffn; the router takes E <= 256); OOM when ws_bytes is below
  * moe_workspace_size(); CACHE_FULL when the cache cannot hold the layer's
  * experts, with the table left unchanged. */

@@ -110,6 +110,34 @@ def test_layer_forward_checks():
     assert f"< {need}" in _err()
 
 
+def test_misaligned_arrays_are_rejected():
+    """Non-NULL but misaligned pointers (never dereferenced: the checks return first)."""
+    L = moe.lib()
+    A = 1 << 24                 # 256-byte aligned
+    odd2, odd8 = A + 2, A + 8   # 2 bytes off (breaks int32/fp32), 8 bytes off (breaks 16-byte vectors)
+    route = lambda idx=A, w=A, logits=None, bias=None, ws=A: L.moe_route_topk(
+        A, 4, 256, A, 0, bias, 8, 2, idx, w, logits, ws, 1 << 30, None)
+    for kw in (dict(idx=odd2), dict(w=odd2), dict(logits=odd2), dict(bias=odd2), dict(ws=odd8)):
+        assert route(**kw) == INVALID_ARG, kw
+    perm = lambda idx=A, off=A, sp=A, pr=A, ws=A: L.moe_permute(idx, 4, 2, 8, None, 0, off, sp, pr, None, ws,
+                                                                1 << 30, None)
+    for kw in (dict(idx=odd2), dict(off=odd2), dict(sp=odd2), dict(pr=odd2), dict(ws=odd8)):
+        assert perm(**kw) == INVALID_ARG, kw
+    comb = lambda pr=A, w=A, y=A, out=A: L.moe_combine(y, 0, pr, w, 4, 2, 256, out, None)
+    for kw in (dict(pr=odd2), dict(w=odd2), dict(y=odd8), dict(out=odd8)):
+        assert comb(**kw) == INVALID_ARG, kw
+    ffn = lambda ex, off=A, y=A: L.moe_grouped_ffn(A, 4, off, ex, y, 0, A, 1 << 40, None)
+    ex = _experts(w=A)
+    assert ffn(ex, off=odd2) == INVALID_ARG
+    assert ffn(ex, y=odd8) == INVALID_ARG
+    assert ffn(_experts(fmt="nvfp4", w=A, scale=A, tscale=odd2)) == INVALID_ARG
+    assert L.moe_dequantize(FMT["fp8"], A, odd2, 1.0, 4, 128, A, None) == INVALID_ARG
+    lay = lambda bias=None, idx=None, w=None, out=A: L.moe_layer_forward(A, 4, A, 0, bias, 2, ex, None, 0, 0, out,
+                                                                         idx, w, A, 1 << 40, None)
+    for kw in (dict(bias=odd2), dict(idx=odd2), dict(w=odd2), dict(out=odd8)):
+        assert lay(**kw) == INVALID_ARG, kw
+
+
 def test_cache_init_checks_the_layers_first():
     L = moe.lib()
     h = ctypes.c_void_p()
