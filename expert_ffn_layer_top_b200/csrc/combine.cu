@@ -18,7 +18,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
     __shared__ int rows[kMaxTopK];
     __shared__ float ws[kMaxTopK];
     if (threadIdx.x < k) {
-        rows[threadIdx.x] = pair_row[(int64_t)t * k + threadIdx.x];
+        int r = pair_row[(int64_t)t * k + threadIdx.x];
+        // a row outside y_perm's T*k rows is reported, and row 0 read in its place
+        if (r < 0 || (int64_t)r >= (int64_t)gridDim.x * k) {
+            flag_error(2);
+            r = 0;
+        }
+        rows[threadIdx.x] = r;
         ws[threadIdx.x] = w[(int64_t)t * k + threadIdx.x];
     }
     __syncthreads();

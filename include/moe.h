@@ -205,7 +205,9 @@ moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offset
  *   y_perm: [T*k][H] bf16 or fp32 (y_is_fp32); out: bf16 [T][H]. H % 8 == 0.
  *   T == 0 is a no-op. Errors: INVALID_ARG for T < 0, k outside 1..16, H not a
  *   positive multiple of 8, NULL pointers, y_perm or out not 16-byte aligned, or
- *   pair_row or w not 4-byte aligned. */
+ *   pair_row or w not 4-byte aligned. A pair_row entry outside 0..T*k-1 is found
+ *   on the device: it sets the device error word to 2 (moe_device_error) and row
+ *   0 is read in its place. */
 moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
                        int H, void *out, moe_stream_t stream);
 
