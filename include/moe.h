@@ -181,6 +181,10 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
  *   h = silu(Wg_e . x_perm[r]) * (Wu_e . x_perm[r]), rounded to bf16;
  *   y_perm[r] = W2_e . h   (bf16, or fp32 if y_is_fp32).
  *   x_perm: bf16 [n_rows][H] in the interleaved layout written by moe_permute.
+ *   offsets: int32 [E+1] as moe_permute writes them: offsets[0] = 0,
+ *     non-decreasing, offsets[E] = n_rows. The kernels take them as given (they
+ *     are read on the device only); other values make them read and write
+ *     outside x_perm and y_perm.
  *   y_perm: [n_rows][H], natural column order.
  *   ws: scratch; moe_workspace_size(n_rows, H, I, E, 1, y_is_fp32) bytes
  *   always suffice. The decoding path (row-major experts, BF16, FP8, and
