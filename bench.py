@@ -218,13 +218,11 @@ def time_ffn_only(moe, lb: LayerBench, K: int, W: int, device):
     """Average duration of the grouped FFN call (gate/up + down launches) on the same data."""
     T, k = lb.T, lb.k
     P = T * k
-    j0 = 0
     # permuted operands per set, prepared once (untimed)
     prep = []
     for j in range(len(lb.sets)):
-        off, sp, pr, xp = moe.moe_permute(lb.idx[j], lb.layer.E, lb.xs[j])
+        off, _, _, xp = moe.moe_permute(lb.idx[j], lb.layer.E, lb.xs[j])
         prep.append((xp, off))
-    y = torch.empty(P, lb.layer.H, dtype=torch.float32 if lb.y32 else torch.bfloat16, device=device)
     ws = torch.empty(moe.moe_workspace_size(P, lb.layer.H, lb.layer.I, lb.layer.E, 1, lb.y32), dtype=torch.uint8,
                      device=device)
 
