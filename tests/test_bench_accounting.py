@@ -35,9 +35,11 @@ def test_expert_bytes_closed_form(fmt):
         assert synthetic.expert_bytes(fmt, H, I) == want
 
 
-def test_decode_expert_is_2506752_bytes():
-    # w13 [1536][2048] and w2 [2048][768] at 0.53125 bytes per element
+def test_per_expert_bytes_of_the_workloads():
+    # decode: w13 [1536][2048] and w2 [2048][768] at 0.53125 bytes per element
     assert synthetic.expert_bytes("mxfp4", 2048, 768) == 2_506_752
+    # Large: [4096][4096] and [4096][2048] at 0.5625 bytes per element, plus two fp32 tensor scales
+    assert synthetic.expert_bytes("nvfp4", 4096, 2048) == 14_155_784
 
 
 def test_active_expert_bytes_count_each_used_expert_once():
