@@ -273,6 +273,52 @@ def test_layer_matches_per_token_brute_force_fp64():
     assert np.abs(r["out"] - out).max() <= 1e-3 * np.abs(out).max()
 
 
+def _e2m1_table():
+    return {int(c): float(v) for c, v in (l.split() for l in open(os.path.join(GOLDEN, "e2m1_table.txt"))
+                                          if l.strip() and not l.startswith("#"))}
+
+
+def _decode_np(fmt, codes, scale, tscale):
+    """Independent fp64 decode of one expert tensor [R, K] (codes as stored, NumPy and torch only)."""
+    codes = codes.numpy()
+    if fmt == "fp8":
+        q = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+        return q * np.repeat(scale.double().numpy(), 128, axis=1)
+    tab = _e2m1_table()
+    lo, hi = codes & 15, codes >> 4
+    nib = np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1)     # low nibble = lower K index
+    q = np.vectorize(tab.get)(nib).astype(np.float64)
+    if fmt == "mxfp4":
+        return q * np.repeat(np.exp2(scale.numpy().astype(np.float64) - 127), 32, axis=1)
+    sb = torch.from_numpy(scale.numpy()).view(torch.float8_e4m3fn).double().numpy()
+    return q * np.repeat(sb, 16, axis=1) * float(tscale)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "mxfp4", "nvfp4"])
+def test_quantised_layer_matches_per_token_brute_force_fp64(fmt):
+    """Per-expert scale planes, strides and tensor scales of the quantised formats, against an fp64
+    per-token evaluation that decodes every expert independently of the oracle's decoder."""
+    H, I, E, k = 128, 128, 4, 2
+    L = synthetic.make_layer(dict(H=H, E=E, k=k, I=I, fmt=fmt), 11)
+    x = synthetic.make_tokens(6, H, 11)
+    r = oracle.layer_forward(x, L)
+    xf = x.double().numpy()
+    w13 = [_decode_np(fmt, L.w13[e], None if L.w13_scale is None else L.w13_scale[e],
+                      None if L.w13_tscale is None else L.w13_tscale[e]) for e in range(E)]
+    w2 = [_decode_np(fmt, L.w2[e], None if L.w2_scale is None else L.w2_scale[e],
+                     None if L.w2_tscale is None else L.w2_tscale[e]) for e in range(E)]
+    out = np.zeros_like(xf)
+    for t in range(xf.shape[0]):
+        for j in range(k):
+            e = r["idx"][t, j]
+            g = w13[e][:I] @ xf[t]
+            u = w13[e][I:] @ xf[t]
+            h = _bf16_round_np(g / (1 + np.exp(-g)) * u).astype(np.float64)
+            out[t] += r["w"][t, j] * (w2[e] @ h)
+    assert len(set(r["idx"].ravel().tolist())) > 1           # several experts, so strides matter
+    assert np.abs(r["out"] - out).max() <= 1e-3 * np.abs(out).max()
+
+
 def test_token_rows_agree_with_layer():
     L = synthetic.make_layer(dict(H=128, E=16, k=4, I=64, fmt="nvfp4"), 9)
     x = synthetic.make_tokens(20, 128, 9)

@@ -20,7 +20,9 @@ from conftest import ROOT
 
 _DIR = os.path.join(ROOT, "_build", "planted")
 
-# (name, exact text in oracle.c, replacement). The text must occur once.
+# (name, exact text in oracle.c, replacement[, occurrences]). The text must occur exactly that many
+# times (once unless stated); every occurrence is edited, so a mistake can sit in both the layer path
+# and the per-token path at once.
 C_PLANTS = [
     ("e2m1_exponent_bias", "ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)"),
     ("e2m1_subnormal_step", "(e == 0) ? 0.5 * m", "(e == 0) ? 1.0 * m"),
@@ -65,6 +67,11 @@ C_PLANTS = [
     ("combine_first_gate_only", "acc += w[(size_t)t * k + j] * y_perm[(size_t)r * H + c];",
      "acc += w[(size_t)t * k] * y_perm[(size_t)r * H + c];"),
     ("combine_skips_pair_row", "int r = pair_row[(size_t)t * k + j];", "int r = t * k + j;"),
+    ("w13_scale_stride_of_w2", "w13s ? (const char *)w13s + e * s13 : 0,", "w13s ? (const char *)w13s + e * s2 : 0,",
+     2),
+    ("w2_scale_of_expert_0", "w2s ? (const char *)w2s + e * s2 : 0,", "w2s ? (const char *)w2s : 0,", 2),
+    ("w13_tensor_scale_of_expert_0", "w13t ? w13t[e] : 1.0f", "w13t ? w13t[0] : 1.0f", 2),
+    ("w2_tensor_scale_of_expert_0", "w2t ? w2t[e] : 1.0f", "w2t ? w2t[0] : 1.0f", 2),
 ]
 
 # (name, exact text in lru.py, replacement).
@@ -82,7 +89,8 @@ LRU_PLANTS = [
     ("evict_ignores_ids", "            if ids is not None and o[1] not in set(ids):\n                continue\n", ""),
 ]
 
-PARAMS = {"test_permutation_is_stable_counting_sort": [(16, 2, 8), (64, 8, 128)]}
+PARAMS = {"test_permutation_is_stable_counting_sort": [(16, 2, 8), (64, 8, 128)],
+          "test_quantised_layer_matches_per_token_brute_force_fp64": [("fp8",), ("mxfp4",), ("nvfp4",)]}
 
 
 def _pins():
@@ -105,8 +113,8 @@ def _failing_pins():
     return failed
 
 
-def _plant(text, old, new):
-    assert text.count(old) == 1, f"planting text occurs {text.count(old)} times: {old!r}"
+def _plant(text, old, new, n=1):
+    assert text.count(old) == n, f"planting text occurs {text.count(old)} times, not {n}: {old!r}"
     return text.replace(old, new)
 
 
@@ -114,10 +122,11 @@ def test_unplanted_oracle_passes_every_pin():
     assert _failing_pins() == []
 
 
-@pytest.mark.parametrize("name,old,new", C_PLANTS, ids=[p[0] for p in C_PLANTS])
-def test_planted_c_mistake_is_caught(name, old, new, monkeypatch):
+@pytest.mark.parametrize("plant", C_PLANTS, ids=[p[0] for p in C_PLANTS])
+def test_planted_c_mistake_is_caught(plant, monkeypatch):
+    name = plant[0]
     os.makedirs(_DIR, exist_ok=True)
-    src = _plant(open(oracle._SRC).read(), old, new)
+    src = _plant(open(oracle._SRC).read(), *plant[1:])
     c = os.path.join(_DIR, f"{name}.c")
     so = os.path.join(_DIR, f"{name}.{os.getpid()}.so")
     with open(c, "w") as f:
