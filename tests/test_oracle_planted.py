@@ -67,6 +67,23 @@ C_PLANTS = [
     ("combine_first_gate_only", "acc += w[(size_t)t * k + j] * y_perm[(size_t)r * H + c];",
      "acc += w[(size_t)t * k] * y_perm[(size_t)r * H + c];"),
     ("combine_skips_pair_row", "int r = pair_row[(size_t)t * k + j];", "int r = t * k + j;"),
+    ("logits_written_before_bias",
+     "            float lf = (float)acc;\n            if (bias) lf = lf + bias[e];\n            l[e] = lf;\n"
+     "            if (logits) logits[(size_t)t * E + e] = lf;",
+     "            float lf = (float)acc;\n            if (logits) logits[(size_t)t * E + e] = lf;\n"
+     "            if (bias) lf = lf + bias[e];\n            l[e] = lf;"),
+    ("router_bf16_weight_transposed", "bf16_to_f32(((const uint16_t *)wr)[(size_t)h * E + e])",
+     "bf16_to_f32(((const uint16_t *)wr)[(size_t)e * H + h])"),
+    ("gating_sum_skips_last", "for (int j = 0; j < k; ++j) z += expf(l[order[j]] - l0);",
+     "for (int j = 0; j + 1 < k; ++j) z += expf(l[order[j]] - l0);"),
+    ("offsets_scan_stops_early", "for (int e = 0; e < E; ++e) offsets[e + 1] += offsets[e];",
+     "for (int e = 0; e + 1 < E; ++e) offsets[e + 1] += offsets[e];"),
+    ("nvfp4_multiplication_order", "v = (q * s) * tscale;", "v = q * (s * tscale);"),
+    ("silu_of_up_instead_of_gate", "float hv = bf16_to_f32(f32_to_bf16(silu(g) * u));",
+     "float hv = bf16_to_f32(f32_to_bf16(silu(u) * g));"),
+    ("down_projection_drops_last_channel", "for (int i = 0; i < I; ++i) acc += hbuf[i] * w2r[i];",
+     "for (int i = 0; i + 1 < I; ++i) acc += hbuf[i] * w2r[i];"),
+    ("combine_pair_row_transposed", "int r = pair_row[(size_t)t * k + j];", "int r = pair_row[(size_t)j * T + t];"),
     ("w13_scale_stride_of_w2", "w13s ? (const char *)w13s + e * s13 : 0,", "w13s ? (const char *)w13s + e * s2 : 0,",
      2),
     ("w2_scale_of_expert_0", "w2s ? (const char *)w2s + e * s2 : 0,", "w2s ? (const char *)w2s : 0,", 2),
