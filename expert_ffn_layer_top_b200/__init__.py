@@ -20,6 +20,9 @@ from ._lib import (  # noqa: F401
     moe_permute,
     moe_permute_static,
     moe_prepack,
+    moe_selftest_wait,
+    moe_set_wait_limit_ns,
+    PREFETCH,
     moe_prepacked_expert_bytes,
     LAYOUT_STANDARD,
     LAYOUT_TILED,

@@ -37,6 +37,18 @@ class _Experts(C.Structure):
     ]
 
 
+class _CacheReport(C.Structure):
+    _fields_ = [
+        ("table_s", C.c_double), ("host_wait_s", C.c_double), ("issue_s", C.c_double), ("copy_s", C.c_double),
+        ("compute_s", C.c_double), ("overlap_s", C.c_double), ("h2d_gbs", C.c_double),
+        ("calls", C.c_uint64), ("prefetched", C.c_uint64), ("moved", C.c_uint64),
+        ("n_slots", C.c_int), ("last_depth", C.c_int),
+    ]
+
+
+PREFETCH = {"none": 0, "predicted": 1, "full_layer": 2, "adaptive": 3}
+
+
 def lib():
     """Load (building first if missing or stale) libmoe.so; raises if that fails."""
     global _lib_handle
@@ -81,6 +93,16 @@ def lib():
             L.expert_cache_stats.restype = st
             L.expert_cache_stats.argtypes = [_P, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64),
                                              C.POINTER(C.c_uint64), C.POINTER(C.c_double)]
+            L.expert_cache_set_prefetch.restype = st
+            L.expert_cache_set_prefetch.argtypes = [_P, _I, _I]
+            L.expert_cache_resize.restype = st
+            L.expert_cache_resize.argtypes = [_P, C.c_size_t]
+            L.expert_cache_report.restype = st
+            L.expert_cache_report.argtypes = [_P, C.POINTER(_CacheReport)]
+            L.moe_set_wait_limit_ns.restype = st
+            L.moe_set_wait_limit_ns.argtypes = [C.c_uint64]
+            L.moe_selftest_wait.restype = st
+            L.moe_selftest_wait.argtypes = [_P]
             L.expert_cache_slot_of.restype = st
             L.expert_cache_slot_of.argtypes = [_P, _I, _I, C.POINTER(C.c_int32)]
             L.expert_cache_destroy.restype = st
@@ -130,6 +152,16 @@ def moe_device_error() -> int:
     code = C.c_int(0)
     _check(lib().moe_device_error(C.byref(code)))
     return code.value
+
+
+def moe_set_wait_limit_ns(ns: int) -> None:
+    """Limit of the bounded device waits in ns (0 = the 2 s default); a test hook."""
+    _check(lib().moe_set_wait_limit_ns(int(ns)))
+
+
+def moe_selftest_wait(stream=None) -> None:
+    """Enqueue the kernel whose bounded wait must give up (sets device error 1)."""
+    _check(lib().moe_selftest_wait(_stream(stream)))
 
 
 def moe_workspace_size(T: int, H: int, I: int, E: int, k: int, y_fp32: bool = False) -> int:
@@ -302,6 +334,18 @@ class ExpertCache:
         s = C.c_double()
         _check(lib().expert_cache_stats(self.handle, C.byref(h), C.byref(m), C.byref(b), C.byref(s)))
         return dict(hits=h.value, misses=m.value, bytes_h2d=b.value, copy_s=s.value)
+
+    def set_prefetch(self, policy: str, depth: int = -1):
+        """Next-layer prefetch: 'none', 'predicted' (first `depth`, -1 all), 'full_layer', 'adaptive'."""
+        _check(lib().expert_cache_set_prefetch(self.handle, PREFETCH[policy], int(depth)))
+
+    def resize(self, capacity_bytes: int):
+        _check(lib().expert_cache_resize(self.handle, int(capacity_bytes)))
+
+    def report(self) -> dict:
+        r = _CacheReport()
+        _check(lib().expert_cache_report(self.handle, C.byref(r)))
+        return {name: getattr(r, name) for name, _ in _CacheReport._fields_}
 
     def slot_of(self, layer: int, e: int) -> int:
         v = C.c_int32()

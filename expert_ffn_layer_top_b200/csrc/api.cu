@@ -385,7 +385,23 @@ static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
 
 moe_status cache_resolve_and_map(struct expert_cache *c, int layer, const int32_t *idx, int T, int k,
                                  const moe_experts *shape, moe_experts *dev_view, cudaStream_t st);
+void cache_compute_end(struct expert_cache *c, cudaStream_t st);
 int cache_layout(const struct expert_cache *c);
+
+// A kernel that waits, with the bounded wait of the FFN kernels, on an mbarrier that
+// nothing completes; no copy or MMA is in flight. The wait gives up, flags error 1 and
+// the kernel returns.
+__global__ void __launch_bounds__(32) wait_selftest_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    mbar_wait(&bar, 0, &abort_flag);
+}
 
 }  // namespace moe
 
@@ -589,15 +605,32 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     if (cache) {
         r = cache_resolve_and_map(cache, layer, idx, T, k, experts, &view, st);
         if (r != MOE_OK) return r;
-        if ((r = check_experts(&view)) != MOE_OK) return r;
     }
-    if (is_mx(view, T * k) != mx) return set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
-    if (mx)
-        r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
-    else
-        r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
-    if (r != MOE_OK) return r;
-    return moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
+    r = check_experts(&view);
+    if (r == MOE_OK && is_mx(view, T * k) != mx)
+        r = set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
+    if (r == MOE_OK) {
+        if (mx)
+            r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+        else
+            r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+    }
+    if (r == MOE_OK) r = moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
+    if (cache) cache_compute_end(cache, st);   // closes the call's timing record in every case
+    return r;
+}
+
+moe_status moe_set_wait_limit_ns(uint64_t ns) {
+    const uint64_t v = ns ? ns : kWaitLimitNs;
+    cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "wait limit");
+}
+
+moe_status moe_selftest_wait(moe_stream_t stream) {
+    count_launch();
+    wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "wait self-test launch");
 }
 
 }  // extern "C"

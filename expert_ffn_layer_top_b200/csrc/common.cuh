@@ -73,7 +73,14 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, then give up and flag
+// Bounded waits. A wait on an mbarrier that another role of the CTA completes
+// gives up after g_wait_limit_ns (2 s unless moe_set_wait_limit_ns changed it,
+// read from memory only once the first poll has failed) and flags error 1. The
+// waits that keep a CTA alive until its own bulk copies and MMAs have landed
+// always use the fixed kWaitLimitNs: they must not end while an asynchronous
+// write into the CTA's shared memory or TMEM is still in flight.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -120,15 +127,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Gives up after
-// kWaitLimitNs, or as soon as another role of the CTA has given up (*abort),
+// g_wait_limit_ns, or as soon as another role of the CTA has given up (*abort),
 // setting the CTA abort flag and the device error word. Returns false then.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    const uint64_t limit = *reinterpret_cast<volatile uint64_t *>(&g_wait_limit_ns);
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit) {
             *abort_flag = 1;
             flag_error(1);
             return false;

@@ -65,15 +65,18 @@ __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
 }
 
 // Exact widening to fp64 by moving the bit fields (the exponent is rebiased by
-// 1023 - 127 = 896); zeros and subnormals take the conversion instruction.
+// 1023 - 127 = 896); zeros, subnormals, infinities and NaNs (exponent field 0
+// or all ones) take the conversion instruction, which keeps Inf and NaN.
 __device__ __forceinline__ double bf16_bits_to_f64(uint32_t b) {
-    if ((b & 0x7F80u) == 0) return (double)__uint_as_float(b << 16);
+    const uint32_t ex = b & 0x7F80u;
+    if (ex == 0 || ex == 0x7F80u) return (double)__uint_as_float(b << 16);
     const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + (896u << 20));
     return __hiloint2double((int)hi, 0);
 }
 
 __device__ __forceinline__ double f32_bits_to_f64(uint32_t f) {
-    if ((f & 0x7F800000u) == 0) return (double)__uint_as_float(f);
+    const uint32_t ex = f & 0x7F800000u;
+    if (ex == 0 || ex == 0x7F800000u) return (double)__uint_as_float(f);
     const uint32_t hi = (f & 0x80000000u) | (((f & 0x7FFFFFFFu) >> 3) + (896u << 20));
     return __hiloint2double((int)hi, (int)(f << 29));
 }
@@ -590,8 +593,8 @@ static cudaError_t launch_router_cluster(const RouterClusterShape &sh, const voi
 // The ticket counter of (device, stream): launches on one stream run in order, so
 // one counter per stream is never shared by two launches at once. Slots are
 // handed out per (device, stream) on first use; a device holds kTicketSlots of
-// them (after that many streams, slots are reused round-robin). Null if the
-// counters cannot be found, and the caller permutes in its own launch.
+// them. Null once a device's slots are all taken (its later streams route and
+// permute in two launches) or if the counters cannot be found.
 static unsigned int *route_ticket(cudaStream_t st) {
     struct Slot { int dev; cudaStream_t st; int idx; };
     static std::mutex mu;

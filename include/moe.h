@@ -309,6 +309,75 @@ moe_status expert_cache_evict(struct expert_cache *cache, int layer, const int32
 moe_status expert_cache_stats(struct expert_cache *cache, uint64_t *hits, uint64_t *misses, uint64_t *bytes_h2d,
                               double *copy_s);
 
+/* Prefetch of the next layer, decided per cached layer call ([P4] "Three
+ * Engineering Cores": full-layer double-buffered streaming; [P3] "FreeToken's
+ * Three-Layer Mechanism": the transfer adapts to the bandwidth it measures).
+ * After a call resolves layer l, experts of layer l+1 are loaded behind that
+ * layer's own misses on the copy stream, so they arrive while layer l computes.
+ * The prediction for layer l+1 is the set of experts its previous call used,
+ * ranked by the pairs each received (more first, ties to the lower id).
+ *   MOE_PREFETCH_NONE        nothing.
+ *   MOE_PREFETCH_PREDICTED   the first `depth` experts of the prediction
+ *                            (depth < 0: all of it). The default, depth -1.
+ *   MOE_PREFETCH_FULL_LAYER  every expert of layer l+1 (prefill: the next call
+ *                            touches nearly every expert).
+ *   MOE_PREFETCH_ADAPTIVE    per call: the full layer when the call's T tokens
+ *                            are expected to reach at least half of the E
+ *                            experts (E (1 - (1 - k/E)^T) >= E/2); otherwise
+ *                            the first floor(bw * t / expert_bytes) of the
+ *                            prediction, bw being the measured host-to-device
+ *                            rate and t the measured time of a cached layer's
+ *                            FFN and combine (running averages); the whole
+ *                            prediction until both have been measured.
+ * A prefetch that does not fit in the free and evictable slots is skipped. */
+typedef enum {
+    MOE_PREFETCH_NONE = 0,
+    MOE_PREFETCH_PREDICTED = 1,
+    MOE_PREFETCH_FULL_LAYER = 2,
+    MOE_PREFETCH_ADAPTIVE = 3
+} moe_prefetch_policy;
+
+/* Set the prefetch policy (host call, takes effect at the next layer call).
+ * Errors: INVALID_ARG for a NULL cache or an unknown policy. */
+moe_status expert_cache_set_prefetch(struct expert_cache *cache, int policy, int depth);
+
+/* Resize the slot pool to floor(capacity_bytes / slot bytes) slots without
+ * fetching any resident expert again ([P4] "Three Engineering Cores": elastic
+ * memory management without weight reloads). The pool is a reserved virtual
+ * address range backed by physical chunks: growing maps more chunks and adds
+ * free slots; shrinking keeps the most recently used experts that fit, moves
+ * those above the new end into the lowest free slots (least recent first, by
+ * device-to-device copy on the cache's copy stream), drops the rest and unmaps
+ * the chunks past the new end. Synchronous: it waits for the device, so no
+ * layer call may be in flight on another thread. The table change follows the
+ * rule of the cache's policy exactly.
+ * Errors: INVALID_ARG for a NULL cache; CACHE_FULL for a capacity below one
+ * expert; UNSUPPORTED when the pool could not be built on reserved addresses
+ * (then only sizes within the first allocation are accepted) or the capacity
+ * exceeds the reserved range (the device's memory); OOM or CUDA when mapping
+ * fails, with the cache unchanged. */
+moe_status expert_cache_resize(struct expert_cache *cache, size_t capacity_bytes);
+
+/* What the cache measured since init. Seconds are summed over the cached layer
+ * calls whose events have completed. */
+typedef struct {
+    double table_s;      /* device time of the table updates (event-timed) */
+    double host_wait_s;  /* host time spent waiting for a table update to finish */
+    double issue_s;      /* host time spent enqueueing copies */
+    double copy_s;       /* time the copy stream spent copying (event-timed) */
+    double compute_s;    /* caller-stream time of the cached calls' FFN and combine */
+    double overlap_s;    /* copy time that fell inside those FFN-and-combine intervals */
+    double h2d_gbs;      /* running average of the measured host-to-device rate, GB/s (0: none yet) */
+    uint64_t calls;      /* cached layer calls */
+    uint64_t prefetched; /* experts loaded by next-layer prefetches */
+    uint64_t moved;      /* experts moved device-to-device by resizes */
+    int n_slots;         /* slots in the pool now */
+    int last_depth;      /* depth of the last call's prefetch (-1: whole prediction; E: whole layer) */
+} moe_cache_report;
+
+/* Fill *out (waits for the copy stream first). Errors: INVALID_ARG for NULL. */
+moe_status expert_cache_report(struct expert_cache *cache, moe_cache_report *out);
+
 /* Device slot of (layer, e), or -1 (synchronous read; for tests and tools). */
 moe_status expert_cache_slot_of(struct expert_cache *cache, int layer, int e, int32_t *slot);
 
@@ -324,6 +393,21 @@ const char *moe_last_error_string(void);
  * checks (0 = none; 1 = a wait timed out; 2 = bad argument seen on device).
  * Synchronises the device. */
 moe_status moe_device_error(int *code);
+
+/* Limit of the bounded device-side waits (the kernels' waits on barriers that
+ * another role of the same CTA completes), in nanoseconds, on the current
+ * device; 0 restores the default of 2 s. Waits that keep a CTA alive until its
+ * own bulk copies and MMAs have landed keep the 2 s limit whatever is set. No
+ * counterpart in the pages: a test hook for the failure path of the bounded
+ * waits. Synchronous. Errors: CUDA. */
+moe_status moe_set_wait_limit_ns(uint64_t ns);
+
+/* Enqueue one small kernel that waits, through the same bounded-wait code as
+ * the grouped FFN, on a barrier that nothing completes, with no copy or MMA in
+ * flight. It gives up after the wait limit, sets the device error word to 1
+ * and returns, leaving the context usable. No counterpart in the pages: the
+ * test of the bounded waits. Errors: CUDA for a failed launch. */
+moe_status moe_selftest_wait(moe_stream_t stream);
 
 /* Library version, for logs. */
 const char *moe_version(void);

@@ -18,6 +18,18 @@ and the final table are fully determined:
   prefetch) counts its bytes.
 * If every occupied slot is protected and none is free the call fails with
   CACHE_FULL and leaves the table as it was before the call.
+* Prediction of a layer's next call (aimodeling.com English page, "Three
+  Engineering Cores": full-layer double-buffered streaming; winzheng.com,
+  "FreeToken's Three-Layer Mechanism": transfers sized to the bandwidth
+  measured): the experts its last resolve used, ranked by the pairs each
+  received, more first, ties to the lower id (counts above 2^20 - 1 rank as
+  equal). A prefetch of depth d takes the first d of them; a full-layer
+  prefetch takes every expert of the layer.
+* Resize to S' slots (aimodeling.com, "Three Engineering Cores": elastic memory
+  without weight reloads): growing adds free slots. Shrinking keeps the
+  min(occupied, S') most recently referenced experts and drops the others;
+  kept experts in slots >= S' then move, least recent first, each to the
+  lowest free slot below S', keeping their recency and call index.
 
 Independent of the device code: this keeps explicit integer stamps and scans
 for the minimum, where the kernel keeps an intrusive linked list.
@@ -43,6 +55,8 @@ class LruSim:
         self.calls = 0
         self.hits = self.misses = self.loads = 0
         self.bytes_h2d = 0
+        self.moves = 0
+        self.last_counts: Dict[int, Dict[int, int]] = {}   # layer -> {expert: pairs} at its last resolve
 
     def _call(self, layer: int, ids: Iterable[int], count: bool) -> List[Tuple[int, int]]:
         ids = sorted(set(int(i) for i in ids))
@@ -82,8 +96,56 @@ class LruSim:
         return loads
 
     def resolve(self, layer: int, ids: Iterable[int]) -> List[Tuple[int, int]]:
-        """Map the experts a layer needs to slots; returns the (expert, slot) loads."""
-        return self._call(layer, ids, True)
+        """Map the experts a layer needs to slots; returns the (expert, slot) loads.
+
+        ``ids`` may repeat an expert once per pair routed to it: the number of
+        repeats is the pair count that ranks the layer's next prediction."""
+        ids = [int(i) for i in ids]
+        loads = self._call(layer, ids, True)
+        counts: Dict[int, int] = {}
+        for e in ids:
+            counts[e] = counts.get(e, 0) + 1
+        self.last_counts[layer] = counts
+        return loads
+
+    def predict(self, layer: int, depth: int = -1, full: bool = False) -> List[int]:
+        """Experts a prefetch of ``layer`` loads: all E when ``full``, else the
+        first ``depth`` of the layer's prediction in rank order (depth < 0: all)."""
+        if full:
+            return list(range(self.E))
+        counts = self.last_counts.get(layer, {})
+        ranked = sorted(counts, key=lambda e: (-min(counts[e], (1 << 20) - 1), e))
+        return sorted(ranked if depth < 0 else ranked[:depth])
+
+    def resize(self, n_slots: int) -> List[Tuple[int, int]]:
+        """Change the pool to ``n_slots`` slots; returns the (from, to) slot moves."""
+        S = self.S
+        if n_slots >= S:
+            self.owner += [None] * (n_slots - S)
+            self.stamp += [-1] * (n_slots - S)
+            self.ref_call += [-(10**9)] * (n_slots - S)
+            self.S = n_slots
+            return []
+        occ = sorted((i for i in range(S) if self.owner[i] is not None), key=lambda i: self.stamp[i])
+        keep = occ[len(occ) - min(len(occ), n_slots):]
+        for i in occ[: len(occ) - len(keep)]:
+            del self.slot_of[self.owner[i]]
+            self.owner[i] = None
+            self.stamp[i] = -1
+            self.ref_call[i] = -(10**9)
+        moves = []
+        for i in keep:   # least recent first
+            if i < n_slots:
+                continue
+            f = min(j for j in range(n_slots) if self.owner[j] is None)
+            self.owner[f], self.stamp[f], self.ref_call[f] = self.owner[i], self.stamp[i], self.ref_call[i]
+            self.slot_of[self.owner[f]] = f
+            self.owner[i], self.stamp[i], self.ref_call[i] = None, -1, -(10**9)
+            moves.append((i, f))
+        del self.owner[n_slots:], self.stamp[n_slots:], self.ref_call[n_slots:]
+        self.S = n_slots
+        self.moves += len(moves)
+        return moves
 
     def prefetch(self, layer: int, ids: Iterable[int]) -> List[Tuple[int, int]]:
         return self._call(layer, ids, False)

@@ -384,3 +384,205 @@ def test_bad_arguments_are_rejected(moe):
     assert ei.value.name == "UNSUPPORTED"
     with pytest.raises(moe.MoeError):
         moe.moe_route_topk(x, L.wr, 17)                        # k > 16
+
+
+# ----------------------------------------------------------------------------- wider full-size sampling
+
+
+def _sample_rows(L, x, n_random, seed, BN=128):
+    """Tokens whose outputs are checked at full size: rows at the start, end and every
+    token-tile boundary (multiples of BN) of the three most-routed experts, the first and
+    last row of every expert that has any, and random tokens; about 64-100 in all."""
+    idx_o, _, _ = oracle.route(x, L.wr, L.k, bias=L.bias, with_logits=False)
+    off, sp, _ = oracle.permute(idx_o, L.E)
+    n = np.diff(off)
+    rows = []
+    for e in np.argsort(-n, kind="stable")[:3]:
+        b, c = int(off[e]), int(n[e])
+        for r in range(0, c, BN):
+            rows += [b + r, b + r - 1] if r else [b]
+        rows.append(b + c - 1)
+    busy = [e for e in range(L.E) if n[e] > 0]
+    g = np.random.default_rng(seed)
+    for e in g.choice(busy, size=min(len(busy), 16), replace=False):
+        rows += [int(off[e]), int(off[e + 1]) - 1]
+    toks = set(int(sp[r]) // L.k for r in rows if 0 <= r < len(sp))
+    toks |= set(int(t) for t in g.choice(x.shape[0], n_random, replace=False))
+    return sorted(toks)
+
+
+def test_layer_prefill_nvfp4_full_size_wide_sample(moe, prefill_layer):
+    x = synthetic.make_tokens(4096, 2048, seed=12)
+    sample = _sample_rows(prefill_layer, x, 16, 12)
+    assert len(sample) >= 64
+    _layer_check(moe, prefill_layer, x, sample=sample)
+
+
+def test_layer_large_prefill_wide_sample(moe, large_layer):
+    x = synthetic.make_tokens(8192, 4096, seed=14)
+    sample = _sample_rows(large_layer, x, 16, 14)
+    assert len(sample) >= 64
+    _layer_check(moe, large_layer, x, y_fp32=True, sample=sample)
+
+
+def test_layer_large_decode_every_row(moe, large_layer):
+    x = synthetic.make_tokens(32, 4096, seed=13)
+    _layer_check(moe, large_layer, x, y_fp32=True, sample=list(range(32)))
+
+
+# ----------------------------------------------------------------------------- the boundary's limits
+
+
+def test_router_top16(moe):
+    cfg = dict(H=512, E=256, k=16, wr_fp32=False, zipf=None)
+    wr, _ = synthetic.make_router(cfg, seed=31)
+    for T in (5, 300):   # the cluster path and the fp64 tensor-core path
+        x = synthetic.make_tokens(T, 512, seed=31 + T)
+        idx_o, w_o, lg_o = oracle.route(x, wr, 16)
+        idx, w, lg = moe.moe_route_topk(x.cuda(), wr.cuda(), 16, want_logits=True)
+        assert np.array_equal(idx.cpu().numpy(), idx_o)
+        assert _ulp_close(lg.cpu().numpy(), lg_o, 1)
+        assert np.allclose(w.cpu().numpy(), w_o, rtol=0, atol=2e-6)
+
+
+def test_router_infinite_input(moe):
+    """An infinite activation makes every logit of its token +-Inf: the experts tie and go
+    in index order, as in the oracle; the other tokens are unaffected."""
+    wr, _ = synthetic.make_router("decode", seed=32)
+    for T in (6, 300):
+        x = synthetic.make_tokens(T, 2048, seed=32)
+        x[2, 100] = float("inf")
+        idx_o, w_o, lg_o = oracle.route(x, wr, 8)
+        idx, w, lg = moe.moe_route_topk(x.cuda(), wr.cuda(), 8, want_logits=True)
+        assert np.array_equal(idx.cpu().numpy(), idx_o)
+        lg, w = lg.cpu().numpy(), w.cpu().numpy()
+        assert np.array_equal(np.isinf(lg), np.isinf(lg_o)) and np.isinf(lg_o[2]).all()
+        fin = np.isfinite(lg_o)
+        assert _ulp_close(lg[fin], lg_o[fin], 1)
+        assert np.array_equal(np.isnan(w), np.isnan(w_o))
+        ok = ~np.isnan(w_o)
+        assert np.allclose(w[ok], w_o[ok], rtol=0, atol=2e-6)
+
+
+@pytest.mark.parametrize("T,k,E", [(512, 16, 1024), (3000, 16, 1024), (20000, 8, 1024)])
+def test_permute_at_the_limits(moe, T, k, E):
+    idx = _rand_idx(T, k, E, 17 + T)
+    x = synthetic.make_tokens(T, 64, seed=17)
+    off_o, sp_o, pr_o = oracle.permute(idx, E)
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), E, x.cuda())
+    assert np.array_equal(off.cpu().numpy(), off_o)
+    assert np.array_equal(sp.cpu().numpy(), sp_o)
+    assert np.array_equal(pr.cpu().numpy(), pr_o)
+    got = deinterleave_cols(xp.view(torch.int16).cpu().numpy())
+    assert np.array_equal(got, x.view(torch.int16).numpy()[sp_o // k])
+
+
+@pytest.mark.parametrize("fmt,tiled", [("mxfp4", True), ("bf16", False)])
+def test_grouped_ffn_1024_experts(moe, fmt, tiled):
+    """E = 1024 experts (the grouped FFN's limit), most with a row or two, some empty."""
+    E, T, k = 1024, 700, 2
+    cfg = dict(H=256, E=E, k=k, I=256, fmt=fmt, wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=19, device="cuda").to("cpu")
+    x = synthetic.make_tokens(T, 256, seed=19)
+    idx = _rand_idx(T, k, E, 19)
+    off_o, sp_o, _ = oracle.permute(idx, E)
+    y_o = oracle.ffn(x, L, off_o, sp_o, k)
+    ex = moe.Experts.from_layer(L.to("cuda"))
+    if tiled:
+        ex = moe.moe_prepack(ex)
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), E, x.cuda())
+    y = moe.moe_grouped_ffn(xp, off, ex)
+    torch.cuda.synchronize()
+    assert rel_err(bf16_np(y), y_o) < TOL
+    assert moe.moe_device_error() == 0
+
+
+def test_combine_top16(moe):
+    g = torch.Generator().manual_seed(23)
+    T, k, H = 29, 16, 256
+    y = torch.randn(T * k, H, generator=g).to(torch.bfloat16)
+    pr = torch.randperm(T * k, generator=g).to(torch.int32)
+    w = torch.rand(T, k, generator=g)
+    ref = oracle.combine(y.float().numpy(), pr.numpy(), w.numpy(), T, k)
+    out = moe.moe_combine(y.cuda(), pr.cuda(), w.cuda())
+    assert rel_err(bf16_np(out), ref) < 4e-3
+
+
+def test_layer_top16(moe):
+    cfg = dict(H=256, E=64, k=16, I=256, fmt="mxfp4", wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=24)
+    x = synthetic.make_tokens(40, 256, seed=24)
+    _layer_check(moe, L, x)
+    _layer_check(moe, L, x, tiled=False)
+
+
+def test_layer_block_scaled_unfused_routing(moe):
+    """Prepacked MXFP4 with more than 8192 pairs: routing and permutation run in separate
+    launches (the fused one-block sort stops at 8192 pairs), then the block-scaled path."""
+    cfg = dict(H=512, E=16, k=8, I=256, fmt="mxfp4", wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=25)
+    x = synthetic.make_tokens(1100, 512, seed=25)
+    n0 = moe.moe_kernel_launch_count()
+    _layer_check(moe, L, x)
+    assert moe.moe_kernel_launch_count() - n0 > 5
+
+
+def test_layer_on_more_streams_than_ticket_counters(moe, decode_layer):
+    """Each stream gets one of 256 ticket counters for the fused routing + permutation;
+    calls on further streams permute in their own launch. Every stream's output must equal
+    the default stream's, bit for bit, on both sides of that limit."""
+    from cuda.bindings import runtime as rt
+
+    L = decode_layer.to("cuda")
+    ex = moe.moe_prepack(moe.Experts.from_layer(L))
+    T = 16
+    x = synthetic.make_tokens(T, L.H, seed=26).cuda()
+    ws = torch.empty(moe.moe_workspace_size(T, L.H, L.I, L.E, L.k), dtype=torch.uint8, device="cuda")
+    ref = moe.moe_layer_forward(x, L.wr, L.k, ex, ws=ws).clone()
+    out = torch.empty_like(ref)      # nothing is allocated on the streams created below
+    torch.cuda.synchronize()
+    handles, launches = [], []
+    try:
+        for _ in range(300):
+            err, h = rt.cudaStreamCreateWithFlags(1)
+            assert int(err) == 0
+            handles.append(h)
+            s = torch.cuda.ExternalStream(int(h))
+            s.wait_stream(torch.cuda.current_stream())
+            n0 = moe.moe_kernel_launch_count()
+            out.zero_()
+            torch.cuda.synchronize()
+            with torch.cuda.stream(s):
+                moe.moe_layer_forward(x, L.wr, L.k, ex, ws=ws, out=out)
+            launches.append(moe.moe_kernel_launch_count() - n0)
+            s.synchronize()
+            assert torch.equal(out, ref)
+    finally:
+        torch.cuda.synchronize()
+        for h in handles:
+            rt.cudaStreamDestroy(h)
+    # fused (5 launches) while counters last, then routing and permutation apart (6)
+    assert launches[-1] == 6 and set(launches) <= {5, 6}
+    assert launches == sorted(launches)
+    assert moe.moe_device_error() == 0
+
+
+# ----------------------------------------------------------------------------- bounded waits
+
+
+def test_bounded_wait_gives_up_and_reports(moe):
+    """A kernel waits, through the FFN kernels' bounded wait, on a barrier that nothing
+    completes (no copy or MMA in flight). With a 1 ms limit it returns, the device error
+    word reads 1 (a wait timed out), and with the default limit back the next layer runs."""
+    assert moe.moe_device_error() == 0
+    moe.moe_set_wait_limit_ns(1_000_000)
+    try:
+        moe.moe_selftest_wait()
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_wait_limit_ns(0)
+    assert moe.moe_device_error() == 1
+    assert moe.moe_device_error() == 0          # read and cleared
+    L = synthetic.make_layer("tiny", 0)
+    x = synthetic.make_tokens(16, L.H, 0)
+    _layer_check(moe, L, x)

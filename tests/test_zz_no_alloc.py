@@ -40,6 +40,34 @@ def _same(a, b):
 CASES = [(4096, 8, 128, 2048), (2048, 8, 64, 256), (64, 8, 128, 2048)]
 
 
+def _matches_oracle(got, idx, E, x=None):
+    import oracle
+    from gpu_util import deinterleave_cols
+
+    off_o, sp_o, pr_o = oracle.permute(idx.cpu().numpy(), E)
+    off, sp, pr, xp = got
+    assert np.array_equal(off.cpu().numpy(), off_o)
+    assert np.array_equal(sp.cpu().numpy(), sp_o)
+    assert np.array_equal(pr.cpu().numpy(), pr_o)
+    if x is not None:
+        k = idx.shape[1]
+        want = x.cpu().view(torch.int16).numpy()[sp_o // k]
+        assert np.array_equal(deinterleave_cols(xp.view(torch.int16).cpu().numpy()), want)
+
+
+def test_static_permute_matches_the_oracle(moe):
+    """Offsets, sorted pairs, pair rows and the gathered rows, bit for bit against the
+    oracle's counting sort, for each case and for the largest accepted size."""
+    for i, (T, k, E, H) in enumerate(CASES):
+        idx = _idx(T, k, E, 30 + i)
+        x = synthetic.make_tokens(T, H, seed=30 + i).cuda()
+        _matches_oracle(moe.moe_permute_static(idx, E, x), idx, E, x)
+    E, k = 1024, 8
+    T2 = (LIMIT // 2 // (E * 4)) * 1024 // k
+    idx2 = _idx(T2, k, E, 33)
+    _matches_oracle(moe.moe_permute_static(idx2, E), idx2, E)
+
+
 def test_static_permute_two_calls_in_a_row_match_workspace_permute(moe):
     ins = [(_idx(T, k, E, 10 + i), synthetic.make_tokens(T, H, seed=10 + i).cuda(), E)
            for i, (T, k, E, H) in enumerate(CASES)]
