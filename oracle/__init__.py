@@ -27,6 +27,7 @@ _SO = os.path.join(_HERE, "_oracle.so")
 _lib = None
 
 FMT = {"bf16": 0, "fp8": 1, "mxfp4": 2, "nvfp4": 3}
+ACT = {"a16": 0, "a4": 1}
 
 
 def build(force: bool = False) -> str:
@@ -59,13 +60,21 @@ def _bind(path: str):
     L.oracle_permute.restype = None
     L.oracle_permute.argtypes = [P, i, i, i, P, P, P]
     L.oracle_ffn.restype = i
-    L.oracle_ffn.argtypes = [P, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
+    L.oracle_ffn.argtypes = [P, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P, i]
     L.oracle_combine.restype = None
     L.oracle_combine.argtypes = [P, P, P, i, i, i, P]
     L.oracle_layer.restype = i
-    L.oracle_layer.argtypes = [P, i, i, P, i, P, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P, P]
+    L.oracle_layer.argtypes = [P, i, i, P, i, P, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P, P, i]
     L.oracle_token_rows.restype = i
-    L.oracle_token_rows.argtypes = [P, i, i, i, i, P, P, P, P, P, P, P, P, P, i, P]
+    L.oracle_token_rows.argtypes = [P, i, i, i, i, P, P, P, P, P, P, P, P, P, i, P, i, i]
+    L.oracle_e4m3_encode.restype = i
+    L.oracle_e4m3_encode.argtypes = [f]
+    L.oracle_e2m1_encode.restype = i
+    L.oracle_e2m1_encode.argtypes = [f]
+    L.oracle_a4_tensor_scale.restype = f
+    L.oracle_a4_tensor_scale.argtypes = [P, C.c_size_t]
+    L.oracle_a4_quant.restype = None
+    L.oracle_a4_quant.argtypes = [P, i, f, P, P, P]
     L.oracle_threads.restype = i
     L.oracle_threads.argtypes = []
     return L
@@ -119,6 +128,35 @@ def bf16_round(v: float) -> float:
     return lib().oracle_bf16_round(v)
 
 
+def e4m3_encode(v: float) -> int:
+    """Nearest E4M3 code of a magnitude (ties to the even code, saturating at 448)."""
+    return lib().oracle_e4m3_encode(float(v))
+
+
+def e2m1_encode(v: float) -> int:
+    """Nearest E2M1 code (ties to the even code, saturating at 6; bit 3 = sign)."""
+    return lib().oracle_e2m1_encode(float(v))
+
+
+def a4_tensor_scale(x) -> float:
+    """Per-tensor scale of activations x in the A4 form: amax / (6 * 448) (1 if all zero)."""
+    xn = _np(x)
+    return float(lib().oracle_a4_tensor_scale(_p(xn), xn.size))
+
+
+def a4_quant(v, s_g: float):
+    """A4 form of rows v[n, K] (fp32, K % 16 == 0) with tensor scale s_g.
+    Returns (values, E2M1 codes [n, K], E4M3 scale codes [n, K/16])."""
+    v = np.ascontiguousarray(v, np.float32)
+    n, K = v.shape
+    out = np.empty_like(v)
+    codes = np.empty((n, K), np.uint8)
+    scales = np.empty((n, K // 16), np.uint8)
+    for r in range(n):
+        lib().oracle_a4_quant(_p(v[r]), K, float(s_g), _p(out[r]), _p(codes[r]), _p(scales[r]))
+    return out, codes, scales
+
+
 def threads() -> int:
     return lib().oracle_threads()
 
@@ -167,7 +205,7 @@ def _layer_arrays(layer):
             _np(layer.w2), _np(layer.w2_scale), _np(layer.w2_tscale, np.float32))
 
 
-def ffn(x, layer, offsets, sorted_pair, k: int, want_h: bool = False):
+def ffn(x, layer, offsets, sorted_pair, k: int, want_h: bool = False, act: str = "a16"):
     xn = _np(x)
     T, H = xn.shape
     f, w13, s13, t13, w2, s2, t2 = _layer_arrays(layer)
@@ -176,7 +214,7 @@ def ffn(x, layer, offsets, sorted_pair, k: int, want_h: bool = False):
     h = np.empty((P, layer.I), np.float32) if want_h else None
     rc = lib().oracle_ffn(_p(xn), T, H, layer.I, layer.E, k, f, _p(w13), _p(s13), _p(t13), _p(w2), _p(s2), _p(t2),
                           _p(np.ascontiguousarray(offsets, np.int32)), _p(np.ascontiguousarray(sorted_pair, np.int32)),
-                          _p(y), _p(h))
+                          _p(y), _p(h), ACT[act])
     if rc:
         raise ValueError("bad format")
     return (y, h) if want_h else y
@@ -191,7 +229,7 @@ def combine(y_perm: np.ndarray, pair_row: np.ndarray, w: np.ndarray, T: int, k: 
     return out
 
 
-def layer_forward(x, layer, bias="layer"):
+def layer_forward(x, layer, bias="layer", act: str = "a16"):
     """Whole layer. Returns dict(idx, w, offsets, sorted_pair, pair_row, y_perm, out)."""
     xn = _np(x)
     T, H = xn.shape
@@ -206,14 +244,15 @@ def layer_forward(x, layer, bias="layer"):
              pair_row=np.empty(P, np.int32), y_perm=np.empty((P, H), np.float32), out=np.empty((T, H), np.float32))
     rc = lib().oracle_layer(_p(xn), T, H, _p(wrn), int(wrn.dtype == np.float32), _p(bn), layer.E, k, layer.I, f,
                             _p(w13), _p(s13), _p(t13), _p(w2), _p(s2), _p(t2), _p(r["idx"]), _p(r["w"]),
-                            _p(r["offsets"]), _p(r["sorted_pair"]), _p(r["pair_row"]), _p(r["y_perm"]), _p(r["out"]))
+                            _p(r["offsets"]), _p(r["sorted_pair"]), _p(r["pair_row"]), _p(r["y_perm"]), _p(r["out"]),
+                            ACT[act])
     if rc:
         raise ValueError("bad format")
     return r
 
 
-def token_rows(x, layer, idx, w, tokens):
-    """out rows for the listed tokens given the batch routing (idx, w)."""
+def token_rows(x, layer, idx, w, tokens, act: str = "a16"):
+    """out rows for the listed tokens given the batch routing (idx, w); x is the whole batch."""
     xn = _np(x)
     T, H = xn.shape
     f, w13, s13, t13, w2, s2, t2 = _layer_arrays(layer)
@@ -221,7 +260,7 @@ def token_rows(x, layer, idx, w, tokens):
     out = np.empty((len(toks), H), np.float32)
     rc = lib().oracle_token_rows(_p(xn), H, layer.I, layer.k, f, _p(w13), _p(s13), _p(t13), _p(w2), _p(s2), _p(t2),
                                  _p(np.ascontiguousarray(idx, np.int32)), _p(np.ascontiguousarray(w, np.float32)),
-                                 _p(toks), len(toks), _p(out))
+                                 _p(toks), len(toks), _p(out), T, ACT[act])
     if rc:
         raise ValueError("bad format")
     return out

@@ -47,6 +47,7 @@
 #endif
 
 enum { OF_BF16 = 0, OF_FP8 = 1, OF_MXFP4 = 2, OF_NVFP4 = 3 };
+enum { ACT_A16 = 0, ACT_A4 = 1 };
 
 /* ---------------------------------------------------------------- scalars */
 
@@ -144,6 +145,84 @@ static size_t scale_bytes(int fmt, int rows, int K) {
     return fmt == OF_FP8 ? 4 * (n / 128) : fmt == OF_MXFP4 ? n / 32 : fmt == OF_NVFP4 ? n / 16 : 0;
 }
 
+/* --------------------------------------------------- activation format A4 */
+
+/* READING (activation format). Besides the plain form (A16: x as given in bf16,
+ * h rounded to bf16), the layer's activations may be carried in the NVFP4 form
+ * the aimodeling.com page names among its formats ("Reported Numbers and
+ * Ecosystem Position"), so that both operands of every expert GEMM are FP4:
+ *   x: one per-tensor scale s_g = amax(|x|) / (6 * 448) over the whole [T, H]
+ *      batch (s_g = 1 when every element is 0);
+ *   h: s_g = 1 (h is quantised row by row as it is produced);
+ *   per 16 consecutive elements along K: s_b = E4M3_RN_sat((amax_b / 6) / s_g);
+ *   codes q = E2M1_RNE_sat(v / (s_b * s_g)), 0 where s_b * s_g is 0;
+ *   the value the GEMM sees is (q * s_b) * s_g.
+ * Every step is one binary32 operation in the order written. E4M3_RN_sat and
+ * E2M1_RNE_sat round to the nearest representable value, ties to the even
+ * code (mantissa bit 0), and clamp magnitudes beyond the largest value (448,
+ * 6) to it. */
+
+/* Nearest E4M3 code of a magnitude v >= 0 (ties to the even code, saturating). */
+static int e4m3_rn_sat(float v) {
+    if (!(v > 0.0f)) return 0;
+    if (v >= 448.0f) return 0x7E;
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(oracle_e4m3(c) - (double)v);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return best;
+}
+
+/* Nearest E2M1 code of v (ties to the even code, saturating at 6); bit 3 = sign. */
+static int e2m1_rne_sat(float v) {
+    int sgn = v < 0.0f ? 8 : 0;
+    double a = fabs((double)v);
+    if (a >= 6.0) return 7 | sgn;   /* saturate (far beyond 6 the distances would tie in binary64) */
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        double d = fabs(oracle_e2m1(c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return best | sgn;
+}
+
+int oracle_e4m3_encode(float v) { return e4m3_rn_sat(v); }
+int oracle_e2m1_encode(float v) { return e2m1_rne_sat(v); }
+
+/* Per-tensor scale of x in A4 form: amax(|x|) / (6 * 448), or 1 for an all-zero x. */
+float oracle_a4_tensor_scale(const uint16_t *x, size_t n) {
+    float amax = 0.0f;
+    for (size_t i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(bf16_to_f32(x[i])));
+    return amax > 0.0f ? amax / (6.0f * 448.0f) : 1.0f;
+}
+
+/* A4 form of v[K] (K a multiple of 16) with tensor scale s_g: out = (q * s_b) * s_g;
+ * codes (nullable) get the E2M1 codes, scales (nullable) the E4M3 codes, one per block. */
+void oracle_a4_quant(const float *v, int K, float s_g, float *out, uint8_t *codes, uint8_t *scales) {
+    for (int b = 0; b < K; b += 16) {
+        float amax = 0.0f;
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[b + i]));
+        int sc = e4m3_rn_sat((amax / 6.0f) / s_g);
+        float sb = (float)oracle_e4m3(sc);
+        float den = sb * s_g;
+        if (scales) scales[b / 16] = (uint8_t)sc;
+        for (int i = 0; i < 16; ++i) {
+            int q = den > 0.0f ? e2m1_rne_sat(v[b + i] / den) : 0;
+            if (codes) codes[b + i] = (uint8_t)q;
+            out[b + i] = ((float)oracle_e2m1(q) * sb) * s_g;
+        }
+    }
+}
+
 /* ---------------------------------------------------------------- router */
 
 /* Router logits, top-k and gating for T tokens.
@@ -231,19 +310,25 @@ static float silu(float z) { return z / (1.0f + expf(-z)); }
  * READING: h is rounded to bf16 (to nearest even) before the down projection;
  * y = h.W2^T in binary32. w13f [2I, H] (gate rows then up rows), w2f [H, I]. */
 static void ffn_rows(const uint16_t *x, const int32_t *tok_of_row, int nrows, int H, int I, const float *w13f,
-                     const float *w2f, float *hbuf, float *y, float *h_out) {
+                     const float *w2f, float *hbuf, float *y, float *h_out, int act, float s_gx) {
     float *xr = (float *)malloc(sizeof(float) * H);
     for (int r = 0; r < nrows; ++r) {
         int t = tok_of_row[r];
         for (int c = 0; c < H; ++c) xr[c] = bf16_to_f32(x[(size_t)t * H + c]);
+        if (act == ACT_A4) oracle_a4_quant(xr, H, s_gx, xr, 0, 0);   /* READING: activation format A4 */
         for (int i = 0; i < I; ++i) {
             float g = 0.0f, u = 0.0f;
             const float *wg = w13f + (size_t)i * H, *wu = w13f + (size_t)(I + i) * H;
             for (int c = 0; c < H; ++c) g += xr[c] * wg[c];
             for (int c = 0; c < H; ++c) u += xr[c] * wu[c];
             float hv = bf16_to_f32(f32_to_bf16(silu(g) * u));
+            if (act == ACT_A4) hv = silu(g) * u;   /* quantised below, with the whole row */
             hbuf[i] = hv;
             if (h_out) h_out[(size_t)r * I + i] = hv;
+        }
+        if (act == ACT_A4) {
+            oracle_a4_quant(hbuf, I, 1.0f, hbuf, 0, 0);
+            if (h_out) memcpy(h_out + (size_t)r * I, hbuf, sizeof(float) * I);
         }
         for (int j = 0; j < H; ++j) {
             float acc = 0.0f;
@@ -261,9 +346,10 @@ static void ffn_rows(const uint16_t *x, const int32_t *tok_of_row, int nrows, in
  * Returns 0, or -1 on a bad format. */
 int oracle_ffn(const uint16_t *x, int T, int H, int I, int E, int k, int fmt, const void *w13, const void *w13s,
                const float *w13t, const void *w2, const void *w2s, const float *w2t, const int32_t *offsets,
-               const int32_t *sorted_pair, float *y_perm, float *h_out) {
+               const int32_t *sorted_pair, float *y_perm, float *h_out, int act) {
     size_t b13 = tensor_bytes(fmt, 2 * I, H), s13 = scale_bytes(fmt, 2 * I, H);
     size_t b2 = tensor_bytes(fmt, H, I), s2 = scale_bytes(fmt, H, I);
+    float s_gx = act == ACT_A4 ? oracle_a4_tensor_scale(x, (size_t)T * H) : 1.0f;
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int e = 0; e < E; ++e) {
@@ -279,7 +365,7 @@ int oracle_ffn(const uint16_t *x, int T, int H, int I, int E, int k, int fmt, co
                               w2t ? w2t[e] : 1.0f, w2f) != 0;
         for (int r = 0; r < n; ++r) tok[r] = sorted_pair[offsets[e] + r] / k;
         ffn_rows(x, tok, n, H, I, w13f, w2f, hbuf, y_perm + (size_t)offsets[e] * H,
-                 h_out ? h_out + (size_t)offsets[e] * I : 0);
+                 h_out ? h_out + (size_t)offsets[e] * I : 0, act, s_gx);
         free(w13f);
         free(w2f);
         free(hbuf);
@@ -313,7 +399,7 @@ void oracle_combine(const float *y_perm, const int32_t *pair_row, const float *w
 int oracle_layer(const uint16_t *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E, int k,
                  int I, int fmt, const void *w13, const void *w13s, const float *w13t, const void *w2,
                  const void *w2s, const float *w2t, int32_t *idx_out, float *w_out, int32_t *offsets_out,
-                 int32_t *sorted_out, int32_t *pair_row_out, float *y_perm_out, float *out) {
+                 int32_t *sorted_out, int32_t *pair_row_out, float *y_perm_out, float *out, int act) {
     int P = T * k;
     int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (P ? P : 1));
     float *w = (float *)malloc(sizeof(float) * (P ? P : 1));
@@ -323,7 +409,7 @@ int oracle_layer(const uint16_t *x, int T, int H, const void *wr, int wr_is_fp32
     float *y = (float *)malloc(sizeof(float) * (size_t)(P ? P : 1) * H);
     oracle_route(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, 0);
     oracle_permute(idx, T, k, E, off, sp, pr);
-    int rc = oracle_ffn(x, T, H, I, E, k, fmt, w13, w13s, w13t, w2, w2s, w2t, off, sp, y, 0);
+    int rc = oracle_ffn(x, T, H, I, E, k, fmt, w13, w13s, w13t, w2, w2s, w2t, off, sp, y, 0, act);
     oracle_combine(y, pr, w, T, k, H, out);
     if (idx_out) memcpy(idx_out, idx, sizeof(int32_t) * P);
     if (w_out) memcpy(w_out, w, sizeof(float) * P);
@@ -346,9 +432,10 @@ int oracle_layer(const uint16_t *x, int T, int H, const void *wr, int wr_is_fp32
  * independent of T. Used to check full-size runs on sampled outputs. */
 int oracle_token_rows(const uint16_t *x, int H, int I, int k, int fmt, const void *w13, const void *w13s,
                       const float *w13t, const void *w2, const void *w2s, const float *w2t, const int32_t *idx,
-                      const float *w, const int32_t *tokens, int ntok, float *out_rows) {
+                      const float *w, const int32_t *tokens, int ntok, float *out_rows, int T, int act) {
     size_t b13 = tensor_bytes(fmt, 2 * I, H), s13 = scale_bytes(fmt, 2 * I, H);
     size_t b2 = tensor_bytes(fmt, H, I), s2 = scale_bytes(fmt, H, I);
+    float s_gx = act == ACT_A4 ? oracle_a4_tensor_scale(x, (size_t)T * H) : 1.0f;   /* over the whole batch */
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int i = 0; i < ntok; ++i) {
@@ -366,7 +453,7 @@ int oracle_token_rows(const uint16_t *x, int H, int I, int k, int fmt, const voi
             bad |= oracle_dequant(fmt, H, I, (const char *)w2 + e * b2, w2s ? (const char *)w2s + e * s2 : 0,
                                   w2t ? w2t[e] : 1.0f, w2f) != 0;
             int32_t tok = t;
-            ffn_rows(x, &tok, 1, H, I, w13f, w2f, hbuf, y, 0);
+            ffn_rows(x, &tok, 1, H, I, w13f, w2f, hbuf, y, 0, act, s_gx);
             for (int c = 0; c < H; ++c) acc[c] += w[(size_t)t * k + j] * y[c];
         }
         free(w13f);

@@ -190,31 +190,6 @@ def test_prefetch_depths_full_layers_and_resizes_match_the_simulation(lib, block
     assert moves > 0
 
 
-def test_resize_by_hand():
-    """Hand-worked: 4 slots hold (0,0) (0,1) (0,2) (0,3), referenced in that order.
-    Shrinking to 2 keeps the two most recent, (0,2) and (0,3), which sit in slots 2 and
-    3 and move, least recent first, to the free slots 0 and 1. Growing back to 3 adds
-    one free slot, which the next miss takes."""
-    sim = LruSim(4, 1, 8, 1)
-    for e in range(4):
-        sim.resolve(0, [e])
-    assert sim.resize(2) == [(2, 0), (3, 1)]
-    assert sim.table()[:4] == [-1, -1, 0, 1]
-    assert sim.resize(3) == []
-    assert sim.resolve(0, [5]) == [(5, 2)]
-
-
-def test_prediction_ranks_by_pair_count_by_hand():
-    """Experts 4 (three pairs), 1 (two), 6 and 2 (one each): depth 2 takes 4 and 1, depth 3
-    adds 2 (ties to the lower id)."""
-    sim = LruSim(16, 2, 8, 1)
-    sim.resolve(1, [4, 1, 6, 4, 2, 1, 4])
-    assert sim.predict(1, 2) == [1, 4]
-    assert sim.predict(1, 3) == [1, 2, 4]
-    assert sim.predict(1, -1) == [1, 2, 4, 6]
-    assert sim.predict(1, 0, full=True) == list(range(8))
-
-
 def test_prefetch_plan(lib):
     """The per-call decision: fixed policies pass through; the adaptive one streams the
     whole next layer when the call is expected to reach half of the experts, else the

@@ -411,3 +411,152 @@ def test_lru_large_cache_never_evicts():
             sim.resolve(l, ids)
             seen |= {(l, int(e)) for e in ids}
     assert sim.misses == len(seen) and sim.loads == len(seen)
+
+
+# ----------------------------------------------------------------------------- activation format A4
+
+
+def test_e2m1_encode_ties_saturation_and_identity():
+    """The A4 rounding of activations: nearest E2M1 value, ties to the even code (the
+    hand-worked cases 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4), magnitudes
+    beyond 6 clamp to 6, and every representable value maps to its own code."""
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6, -0.75: 10, -5.0: 14}
+    for v, c in ties.items():
+        assert oracle.e2m1_encode(v) == c, v
+    for v in (6.5, 7.0, 100.0, 1e30):
+        assert oracle.e2m1_encode(v) == 7 and oracle.e2m1_encode(-v) == 15
+    tab = _e2m1_table()
+    for c, v in tab.items():
+        if v != 0.0:
+            assert oracle.e2m1_encode(v) == c
+    assert oracle.e2m1_encode(0.24) == 0 and oracle.e2m1_encode(0.26) == 1
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    """E4M3 round-to-nearest-even of scale values against torch's float8_e4m3fn cast on
+    random magnitudes and on every exact midpoint between neighbouring values; beyond 448
+    the scale saturates."""
+    g = np.random.default_rng(5)
+    vals = np.concatenate([np.exp2(g.uniform(-12, 8.8, 3000)), g.uniform(0, 448, 1000)]).astype(np.float32)
+    grid = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)
+    vals = np.concatenate([vals, mids[(mids.astype(np.float64) == (grid[1:] + grid[:-1]) / 2)]])
+    want = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in vals])
+    assert np.array_equal(got, want)
+    for v in (448.0, 449.0, 463.9, 1e6):
+        assert oracle.e4m3_encode(v) == 0x7E
+    assert oracle.e4m3_encode(0.0) == 0
+
+
+def test_a4_tensor_scale_is_amax_over_6_times_448():
+    x = synthetic.make_tokens(5, 64, 3)
+    amax = float(x.float().abs().max())
+    assert oracle.a4_tensor_scale(x) == float(np.float32(amax) / np.float32(2688.0))
+    assert oracle.a4_tensor_scale(torch.zeros(3, 16, dtype=torch.bfloat16)) == 1.0
+
+
+def test_a4_blocks_hand_worked():
+    for line in open(os.path.join(GOLDEN, "a4_blocks.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        sg, v, sc, codes, vals = [p.split() for p in line.split("|")]
+        out, c, s = oracle.a4_quant(np.array([[float(t) for t in v]], np.float32), float(sg[0]))
+        assert s[0, 0] == int(sc[0]), line
+        assert c[0].tolist() == [int(t) for t in codes], line
+        assert out[0].tolist() == [float(t) for t in vals], line
+
+
+def test_a4_round_trip_of_representable_values_is_the_identity():
+    """Blocks built as q * s_b * s_g from E2M1 values q (largest 6) and power-of-two scales
+    come back unchanged."""
+    g = np.random.default_rng(6)
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    for s_g in (1.0, 2.0 ** -10, 2.0 ** 3):
+        q = mags[g.integers(0, 8, (8, 64))] * np.where(g.random((8, 64)) < 0.5, -1, 1).astype(np.float32)
+        q[:, ::16] = 6.0
+        sb = np.exp2(g.integers(-6, 8, (8, 4))).astype(np.float32)
+        v = (q.reshape(8, 4, 16) * sb[..., None] * np.float32(s_g)).reshape(8, 64).astype(np.float32)
+        out, _, _ = oracle.a4_quant(v, s_g)
+        assert np.array_equal(out, v)
+
+
+def _a4_np(v, s_g):
+    """Independent A4 form of fp32 rows v[n, K]: torch's float8_e4m3fn cast for the scales
+    and the input generator's E2M1 encoder for the codes."""
+    v = np.asarray(v, np.float32)
+    n, K = v.shape
+    b = v.reshape(n, K // 16, 16)
+    amax = np.abs(b).max(-1).astype(np.float32)
+    t = ((amax / np.float32(6.0)) / np.float32(s_g)).astype(np.float32)
+    sb = torch.from_numpy(np.minimum(t, np.float32(448.0))).to(torch.float8_e4m3fn).float().numpy()
+    den = (sb * np.float32(s_g)).astype(np.float32)
+    arg = np.where(den[..., None] > 0, b / np.where(den > 0, den, 1)[..., None], 0).astype(np.float32)
+    codes = synthetic.gen._e2m1_encode(torch.from_numpy(arg)).numpy()
+    tab = _e2m1_table()
+    q = np.vectorize(tab.get)(codes).astype(np.float32)
+    return ((q * sb[..., None]).astype(np.float32) * np.float32(s_g)).astype(np.float32).reshape(n, K)
+
+
+def test_a4_layer_matches_per_token_brute_force():
+    """NVFP4 layer in the A4 activation form against an fp64 per-token evaluation whose
+    decoder and quantiser are written independently: x quantised with the batch's tensor
+    scale, h (computed, then rounded to fp32) quantised with tensor scale 1."""
+    H, I, E, k = 128, 64, 4, 2
+    L = synthetic.make_layer(dict(H=H, E=E, k=k, I=I, fmt="nvfp4"), 13)
+    x = synthetic.make_tokens(6, H, 13)
+    r = oracle.layer_forward(x, L, act="a4")
+    s_g = np.float32(float(x.float().abs().max())) / np.float32(2688.0)
+    xq = _a4_np(x.float().numpy(), s_g).astype(np.float64)
+    w13 = [_decode_np("nvfp4", L.w13[e], L.w13_scale[e], L.w13_tscale[e]) for e in range(E)]
+    w2 = [_decode_np("nvfp4", L.w2[e], L.w2_scale[e], L.w2_tscale[e]) for e in range(E)]
+    out = np.zeros((6, H))
+    for t in range(6):
+        for j in range(k):
+            e = r["idx"][t, j]
+            g = w13[e][:I] @ xq[t]
+            u = w13[e][I:] @ xq[t]
+            h = _a4_np((g / (1 + np.exp(-g)) * u).astype(np.float32)[None], 1.0)[0].astype(np.float64)
+            out[t] += r["w"][t, j] * (w2[e] @ h)
+    assert np.abs(r["out"] - out).max() <= 1e-3 * np.abs(out).max()
+    # the token-row path agrees with the layer path (the tensor scale comes from the whole batch)
+    rows = oracle.token_rows(x, L, r["idx"], r["w"], [1, 5], act="a4")
+    assert np.array_equal(rows, r["out"][[1, 5]])
+
+
+def test_a4_changes_the_layer_by_the_quantisation_error():
+    """The A4 form is a different computation from A16: on an NVFP4 layer the two differ
+    by a few percent (FP4 activations), not by rounding noise, and not by more than 25%."""
+    L = synthetic.make_layer(dict(H=256, E=8, k=2, I=256, fmt="nvfp4"), 14)
+    x = synthetic.make_tokens(16, 256, 14)
+    a16 = oracle.layer_forward(x, L)["out"]
+    a4 = oracle.layer_forward(x, L, act="a4")["out"]
+    d = np.abs(a4 - a16).max() / np.abs(a16).max()
+    assert 5e-3 < d < 0.25, d
+
+
+def test_lru_resize_by_hand():
+    """4 slots hold (0,0) (0,1) (0,2) (0,3), referenced in that order. Shrinking to 2 keeps
+    the two most recent, (0,2) and (0,3), which sit in slots 2 and 3 and move, least recent
+    first, to the free slots 0 and 1. Growing to 3 adds one free slot, which the next miss
+    takes; shrinking to 1 keeps the most recent expert only."""
+    sim = LruSim(4, 1, 8, 1)
+    for e in range(4):
+        sim.resolve(0, [e])
+    assert sim.resize(2) == [(2, 0), (3, 1)]
+    assert sim.table()[:4] == [-1, -1, 0, 1]
+    assert sim.resize(3) == []
+    assert sim.resolve(0, [5]) == [(5, 2)]
+    assert sim.resize(1) == [(2, 0)]
+    assert sim.table()[5] == 0 and sum(v >= 0 for v in sim.table()) == 1
+
+
+def test_lru_prediction_ranks_by_pair_count_by_hand():
+    """Experts 4 (three pairs), 1 (two), 6 and 2 (one each): depth 2 takes 4 and 1, depth 3
+    adds 2 (ties to the lower id); the whole layer is every expert."""
+    sim = LruSim(16, 2, 8, 1)
+    sim.resolve(1, [4, 1, 6, 4, 2, 1, 4])
+    assert sim.predict(1, 2) == [1, 4]
+    assert sim.predict(1, 3) == [1, 2, 4]
+    assert sim.predict(1, -1) == [1, 2, 4, 6]
+    assert sim.predict(1, 0, full=True) == list(range(8))

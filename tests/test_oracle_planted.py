@@ -89,6 +89,28 @@ C_PLANTS = [
     ("w2_scale_of_expert_0", "w2s ? (const char *)w2s + e * s2 : 0,", "w2s ? (const char *)w2s : 0,", 2),
     ("w13_tensor_scale_of_expert_0", "w13t ? w13t[e] : 1.0f", "w13t ? w13t[0] : 1.0f", 2),
     ("w2_tensor_scale_of_expert_0", "w2t ? w2t[e] : 1.0f", "w2t ? w2t[0] : 1.0f", 2),
+    # activation format A4
+    ("a4_e2m1_ties_to_odd", "if (d < bd || (d == bd && (c & 1) == 0)) {\n            best = c;\n            bd = d;\n"
+     "        }\n    }\n    return best | sgn;",
+     "if (d < bd || (d == bd && (c & 1) == 1)) {\n            best = c;\n            bd = d;\n"
+     "        }\n    }\n    return best | sgn;"),
+    ("a4_e4m3_ties_to_odd", "if (d < bd || (d == bd && (c & 1) == 0)) {\n            best = c;\n            bd = d;\n"
+     "        }\n    }\n    return best;",
+     "if (d < bd || (d == bd && (c & 1) == 1)) {\n            best = c;\n            bd = d;\n"
+     "        }\n    }\n    return best;"),
+    ("a4_e2m1_saturates_at_4", "if (a >= 6.0) return 7 | sgn;", "if (a >= 4.0) return 6 | sgn;"),
+    ("a4_tensor_scale_without_6", "amax / (6.0f * 448.0f)", "amax / 448.0f"),
+    ("a4_block_scale_without_6", "int sc = e4m3_rn_sat((amax / 6.0f) / s_g);", "int sc = e4m3_rn_sat(amax / s_g);"),
+    ("a4_block_amax_first_half", "for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[b + i]));",
+     "for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[b + i]));"),
+    ("a4_block_scale_not_rounded", "float sb = (float)oracle_e4m3(sc);",
+     "float sb = (amax / 6.0f) / s_g; (void)sc;"),
+    ("a4_x_not_quantised", "if (act == ACT_A4) oracle_a4_quant(xr, H, s_gx, xr, 0, 0);", ""),
+    ("a4_h_with_the_tensor_scale_of_x", "oracle_a4_quant(hbuf, I, 1.0f, hbuf, 0, 0);",
+     "oracle_a4_quant(hbuf, I, s_gx, hbuf, 0, 0);"),
+    ("a4_h_not_quantised", "            oracle_a4_quant(hbuf, I, 1.0f, hbuf, 0, 0);\n", ""),
+    ("a4_tensor_scale_of_first_token", "oracle_a4_tensor_scale(x, (size_t)T * H)", "oracle_a4_tensor_scale(x, (size_t)H)",
+     2),
 ]
 
 # (name, exact text in lru.py, replacement).
@@ -104,6 +126,13 @@ LRU_PLANTS = [
     ("hit_not_refreshed", "                hits += 1\n", "                hits += 1\n                continue\n"),
     ("evict_ignores_layer", "            if layer >= 0 and o[0] != layer:\n                continue\n", ""),
     ("evict_ignores_ids", "            if ids is not None and o[1] not in set(ids):\n                continue\n", ""),
+    ("prediction_least_routed_first", "ranked = sorted(counts, key=lambda e: (-min(counts[e], (1 << 20) - 1), e))",
+     "ranked = sorted(counts, key=lambda e: (min(counts[e], (1 << 20) - 1), e))"),
+    ("prediction_ties_to_higher_id", "ranked = sorted(counts, key=lambda e: (-min(counts[e], (1 << 20) - 1), e))",
+     "ranked = sorted(counts, key=lambda e: (-min(counts[e], (1 << 20) - 1), -e))"),
+    ("resize_keeps_least_recent", "keep = occ[len(occ) - min(len(occ), n_slots):]", "keep = occ[:min(len(occ), n_slots)]"),
+    ("resize_moves_to_highest_free", "f = min(j for j in range(n_slots) if self.owner[j] is None)",
+     "f = max(j for j in range(n_slots) if self.owner[j] is None)"),
 ]
 
 PARAMS = {"test_permutation_is_stable_counting_sort": [(16, 2, 8), (64, 8, 128)],
