@@ -130,8 +130,8 @@ def active_expert_bytes(idx: torch.Tensor, layer) -> int:
 class LayerBench:
     """One layer configuration: NSETS weight copies, NSETS token batches, a graph per pair."""
 
-    def __init__(self, moe, cfg: str, T: int, device, seed: int = 0, nsets: int = NSETS):
-        self.moe, self.cfg, self.T, self.dev = moe, cfg, T, device
+    def __init__(self, moe, cfg: str, T: int, device, seed: int = 0, nsets: int = NSETS, act: str = "a16"):
+        self.moe, self.cfg, self.T, self.dev, self.act = moe, cfg, T, device, act
         c = synthetic.CONFIGS[cfg]
         self.k, self.y32 = c["k"], c["y_fp32"]
         base = synthetic.make_layer(cfg, seed, device=device)
@@ -159,7 +159,7 @@ class LayerBench:
         j = i % len(self.sets)
         s = self.sets[j]
         self.moe.moe_layer_forward(self.xs[j], s.wr, self.k, self.experts[j], bias=s.bias, y_fp32=self.y32,
-                                   ws=self.ws, out=self.out, idx_out=self.idx[j], w_out=self.w[j])
+                                   ws=self.ws, out=self.out, idx_out=self.idx[j], w_out=self.w[j], act=self.act)
 
     def capture(self):
         self.graphs = []
@@ -275,6 +275,21 @@ def traffic_for(key: str):
 
 
 # ------------------------------------------------------------------------------------------- arms
+
+
+def tensor_peaks(moe) -> dict:
+    """Dense tensor-core peaks of this GPU for the FFN's MMA kinds, from the library's own
+    MMA loop (tcgen05, operands resident in shared memory, no memory traffic): TFLOP/s."""
+    out = {}
+    fn = getattr(moe, "moe_tensor_peak_tflops", None)
+    if fn is None:
+        return out
+    for kind in ("bf16", "fp8", "mxfp4", "nvfp4"):
+        try:
+            out[f"{kind}_tflops"] = fn(kind)
+        except Exception as exc:   # report, do not fail the bench
+            out[f"{kind}_error"] = str(exc)[:120]
+    return out
 
 
 def cpu_oracle_tokens_per_s(cfg: str, T: int, budget_s: float = 12.0):
@@ -577,21 +592,41 @@ def run_ours(args, rank, world, device):
     # side measurements (not the headline): other batch sizes, the prefill-shaped and large layers,
     # and the streaming stack
     if not args.quick and world == 1:   # the side workloads run on one GPU only
-        for cfg, T in (("decode", 1), ("decode", 8), ("prefill", 4096), ("large", 32), ("large", 8192)):
+        peaks = tensor_peaks(moe)
+        extra["tensor_peaks"] = peaks
+        outs = {}
+        for cfg, T, act in (("decode", 1, "a16"), ("decode", 8, "a16"), ("prefill", 4096, "a16"),
+                            ("prefill", 4096, "a4"), ("large", 32, "a16"), ("large", 32, "a4"),
+                            ("large", 8192, "a16"), ("large", 8192, "a4")):
             nsets = NSETS if cfg == "decode" else (2 if cfg == "large" else 4)
-            b = lb if (cfg == "decode" and T == 64) else LayerBench(moe, cfg, T, device, nsets=nsets)
+            b = lb if (cfg == "decode" and T == 64) else LayerBench(moe, cfg, T, device, nsets=nsets, act=act)
             b.capture()
             nsteps = max(10, args.steps // 2) if T < 8192 else max(10, min(args.steps // 2, 40))
             s = time_steps(b.step, nsteps, args.warmup, device, barrier)
             ms_b = s / nsteps * 1e3
             n_alg = [b.algorithmic_bytes(args.warmup + i) for i in range(min(8, len(b.sets)))]
             gbs = sum(n_alg) / len(n_alg) / (ms_b * 1e-3) / 1e9
-            extra[f"{cfg}_T{T}"] = {"tokens_per_s": T / (ms_b * 1e-3) * world, "ms_per_layer": ms_b,
-                                    "layer_gbs": gbs, "frac_hbm": gbs / hbm,
-                                    "tflops": b.flops() / (ms_b * 1e-3) / 1e12,
-                                    "frac_bf16_peak": b.flops() / (ms_b * 1e-3) / 1e12 / bf16_tf}
+            tf = b.flops() / (ms_b * 1e-3) / 1e12
+            key = f"{cfg}_T{T}" + ("_a4" if act == "a4" else "")
+            extra[key] = {"tokens_per_s": T / (ms_b * 1e-3) * world, "ms_per_layer": ms_b, "act": act,
+                          "layer_gbs": gbs, "frac_hbm": gbs / hbm, "tflops": tf, "frac_bf16_peak": tf / bf16_tf}
+            if cfg != "decode":
+                # the FP4-weight layers against the dense FP4 tensor peak measured above (the
+                # format's own peak applies to A4, where both operands are FP4)
+                if peaks.get("nvfp4_tflops"):
+                    extra[key]["frac_fp4_peak"] = tf / peaks["nvfp4_tflops"]
+                b.call(0)
+                torch.cuda.synchronize(device)
+                outs[(cfg, T, act)] = b.out.float().clone()
             del b
             torch.cuda.empty_cache()
+        # the A4 form is a different computation: its distance from A16 on the same inputs
+        # (GPU outputs of both) is quantisation error, reported beside the parity tests'
+        # oracle comparison
+        for cfg, T in (("prefill", 4096), ("large", 32), ("large", 8192)):
+            a, q = outs.get((cfg, T, "a16")), outs.get((cfg, T, "a4"))
+            if a is not None and q is not None:
+                extra[f"{cfg}_T{T}_a4"]["a4_vs_a16_max_rel"] = float((q - a).abs().max() / a.abs().max())
         extra["stack"] = run_stack(moe, device, args.stack_steps)
         extra["prefill_stack"] = run_prefill_stack(moe, device)
 
@@ -621,8 +656,8 @@ def run_profile(args, device):
     """W + K plain (non-graph) layer forwards of one workload; for ncu launch lists."""
     import expert_ffn_layer_top_b200 as moe
 
-    cfg, T = args.profile.split(":")
-    lb = LayerBench(moe, cfg, int(T), device, nsets=4)
+    cfg, T, *rest = args.profile.split(":")
+    lb = LayerBench(moe, cfg, int(T), device, nsets=4, act=rest[0] if rest else "a16")
     for i in range(args.warmup + args.steps):
         lb.call(i)
     torch.cuda.synchronize(device)
@@ -638,7 +673,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--stack-steps", type=int, default=512, help="decode steps of the streaming-stack run")
-    ap.add_argument("--profile", default=None, help="plain launches of one workload (cfg:T, e.g. decode:64) for ncu")
+    ap.add_argument("--profile", default=None, help="plain launches of one workload (cfg:T[:act], e.g. decode:64 or prefill:4096:a4) for ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -7,6 +7,7 @@ CUDA kernels. There is no fallback: if the library cannot be loaded, every call
 raises.
 """
 from ._lib import (  # noqa: F401
+    ACT,
     FMT,
     ExpertCache,
     Experts,
@@ -21,6 +22,7 @@ from ._lib import (  # noqa: F401
     moe_permute_static,
     moe_prepack,
     moe_selftest_wait,
+    moe_tensor_peak_tflops,
     moe_set_wait_limit_ns,
     PREFETCH,
     moe_prepacked_expert_bytes,

@@ -11,6 +11,7 @@ import torch
 from . import build as _build
 
 FMT = {"bf16": 0, "fp8": 1, "mxfp4": 2, "nvfp4": 3}
+ACT = {"a16": 0, "a4": 1}
 _STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "OOM", 5: "TIMEOUT", 6: "CACHE_FULL"}
 
 _P = C.c_void_p
@@ -66,24 +67,24 @@ def lib():
             L.moe_route_topk.restype = st
             L.moe_route_topk.argtypes = [_P, _I, _I, _P, _I, _P, _I, _I, _P, _P, _P, _P, C.c_size_t, _P]
             L.moe_permute.restype = st
-            L.moe_permute.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, C.c_size_t, _P]
+            L.moe_permute.argtypes = [_P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _P, _P, C.c_size_t, _P]
             L.moe_permute_static.restype = st
             L.moe_permute_static.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P]
             L.moe_grouped_ffn.restype = st
-            L.moe_grouped_ffn.argtypes = [_P, _I, _P, C.POINTER(_Experts), _P, _I, _P, C.c_size_t, _P]
+            L.moe_grouped_ffn.argtypes = [_P, _I, _P, C.POINTER(_Experts), _I, _P, _I, _P, C.c_size_t, _P]
             L.moe_combine.restype = st
             L.moe_combine.argtypes = [_P, _I, _P, _P, _I, _I, _I, _P, _P]
             L.moe_dequantize.restype = st
             L.moe_dequantize.argtypes = [_I, _P, _P, C.c_float, _I, _I, _P, _P]
             L.moe_layer_forward.restype = st
-            L.moe_layer_forward.argtypes = [_P, _I, _P, _I, _P, _I, C.POINTER(_Experts), _P, _I, _I, _P, _P, _P,
-                                            _P, C.c_size_t, _P]
+            L.moe_layer_forward.argtypes = [_P, _I, _P, _I, _P, _I, C.POINTER(_Experts), _I, _P, _I, _I, _P, _P,
+                                            _P, _P, C.c_size_t, _P]
             L.moe_prepacked_expert_bytes.restype = C.c_size_t
             L.moe_prepacked_expert_bytes.argtypes = [_I, _I, _I, _I]
             L.moe_prepack.restype = st
             L.moe_prepack.argtypes = [C.POINTER(_Experts), _P, _P, _P]
             L.moe_workspace_size.restype = C.c_size_t
-            L.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
+            L.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I]
             L.expert_cache_init.restype = st
             L.expert_cache_init.argtypes = [C.POINTER(_P), C.c_size_t, _I, C.POINTER(_Experts), _I]
             L.expert_cache_prefetch.restype = st
@@ -101,6 +102,8 @@ def lib():
             L.expert_cache_report.argtypes = [_P, C.POINTER(_CacheReport)]
             L.moe_set_wait_limit_ns.restype = st
             L.moe_set_wait_limit_ns.argtypes = [C.c_uint64]
+            L.moe_tensor_peak.restype = st
+            L.moe_tensor_peak.argtypes = [_I, _I, C.POINTER(C.c_double)]
             L.moe_selftest_wait.restype = st
             L.moe_selftest_wait.argtypes = [_P]
             L.expert_cache_slot_of.restype = st
@@ -164,8 +167,18 @@ def moe_selftest_wait(stream=None) -> None:
     _check(lib().moe_selftest_wait(_stream(stream)))
 
 
-def moe_workspace_size(T: int, H: int, I: int, E: int, k: int, y_fp32: bool = False) -> int:
-    return int(lib().moe_workspace_size(T, H, I, E, k, int(y_fp32)))
+_PEAK_KIND = {"bf16": 0, "fp8": 1, "mxfp4": 2, "nvfp4": 3}
+
+
+def moe_tensor_peak_tflops(kind: str, iters: int = 4000) -> float:
+    """Dense tensor-core TFLOP/s of the current device for one MMA kind (library MMA loop)."""
+    v = C.c_double()
+    _check(lib().moe_tensor_peak(_PEAK_KIND[kind], int(iters), C.byref(v)))
+    return v.value
+
+
+def moe_workspace_size(T: int, H: int, I: int, E: int, k: int, y_fp32: bool = False, act: str = "a16") -> int:
+    return int(lib().moe_workspace_size(T, H, I, E, k, int(y_fp32), ACT[act]))
 
 
 def _ws(nbytes: int, device) -> torch.Tensor:
@@ -228,7 +241,8 @@ def moe_route_topk(x: torch.Tensor, wr: torch.Tensor, k: int, bias: Optional[tor
     return (idx, w, logits) if want_logits else (idx, w)
 
 
-def moe_permute(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+def moe_permute(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                act: str = "a16"):
     _need_cuda(idx, x)
     T, k = idx.shape
     dev = idx.device
@@ -240,8 +254,8 @@ def moe_permute(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = None, ws:
     x_perm = torch.empty(max(P, 1), H, dtype=torch.bfloat16, device=dev) if x is not None else None
     if ws is None:
         ws = _ws(moe_workspace_size(T, max(H, 8), 128, E, k), dev)
-    _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(x), H, _ptr(offsets), _ptr(sp), _ptr(pr), _ptr(x_perm),
-                             _ptr(ws), ws.numel(), _stream()))
+    _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(x), H, ACT[act], _ptr(offsets), _ptr(sp), _ptr(pr),
+                             _ptr(x_perm), _ptr(ws), ws.numel(), _stream()))
     return offsets, sp[:P], pr[:P], (x_perm[:P] if x_perm is not None else None)
 
 
@@ -262,14 +276,14 @@ def moe_permute_static(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = No
 
 
 def moe_grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, experts: Experts, y_fp32: bool = False,
-                    ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+                    ws: Optional[torch.Tensor] = None, act: str = "a16") -> torch.Tensor:
     _need_cuda(x_perm, offsets)
     n = x_perm.shape[0]
     y = torch.empty(max(n, 1), experts.H, dtype=torch.float32 if y_fp32 else torch.bfloat16, device=x_perm.device)
     if ws is None:
         ws = _ws(moe_workspace_size(max(n, 1), experts.H, experts.I, experts.E, 1, y_fp32), x_perm.device)
-    _check(lib().moe_grouped_ffn(_ptr(x_perm), n, _ptr(offsets), C.byref(experts.c), _ptr(y), int(y_fp32), _ptr(ws),
-                                 ws.numel(), _stream()))
+    _check(lib().moe_grouped_ffn(_ptr(x_perm), n, _ptr(offsets), C.byref(experts.c), ACT[act], _ptr(y), int(y_fp32),
+                                 _ptr(ws), ws.numel(), _stream()))
     return y[:n]
 
 
@@ -294,7 +308,8 @@ def moe_dequantize(fmt: str, w: torch.Tensor, scale: Optional[torch.Tensor], tsc
 def moe_layer_forward(x: torch.Tensor, wr: torch.Tensor, k: int, experts: Experts,
                       bias: Optional[torch.Tensor] = None, cache: Optional["ExpertCache"] = None, layer: int = 0,
                       y_fp32: bool = False, ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                      idx_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                      idx_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None,
+                      act: str = "a16") -> torch.Tensor:
     _need_cuda(x, wr, bias, ws, out, idx_out, w_out)
     T, H = x.shape
     if out is None:
@@ -302,7 +317,7 @@ def moe_layer_forward(x: torch.Tensor, wr: torch.Tensor, k: int, experts: Expert
     if ws is None:
         ws = _ws(moe_workspace_size(T, H, experts.I, experts.E, k, y_fp32), x.device)
     _check(lib().moe_layer_forward(_ptr(x), T, _ptr(wr), int(wr.dtype == torch.float32), _ptr(bias), k,
-                                   C.byref(experts.c), cache.handle if cache is not None else None, layer,
+                                   C.byref(experts.c), ACT[act], cache.handle if cache is not None else None, layer,
                                    int(y_fp32), _ptr(out), _ptr(idx_out), _ptr(w_out), _ptr(ws), ws.numel(),
                                    _stream()))
     return out

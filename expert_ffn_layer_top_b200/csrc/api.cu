@@ -2,6 +2,7 @@
 // workspace carving, TMA descriptor construction and kernel launches.
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -215,20 +216,23 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 // atoms) of x and of h; NVFP4 also keeps h in bf16 at offset 0 and the per-row
 // exponent offsets of x and h.
 struct FfnWs {
-    size_t h, re1, re2, b1, b2, total;
+    size_t h, re1, re2, a4, b1, b2, total;
 };
 
 // h: bf16 [n][I] (the decoding paths' h buffer; NVFP4: h before its
-// quantisation); re1, re2: NVFP4 per-row exponent offsets of x and h; b1, b2:
-// activation blobs of x and h for the block-scaled FP4 path.
+// quantisation); re1, re2: NVFP4 per-row exponent offsets of x and h; a4: the A4
+// tensor scale of x, then the partial maxima of |x|; b1, b2: activation blobs of
+// x and h for the block-scaled FP4 path (four planes, or one in A4 form: the
+// larger of the two sizes).
 static FfnWs ffn_ws(int n, int H, int I, int E) {
     FfnWs W;
     size_t o = 0;
     W.h = o; o += align_up((size_t)n * I * 2, 256);
     W.re1 = o; o += align_up((size_t)n * 4, 256);
     W.re2 = o; o += align_up((size_t)n * 4, 256);
-    W.b1 = o; o += mx_blob_bytes(n, H, E);
-    W.b2 = o; o += mx_blob_bytes(n, I, E);
+    W.a4 = o; o += align_up((size_t)(1 + kA4Parts) * 4, 256);
+    W.b1 = o; o += std::max(mx_blob_bytes(n, H, E), a4_blob_bytes(n, H, E));
+    W.b2 = o; o += std::max(mx_blob_bytes(n, I, E), a4_blob_bytes(n, I, E));
     W.total = o;
     return W;
 }
@@ -298,6 +302,59 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
+}
+
+// A4 grouped FFN (activations in NVFP4 form; prepacked NVFP4 experts). The tensor
+// scale of x comes from the rows the maxima are taken over: the token rows x [T][H]
+// when gathering (every token appears k times among the pairs), else x_perm.
+static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_src, int64_t amax_elems,
+                              const int32_t *sorted_pair, int k, int n_rows, const int32_t *offsets,
+                              const moe_experts *x, void *y_perm, int y_is_fp32, void *ws, cudaStream_t st) {
+    if (n_rows == 0) return MOE_OK;
+    if (x->fmt != MOE_NVFP4 || x->layout != MOE_LAYOUT_TILED)
+        return set_error(MOE_ERR_UNSUPPORTED, "A4 activations need prepacked NVFP4 experts");
+    const int E = x->E, H = x->H, I = x->I;
+    const Strides s = default_strides(*x);
+    const int BN = choose_bn_a4(n_rows, E);
+    const int nsm = num_sms(current_device());
+    const FfnWs W = ffn_ws(n_rows, H, I, E);
+    uint8_t *b = reinterpret_cast<uint8_t *>(ws);
+    float *xscale = reinterpret_cast<float *>(b + W.a4), *parts = xscale + 1;
+    moe_status r = launch_a4_amax(amax_src, amax_elems, parts, st);
+    if (r == MOE_OK)
+        r = launch_a4_quant(x_src, gather ? 1 : 2, sorted_pair, k, n_rows, H, offsets, E, BN, parts, xscale, b + W.b1,
+                            nsm, st);
+    if (r != MOE_OK) return r;
+    MxParams p;
+    memset(&p, 0, sizeof(p));
+    p.offsets = offsets;
+    p.expert_map = x->expert_map;
+    p.E = E;
+    p.H = H;
+    p.I = I;
+    p.n_rows = n_rows;
+    // ---- gate/up + SwiGLU; the epilogue writes h in A4 form for the down pass
+    p.K = H;
+    p.m_tiles = I / 64;
+    p.wbase = reinterpret_cast<const uint8_t *>(x->w13);
+    p.w_estride = s.w13;
+    p.bblob = b + W.b1;
+    p.tscale = x->w13_tscale;
+    p.bblob_out = b + W.b2;
+    p.xscale = xscale;
+    if ((r = launch_mx_phase(kBsNv, kPhaseUp, BN, p, nsm, st, 1)) != MOE_OK) return r;
+    // ---- down projection
+    p.K = I;
+    p.m_tiles = H / 128;
+    p.wbase = reinterpret_cast<const uint8_t *>(x->w2);
+    p.w_estride = s.w2;
+    p.bblob = b + W.b2;
+    p.tscale = x->w2_tscale;
+    p.bblob_out = nullptr;
+    p.xscale = nullptr;
+    p.out = y_perm;
+    p.out_fp32 = y_is_fp32;
+    return launch_mx_phase(kBsNv, kPhaseDown, BN, p, nsm, st, 1);
 }
 
 // grouped FFN with explicit h buffer
@@ -427,8 +484,8 @@ moe_status moe_device_error(int *code) {
     return MOE_OK;
 }
 
-size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32) {
-    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return 0;
+size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32, int af) {
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || (af != MOE_ACT_A16 && af != MOE_ACT_A4)) return 0;
     return layer_ws(T, H, I, E, k, y_is_fp32).total;
 }
 
@@ -449,11 +506,12 @@ moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is
                          num_sms(current_device()), (cudaStream_t)stream);
 }
 
-moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int af, int32_t *offsets,
                        int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
                        moe_stream_t stream) {
     if (T < 0 || k < 1 || k > kMaxTopK || E < 1 || E > kMaxExperts)
         return set_error(MOE_ERR_INVALID_ARG, "bad T/k/E (%d %d %d)", T, k, E);
+    if (af != MOE_ACT_A16 && af != MOE_ACT_A4) return set_error(MOE_ERR_INVALID_ARG, "unknown activation format %d", af);
     if (!offsets) return set_error(MOE_ERR_INVALID_ARG, "offsets is NULL");
     if (T > 0 && (!idx || !sorted_pair || !pair_row || (x_perm && !x) || !ws))
         return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
@@ -464,7 +522,7 @@ moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, i
         misaligned(ws, 16))
         return set_error(MOE_ERR_INVALID_ARG, "int32 arrays must be 4-byte aligned, ws 16-byte aligned");
     return launch_permute(idx, T, k, E, x, H, offsets, sorted_pair, pair_row, x_perm, ws, ws_bytes,
-                          (cudaStream_t)stream);
+                          (cudaStream_t)stream, af == MOE_ACT_A4);
 }
 
 moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
@@ -478,24 +536,31 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
     void *scratch = nullptr;
     moe_status r = permute_scratch_address(&scratch);
     if (r != MOE_OK) return r;
-    return moe_permute(idx, T, k, E, x, H, offsets, sorted_pair, pair_row, x_perm, scratch,
+    return moe_permute(idx, T, k, E, x, H, MOE_ACT_A16, offsets, sorted_pair, pair_row, x_perm, scratch,
                        MOE_PERMUTE_STATIC_SCRATCH_BYTES, stream);
 }
 
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
-                           void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream) {
+                           int af, void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream) {
     moe_status r = check_experts(experts);
     if (r != MOE_OK) return r;
+    if (af != MOE_ACT_A16 && af != MOE_ACT_A4) return set_error(MOE_ERR_INVALID_ARG, "unknown activation format %d", af);
+    if (af == MOE_ACT_A4 && (experts->fmt != MOE_NVFP4 || experts->layout != MOE_LAYOUT_TILED))
+        return set_error(MOE_ERR_UNSUPPORTED, "A4 activations need prepacked NVFP4 experts");
     if (n_rows < 0) return set_error(MOE_ERR_INVALID_ARG, "n_rows < 0");
     if (n_rows == 0) return MOE_OK;
     if (!x_perm || !offsets || !y_perm || !ws) return set_error(MOE_ERR_INVALID_ARG, "NULL pointer");
-    const size_t need = is_mx(*experts, n_rows) ? ffn_ws_bytes(n_rows, experts->H, experts->I, experts->E)
-                                        : align_up((size_t)n_rows * experts->I * 2, 256);
+    const size_t need = (af == MOE_ACT_A4 || is_mx(*experts, n_rows))
+                            ? ffn_ws_bytes(n_rows, experts->H, experts->I, experts->E)
+                            : align_up((size_t)n_rows * experts->I * 2, 256);
     if (ws_bytes < need) return set_error(MOE_ERR_OOM, "FFN workspace too small (%zu < %zu)", ws_bytes, need);
     if ((reinterpret_cast<uintptr_t>(x_perm) | reinterpret_cast<uintptr_t>(ws)) & 15)
         return set_error(MOE_ERR_INVALID_ARG, "x_perm and ws must be 16-byte aligned");
     if (misaligned(y_perm, 16) || misaligned(offsets, 4))
         return set_error(MOE_ERR_INVALID_ARG, "y_perm must be 16-byte aligned, offsets 4-byte aligned");
+    if (af == MOE_ACT_A4)
+        return a4_ffn_impl(x_perm, 0, x_perm, (int64_t)n_rows * experts->H, nullptr, 1, n_rows, offsets, experts, y_perm,
+                           y_is_fp32, ws, (cudaStream_t)stream);
     if (is_mx(*experts, n_rows))
         return mx_ffn_impl(x_perm, 0, nullptr, 1, n_rows, offsets, experts, y_perm, y_is_fp32, ws,
                            (cudaStream_t)stream);
@@ -548,12 +613,13 @@ moe_status moe_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_ro
 }
 
 moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp32, const float *bias, int k,
-                             const moe_experts *experts, struct expert_cache *cache, int layer, int y_is_fp32,
-                             void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                             const moe_experts *experts, int af, struct expert_cache *cache, int layer,
+                             int y_is_fp32, void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
                              moe_stream_t stream) {
     if (!experts) return set_error(MOE_ERR_INVALID_ARG, "experts is NULL");
     const int E = experts->E, H = experts->H, I = experts->I;
     if (T < 0) return set_error(MOE_ERR_INVALID_ARG, "T < 0");
+    if (af != MOE_ACT_A16 && af != MOE_ACT_A4) return set_error(MOE_ERR_INVALID_ARG, "unknown activation format %d", af);
     if (T == 0) return MOE_OK;
     if (k < 1 || k > kMaxTopK || k > E)
         return set_error(MOE_ERR_INVALID_ARG, "k=%d outside 1..min(%d, E=%d)", k, kMaxTopK, E);
@@ -579,7 +645,11 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     // The block-scaled FP4 path gathers the token rows itself while quantising them, so
     // it needs no x_perm, and for small batches the router kernel also permutes.
     const int layout = cache ? cache_layout(cache) : experts->layout;
-    const bool mx = use_bs(experts->fmt, layout, T * k, E);
+    const bool a4 = af == MOE_ACT_A4;
+    if (a4 && (experts->fmt != MOE_NVFP4 || layout != MOE_LAYOUT_TILED))
+        return set_error(MOE_ERR_UNSUPPORTED, "A4 activations need prepacked NVFP4 experts");
+    // both FP4-operand paths gather the token rows while quantising them (no x_perm)
+    const bool mx = a4 || use_bs(experts->fmt, layout, T * k, E);
     moe_status r;
     int fused = 0;
     if (mx) {
@@ -597,8 +667,8 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     }
     if (r != MOE_OK) return r;
     if (!fused) {
-        r = moe_permute(idx, T, k, E, x, H, offsets, sorted, prow, mx ? nullptr : b + L.x_perm, b + L.perm,
-                        L.x_perm - L.perm, stream);
+        r = moe_permute(idx, T, k, E, x, H, MOE_ACT_A16, offsets, sorted, prow, mx ? nullptr : b + L.x_perm,
+                        b + L.perm, L.x_perm - L.perm, stream);
         if (r != MOE_OK) return r;
     }
     moe_experts view = *experts;
@@ -607,10 +677,12 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
         if (r != MOE_OK) return r;
     }
     r = check_experts(&view);
-    if (r == MOE_OK && is_mx(view, T * k) != mx)
+    if (r == MOE_OK && !a4 && is_mx(view, T * k) != mx)
         r = set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
     if (r == MOE_OK) {
-        if (mx)
+        if (a4)
+            r = a4_ffn_impl(x, 1, x, (int64_t)T * H, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+        else if (mx)
             r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
         else
             r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);

@@ -33,6 +33,13 @@
 // puts atom row l into TMEM lanes l, l+32, l+64, l+96 (4 columns), where the
 // MMA reads the scale of row r: lane r, column r / 32, byte j.
 //
+// Activation format A4 (NVFP4 only): the activations are themselves in NVFP4
+// form, one plane: x with the per-tensor scale s_g = amax|x| / (6 * 448), h with
+// s_g = 1; E4M3 scales E4M3_RN_sat((amax_16 / 6) / s_g) per 16 K elements and
+// E2M1 codes of v / (s_b s_g), ties to even. The B operand then has N = BN rows
+// (one per token), and the epilogue multiplies by s_g and the weights' tensor
+// scale. The UP epilogue writes h in this form for the down pass.
+//
 // Every wait is bounded; on timeout the CTA sets the device error word, drains
 // its copies and MMAs and exits.
 #include "common.cuh"
@@ -148,6 +155,40 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi, float *qlo, float
     *qlo = f.x;
     *qhi = f.y;
     return w;
+}
+
+// E2M1 codes (nearest, ties to even, saturating at 6) of the pair (lo, hi): one byte,
+// lo in bits 0-3.
+__device__ __forceinline__ uint32_t e2m1x2_code(float lo, float hi) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "mov.b32 %0, {t, 0, 0, 0};\n\t}"
+        : "=r"(w)
+        : "f"(lo), "f"(hi));
+    return w;
+}
+
+// E4M3 code of v (nearest, ties to even, saturating at 448), in the low byte.
+__device__ __forceinline__ uint32_t e4m3_code(float v) {
+    uint32_t w;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 t, %2, %1;\n\t"
+        "cvt.u32.u16 %0, t;\n\t}"
+        : "=r"(w)
+        : "f"(v), "f"(0.0f));
+    return w & 0xFFu;
+}
+
+// Value of an E4M3 code (exact: every E4M3 value is an fp16 value).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h)
+        : "r"(code & 0xFFu));
+    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
 }
 
 // Biased E8M0 exponent s of plane 0 for a block with maximum magnitude amax:
@@ -381,6 +422,94 @@ __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__
     }
 }
 
+// ------------------------------------------------------------------ A4 activations
+
+// Partial maxima of |src| (bf16, n8 groups of 8): part[b] = the maximum over block b's
+// share (grid-stride). Maxima are exact, so the tensor scale does not depend on the split.
+__global__ void __launch_bounds__(256) a4_amax_kernel(const uint4 *__restrict__ src, int64_t n8,
+                                                      float *__restrict__ part) {
+    __shared__ uint32_t s_max[8];
+    pdl_wait();
+    pdl_release();
+    float amax = 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (int64_t)gridDim.x * 256) {
+        float v[8];
+        bf16x8_to_float(__ldg(src + i), v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    }
+    // non-negative floats order like their bit patterns
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = wmax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t m = s_max[0];
+        for (int w = 1; w < 8; ++w) m = max(m, s_max[w]);
+        part[blockIdx.x] = __uint_as_float(m);
+    }
+}
+
+// A4 form of the activation rows into the blobs of the FFN's token tiles. The block
+// first reduces the kA4Parts partial maxima to s_g = amax / (6 * 448) (1 for an all-zero
+// x; block 0 stores it in *xscale for the UP epilogue). Then one warp per (row r,
+// 256-wide stage), 8 consecutive elements per lane, two lanes per 16-block:
+// s_b = E4M3(((amax_16 / 6) / s_g)), codes E2M1(v / (s_b s_g)) (0 when s_b s_g = 0),
+// every step a correctly rounded binary32 operation. Rows: x[sorted_pair[r] / k]
+// (mode 1) or src[r] (mode 2), natural order; placement as in mx_quant_kernel, one plane.
+__global__ void __launch_bounds__(256) a4_quant_kernel(const uint4 *__restrict__ src, int mode,
+                                                       const int32_t *__restrict__ sorted_pair, int k, int P, int K,
+                                                       const int32_t *__restrict__ offsets, int E, int BN,
+                                                       const float *__restrict__ part, float *__restrict__ xscale,
+                                                       uint8_t *__restrict__ bblob) {
+    __shared__ int s_off[kMaxExperts + 1];
+    __shared__ int s_tile[kMaxExperts + 1];
+    __shared__ int s_wsum[8];
+    __shared__ float s_sg;
+    pdl_wait();
+    pdl_release();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
+    if (warp == 0) {
+        uint32_t m = 0u;
+        for (int i = lane; i < kA4Parts; i += 32) m = max(m, __float_as_uint(__ldcg(part + i)));
+        m = __reduce_max_sync(0xffffffffu, m);
+        const float amax = __uint_as_float(m);
+        const float sg = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+        if (lane == 0) {
+            s_sg = sg;
+            if (blockIdx.x == 0) *xscale = sg;
+        }
+    }
+    __syncthreads();
+    const float sg = s_sg;
+    const int K8 = K / 8, KST = K / kMxStageK, BB = bs_bblob_bytes(kBsNv, BN, 1);
+    const int64_t units = (int64_t)P * KST;
+    const int64_t nw = (int64_t)gridDim.x * 8;
+    for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += nw) {
+        const int r = (int)(u / KST), st = (int)(u - (int64_t)r * KST);
+        const int e = expert_of_row(s_off, E, r);
+        const int rel = r - s_off[e];
+        const int tile = s_tile[e] + rel / BN, n = rel % BN;
+        const uint4 uv = src[(int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8 + st * 32 + lane];
+        float v[8];
+        bf16x8_to_float(uv, v);
+        float bmax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));   // two lanes per 16-block
+        const uint32_t sc = e4m3_code(__fdiv_rn(__fdiv_rn(bmax, 6.0f), sg));
+        const float den = __fmul_rn(e4m3_value(sc), sg);
+        float t[8], q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = den > 0.0f ? __fdiv_rn(v[i], den) : 0.0f;
+        const uint32_t word = e2m1x8(t, q);
+        uint8_t *blob = bblob + ((int64_t)tile * KST + st) * BB;
+        *reinterpret_cast<uint32_t *>(blob + sw128_chunk(n, lane >> 2) + (lane & 3) * 4) = word;
+        const int b16 = lane >> 1;   // 16-block within the stage
+        if ((lane & 1) == 0) blob[BN * 128 + (b16 >> 2) * 512 + atom_offset(n, b16 & 3)] = (uint8_t)sc;
+    }
+}
+
 // ------------------------------------------------------------------ grouped FFN kernel
 
 struct MxSmem {
@@ -439,14 +568,15 @@ __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int
 // TMEM columns: accumulator (buffer a, pipeline w) at (a NW + w) N; from 2 NW N
 // on, 16 NA scale columns per pipeline (two rotating groups of 8 NA: the NA
 // weight atoms, then the NA activation atoms, 4 columns each).
-template <int FMT, int PHASE, int BN>
+template <int FMT, int PHASE, int BN, int PL>
 __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_constant__ MxParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    constexpr int N = kMxPlanes * BN;                       // MMA N: the planes' rows
+    static_assert(PL == kMxPlanes || (PL == 1 && FMT == kBsNv), "A4 activations are NVFP4");
+    constexpr int N = PL * BN;                              // MMA N: the planes' rows
     constexpr int NW = N <= 32 ? 4 : (N <= 64 ? 2 : 1);    // pipelines TMEM has room for
     constexpr int NA = bs_atoms(FMT);                       // scale atoms per operand and stage
     constexpr int ABLOB = bs_ablob_bytes(FMT);
-    constexpr int BBLOB = bs_bblob_bytes(FMT, BN);
+    constexpr int BBLOB = bs_bblob_bytes(FMT, BN, PL);
     constexpr int STAGE = ABLOB + BBLOB;                    // a multiple of 1024
     constexpr uint32_t SFCOL = 2 * NW * N;
     static_assert(SFCOL + NW * 16 * NA <= 512, "TMEM columns");
@@ -648,7 +778,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                 for (int j = 0; j < 16; ++j) val[j] = 0.0f;
                 constexpr float kPw[kMxPlanes] = {1.0f, FMT == kBsNv ? 0.125f : 1.0f, FMT == kBsNv ? 0.015625f : 1.0f,
                                                   FMT == kBsNv ? 0.001953125f : 1.0f};
-                if constexpr (BN <= 8) {
+                if constexpr (BN <= 8 && PL == kMxPlanes) {
                     for (int w = wlo; w < whi; ++w) {   // all N <= 32 columns of pipeline w
                         uint32_t v0[16], v1[16];
                         tmem_ld16(acc0 + w * N, v0);
@@ -665,17 +795,21 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                     }
                 } else {
                     for (int w = wlo; w < whi; ++w) {
-                        uint32_t v[kMxPlanes][16];
+                        uint32_t v[PL][16];
 #pragma unroll
-                        for (int pl = 0; pl < kMxPlanes; ++pl) tmem_ld16(acc0 + w * N + pl * BN + c0, v[pl]);
+                        for (int pl = 0; pl < PL; ++pl) tmem_ld16(acc0 + w * N + pl * BN + c0, v[pl]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int pl = 0; pl < kMxPlanes; ++pl)
+                        for (int pl = 0; pl < PL; ++pl)
 #pragma unroll
                             for (int j = 0; j < 16; ++j) val[j] = fmaf(__uint_as_float(v[pl][j]), kPw[pl], val[j]);
                     }
                 }
-                if constexpr (FMT == kBsNv) {   // 2^-C of each token row, times the expert's tensor scale
+                if constexpr (PL == 1) {   // A4: the tensor scales of x (UP; h has 1) and of the weights
+                    const float f = (PHASE == kPhaseUp ? __ldcg(p.xscale) : 1.0f) * p.tscale[it.e];
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) val[j] *= f;
+                } else if constexpr (FMT == kBsNv) {   // 2^-C of each token row, times the expert's tensor scale
                     const float ts = p.tscale[it.e];
 #pragma unroll
                     for (int j = 0; j < CH; ++j) {
@@ -715,6 +849,36 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                     // channel ch = 64 m + 32 pr + lane: this warp holds one 32-block of h,
                     // which is one 16-byte chunk of a row of the down pass's activation blob
                     const int ch = it.m * 64 + pr * 32 + lane;
+                    if constexpr (PL == 1) {
+                        // A4: h in NVFP4 form with tensor scale 1. A 16-block of channels is 16 lanes:
+                        // scale E4M3(amax / 6), codes E2M1(h / scale); lane pairs share a byte.
+                        const int c16 = (ch >> 5) & 7, b16 = (ch & 255) >> 4;
+                        uint8_t *blob = p.bblob_out + ((int64_t)it.rt * (p.I / kMxStageK) + (ch >> 8)) * BBLOB;
+#pragma unroll
+                        for (int j = 0; j < HCH; ++j) {
+                            const float g = gate ? val[j] : other[j];
+                            const float uu = gate ? other[j] : val[HCH + j];
+                            const float hv = g / (1.0f + expf(-g)) * uu;
+                            float amax = fabsf(hv);
+#pragma unroll
+                            for (int d = 1; d < 16; d <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+                            const uint32_t sc = e4m3_code(__fdiv_rn(amax, 6.0f));
+                            const float sb = e4m3_value(sc);
+                            const float t = sb > 0.0f ? __fdiv_rn(hv, sb) : 0.0f;
+                            const float to = __shfl_xor_sync(0xffffffffu, t, 1);
+                            const bool odd = lane & 1;
+                            uint32_t wv = e2m1x2_code(odd ? to : t, odd ? t : to) << (8 * ((lane >> 1) & 3));
+                            wv |= __shfl_xor_sync(0xffffffffu, wv, 2);
+                            wv |= __shfl_xor_sync(0xffffffffu, wv, 4);
+                            const int tok = c0 + t0 + j;
+                            if (tok < it.nvalid) {   // warp-uniform
+                                if ((lane & 7) == 0)
+                                    *reinterpret_cast<uint32_t *>(blob + sw128_chunk(tok, c16) + (lane >> 3) * 4) = wv;
+                                if ((lane & 15) == 0) blob[N * 128 + (b16 >> 2) * 512 + atom_offset(tok, b16 & 3)] = (uint8_t)sc;
+                            }
+                        }
+                        continue;
+                    }
                     if constexpr (FMT == kBsNv) {   // h in bf16; the NVFP4 quantiser makes its planes
 #pragma unroll
                         for (int j = 0; j < HCH; ++j) {
@@ -791,22 +955,37 @@ size_t mx_tiles_ub(int n_rows, int E) {
     return (size_t)(n_rows + BN - 1) / BN + (size_t)E;
 }
 
+// Token tile of the A4 path (one plane, so up to 128 tokens fill N = 128): from the
+// mean rows per expert, 32, 64 or 128.
+int choose_bn_a4(int n_rows, int E) {
+    const int avg = (n_rows + E - 1) / (E > 0 ? E : 1);
+    if (avg <= 32) return 32;
+    if (avg <= 64) return 64;
+    return 128;
+}
+
+size_t a4_blob_bytes(int n_rows, int K, int E) {
+    const int BN = choose_bn_a4(n_rows, E);
+    const size_t tiles = (size_t)(n_rows + BN - 1) / BN + (size_t)E;
+    return align_up(tiles * (K / kMxStageK) * bs_bblob_bytes(kBsNv, BN, 1), 256);
+}
+
 // Activation blob bytes of n_rows rows and reduction K, sized for NVFP4 (the
 // larger of the two formats' blobs).
 size_t mx_blob_bytes(int n_rows, int K, int E) {
     return align_up(mx_tiles_ub(n_rows, E) * (K / kMxStageK) * bs_bblob_bytes(kBsNv, choose_bn_mx(n_rows, E)), 256);
 }
 
-static size_t mx_smem_bytes(int fmt, int phase, int BN, int stages, int E) {
-    const size_t stage = (size_t)bs_ablob_bytes(fmt) + bs_bblob_bytes(fmt, BN);
+static size_t mx_smem_bytes(int fmt, int phase, int BN, int stages, int E, int planes) {
+    const size_t stage = (size_t)bs_ablob_bytes(fmt) + bs_bblob_bytes(fmt, BN, planes);
     return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 128 * kMxXch * 4 : 0) + sizeof(MxSmem) +
            (size_t)(3 * E + 2) * sizeof(int);
 }
 
-template <int FMT, int PHASE, int BN>
+template <int FMT, int PHASE, int BN, int PL>
 static cudaError_t mx_launch_one(const MxParams &p, int grid, size_t smem, cudaStream_t st) {
-    auto kfn = ffn_mx_kernel<FMT, PHASE, BN>;
-    cudaError_t e = ensure_max_smem<ffn_mx_kernel<FMT, PHASE, BN>>((int)smem);
+    auto kfn = ffn_mx_kernel<FMT, PHASE, BN, PL>;
+    cudaError_t e = ensure_max_smem<ffn_mx_kernel<FMT, PHASE, BN, PL>>((int)smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kfn, dim3(grid), dim3(kMxThreads), smem, st, p);
     return e == cudaSuccess ? cudaGetLastError() : e;
@@ -815,9 +994,18 @@ static cudaError_t mx_launch_one(const MxParams &p, int grid, size_t smem, cudaS
 template <int FMT, int PHASE>
 static cudaError_t mx_launch_bn(int BN, const MxParams &p, int grid, size_t smem, cudaStream_t st) {
     switch (BN) {
-        case 8: return mx_launch_one<FMT, PHASE, 8>(p, grid, smem, st);
-        case 16: return mx_launch_one<FMT, PHASE, 16>(p, grid, smem, st);
-        default: return mx_launch_one<FMT, PHASE, 32>(p, grid, smem, st);
+        case 8: return mx_launch_one<FMT, PHASE, 8, kMxPlanes>(p, grid, smem, st);
+        case 16: return mx_launch_one<FMT, PHASE, 16, kMxPlanes>(p, grid, smem, st);
+        default: return mx_launch_one<FMT, PHASE, 32, kMxPlanes>(p, grid, smem, st);
+    }
+}
+
+template <int PHASE>
+static cudaError_t a4_launch_bn(int BN, const MxParams &p, int grid, size_t smem, cudaStream_t st) {
+    switch (BN) {
+        case 32: return mx_launch_one<kBsNv, PHASE, 32, 1>(p, grid, smem, st);
+        case 64: return mx_launch_one<kBsNv, PHASE, 64, 1>(p, grid, smem, st);
+        default: return mx_launch_one<kBsNv, PHASE, 128, 1>(p, grid, smem, st);
     }
 }
 
@@ -826,12 +1014,12 @@ static cudaError_t mx_launch_bn(int BN, const MxParams &p, int grid, size_t smem
 // at least two slots each in the shared memory of one CTA. False if none fits.
 // When that leaves one stage per item and pipeline, every stage would be an
 // item boundary for its MMA warp: the pipelines take whole items instead.
-bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl) {
+bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl, int planes) {
     const int KST = K / kMxStageK;
-    const int N = kMxPlanes * BN;
+    const int N = planes * BN;
     const int nw = N <= 32 ? 4 : (N <= 64 ? 2 : 1);
     int fit = kMxMaxStages;
-    while (fit > 0 && mx_smem_bytes(fmt, phase, BN, fit, E) > (size_t)kMxSmemCap) --fit;
+    while (fit > 0 && mx_smem_bytes(fmt, phase, BN, fit, E, planes) > (size_t)kMxSmemCap) --fit;
     for (int np = nw < KST ? nw : KST; np >= 1; --np) {
         if (KST % np) continue;
         const int nsw = fit / np;
@@ -844,20 +1032,24 @@ bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl) {
     return false;
 }
 
-moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st) {
+moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st, int planes) {
     if (p.K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", p.K, kMxStageK);
+    if (planes != kMxPlanes && (planes != 1 || fmt != kBsNv))
+        return set_error(MOE_ERR_UNSUPPORTED, "A4 activations need NVFP4 experts");
     MxPlan pl;
-    if (!mx_plan(fmt, phase, BN, p.K, p.E, &pl))
+    if (!mx_plan(fmt, phase, BN, p.K, p.E, &pl, planes))
         return set_error(MOE_ERR_UNSUPPORTED, "K=%d: no pipeline plan for the block-scaled FP4 path", p.K);
     p.pipes = pl.pipes;
     p.stages = pl.stages;
     p.itempar = pl.itempar;
-    size_t smem = mx_smem_bytes(fmt, phase, BN, pl.stages, p.E);
+    size_t smem = mx_smem_bytes(fmt, phase, BN, pl.stages, p.E, planes);
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: it allocates all 512 TMEM columns
     const int64_t items_ub = ((int64_t)p.n_rows / BN + p.E) * p.m_tiles;
     const int grid = (int)(items_ub < num_sms ? (items_ub > 0 ? items_ub : 1) : num_sms);
     cudaError_t e;
-    if (fmt == kBsNv)
+    if (planes == 1)
+        e = phase == kPhaseUp ? a4_launch_bn<kPhaseUp>(BN, p, grid, smem, st) : a4_launch_bn<kPhaseDown>(BN, p, grid, smem, st);
+    else if (fmt == kBsNv)
         e = phase == kPhaseUp ? mx_launch_bn<kBsNv, kPhaseUp>(BN, p, grid, smem, st)
                               : mx_launch_bn<kBsNv, kPhaseDown>(BN, p, grid, smem, st);
     else
@@ -887,6 +1079,33 @@ moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *so
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "block-scaled quantiser launch");
+}
+
+}  // namespace moe
+
+namespace moe {
+
+moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cudaStream_t st) {
+    const int64_t n8 = n_elems / 8;
+    cudaError_t e = launch_pdl(a4_amax_kernel, dim3(kA4Parts), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
+                               n8, partials);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 amax launch");
+}
+
+moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
+                           const int32_t *offsets, int E, int BN, const float *partials, float *xscale, void *bblob,
+                           int num_sms, cudaStream_t st) {
+    if (P == 0) return MOE_OK;
+    if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
+    if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
+    const int64_t units = (int64_t)P * (K / kMxStageK);
+    const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
+    cudaError_t e = launch_pdl(a4_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
+                               mode, sorted_pair, k, P, K, offsets, E, BN, partials, xscale,
+                               reinterpret_cast<uint8_t *>(bblob));
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 quantiser launch");
 }
 
 }  // namespace moe

@@ -48,8 +48,13 @@ constexpr int kMxPlanes = 4;                     // E2M1 planes per activation v
 __host__ __device__ constexpr int bs_atoms(int f) { return f == kBsNv ? 4 : 2; }
 // Bytes of one weight blob (M tile, stage): codes, then the scale atoms.
 __host__ __device__ constexpr int bs_ablob_bytes(int f) { return kMxCodeBytes + 512 * bs_atoms(f); }
-// Bytes of one activation blob (N tile of BN rows, stage): 4 BN rows of 128 B, then the scale atoms.
-__host__ __device__ constexpr int bs_bblob_bytes(int f, int BN) { return kMxPlanes * BN * 128 + 512 * bs_atoms(f); }
+// Bytes of one activation blob (N tile of BN rows, stage): `planes` BN rows of 128 B, then the
+// scale atoms. Four planes carry bf16 activations (A16); one plane is the activation itself in
+// NVFP4 form (A4).
+__host__ __device__ constexpr int bs_bblob_bytes(int f, int BN, int planes = kMxPlanes) {
+    return planes * BN * 128 + 512 * bs_atoms(f);
+}
+constexpr int kA4Parts = 592;   // partial maxima of |x| (A4 tensor scale), 4 per SM of a 148-SM part
 
 struct MxParams {
     const int32_t *offsets;     // [E+1]
@@ -68,8 +73,9 @@ struct MxParams {
     const float *tscale;        // NVFP4: per-expert tensor scale of this phase's weights [E]
     void *out;                  // down: y [n_rows][H] (bf16 or fp32)
     int out_fp32;
-    uint8_t *bblob_out;         // MXFP4 up: blobs of h for the down pass [tiles][I/256]
+    uint8_t *bblob_out;         // MXFP4 and A4 up: blobs of h for the down pass [tiles][I/256]
     void *hout;                 // NVFP4 up: h bf16 [n_rows][I]
+    const float *xscale;        // A4 up: device word with the per-tensor scale of x
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -91,10 +97,20 @@ int choose_bn_mx(int n_rows, int E);
 struct MxPlan {
     int pipes, stages, itempar;
 };
-bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl);
+bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl, int planes = kMxPlanes);
 size_t mx_tiles_ub(int n_rows, int E);
 size_t mx_blob_bytes(int n_rows, int K, int E);
-moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st);
+// planes: kMxPlanes (A16 activations) or 1 (A4, NVFP4 only)
+moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st,
+                           int planes = kMxPlanes);
+// A4 (activations in NVFP4 form): token tile, workspace of the activation blobs, the
+// partial maxima of |x| and the quantiser (src rows as launch_mx_quant modes 1 and 2).
+int choose_bn_a4(int n_rows, int E);
+size_t a4_blob_bytes(int n_rows, int K, int E);
+moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cudaStream_t st);
+moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
+                           const int32_t *offsets, int E, int BN, const float *partials, float *xscale, void *bblob,
+                           int num_sms, cudaStream_t st);
 // src rows: mode 0 x_perm[r] (operand order), 1 x[sorted_pair[r] / k] (natural
 // order), 2 src[r] (natural order; NVFP4 only). rowexp: NVFP4 only.
 moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
@@ -120,9 +136,11 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
 // permutation (permute.cu)
 size_t permute_ws_bytes(int T, int k, int E);
 size_t permute_scratch_bytes(int T, int k, int E);
+// natural: x_perm rows in natural column order (A4 activations), else in the operand order
+// 0,4,1,5,2,6,3,7 of every group of 8 (A16)
 moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
                           int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
-                          cudaStream_t st);
+                          cudaStream_t st, int natural = 0);
 
 // combine (combine.cu)
 moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,

@@ -8,3 +8,4 @@
 #include "ffn_mx.cu"
 #include "prepack.cu"
 #include "cache.cu"
+#include "peak.cu"

@@ -140,7 +140,7 @@ size_t permute_scratch_bytes(int T, int k, int E) {
 
 __global__ void __launch_bounds__(256) perm_gather_kernel(const uint4 *__restrict__ x, int H8, int k,
                                                          const int32_t *__restrict__ sorted_pair, int P,
-                                                         uint4 *__restrict__ x_perm) {
+                                                         uint4 *__restrict__ x_perm, int natural) {
     pdl_wait();
     pdl_release();
     const int64_t total = (int64_t)P * H8;
@@ -148,13 +148,14 @@ __global__ void __launch_bounds__(256) perm_gather_kernel(const uint4 *__restric
         const int64_t r = i / H8;
         const int c = (int)(i - r * H8);
         const int t = sorted_pair[r] / k;
-        x_perm[i] = interleave8(x[(int64_t)t * H8 + c]);
+        const uint4 v = x[(int64_t)t * H8 + c];
+        x_perm[i] = natural ? v : interleave8(v);
     }
 }
 
 moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
                           int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
-                          cudaStream_t st) {
+                          cudaStream_t st, int natural) {
     const int P = T * k;
     if (P == 0) {
         cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
@@ -193,7 +194,7 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
         int blocks = (int)((total + 255) / 256);
         if (blocks > 148 * 16) blocks = 148 * 16;
         e = launch_pdl(perm_gather_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(x), H8, k,
-                       (const int32_t *)sorted_pair, P, reinterpret_cast<uint4 *>(x_perm));
+                       (const int32_t *)sorted_pair, P, reinterpret_cast<uint4 *>(x_perm), natural);
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return set_cuda_error(e, "gather launch");
     }

@@ -73,6 +73,22 @@ typedef enum {
  *                     tscale: one fp32 per expert and tensor. */
 typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3_K128 = 1, MOE_MXFP4 = 2, MOE_NVFP4 = 3 } moe_wfmt;
 
+/* Activation format inside the expert GEMMs. The pages name the weight formats
+ * ([P4] "Reported Numbers and Ecosystem Position") but not the precision the
+ * activations enter the GEMMs in; this library offers two, and the math of the
+ * layer depends on the choice:
+ *   MOE_ACT_A16  the activations as given: x in bf16, h rounded to bf16 before
+ *                the down projection. The default.
+ *   MOE_ACT_A4   the activations in NVFP4 form, so that both operands of every
+ *                expert GEMM are FP4 (block-scaled FP4 tensor-core MMA): x with
+ *                one per-tensor scale s_g = amax|x| / (6 * 448) over the whole
+ *                [T][H] batch (1 if x is all zero), h with s_g = 1; per 16
+ *                elements along K an E4M3 scale s_b = E4M3((amax_16 / 6) / s_g)
+ *                and E2M1 codes of v / (s_b * s_g), both rounded to nearest,
+ *                ties to even, saturating; the GEMM sees q * s_b * s_g.
+ *                Prepacked NVFP4 experts only (MOE_ERR_UNSUPPORTED otherwise). */
+typedef enum { MOE_ACT_A16 = 0, MOE_ACT_A4 = 1 } moe_actfmt;
+
 /* Memory layout of the expert codes. STANDARD: row-major as described above.
  * TILED: produced by moe_prepack. The values are the same and so is the byte
  * count (codes plus scales); only the byte order differs. Weight rows form M
@@ -141,20 +157,21 @@ moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is
  * Times"): a counting sort of the T*k pairs p = t*k + j by expert, stable in p.
  *   offsets: int32 [E+1], exclusive scan of per-expert counts (offsets[E] = T*k).
  *   sorted_pair: int32 [T*k], the pairs in expert order; pair_row: its inverse.
- *   x_perm (nullable): bf16 [T*k][H], row r = x[sorted_pair[r] / k], with the
- *     columns of every aligned group of 8 stored in the order 0,4,1,5,2,6,3,7
- *     (the operand layout of moe_grouped_ffn).
+ *   x_perm (nullable): bf16 [T*k][H], row r = x[sorted_pair[r] / k], laid out for
+ *     moe_grouped_ffn with the same activation format `af`: MOE_ACT_A16 stores the
+ *     columns of every aligned group of 8 in the order 0,4,1,5,2,6,3,7; MOE_ACT_A4
+ *     stores them in natural order (the A4 FFN quantises the rows itself).
  *   Bit-exact and deterministic. Requires H % 8 == 0.
- *   Errors: INVALID_ARG for T < 0, k outside 1..16, E outside 1..1024, NULL
- *   offsets, NULL idx, sorted_pair, pair_row or ws when T > 0, x_perm without x,
- *   H not a positive multiple of 8 or x or x_perm not 16-byte aligned when x_perm
- *   is given, int32 arrays not 4-byte aligned, or ws not 16-byte aligned; OOM
- *   when ws_bytes is below what the call needs. */
-moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
+ *   Errors: INVALID_ARG for T < 0, k outside 1..16, E outside 1..1024, an unknown
+ *   af, NULL offsets, NULL idx, sorted_pair, pair_row or ws when T > 0, x_perm
+ *   without x, H not a positive multiple of 8 or x or x_perm not 16-byte aligned
+ *   when x_perm is given, int32 arrays not 4-byte aligned, or ws not 16-byte
+ *   aligned; OOM when ws_bytes is below what the call needs. */
+moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, int H, int af, int32_t *offsets,
                        int32_t *sorted_pair, int32_t *pair_row, void *x_perm, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
 
-/* moe_permute without a caller workspace: the same permutation, bit for bit,
+/* moe_permute (with af = MOE_ACT_A16) without a caller workspace: the same permutation, bit for bit,
  * with the scratch taken from a fixed device array inside the library instead
  * of `ws`. The pages have no counterpart; it exists for callers that cannot
  * hand over device memory (no allocation happens anywhere on this path).
@@ -176,11 +193,18 @@ moe_status moe_permute(const int32_t *idx, int T, int k, int E, const void *x, i
 moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const void *x, int H, int32_t *offsets,
                               int32_t *sorted_pair, int32_t *pair_row, void *x_perm, moe_stream_t stream);
 
-/* Grouped SwiGLU expert FFN over the permuted rows ([P4] formats): for every
- * expert e and row r in [offsets[e], offsets[e+1]):
- *   h = silu(Wg_e . x_perm[r]) * (Wu_e . x_perm[r]), rounded to bf16;
+/* Grouped SwiGLU expert FFN over the permuted rows ([P4] formats; the routed
+ * experts of [P3] "Why Now of All Times"): for every expert e and row r in
+ * [offsets[e], offsets[e+1]):
+ *   h = silu(Wg_e . x_perm[r]) * (Wu_e . x_perm[r]), rounded to bf16 (A16) or
+ *       put in NVFP4 form with tensor scale 1 (A4);
  *   y_perm[r] = W2_e . h   (bf16, or fp32 if y_is_fp32).
- *   x_perm: bf16 [n_rows][H] in the interleaved layout written by moe_permute.
+ *   x_perm: bf16 [n_rows][H] as moe_permute writes it for the same `af` (A16:
+ *     interleaved columns; A4: natural order, quantised here with the tensor
+ *     scale of the n_rows rows, which equals that of x when every token is
+ *     among them).
+ *   af: moe_actfmt; MOE_ACT_A4 needs prepacked NVFP4 experts (UNSUPPORTED else)
+ *     and runs the block-scaled FP4 path with one plane per activation.
  *   offsets: int32 [E+1] as moe_permute writes them: offsets[0] = 0,
  *     non-decreasing, offsets[E] = n_rows. The kernels take them as given (they
  *     are read on the device only); other values make them read and write
@@ -202,10 +226,12 @@ moe_status moe_permute_static(const int32_t *idx, int T, int k, int E, const voi
  *   4-byte aligned, or n_rows < 0; OOM when ws_bytes is below what the call
  *   needs. */
 moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offsets, const moe_experts *experts,
-                           void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
+                           int af, void *y_perm, int y_is_fp32, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Gate-weighted combine: out[t] = sum_{j<k} w[t,j] * y_perm[pair_row[t*k+j]],
- * accumulated in fp32 in order of j, rounded to bf16.
+ * accumulated in fp32 in order of j, rounded to bf16 (the outputs of a token's
+ * k routed experts, [P3] "Why Now of All Times", weighted by its gates; the
+ * pages give no formula, this is the standard top-k mixture).
  *   y_perm: [T*k][H] bf16 or fp32 (y_is_fp32); out: bf16 [T][H]. H % 8 == 0.
  *   T == 0 is a no-op. Errors: INVALID_ARG for T < 0, k outside 1..16, H not a
  *   positive multiple of 8, NULL pointers, y_perm or out not 16-byte aligned, or
@@ -246,7 +272,12 @@ moe_status moe_prepack(const moe_experts *in, void *out_w13, void *out_w2, moe_s
 
 struct expert_cache;
 
-/* The whole layer: route -> permute -> grouped FFN -> combine.
+/* The whole layer: route -> permute -> grouped FFN -> combine (the MoE layer of
+ * [P3] "Why Now of All Times": each token runs through its k routed experts;
+ * with a cache, the experts come from the device cache fed by host streaming of
+ * [P3] "FreeToken's Three-Layer Mechanism" and [P4] "Three Engineering Cores").
+ *   af: moe_actfmt of the expert GEMMs (MOE_ACT_A4: prepacked NVFP4 experts;
+ *     with a cache, a cache built on prepacked NVFP4 layers).
  *   cache: nullable. When set, `experts` gives the layer's shape and format
  *     only, the weights come from the cache's device slots for `layer`, and
  *     missing experts are streamed from the cache's pinned host pool first
@@ -254,19 +285,24 @@ struct expert_cache;
  *   idx_out, w_out: nullable copies of the routing.
  *   y_is_fp32: keep the expert outputs in fp32 before the combine.
  * T == 0 is a no-op. Errors: INVALID_ARG for NULL experts, x, wr, out or ws,
- * T < 0, k outside 1..min(16, E), x, wr or out not 16-byte aligned, bias,
- * idx_out or w_out not 4-byte aligned, or ws not 256-byte aligned; UNSUPPORTED for a shape or format outside the kernels (as
- * for moe_grouped_ffn; the router takes E <= 256); OOM when ws_bytes is below
+ * T < 0, an unknown af, k outside 1..min(16, E), x, wr or out not 16-byte
+ * aligned, bias, idx_out or w_out not 4-byte aligned, or ws not 256-byte
+ * aligned; UNSUPPORTED for a shape or format outside the kernels (as for
+ * moe_grouped_ffn; the router takes E <= 256); OOM when ws_bytes is below
  * moe_workspace_size(); CACHE_FULL when the cache cannot hold the layer's
  * experts, with the table left unchanged. */
 moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp32, const float *bias, int k,
-                             const moe_experts *experts, struct expert_cache *cache, int layer, int y_is_fp32,
-                             void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                             const moe_experts *experts, int af, struct expert_cache *cache, int layer,
+                             int y_is_fp32, void *out, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
                              moe_stream_t stream);
 
 /* Scratch bytes needed by moe_layer_forward / moe_route_topk / moe_permute /
- * moe_grouped_ffn for these sizes (an upper bound; host-only, no CUDA call). */
-size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32);
+ * moe_grouped_ffn for these sizes and activation format (an upper bound that
+ * covers every path the sizes can take: the router's fp64 partial sums, the
+ * routing, the permutation, x_perm, h or the FP4 activation blobs, y). No
+ * counterpart in the pages: it is what lets every call run without allocating.
+ * Host-only, no CUDA call; 0 for non-positive sizes or an unknown af. */
+size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32, int af);
 
 /* ---------------------------------------------------------------- cache */
 /* Device LRU expert cache with streaming from pinned host memory ([P3]
@@ -408,6 +444,17 @@ moe_status moe_set_wait_limit_ns(uint64_t ns);
  * and returns, leaving the context usable. No counterpart in the pages: the
  * test of the bounded waits. Errors: CUDA for a failed launch. */
 moe_status moe_selftest_wait(moe_stream_t stream);
+
+/* Dense tensor-core throughput of the current device for one MMA kind of the
+ * grouped FFN (kind 0: bf16 kind::f16; 1: FP8 E4M3 kind::f8f6f4; 2: MXFP4
+ * kind::mxf4; 3: NVFP4 kind::mxf4nvf4), measured by this library's own MMA loop:
+ * one CTA per SM issues `iters` x 4 MMAs of M = 128, N = 256 on operands held in
+ * shared memory (no memory traffic), a warm-up launch and three timed ones
+ * (CUDA events). *tflops: the measured rate. No counterpart in the pages: the
+ * roofline denominators of the FFN kernels. Synchronous; creates and destroys
+ * its own stream and events. Errors: INVALID_ARG for an unknown kind, iters < 1
+ * or NULL tflops; CUDA. */
+moe_status moe_tensor_peak(int kind, int iters, double *tflops);
 
 /* Library version, for logs. */
 const char *moe_version(void);

@@ -238,7 +238,7 @@ def test_grouped_ffn_fp32_output(moe):
 # ----------------------------------------------------------------------------- whole layer
 
 
-def _layer_check(moe, L, x, y_fp32=False, sample=None, tiled=True):
+def _layer_check(moe, L, x, y_fp32=False, sample=None, tiled=True, act="a16"):
     """Run the layer on the GPU; compare routing bit-exactly and outputs (all or sampled rows)."""
     Ld = L.to("cuda")
     T = x.shape[0]
@@ -248,17 +248,17 @@ def _layer_check(moe, L, x, y_fp32=False, sample=None, tiled=True):
     if tiled:
         ex = moe.moe_prepack(ex)
         del Ld.w13, Ld.w2          # keep device memory low for the large layer
-    out = moe.moe_layer_forward(x.cuda(), Ld.wr, L.k, ex, bias=Ld.bias, y_fp32=y_fp32, idx_out=idx, w_out=w)
+    out = moe.moe_layer_forward(x.cuda(), Ld.wr, L.k, ex, bias=Ld.bias, y_fp32=y_fp32, idx_out=idx, w_out=w, act=act)
     torch.cuda.synchronize()
     idx_o, w_o, _ = oracle.route(x, L.wr, L.k, bias=L.bias, with_logits=False)
     assert np.array_equal(idx.cpu().numpy(), idx_o)
     assert np.allclose(w.cpu().numpy(), w_o, atol=2e-6, rtol=0)
     got = bf16_np(out)
     if sample is None:
-        ref = oracle.layer_forward(x, L)["out"]
+        ref = oracle.layer_forward(x, L, act=act)["out"]
         err = rel_err(got, ref)
     else:
-        ref = oracle.token_rows(x, L, idx_o, w_o, sample)
+        ref = oracle.token_rows(x, L, idx_o, w_o, sample, act=act)
         err = rel_err(got[sample], ref)
     assert err < TOL, f"layer output error {err:.3e}"
     assert moe.moe_device_error() == 0
@@ -586,3 +586,81 @@ def test_bounded_wait_gives_up_and_reports(moe):
     L = synthetic.make_layer("tiny", 0)
     x = synthetic.make_tokens(16, L.H, 0)
     _layer_check(moe, L, x)
+
+
+# ----------------------------------------------------------------------------- activation format A4
+
+
+@pytest.mark.parametrize("E,T,H,I,y32", [(8, 40, 256, 512, False), (8, 100, 512, 256, False), (8, 300, 256, 256, False),
+                                         (8, 3, 256, 256, False), (16, 700, 512, 512, True), (4, 129, 256, 768, False)])
+def test_grouped_ffn_a4_parity(moe, E, T, H, I, y32):
+    """Activations in NVFP4 form (A4) on prepacked NVFP4 experts: token tiles of 32, 64 and
+    128 (mean rows per expert 2T/E), ragged tails, one and several stages per item, the
+    down projection at 3 stages (I = 768), bf16 and fp32 outputs; against the oracle's A4
+    FFN on the same permutation."""
+    cfg = dict(H=H, E=E, k=2, I=I, fmt="nvfp4", wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=40 + T)
+    x = synthetic.make_tokens(T, H, seed=40 + T)
+    idx = _rand_idx(T, 2, E, T + 1)
+    off_o, sp_o, _ = oracle.permute(idx, E)
+    y_o = oracle.ffn(x, L, off_o, sp_o, 2, act="a4")
+    ex = moe.moe_prepack(moe.Experts.from_layer(L.to("cuda")))
+    off, sp, pr, xp = moe.moe_permute(torch.from_numpy(idx).cuda(), E, x.cuda(), act="a4")
+    # A4 rows are in natural column order
+    assert torch.equal(xp.cpu(), x[torch.from_numpy(sp_o // 2).long()])
+    y = moe.moe_grouped_ffn(xp, off, ex, y_fp32=y32, act="a4")
+    torch.cuda.synchronize()
+    err = rel_err(y.float().cpu().numpy(), y_o)
+    assert err < TOL, f"A4 FFN error {err:.3e}"
+    assert moe.moe_device_error() == 0
+
+
+def test_a4_needs_prepacked_nvfp4(moe):
+    L = synthetic.make_layer(dict(H=256, E=8, k=2, I=256, fmt="mxfp4", wr_fp32=False), 3).to("cuda")
+    x = synthetic.make_tokens(8, 256, 3).cuda()
+    for ex in (moe.moe_prepack(moe.Experts.from_layer(L)), moe.Experts.from_layer(L)):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_layer_forward(x, L.wr, 2, ex, act="a4")
+        assert ei.value.name == "UNSUPPORTED"
+
+
+def test_layer_a4_prefill_reduced_batch(moe, prefill_layer):
+    x = synthetic.make_tokens(256, 2048, seed=41)
+    _layer_check(moe, prefill_layer, x, act="a4")
+
+
+def test_layer_a4_prefill_full_size_sampled(moe, prefill_layer):
+    x = synthetic.make_tokens(4096, 2048, seed=42)
+    sample = _sample_rows(prefill_layer, x, 16, 42)
+    _layer_check(moe, prefill_layer, x, sample=sample, act="a4")
+
+
+def test_layer_a4_large_prefill_sampled(moe, large_layer):
+    x = synthetic.make_tokens(8192, 4096, seed=43)
+    sample = _sample_rows(large_layer, x, 16, 43)
+    _layer_check(moe, large_layer, x, y_fp32=True, sample=sample, act="a4")
+
+
+def test_layer_a4_large_decode_every_row(moe, large_layer):
+    x = synthetic.make_tokens(32, 4096, seed=44)
+    _layer_check(moe, large_layer, x, y_fp32=True, sample=list(range(32)), act="a4")
+
+
+def test_layer_a4_through_the_cache_equals_resident(moe):
+    cfg = dict(H=512, E=16, k=4, I=256, fmt="nvfp4", wr_fp32=False)
+    dev = [synthetic.make_layer(cfg, seed=45, layer=l).to("cuda") for l in range(2)]
+    packed = [moe.moe_prepack(moe.Experts.from_layer(L)) for L in dev]
+    host = [moe.Experts(t.fmt, t.E, t.H, t.I, t.w13.cpu().pin_memory(), t.w2.cpu().pin_memory(),
+                        w13_tscale=t.w13_tscale.cpu(), w2_tscale=t.w2_tscale.cpu(), layout=moe.LAYOUT_TILED)
+            for t in packed]
+    cache = moe.ExpertCache(1 << 30, host, device=0)
+    for step in range(3):
+        for l in range(2):
+            x = synthetic.make_tokens(100, 512, seed=46 + 5 * step + l).cuda()
+            out_c = moe.moe_layer_forward(x, dev[l].wr, 4, moe.Experts.from_layer(dev[l]), cache=cache, layer=l,
+                                          act="a4")
+            out_r = moe.moe_layer_forward(x, dev[l].wr, 4, packed[l], act="a4")
+            torch.cuda.synchronize()
+            assert torch.equal(out_c, out_r), (step, l)
+    assert moe.moe_device_error() == 0
+    cache.close()

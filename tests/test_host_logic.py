@@ -46,12 +46,14 @@ def test_route_topk_checks():
 
 def test_permute_checks():
     L = moe.lib()
-    p = lambda T, k, E: L.moe_permute(None, T, k, E, None, 0, None, None, None, None, None, 0, None)
+    p = lambda T, k, E, af=0: L.moe_permute(None, T, k, E, None, 0, af, None, None, None, None, None, 0, None)
     assert p(-1, 2, 8) == INVALID_ARG
     assert p(4, 0, 8) == INVALID_ARG
     assert p(4, 17, 8) == INVALID_ARG
     assert p(4, 2, 2000) == INVALID_ARG            # E above the 1024 experts of the permutation
     assert p(4, 2, 8) == INVALID_ARG               # offsets is NULL
+    assert p(4, 2, 8, af=2) == INVALID_ARG         # unknown activation format
+    assert "activation format" in _err()
     # the fixed scratch of moe_permute_static covers ceil(T*k/1024)*E <= 131072 counters
     assert L.moe_permute_static(None, 1 << 20, 8, 1024, None, 0, None, None, None, None, None) == UNSUPPORTED
     assert "fixed scratch" in _err()
@@ -59,7 +61,7 @@ def test_permute_checks():
 
 def test_grouped_ffn_and_prepack_check_the_experts_first():
     L = moe.lib()
-    g = lambda ex, n=4: L.moe_grouped_ffn(None, n, None, ex, None, 0, None, 0, None)
+    g = lambda ex, n=4, af=0: L.moe_grouped_ffn(None, n, None, ex, af, None, 0, None, 0, None)
     assert g(_experts(H=200)) == UNSUPPORTED        # H not a multiple of 256
     assert g(_experts(I=100)) == UNSUPPORTED
     assert g(_experts(fmt=7)) == UNSUPPORTED
@@ -67,6 +69,11 @@ def test_grouped_ffn_and_prepack_check_the_experts_first():
     assert g(_experts(E=1025)) == UNSUPPORTED
     assert g(_experts()) == INVALID_ARG             # NULL weights
     assert g(None) == INVALID_ARG
+    assert g(_experts(), af=5) == INVALID_ARG
+    # A4 activations: prepacked NVFP4 experts only
+    assert g(_experts(fmt="mxfp4", w=1 << 24, scale=1 << 24), af=1) == UNSUPPORTED
+    assert g(_experts(fmt="nvfp4", w=1 << 24, scale=1 << 24, tscale=1 << 24), af=1) == UNSUPPORTED
+    assert "A4" in _err()
     assert L.moe_prepack(_experts(H=200), None, None, None) == UNSUPPORTED
     assert L.moe_prepack(_experts(), None, None, None) == INVALID_ARG
 
@@ -90,13 +97,14 @@ def test_combine_and_dequantize_checks():
 def test_layer_forward_checks():
     L = moe.lib()
 
-    def f(ex, T=4, k=2, ptr=None, ws_bytes=0):
-        return L.moe_layer_forward(ptr, T, ptr, 0, None, k, ex, None, 0, 0, ptr, None, None, ptr, ws_bytes, None)
+    def f(ex, T=4, k=2, ptr=None, ws_bytes=0, af=0):
+        return L.moe_layer_forward(ptr, T, ptr, 0, None, k, ex, af, None, 0, 0, ptr, None, None, ptr, ws_bytes, None)
 
     ex = _experts()
     assert f(None) == INVALID_ARG
     assert f(ex, T=-1) == INVALID_ARG
     assert f(ex, T=0) == OK
+    assert f(ex, af=3) == INVALID_ARG
     for k in (0, 17, 9):                            # 9 > E = 8
         assert f(ex, k=k) == INVALID_ARG
         assert f"k={k}" in _err()
@@ -119,20 +127,20 @@ def test_misaligned_arrays_are_rejected():
         A, 4, 256, A, 0, bias, 8, 2, idx, w, logits, ws, 1 << 30, None)
     for kw in (dict(idx=odd2), dict(w=odd2), dict(logits=odd2), dict(bias=odd2), dict(ws=odd8)):
         assert route(**kw) == INVALID_ARG, kw
-    perm = lambda idx=A, off=A, sp=A, pr=A, ws=A: L.moe_permute(idx, 4, 2, 8, None, 0, off, sp, pr, None, ws,
+    perm = lambda idx=A, off=A, sp=A, pr=A, ws=A: L.moe_permute(idx, 4, 2, 8, None, 0, 0, off, sp, pr, None, ws,
                                                                 1 << 30, None)
     for kw in (dict(idx=odd2), dict(off=odd2), dict(sp=odd2), dict(pr=odd2), dict(ws=odd8)):
         assert perm(**kw) == INVALID_ARG, kw
     comb = lambda pr=A, w=A, y=A, out=A: L.moe_combine(y, 0, pr, w, 4, 2, 256, out, None)
     for kw in (dict(pr=odd2), dict(w=odd2), dict(y=odd8), dict(out=odd8)):
         assert comb(**kw) == INVALID_ARG, kw
-    ffn = lambda ex, off=A, y=A: L.moe_grouped_ffn(A, 4, off, ex, y, 0, A, 1 << 40, None)
+    ffn = lambda ex, off=A, y=A: L.moe_grouped_ffn(A, 4, off, ex, 0, y, 0, A, 1 << 40, None)
     ex = _experts(w=A)
     assert ffn(ex, off=odd2) == INVALID_ARG
     assert ffn(ex, y=odd8) == INVALID_ARG
     assert ffn(_experts(fmt="nvfp4", w=A, scale=A, tscale=odd2)) == INVALID_ARG
     assert L.moe_dequantize(FMT["fp8"], A, odd2, 1.0, 4, 128, A, None) == INVALID_ARG
-    lay = lambda bias=None, idx=None, w=None, out=A: L.moe_layer_forward(A, 4, A, 0, bias, 2, ex, None, 0, 0, out,
+    lay = lambda bias=None, idx=None, w=None, out=A: L.moe_layer_forward(A, 4, A, 0, bias, 2, ex, 0, None, 0, 0, out,
                                                                          idx, w, A, 1 << 40, None)
     for kw in (dict(bias=odd2), dict(idx=odd2), dict(w=odd2), dict(out=odd8)):
         assert lay(**kw) == INVALID_ARG, kw
@@ -178,6 +186,8 @@ def test_workspace_size_is_monotone_and_rejects_bad_sizes():
     for bad in ((-1, 2048, 768, 128, 8), (4, 0, 768, 128, 8), (4, 2048, 0, 128, 8), (4, 2048, 768, 0, 8),
                 (4, 2048, 768, 128, 0)):
         assert ws(*bad) == 0
+    assert ws(64, 2048, 768, 128, 8, 0, "a4") == ws(64, 2048, 768, 128, 8)   # one bound covers both formats
+    assert moe.lib().moe_workspace_size(64, 2048, 768, 128, 8, 0, 7) == 0
 
 
 @pytest.mark.parametrize("fmt", ["bf16", "fp8", "mxfp4", "nvfp4"])
