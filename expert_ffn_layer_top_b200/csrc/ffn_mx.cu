@@ -297,12 +297,15 @@ __device__ __forceinline__ void bf16x8_to_float(uint4 u, float (&v)[8]) {
 __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
-                                                       uint8_t *__restrict__ bblob) {
+                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ cnt,
+                                                       int ncnt) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     pdl_wait();
     pdl_release();
+    // the fused combine's counters start at zero for the down pass of this call
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsMx, BN);
@@ -347,13 +350,15 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
 __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
-                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp) {
+                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp,
+                                                       int32_t *__restrict__ cnt, int ncnt) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     __shared__ uint32_t s_max[8];
     pdl_wait();
     pdl_release();
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsNv, BN);
@@ -460,13 +465,15 @@ __global__ void __launch_bounds__(256) a4_quant_kernel(const uint4 *__restrict__
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
                                                        const float *__restrict__ part, float *__restrict__ xscale,
-                                                       uint8_t *__restrict__ bblob) {
+                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ cnt,
+                                                       int ncnt) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     __shared__ float s_sg;
     pdl_wait();
     pdl_release();
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     if (warp == 0) {
@@ -523,6 +530,7 @@ struct MxSmem {
     uint32_t tmem_base;
     int abort_flag;
     int total_items;
+    int last_tok[2][128];             // fused combine: token whose last pair an item's row completed, or -1
     // followed by int tile_start[E + 1], off[E + 1], slot[E]
 };
 
@@ -928,6 +936,42 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             if (!ok) break;
             tc_fence_before();
             mbar_arrive(&sm.accempty[bi]);
+            if (PHASE == kPhaseDown && p.comb_out) {
+                // Fused combine. This item's y rows (channels 128 m .. 128 m + 127) are written:
+                // count each row's pair for (token, M tile); the item that brings a count to k
+                // adds that token's k rows for these channels, in order of j, as the combine does.
+                const int gt = lrow;                    // thread index in the epilogue group
+                int *flags = sm.last_tok[grp];
+                __threadfence();                        // y of this thread before the counts below
+                named_bar_sync(1 + grp, 128);
+                for (int tok = gt; tok < it.nvalid; tok += 128) {
+                    const int t = __ldcg(p.sorted_pair + it.row0 + tok) / p.k;
+                    const int old = atomicAdd(p.cnt + (int64_t)t * p.m_tiles + it.m, 1);
+                    flags[tok] = old == p.k - 1 ? t : -1;
+                }
+                named_bar_sync(1 + grp, 128);
+                const int ch = it.m * 128 + lrow;
+                for (int tok = 0; tok < it.nvalid; ++tok) {
+                    const int t = flags[tok];
+                    if (t < 0) continue;
+                    __threadfence();                    // the other pairs' y rows are visible
+                    float acc = 0.0f;
+                    for (int j = 0; j < p.k; ++j) {
+                        int rr = __ldcg(p.pair_row + (int64_t)t * p.k + j);
+                        if (rr < 0 || rr >= p.n_rows) {
+                            flag_error(2);
+                            rr = 0;
+                        }
+                        const float wj = __ldcg(p.gate_w + (int64_t)t * p.k + j);
+                        const int64_t o = (int64_t)rr * p.H + ch;
+                        const float yv = p.out_fp32 ? __ldcg(reinterpret_cast<const float *>(p.out) + o)
+                                                    : __bfloat162float(__ldcg(reinterpret_cast<const __nv_bfloat16 *>(p.out) + o));
+                        acc = fmaf(wj, yv, acc);
+                    }
+                    reinterpret_cast<__nv_bfloat16 *>(p.comb_out)[(int64_t)t * p.H + ch] = __float2bfloat16_rn(acc);
+                }
+                named_bar_sync(1 + grp, 128);           // flags are rewritten by the next item
+            }
         }
     }
 
@@ -1061,7 +1105,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
 
 moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
-                           cudaStream_t st) {
+                           cudaStream_t st, int32_t *cnt, int ncnt) {
     if (P == 0) return MOE_OK;
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
@@ -1069,13 +1113,13 @@ moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *so
     if (fmt == kBsNv) {   // one block per row
         const int blocks = P < num_sms * 8 ? P : num_sms * 8;
         e = launch_pdl(nv_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
-                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp);
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp, cnt, ncnt);
     } else {              // one warp per (row, stage)
         if (mode == 2) return set_error(MOE_ERR_UNSUPPORTED, "MXFP4 quantiser mode 2");
         const int64_t units = (int64_t)P * (K / kMxStageK);
         const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
         e = launch_pdl(mx_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
-                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob));
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), cnt, ncnt);
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "block-scaled quantiser launch");
@@ -1095,7 +1139,7 @@ moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cud
 
 moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, const float *partials, float *xscale, void *bblob,
-                           int num_sms, cudaStream_t st) {
+                           int num_sms, cudaStream_t st, int32_t *cnt, int ncnt) {
     if (P == 0) return MOE_OK;
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
@@ -1103,7 +1147,7 @@ moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair
     const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
     cudaError_t e = launch_pdl(a4_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
                                mode, sorted_pair, k, P, K, offsets, E, BN, partials, xscale,
-                               reinterpret_cast<uint8_t *>(bblob));
+                               reinterpret_cast<uint8_t *>(bblob), cnt, ncnt);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 quantiser launch");
 }
