@@ -216,7 +216,7 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 // atoms) of x and of h; NVFP4 also keeps h in bf16 at offset 0 and the per-row
 // exponent offsets of x and h.
 struct FfnWs {
-    size_t h, re1, re2, a4, b1, b2, total;
+    size_t h, re1, re2, a4, tq, b1, b2, total;
 };
 
 // h: bf16 [n][I] (the decoding paths' h buffer; NVFP4: h before its
@@ -231,6 +231,7 @@ static FfnWs ffn_ws(int n, int H, int I, int E) {
     W.re1 = o; o += align_up((size_t)n * 4, 256);
     W.re2 = o; o += align_up((size_t)n * 4, 256);
     W.a4 = o; o += align_up((size_t)(1 + kA4Parts) * 4, 256);
+    W.tq = o; o += align_up((size_t)n * H / 2, 256) + align_up((size_t)n * H / 16, 256);   // A4 token rows
     W.b1 = o; o += std::max(mx_blob_bytes(n, H, E), a4_blob_bytes(n, H, E));
     W.b2 = o; o += std::max(mx_blob_bytes(n, I, E), a4_blob_bytes(n, I, E));
     W.total = o;
@@ -344,9 +345,18 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
     float *xscale = reinterpret_cast<float *>(b + W.a4), *parts = xscale + 1;
     moe_status r = launch_a4_amax(amax_src, amax_elems, parts, st);
-    if (r == MOE_OK)
-        r = launch_a4_quant(x_src, gather ? 1 : 2, sorted_pair, k, n_rows, H, offsets, E, BN, parts, xscale, b + W.b1,
-                            nsm, st, cf ? cf->cnt : nullptr, cf ? cf->T * (H / 128) : 0);
+    if (r == MOE_OK && gather) {
+        // token rows: quantise each token once (amax_elems / H of them), then place its k pairs
+        const int T = (int)(amax_elems / H);
+        uint8_t *codes = b + W.tq, *scales = codes + align_up((size_t)n_rows * H / 2, 256);
+        r = launch_a4_token_quant(x_src, T, H, parts, xscale, codes, scales, cf ? cf->cnt : nullptr,
+                                  cf ? cf->T * (H / 128) : 0, nsm, st);
+        if (r == MOE_OK)
+            r = launch_a4_scatter(codes, scales, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1, nsm, st);
+    } else if (r == MOE_OK) {
+        r = launch_a4_quant(x_src, 2, sorted_pair, k, n_rows, H, offsets, E, BN, parts, xscale, b + W.b1, nsm, st,
+                            cf ? cf->cnt : nullptr, cf ? cf->T * (H / 128) : 0);
+    }
     if (r != MOE_OK) return r;
     MxParams p;
     memset(&p, 0, sizeof(p));
