@@ -250,32 +250,11 @@ static bool use_bs(int fmt, int layout, int n_rows, int E) {
 }
 static bool is_mx(const moe_experts &x, int n_rows) { return use_bs(x.fmt, x.layout, n_rows, x.E); }
 
-// The combine fused into the down pass of the block-scaled paths (layer forward):
-// out[t] = sum_j w[t,j] y_perm[pair_row[t k + j]], added by the down pass's epilogue
-// once all k rows of a token are written, with per-(token, M tile) counters.
-struct CombineFuse {
-    void *out;
-    const int32_t *pair_row;
-    const float *w;
-    int32_t *cnt;   // [T][H / 128]
-    int T;
-};
-
-static void fuse_combine(MxParams &p, const CombineFuse *cf, const int32_t *sorted_pair, int k) {
-    if (!cf) return;
-    p.comb_out = cf->out;
-    p.sorted_pair = sorted_pair;
-    p.pair_row = cf->pair_row;
-    p.gate_w = cf->w;
-    p.cnt = cf->cnt;
-    p.k = k;
-}
-
 // Block-scaled FP4 grouped FFN. The activations are quantised first: gathered
 // from token rows x[sorted_pair[r] / k] (gather != 0) or read from x_perm.
 static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sorted_pair, int k, int n_rows,
                               const int32_t *offsets, const moe_experts *x, void *y_perm, int y_is_fp32, void *ws,
-                              cudaStream_t st, const CombineFuse *cf = nullptr) {
+                              cudaStream_t st) {
     if (n_rows == 0) return MOE_OK;
     const int E = x->E, H = x->H, I = x->I;
     const int fmt = x->fmt == MOE_NVFP4 ? kBsNv : kBsMx;
@@ -286,7 +265,7 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
     int32_t *re1 = reinterpret_cast<int32_t *>(b + W.re1), *re2 = reinterpret_cast<int32_t *>(b + W.re2);
     moe_status r = launch_mx_quant(fmt, x_src, gather ? 1 : 0, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1,
-                                   re1, nsm, st, cf ? cf->cnt : nullptr, cf ? cf->T * (H / 128) : 0);
+                                   re1, nsm, st);
     if (r != MOE_OK) return r;
     MxParams p;
     memset(&p, 0, sizeof(p));
@@ -323,7 +302,6 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.hout = nullptr;
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
-    fuse_combine(p, cf, sorted_pair, k);
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 
@@ -332,8 +310,7 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
 // when gathering (every token appears k times among the pairs), else x_perm.
 static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_src, int64_t amax_elems,
                               const int32_t *sorted_pair, int k, int n_rows, const int32_t *offsets,
-                              const moe_experts *x, void *y_perm, int y_is_fp32, void *ws, cudaStream_t st,
-                              const CombineFuse *cf = nullptr) {
+                              const moe_experts *x, void *y_perm, int y_is_fp32, void *ws, cudaStream_t st) {
     if (n_rows == 0) return MOE_OK;
     if (x->fmt != MOE_NVFP4 || x->layout != MOE_LAYOUT_TILED)
         return set_error(MOE_ERR_UNSUPPORTED, "A4 activations need prepacked NVFP4 experts");
@@ -349,13 +326,11 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
         // token rows: quantise each token once (amax_elems / H of them), then place its k pairs
         const int T = (int)(amax_elems / H);
         uint8_t *codes = b + W.tq, *scales = codes + align_up((size_t)n_rows * H / 2, 256);
-        r = launch_a4_token_quant(x_src, T, H, parts, xscale, codes, scales, cf ? cf->cnt : nullptr,
-                                  cf ? cf->T * (H / 128) : 0, nsm, st);
+        r = launch_a4_token_quant(x_src, T, H, parts, xscale, codes, scales, nsm, st);
         if (r == MOE_OK)
             r = launch_a4_scatter(codes, scales, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1, nsm, st);
     } else if (r == MOE_OK) {
-        r = launch_a4_quant(x_src, 2, sorted_pair, k, n_rows, H, offsets, E, BN, parts, xscale, b + W.b1, nsm, st,
-                            cf ? cf->cnt : nullptr, cf ? cf->T * (H / 128) : 0);
+        r = launch_a4_quant(x_src, 2, sorted_pair, k, n_rows, H, offsets, E, BN, parts, xscale, b + W.b1, nsm, st);
     }
     if (r != MOE_OK) return r;
     MxParams p;
@@ -387,7 +362,6 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
     p.xscale = nullptr;
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
-    fuse_combine(p, cf, sorted_pair, k);
     return launch_mx_phase(kBsNv, kPhaseDown, BN, p, nsm, st, 1);
 }
 
@@ -453,7 +427,7 @@ static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t
 
 // workspace layout of moe_layer_forward
 struct LayerWs {
-    size_t router, idx, w, offsets, sorted, pair_row, perm, x_perm, h, y, cnt, total;
+    size_t router, idx, w, offsets, sorted, pair_row, perm, x_perm, h, y, total;
 };
 
 static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
@@ -470,7 +444,6 @@ static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
     L.x_perm = o; o += align_up(P * H * 2, 256);
     L.h = o; o += ffn_ws_bytes((int)P, H, I, E);
     L.y = o; o += align_up(P * H * (y32 ? 4 : 2), 256);
-    L.cnt = o; o += align_up((size_t)T * (H / 128 + 1) * 4, 256);
     L.total = o;
     return L;
 }
@@ -714,18 +687,15 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     r = check_experts(&view);
     if (r == MOE_OK && !a4 && is_mx(view, T * k) != mx)
         r = set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
-    // the block-scaled paths combine in their down pass; the decoding path has its own launch
-    const CombineFuse cf{out, prow, w, reinterpret_cast<int32_t *>(b + L.cnt), T};
     if (r == MOE_OK) {
         if (a4)
-            r = a4_ffn_impl(x, 1, x, (int64_t)T * H, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st,
-                            &cf);
+            r = a4_ffn_impl(x, 1, x, (int64_t)T * H, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
         else if (mx)
-            r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st, &cf);
+            r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
         else
             r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
     }
-    if (r == MOE_OK && !mx) r = moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
+    if (r == MOE_OK) r = moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
     if (cache) cache_compute_end(cache, st);   // closes the call's timing record in every case
     return r;
 }

@@ -297,15 +297,12 @@ __device__ __forceinline__ void bf16x8_to_float(uint4 u, float (&v)[8]) {
 __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
-                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ cnt,
-                                                       int ncnt) {
+                                                       uint8_t *__restrict__ bblob) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     pdl_wait();
     pdl_release();
-    // the fused combine's counters start at zero for the down pass of this call
-    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsMx, BN);
@@ -350,15 +347,13 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
 __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
-                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp,
-                                                       int32_t *__restrict__ cnt, int ncnt) {
+                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     __shared__ uint32_t s_max[8];
     pdl_wait();
     pdl_release();
-    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsNv, BN);
@@ -465,15 +460,13 @@ __global__ void __launch_bounds__(256) a4_quant_kernel(const uint4 *__restrict__
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
                                                        const float *__restrict__ part, float *__restrict__ xscale,
-                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ cnt,
-                                                       int ncnt) {
+                                                       uint8_t *__restrict__ bblob) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     __shared__ float s_sg;
     pdl_wait();
     pdl_release();
-    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     if (warp == 0) {
@@ -520,17 +513,14 @@ __global__ void __launch_bounds__(256) a4_quant_kernel(const uint4 *__restrict__
 // A4 form of the token rows, once per token (the layer forward, where each token is
 // in k pairs): the same arithmetic as a4_quant_kernel, one warp per (token t, 256-wide
 // stage), written token-major: codes[t][stage] 128 bytes (natural order, low nibble =
-// lower K index), scales[t][stage] 16 E4M3 bytes. Block 0 also stores s_g in *xscale
-// and every block zeroes its share of the fused combine's counters.
+// lower K index), scales[t][stage] 16 E4M3 bytes. Block 0 also stores s_g in *xscale.
 __global__ void __launch_bounds__(256) a4_token_kernel(const uint4 *__restrict__ x, int T, int K,
                                                        const float *__restrict__ part, float *__restrict__ xscale,
-                                                       uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                                                       int32_t *__restrict__ cnt, int ncnt) {
+                                                       uint8_t *__restrict__ codes, uint8_t *__restrict__ scales) {
     __shared__ float s_sg;
     pdl_wait();
     pdl_release();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = blockIdx.x * 256 + threadIdx.x; i < ncnt; i += gridDim.x * 256) cnt[i] = 0;
     if (warp == 0) {
         uint32_t m = 0u;
         for (int i = lane; i < kA4Parts; i += 32) m = max(m, __float_as_uint(__ldcg(part + i)));
@@ -614,7 +604,6 @@ struct MxSmem {
     uint32_t tmem_base;
     int abort_flag;
     int total_items;
-    int last_tok[2][128];             // fused combine: token whose last pair an item's row completed, or -1
     // followed by int tile_start[E + 1], off[E + 1], slot[E]
 };
 
@@ -1020,42 +1009,6 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             if (!ok) break;
             tc_fence_before();
             mbar_arrive(&sm.accempty[bi]);
-            if (PHASE == kPhaseDown && p.comb_out) {
-                // Fused combine. This item's y rows (channels 128 m .. 128 m + 127) are written:
-                // count each row's pair for (token, M tile); the item that brings a count to k
-                // adds that token's k rows for these channels, in order of j, as the combine does.
-                const int gt = lrow;                    // thread index in the epilogue group
-                int *flags = sm.last_tok[grp];
-                __threadfence();                        // y of this thread before the counts below
-                named_bar_sync(1 + grp, 128);
-                for (int tok = gt; tok < it.nvalid; tok += 128) {
-                    const int t = __ldcg(p.sorted_pair + it.row0 + tok) / p.k;
-                    const int old = atomicAdd(p.cnt + (int64_t)t * p.m_tiles + it.m, 1);
-                    flags[tok] = old == p.k - 1 ? t : -1;
-                }
-                named_bar_sync(1 + grp, 128);
-                const int ch = it.m * 128 + lrow;
-                for (int tok = 0; tok < it.nvalid; ++tok) {
-                    const int t = flags[tok];
-                    if (t < 0) continue;
-                    __threadfence();                    // the other pairs' y rows are visible
-                    float acc = 0.0f;
-                    for (int j = 0; j < p.k; ++j) {
-                        int rr = __ldcg(p.pair_row + (int64_t)t * p.k + j);
-                        if (rr < 0 || rr >= p.n_rows) {
-                            flag_error(2);
-                            rr = 0;
-                        }
-                        const float wj = __ldcg(p.gate_w + (int64_t)t * p.k + j);
-                        const int64_t o = (int64_t)rr * p.H + ch;
-                        const float yv = p.out_fp32 ? __ldcg(reinterpret_cast<const float *>(p.out) + o)
-                                                    : __bfloat162float(__ldcg(reinterpret_cast<const __nv_bfloat16 *>(p.out) + o));
-                        acc = fmaf(wj, yv, acc);
-                    }
-                    reinterpret_cast<__nv_bfloat16 *>(p.comb_out)[(int64_t)t * p.H + ch] = __float2bfloat16_rn(acc);
-                }
-                named_bar_sync(1 + grp, 128);           // flags are rewritten by the next item
-            }
         }
     }
 
@@ -1189,7 +1142,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
 
 moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
-                           cudaStream_t st, int32_t *cnt, int ncnt) {
+                           cudaStream_t st) {
     if (P == 0) return MOE_OK;
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
@@ -1197,13 +1150,13 @@ moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *so
     if (fmt == kBsNv) {   // one block per row
         const int blocks = P < num_sms * 8 ? P : num_sms * 8;
         e = launch_pdl(nv_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
-                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp, cnt, ncnt);
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp);
     } else {              // one warp per (row, stage)
         if (mode == 2) return set_error(MOE_ERR_UNSUPPORTED, "MXFP4 quantiser mode 2");
         const int64_t units = (int64_t)P * (K / kMxStageK);
         const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
         e = launch_pdl(mx_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
-                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), cnt, ncnt);
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob));
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "block-scaled quantiser launch");
@@ -1223,7 +1176,7 @@ moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cud
 
 moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, const float *partials, float *xscale, void *bblob,
-                           int num_sms, cudaStream_t st, int32_t *cnt, int ncnt) {
+                           int num_sms, cudaStream_t st) {
     if (P == 0) return MOE_OK;
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
@@ -1231,7 +1184,7 @@ moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair
     const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
     cudaError_t e = launch_pdl(a4_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
                                mode, sorted_pair, k, P, K, offsets, E, BN, partials, xscale,
-                               reinterpret_cast<uint8_t *>(bblob), cnt, ncnt);
+                               reinterpret_cast<uint8_t *>(bblob));
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 quantiser launch");
 }
@@ -1241,13 +1194,13 @@ moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair
 namespace moe {
 
 moe_status launch_a4_token_quant(const void *x, int T, int K, const float *partials, float *xscale, void *codes,
-                                 void *scales, int32_t *cnt, int ncnt, int num_sms, cudaStream_t st) {
+                                 void *scales, int num_sms, cudaStream_t st) {
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
     const int64_t units = (int64_t)T * (K / kMxStageK);
     const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
     cudaError_t e = launch_pdl(a4_token_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st,
                                reinterpret_cast<const uint4 *>(x), T, K, partials, xscale,
-                               reinterpret_cast<uint8_t *>(codes), reinterpret_cast<uint8_t *>(scales), cnt, ncnt);
+                               reinterpret_cast<uint8_t *>(codes), reinterpret_cast<uint8_t *>(scales));
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 token quantiser launch");
 }

@@ -76,13 +76,6 @@ struct MxParams {
     uint8_t *bblob_out;         // MXFP4 and A4 up: blobs of h for the down pass [tiles][I/256]
     void *hout;                 // NVFP4 up: h bf16 [n_rows][I]
     const float *xscale;        // A4 up: device word with the per-tensor scale of x
-    // down, layer forward only: the combine fused into the epilogue (comb_out = NULL: none)
-    void *comb_out;             // out bf16 [T][H]
-    const int32_t *sorted_pair; // [n_rows]
-    const int32_t *pair_row;    // [n_rows]
-    const float *gate_w;        // [T][k]
-    int32_t *cnt;               // [T][m_tiles], zeroed by the x quantiser of the same call
-    int k;
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -118,18 +111,17 @@ moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cud
 // Token-major A4 rows of x [T][K] (codes [T][K/2], scales [T][K/16]), then their scatter into
 // the blobs of the pairs (the layer forward's path: each token quantised once, not k times).
 moe_status launch_a4_token_quant(const void *x, int T, int K, const float *partials, float *xscale, void *codes,
-                                 void *scales, int32_t *cnt, int ncnt, int num_sms, cudaStream_t st);
+                                 void *scales, int num_sms, cudaStream_t st);
 moe_status launch_a4_scatter(const void *codes, const void *scales, const int32_t *sorted_pair, int k, int P, int K,
                              const int32_t *offsets, int E, int BN, void *bblob, int num_sms, cudaStream_t st);
 moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, const float *partials, float *xscale, void *bblob,
-                           int num_sms, cudaStream_t st, int32_t *cnt = nullptr, int ncnt = 0);
+                           int num_sms, cudaStream_t st);
 // src rows: mode 0 x_perm[r] (operand order), 1 x[sorted_pair[r] / k] (natural
 // order), 2 src[r] (natural order; NVFP4 only). rowexp: NVFP4 only.
-// cnt[0..ncnt) (nullable): counters of the fused combine, zeroed by this launch.
 moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
-                           cudaStream_t st, int32_t *cnt = nullptr, int ncnt = 0);
+                           cudaStream_t st);
 
 moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           cudaStream_t st);

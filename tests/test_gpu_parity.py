@@ -285,8 +285,8 @@ def test_layer_decode_mxfp4(moe, decode_layer, T):
 
 def test_layer_fused_routing_and_permutation(moe, decode_layer):
     """On the block-scaled path a small batch routes and permutes in one router
-    launch (the last cluster to finish sorts the pairs by expert) and the down
-    pass combines, so a layer call is 4 kernels: router, quantiser, UP, DOWN. CUDA-graph replays reuse one launch's arguments, the
+    launch (the last cluster to finish sorts the pairs by expert), so a layer
+    call is 5 kernels: router, quantiser, UP, DOWN, combine. CUDA-graph replays reuse one launch's arguments, the
     ticket epoch included; each replay must give the eager result."""
     L = decode_layer.to("cuda")
     ex = moe.moe_prepack(moe.Experts.from_layer(L))
@@ -296,7 +296,7 @@ def test_layer_fused_routing_and_permutation(moe, decode_layer):
     out = torch.empty(T, L.H, dtype=torch.bfloat16, device="cuda")
     n0 = moe.moe_kernel_launch_count()
     ref = moe.moe_layer_forward(x, L.wr, L.k, ex, bias=L.bias, ws=ws, out=out).clone()
-    assert moe.moe_kernel_launch_count() - n0 == 4
+    assert moe.moe_kernel_launch_count() - n0 == 5
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -561,8 +561,8 @@ def test_layer_on_more_streams_than_ticket_counters(moe, decode_layer):
         torch.cuda.synchronize()
         for h in handles:
             rt.cudaStreamDestroy(h)
-    # fused (4 launches) while counters last, then routing and permutation apart (5)
-    assert launches[-1] == 5 and set(launches) <= {4, 5}
+    # fused (5 launches) while counters last, then routing and permutation apart (6)
+    assert launches[-1] == 6 and set(launches) <= {5, 6}
     assert launches == sorted(launches)
     assert moe.moe_device_error() == 0
 
