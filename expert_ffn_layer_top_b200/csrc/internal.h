@@ -133,6 +133,10 @@ size_t router_ws_bytes(int T, int H, int E);
 struct RouterFuse {
     int32_t *offsets, *sorted_pair, *pair_row;
     unsigned int *ticket;
+    // L2 prefetch of the expert weights the grouped FFN reads first (static data, issued
+    // before the router waits on its predecessor): pf_bytes from pf_base, 0 = none
+    const uint8_t *pf_base;
+    int64_t pf_bytes;
 };
 // fuse may be null; *fused (if given) tells whether the permutation was done.
 moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
