@@ -842,6 +842,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         bool ok = true;
         for (int item = blockIdx.x + grp * gridDim.x; item < total && ok; item += 2 * gridDim.x, lt += 2) {
             const MxItem it = mx_item(tab, p, item, BN);
+            // NVFP4: the expert's tensor scale (A4 UP: times that of x), loaded once per item while
+            // the accumulators are still being computed
+            float iscale = 1.0f;
+            if constexpr (FMT == kBsNv) {
+                iscale = p.tscale[it.e];
+                if constexpr (PL == 1 && PHASE == kPhaseUp) iscale *= __ldcg(p.xscale);
+            }
             // lt: the item's index in this CTA. Item-parallel: pipeline lt % NP, its item lt / NP.
             const int wi = IP ? lt % NP : 0, li = IP ? lt / NP : lt;
             const int a = li & 1, bi = IP ? 2 * wi + a : a;
@@ -886,16 +893,16 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                             for (int j = 0; j < 16; ++j) val[j] = fmaf(__uint_as_float(v[pl][j]), kPw[pl], val[j]);
                     }
                 }
-                if constexpr (PL == 1) {   // A4: the tensor scales of x (UP; h has 1) and of the weights
-                    const float f = (PHASE == kPhaseUp ? __ldcg(p.xscale) : 1.0f) * p.tscale[it.e];
+                if constexpr (PL == 1) {   // A4: the tensor scales of the weights and (UP) of x; h has 1
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) val[j] *= f;
+                    for (int j = 0; j < CH; ++j) val[j] *= iscale;
                 } else if constexpr (FMT == kBsNv) {   // 2^-C of each token row, times the expert's tensor scale
-                    const float ts = p.tscale[it.e];
+                    // one load per lane (token c0 + lane), handed to the other lanes
+                    const int Cl = (lane < CH && c0 + lane < it.nvalid) ? __ldcg(p.rowexp + it.row0 + c0 + lane) : 0;
 #pragma unroll
                     for (int j = 0; j < CH; ++j) {
-                        const int C = c0 + j < it.nvalid ? __ldcg(p.rowexp + it.row0 + c0 + j) : 0;
-                        val[j] *= exp2_neg_biased(C + 127) * ts;
+                        const int C = __shfl_sync(0xffffffffu, Cl, j);
+                        val[j] *= exp2_neg_biased(C + 127) * iscale;
                     }
                 }
                 if (PHASE == kPhaseDown) {
