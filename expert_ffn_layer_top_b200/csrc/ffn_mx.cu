@@ -842,19 +842,20 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         bool ok = true;
         for (int item = blockIdx.x + grp * gridDim.x; item < total && ok; item += 2 * gridDim.x, lt += 2) {
             const MxItem it = mx_item(tab, p, item, BN);
-            // NVFP4: the expert's tensor scale (A4 UP: times that of x), loaded once per item while
-            // the accumulators are still being computed
+            // NVFP4: the expert's tensor scale (static data), loaded once per item while the
+            // accumulators are still being computed
             float iscale = 1.0f;
-            if constexpr (FMT == kBsNv) {
-                iscale = p.tscale[it.e];
-                if constexpr (PL == 1 && PHASE == kPhaseUp) iscale *= __ldcg(p.xscale);
-            }
+            if constexpr (FMT == kBsNv) iscale = p.tscale[it.e];
             // lt: the item's index in this CTA. Item-parallel: pipeline lt % NP, its item lt / NP.
             const int wi = IP ? lt % NP : 0, li = IP ? lt / NP : lt;
             const int a = li & 1, bi = IP ? 2 * wi + a : a;
             const int wlo = IP ? wi : 0, whi = IP ? wi + 1 : NP;   // accumulators to add
             if (!mbar_wait(&sm.accfull[bi], (li >> 1) & 1, abort_flag)) break;
             tc_fence_after();
+            // A4 UP: the tensor scale of x comes from the quantiser just before this kernel. It is
+            // read only now: the accumulators hold its output, so the producer has passed the wait
+            // on that kernel (these warps do not wait on it themselves).
+            if constexpr (PL == 1 && PHASE == kPhaseUp) iscale *= __ldcg(p.xscale);
             const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NW * N);
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
             constexpr int HCH = CH / 2;             // UP: tokens per warp of a gate/up pair
