@@ -600,6 +600,8 @@ struct MxSmem {
                               // item-parallel: [2 pipeline + buffer], that pipeline's MMA warp
     uint64_t accempty[8];     // the epilogue group that read the buffer (128 threads)
     uint64_t mmadone[4];
+    uint64_t sfrdy[4];              // token-major mode: a scale group's copies landed (both helpers)
+    uint64_t hdone[2];              // token-major mode: a helper's last copies landed
     uint64_t xfull[2], xempty[2];   // gate/up exchange, per epilogue group
     uint32_t tmem_base;
     int abort_flag;
@@ -653,6 +655,11 @@ template <int FMT, int PHASE, int BN, int PL>
 __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_constant__ MxParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     static_assert(PL == kMxPlanes || (PL == 1 && FMT == kBsNv), "A4 activations are NVFP4");
+    // Token-major accumulators (A4 with tiles of 128 tokens): the MMA takes the 128 tokens as
+    // its A operand (M) and the 128 weight rows as B (N), so a TMEM lane holds one token's
+    // outputs. The UP epilogue then finds a channel's gate and up values in one thread, and
+    // DOWN writes a token's 128 outputs as whole vectors. Smaller tiles keep the weights on M.
+    constexpr bool TM = PL == 1 && BN == 128;
     constexpr int N = PL * BN;                              // MMA N: the planes' rows
     constexpr int NW = N <= 32 ? 4 : (N <= 64 ? 2 : 1);    // pipelines TMEM has room for
     constexpr int NA = bs_atoms(FMT);                       // scale atoms per operand and stage
@@ -661,6 +668,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
     constexpr int STAGE = ABLOB + BBLOB;                    // a multiple of 1024
     constexpr uint32_t SFCOL = 2 * NW * N;
     static_assert(SFCOL + NW * 16 * NA <= 512, "TMEM columns");
+    static_assert(!TM || SFCOL + 4 * 8 * NA <= 512, "TMEM columns of the token-major mode");
     const int NP = p.pipes;                                 // <= NW; stage-parallel: divides the stages per item
     const int NSW = p.stages / NP;                          // slots per pipeline
 
@@ -695,6 +703,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             mbar_init(&sm.xempty[a], 128);
         }
         for (int w = 0; w < 4; ++w) mbar_init(&sm.mmadone[w], 1);
+        for (int g = 0; g < 4; ++g) mbar_init(&sm.sfrdy[g], 2);
+        for (int h = 0; h < 2; ++h) mbar_init(&sm.hdone[h], 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -783,10 +793,80 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                 }
             }
         }
+    } else if (TM && (warp == 13 || warp == 14) && lane == 0) {
+        // =================================================== scale copies (token-major mode)
+        // One thread issues the stage's scale-atom copies into TMEM at about 23 ns each, so the
+        // MMA thread, left alone, would wait on them: warp 13 copies the weights' atoms and warp
+        // 14 the activations', into one of G rotating column groups, and each commits to the
+        // group's barrier, which the MMA warp waits on. A group is refilled only after the
+        // MMAs of the stage G back (the slot's empty barrier) have completed.
+        const int h = warp - 13;
+        const int G = NSW - 1 < 4 ? NSW - 1 : 4;   // < NSW: empty barriers cannot alias
+        const uint32_t base_u32 = smem_u32(base);
+        int j = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            for (int k = 0; k < KST; ++k, ++j) {
+                const int s = j % NSW;
+                if (!mbar_wait(&sm.full[s], (uint32_t)((j / NSW) & 1), abort_flag)) { ok = false; break; }
+                if (j >= G && !mbar_wait(&sm.empty[(j - G) % NSW], (uint32_t)(((j - G) / NSW) & 1), abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sp = base_u32 + s * STAGE;
+                const uint32_t sfg = tmem + SFCOL + 32 * (j % G) + 16 * h;
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+                    tmem_cp_atom(sfg + 4 * a, sf_atom_desc(h == 0 ? sp + kMxCodeBytes + 512 * a : sp + ABLOB + N * 128 + 512 * a));
+                mma_commit(&sm.sfrdy[j % G]);
+            }
+        }
+        mma_commit(&sm.hdone[h]);   // never leave with a copy into TMEM in flight
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&sm.hdone[h], 0)) {
+            if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
+        }
     } else if (warp >= 12) {
         // =================================================== MMA issuer of pipeline w
         const int w = warp - 12;
-        if (lane == 0 && w < NP) {
+        if (TM && lane == 0 && w == 0) {
+            // token-major mode: the scales come from the helper warps (above)
+            const int G = NSW - 1 < 4 ? NSW - 1 : 4;
+            int loc = 0, lt = 0;
+            bool ok = true;
+            const uint32_t base_u32 = smem_u32(base);
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
+                const int a = lt & 1;
+                if (!mbar_wait(&sm.accempty[a], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(a * N);
+                for (int k = 0; k < KST; ++k, ++loc) {
+                    const int s = loc % NSW, g = loc % G;
+                    if (!mbar_wait(&sm.full[s], (uint32_t)((loc / NSW) & 1), abort_flag) ||
+                        !mbar_wait(&sm.sfrdy[g], (uint32_t)((loc / G) & 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sp = base_u32 + s * STAGE;
+                    const uint32_t sfw = tmem + SFCOL + 32 * g, sfx = sfw + 16;
+                    const uint64_t wdesc = smem_desc_sw128(sp), xdesc = smem_desc_sw128(sp + ABLOB);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)   // tokens as A, weights as B; K = 64 each
+                        mma_nvf4(d, xdesc + (uint64_t)(2 * i), wdesc + (uint64_t)(2 * i), idesc_nvf4(N), sfx + 4 * i,
+                                 sfw + 4 * i, (k | i) != 0);
+                    mma_commit(&sm.empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&sm.accfull[a]);
+            }
+            mma_commit(&sm.mmadone[0]);
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&sm.mmadone[0], 0)) {
+                if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
+            }
+        } else if (!TM && lane == 0 && w < NP) {
             int loc = 0, lt = 0, sc = 0;
             bool ok = true;
             const uint32_t base_u32 = smem_u32(base);
@@ -857,6 +937,78 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             // on that kernel (these warps do not wait on it themselves).
             if constexpr (PL == 1 && PHASE == kPhaseUp) iscale *= __ldcg(p.xscale);
             const uint32_t acc0 = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NW * N);
+            if constexpr (TM) {
+                // this thread's token is TMEM lane tok of the tile
+                const int tok = q * 32 + lane;
+                const bool valid = tok < it.nvalid;
+                if constexpr (PHASE == kPhaseUp) {
+                    // columns 0..63: gate of channels 64 m ..; 64..127: up of the same channels. h
+                    // goes out in A4 form, 16 channels (one scale block) at a time.
+                    uint8_t *blob = p.bblob_out + ((int64_t)it.rt * (p.I / kMxStageK) + ((it.m * 64) >> 8)) * BBLOB;
+#pragma unroll 1
+                    for (int blk = 0; blk < 4; ++blk) {
+                        uint32_t G[16], U[16];
+                        tmem_ld16(acc0 + blk * 16, G);
+                        tmem_ld16(acc0 + 64 + blk * 16, U);
+                        tmem_wait_ld();
+                        float h[16], amax = 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float g = __uint_as_float(G[j]) * iscale, uu = __uint_as_float(U[j]) * iscale;
+                            h[j] = __fdividef(g, 1.0f + __expf(-g)) * uu;
+                            amax = fmaxf(amax, fabsf(h[j]));
+                        }
+                        const uint32_t sc = e4m3_code(__fdiv_rn(amax, 6.0f));
+                        const float sb = e4m3_value(sc);
+                        float t[8], qv[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) t[j] = sb > 0.0f ? __fdiv_rn(h[j], sb) : 0.0f;
+                        const uint32_t w0 = e2m1x8(t, qv);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) t[j] = sb > 0.0f ? __fdiv_rn(h[8 + j], sb) : 0.0f;
+                        const uint32_t w1 = e2m1x8(t, qv);
+                        if (valid) {
+                            const int c = (it.m * 64 + blk * 16) & 255;   // first channel within the stage
+                            *reinterpret_cast<uint2 *>(blob + sw128_chunk(tok, c >> 5) + ((c & 31) >> 1)) =
+                                make_uint2(w0, w1);
+                            const int b16 = c >> 4;
+                            blob[N * 128 + (b16 >> 2) * 512 + atom_offset(tok, b16 & 3)] = (uint8_t)sc;
+                        }
+                    }
+                } else {
+                    // the token's 128 outputs of this M tile, 16 at a time
+                    const int64_t o = (int64_t)(it.row0 + tok) * p.H + it.m * 128;
+#pragma unroll 1
+                    for (int blk = 0; blk < 8; ++blk) {
+                        uint32_t V[16];
+                        tmem_ld16(acc0 + blk * 16, V);
+                        tmem_wait_ld();
+                        if (valid) {
+                            float f[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(V[j]) * iscale;
+                            if (p.out_fp32) {
+                                float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + o + blk * 16);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) dst[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+                            } else {
+                                uint32_t w[8];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * j], f[2 * j + 1]);
+                                    w[j] = *reinterpret_cast<const uint32_t *>(&b2);
+                                }
+                                uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + o + blk * 16);
+                                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.accempty[bi]);
+                continue;
+            }
             constexpr int CH = BN < 16 ? BN : 16;   // tokens per chunk
             constexpr int HCH = CH / 2;             // UP: tokens per warp of a gate/up pair
             for (int c0 = 0; c0 < BN && ok; c0 += CH, ++xc) {
@@ -947,7 +1099,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                         for (int j = 0; j < HCH; ++j) {
                             const float g = gate ? val[j] : other[j];
                             const float uu = gate ? other[j] : val[HCH + j];
-                            const float hv = g / (1.0f + expf(-g)) * uu;
+                            const float hv = __fdividef(g, 1.0f + __expf(-g)) * uu;
                             float amax = fabsf(hv);
 #pragma unroll
                             for (int d = 1; d < 16; d <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
