@@ -976,13 +976,18 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                         }
                     }
                 } else {
-                    // the token's 128 outputs of this M tile, 16 at a time
+                    // the token's 128 outputs of this M tile, 32 at a time (two loads, one wait)
                     const int64_t o = (int64_t)(it.row0 + tok) * p.H + it.m * 128;
 #pragma unroll 1
-                    for (int blk = 0; blk < 8; ++blk) {
-                        uint32_t V[16];
-                        tmem_ld16(acc0 + blk * 16, V);
+                    for (int b2 = 0; b2 < 8; b2 += 2) {
+                        uint32_t V2[2][16];
+                        tmem_ld16(acc0 + b2 * 16, V2[0]);
+                        tmem_ld16(acc0 + b2 * 16 + 16, V2[1]);
                         tmem_wait_ld();
+#pragma unroll
+                        for (int hb = 0; hb < 2; ++hb) {
+                        const int blk = b2 + hb;
+                        const uint32_t (&V)[16] = V2[hb];
                         if (valid) {
                             float f[16];
 #pragma unroll
@@ -1002,6 +1007,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                                 dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
                                 dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                             }
+                        }
                         }
                     }
                 }
