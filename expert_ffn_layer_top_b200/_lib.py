@@ -253,7 +253,7 @@ def moe_permute(idx: torch.Tensor, E: int, x: Optional[torch.Tensor] = None, ws:
     H = x.shape[1] if x is not None else 0
     x_perm = torch.empty(max(P, 1), H, dtype=torch.bfloat16, device=dev) if x is not None else None
     if ws is None:
-        ws = _ws(moe_workspace_size(T, max(H, 8), 128, E, k), dev)
+        ws = _ws(moe_workspace_size(T, max(H, 8), 128, E, k, act=act), dev)
     _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(x), H, ACT[act], _ptr(offsets), _ptr(sp), _ptr(pr),
                              _ptr(x_perm), _ptr(ws), ws.numel(), _stream()))
     return offsets, sp[:P], pr[:P], (x_perm[:P] if x_perm is not None else None)
@@ -281,7 +281,7 @@ def moe_grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, experts: Expert
     n = x_perm.shape[0]
     y = torch.empty(max(n, 1), experts.H, dtype=torch.float32 if y_fp32 else torch.bfloat16, device=x_perm.device)
     if ws is None:
-        ws = _ws(moe_workspace_size(max(n, 1), experts.H, experts.I, experts.E, 1, y_fp32), x_perm.device)
+        ws = _ws(moe_workspace_size(max(n, 1), experts.H, experts.I, experts.E, 1, y_fp32, act), x_perm.device)
     _check(lib().moe_grouped_ffn(_ptr(x_perm), n, _ptr(offsets), C.byref(experts.c), ACT[act], _ptr(y), int(y_fp32),
                                  _ptr(ws), ws.numel(), _stream()))
     return y[:n]
@@ -315,7 +315,7 @@ def moe_layer_forward(x: torch.Tensor, wr: torch.Tensor, k: int, experts: Expert
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
     if ws is None:
-        ws = _ws(moe_workspace_size(T, H, experts.I, experts.E, k, y_fp32), x.device)
+        ws = _ws(moe_workspace_size(T, H, experts.I, experts.E, k, y_fp32, act), x.device)
     _check(lib().moe_layer_forward(_ptr(x), T, _ptr(wr), int(wr.dtype == torch.float32), _ptr(bias), k,
                                    C.byref(experts.c), ACT[act], cache.handle if cache is not None else None, layer,
                                    int(y_fp32), _ptr(out), _ptr(idx_out), _ptr(w_out), _ptr(ws), ws.numel(),

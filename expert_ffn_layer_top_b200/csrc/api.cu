@@ -216,14 +216,15 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 // atoms) of x and of h; NVFP4 also keeps h in bf16 at offset 0 and the per-row
 // exponent offsets of x and h.
 struct FfnWs {
-    size_t h, re1, re2, a4, tq, b1, b2, total;
+    size_t h, re1, re2, a4, tq, b1, b2, sched, total;
 };
 
 // h: bf16 [n][I] (the decoding paths' h buffer; NVFP4: h before its
 // quantisation); re1, re2: NVFP4 per-row exponent offsets of x and h; a4: the A4
 // tensor scale of x, then the partial maxima of |x|; b1, b2: activation blobs of
 // x and h for the block-scaled FP4 path (four planes, or one in A4 form: the
-// larger of the two sizes).
+// larger of the two sizes); sched: the block-scaled kernels' item claim counters (UP,
+// DOWN), zeroed by the quantiser that runs first.
 static FfnWs ffn_ws(int n, int H, int I, int E) {
     FfnWs W;
     size_t o = 0;
@@ -234,6 +235,7 @@ static FfnWs ffn_ws(int n, int H, int I, int E) {
     W.tq = o; o += align_up((size_t)n * H / 2, 256) + align_up((size_t)n * H / 16, 256);   // A4 token rows
     W.b1 = o; o += std::max(mx_blob_bytes(n, H, E), a4_blob_bytes(n, H, E));
     W.b2 = o; o += std::max(mx_blob_bytes(n, I, E), a4_blob_bytes(n, I, E));
+    W.sched = o; o += 256;
     W.total = o;
     return W;
 }
@@ -264,8 +266,9 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     const FfnWs W = ffn_ws(n_rows, H, I, E);
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
     int32_t *re1 = reinterpret_cast<int32_t *>(b + W.re1), *re2 = reinterpret_cast<int32_t *>(b + W.re2);
+    int *sched = reinterpret_cast<int *>(b + W.sched);
     moe_status r = launch_mx_quant(fmt, x_src, gather ? 1 : 0, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1,
-                                   re1, nsm, st);
+                                   re1, nsm, st, sched);
     if (r != MOE_OK) return r;
     MxParams p;
     memset(&p, 0, sizeof(p));
@@ -285,6 +288,7 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.tscale = x->w13_tscale;
     p.bblob_out = b + W.b2;
     p.hout = b + W.h;
+    p.sched = sched;
     if ((r = launch_mx_phase(fmt, kPhaseUp, BN, p, nsm, st)) != MOE_OK) return r;
     if (fmt == kBsNv &&
         (r = launch_mx_quant(fmt, b + W.h, 2, nullptr, 1, n_rows, I, offsets, E, BN, b + W.b2, re2, nsm, st)) !=
@@ -302,6 +306,7 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.hout = nullptr;
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
+    p.sched = sched + 1;
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 
@@ -321,7 +326,8 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
     const FfnWs W = ffn_ws(n_rows, H, I, E);
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
     float *xscale = reinterpret_cast<float *>(b + W.a4), *parts = xscale + 1;
-    moe_status r = launch_a4_amax(amax_src, amax_elems, parts, st);
+    int *sched = reinterpret_cast<int *>(b + W.sched);
+    moe_status r = launch_a4_amax(amax_src, amax_elems, parts, sched, st);
     if (r == MOE_OK && gather) {
         // token rows: quantise each token once (amax_elems / H of them), then place its k pairs
         const int T = (int)(amax_elems / H);
@@ -350,6 +356,7 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
     p.tscale = x->w13_tscale;
     p.bblob_out = b + W.b2;
     p.xscale = xscale;
+    p.sched = sched;
     if ((r = launch_mx_phase(kBsNv, kPhaseUp, BN, p, nsm, st, 1)) != MOE_OK) return r;
     // ---- down projection
     p.K = I;
@@ -362,6 +369,7 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
     p.xscale = nullptr;
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
+    p.sched = sched + 1;
     return launch_mx_phase(kBsNv, kPhaseDown, BN, p, nsm, st, 1);
 }
 

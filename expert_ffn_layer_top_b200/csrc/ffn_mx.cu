@@ -47,7 +47,9 @@
 
 namespace moe {
 
-constexpr int kMxThreads = 512;
+constexpr int kMxThreads = 544;   // 16 role warps + the item scheduler (warp 16)
+constexpr int kMxSchedWarp = 16;
+constexpr int kMxQ = 16;          // entries of the CTA's item queue
 constexpr int kMxMaxStages = 12;
 constexpr int kMxXch = 9;    // padded row of the gate/up exchange (8 values)
 constexpr int kMxSmemCap = 227 * 1024;
@@ -297,12 +299,13 @@ __device__ __forceinline__ void bf16x8_to_float(uint4 u, float (&v)[8]) {
 __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
-                                                       uint8_t *__restrict__ bblob) {
+                                                       uint8_t *__restrict__ bblob, int *__restrict__ sched_zero) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     pdl_wait();
     pdl_release();
+    if (sched_zero && blockIdx.x == 0 && threadIdx.x < 2) sched_zero[threadIdx.x] = 0;   // the FFN's claim counters
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsMx, BN);
@@ -347,13 +350,15 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
 __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__ src, int mode,
                                                        const int32_t *__restrict__ sorted_pair, int k, int P, int K,
                                                        const int32_t *__restrict__ offsets, int E, int BN,
-                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp) {
+                                                       uint8_t *__restrict__ bblob, int32_t *__restrict__ rowexp,
+                                                       int *__restrict__ sched_zero) {
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_tile[kMaxExperts + 1];
     __shared__ int s_wsum[8];
     __shared__ uint32_t s_max[8];
     pdl_wait();
     pdl_release();
+    if (sched_zero && blockIdx.x == 0 && threadIdx.x < 2) sched_zero[threadIdx.x] = 0;   // the FFN's claim counters
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsNv, BN);
@@ -427,10 +432,11 @@ __global__ void __launch_bounds__(256) nv_quant_kernel(const uint4 *__restrict__
 // Partial maxima of |src| (bf16, n8 groups of 8): part[b] = the maximum over block b's
 // share (grid-stride). Maxima are exact, so the tensor scale does not depend on the split.
 __global__ void __launch_bounds__(256) a4_amax_kernel(const uint4 *__restrict__ src, int64_t n8,
-                                                      float *__restrict__ part) {
+                                                      float *__restrict__ part, int *__restrict__ sched_zero) {
     __shared__ uint32_t s_max[8];
     pdl_wait();
     pdl_release();
+    if (sched_zero && blockIdx.x == 0 && threadIdx.x < 2) sched_zero[threadIdx.x] = 0;   // the FFN's claim counters
     float amax = 0.0f;
     for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (int64_t)gridDim.x * 256) {
         float v[8];
@@ -602,6 +608,10 @@ struct MxSmem {
     uint64_t mmadone[4];
     uint64_t sfrdy[4];              // token-major mode: a scale group's copies landed (both helpers)
     uint64_t hdone[2];              // token-major mode: a helper's last copies landed
+    uint64_t qfull[kMxQ];           // item queue: entry published (the scheduler)
+    uint64_t qtake[kMxQ];           // the producers have started the entry's item
+    uint64_t qempty[kMxQ];          // every reader of the entry has read it
+    int qitem[kMxQ];                // the CTA's items in order; -1 ends the sequence
     uint64_t xfull[2], xempty[2];   // gate/up exchange, per epilogue group
     uint32_t tmem_base;
     int abort_flag;
@@ -633,7 +643,17 @@ __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int
     return it;
 }
 
-// Warp roles (512 threads, one CTA per SM, persistent over items). NP
+// Entry j of the CTA's item queue: waits until the scheduler has published it and returns
+// the item (-1: the sequence ended, or a wait gave up: then ok is cleared).
+__device__ __forceinline__ int mx_q_get(MxSmem &sm, int j, volatile int *abort_flag, bool &ok) {
+    if (!mbar_wait(&sm.qfull[j % kMxQ], (uint32_t)((j / kMxQ) & 1), abort_flag)) {
+        ok = false;
+        return -1;
+    }
+    return *reinterpret_cast<volatile int *>(&sm.qitem[j % kMxQ]);
+}
+
+// Warp roles (544 threads, one CTA per SM, persistent over items). NP
 // independent pipelines: pipeline w is producer warp w, MMA warp 12 + w, its own
 // ring of slots and its own double-buffered accumulators. It handles either
 // stages w, w + NP, ... of every item (stage-parallel) or every stage of items
@@ -645,10 +665,17 @@ __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int
 //   warps 12-15 MMA issuers (warp 12 owns TMEM): per stage one tcgen05.cp per
 //               scale atom, four MMAs of K = 64, one commit.
 //   warps 4-7   epilogue of the CTA's even items;
-//   warps 8-11  epilogue of its odd items. The epilogue adds the accumulators
+//   warps 8-11  epilogue of its odd items.
+//   warp 16     item scheduler: publishes the CTA's items in order through a queue
+//               in shared memory. The first (item-parallel: the first NP) are
+//               static, blockIdx.x + j gridDim.x; the rest are claimed one by one
+//               from a counter in global memory (zeroed by the kernel before this
+//               one), each when the producers have started the item L entries
+//               before it, so a CTA that streams faster takes more items and the
+//               CTAs finish together. The epilogue adds the accumulators
 //               of the pipelines that worked on the item (all NP, or the one
 //               owner) and the four planes' columns.
-// TMEM columns: accumulator (buffer a, pipeline w) at (a NW + w) N; from 2 NW N
+// TMEM columns: accumulator (buffer a < NB, pipeline w) at (a NW + w) N; from NB NW N
 // on, 16 NA scale columns per pipeline (two rotating groups of 8 NA: the NA
 // weight atoms, then the NA activation atoms, 4 columns each).
 template <int FMT, int PHASE, int BN, int PL>
@@ -666,9 +693,12 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
     constexpr int ABLOB = bs_ablob_bytes(FMT);
     constexpr int BBLOB = bs_bblob_bytes(FMT, BN, PL);
     constexpr int STAGE = ABLOB + BBLOB;                    // a multiple of 1024
-    constexpr uint32_t SFCOL = 2 * NW * N;
-    static_assert(SFCOL + NW * 16 * NA <= 512, "TMEM columns");
-    static_assert(!TM || SFCOL + 4 * 8 * NA <= 512, "TMEM columns of the token-major mode");
+    static_assert(2 * NW * N + NW * 16 * NA <= 512, "TMEM columns");
+    static_assert(!TM || 2 * NW * N + 4 * 8 * NA <= 512, "TMEM columns of the token-major mode");
+    // accumulator buffers per pipeline: 2, or 3 where the plan found room (never in the
+    // token-major or item-parallel modes); the scale columns follow them
+    const int NB = p.nbuf;
+    const uint32_t SFCOL = (uint32_t)(NB * NW * N);
     const int NP = p.pipes;                                 // <= NW; stage-parallel: divides the stages per item
     const int NSW = p.stages / NP;                          // slots per pipeline
 
@@ -705,6 +735,14 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         for (int w = 0; w < 4; ++w) mbar_init(&sm.mmadone[w], 1);
         for (int g = 0; g < 4; ++g) mbar_init(&sm.sfrdy[g], 2);
         for (int h = 0; h < 2; ++h) mbar_init(&sm.hdone[h], 1);
+        // readers of a queue entry: its producers and MMA warps (all NP, or the owner),
+        // the token-major helpers, and the four warps of its epilogue group
+        const uint32_t readers = (IP ? 2u : 2u * (uint32_t)p.pipes) + (TM ? 2u : 0u) + 4u;
+        for (int e = 0; e < kMxQ; ++e) {
+            mbar_init(&sm.qfull[e], 1);
+            mbar_init(&sm.qtake[e], IP ? 1u : (uint32_t)p.pipes);
+            mbar_init(&sm.qempty[e], readers);
+        }
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -760,18 +798,23 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                           p.wbase + (int64_t)it.slot * p.w_estride + ((int64_t)it.m * KST + st) * ABLOB, ABLOB,
                           fb);
             };
-            // The slots start empty: the weights of this pipeline's first NSW stages go out
-            // before waiting for the kernel that writes the activations.
+            // The slots start empty: the weights of this pipeline's first stages go out before
+            // waiting for the kernel that writes the activations. Its first item is static
+            // (queue entry j0), so they stay within that item.
             int pre = 0;
-            for (int item = blockIdx.x + j0 * gridDim.x; item < total && pre < NSW; item += dj * gridDim.x) {
-                const MxItem it = mx_item(tab, p, item, BN);
+            if (blockIdx.x + j0 * gridDim.x < total) {
+                const MxItem it = mx_item(tab, p, blockIdx.x + j0 * gridDim.x, BN);
                 for (int st = st0; st < KST && pre < NSW; st += dst, ++pre) issue_weights(it, st, w * NSW + pre);
             }
             pdl_wait();
             if (w == 0) pdl_release();
             int loc = 0;   // stages this pipeline has issued
             bool ok = true;
-            for (int item = blockIdx.x + j0 * gridDim.x; item < total && ok; item += dj * gridDim.x) {
+            for (int jq = j0; ok; jq += dj) {   // this pipeline's queue entries
+                const int item = mx_q_get(sm, jq, abort_flag, ok);
+                if (item < 0) break;
+                mbar_arrive(&sm.qtake[jq % kMxQ]);
+                mbar_arrive(&sm.qempty[jq % kMxQ]);
                 const MxItem it = mx_item(tab, p, item, BN);
                 for (int st = st0; st < KST; st += dst, ++loc) {
                     const int s = w * NSW + loc % NSW;
@@ -805,7 +848,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         const uint32_t base_u32 = smem_u32(base);
         int j = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        for (int jq = 0; ok; ++jq) {
+            if (mx_q_get(sm, jq, abort_flag, ok) < 0) break;
+            mbar_arrive(&sm.qempty[jq % kMxQ]);
             for (int k = 0; k < KST; ++k, ++j) {
                 const int s = j % NSW;
                 if (!mbar_wait(&sm.full[s], (uint32_t)((j / NSW) & 1), abort_flag)) { ok = false; break; }
@@ -827,6 +872,48 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         while (!mbar_try_wait(&sm.hdone[h], 0)) {
             if (globaltimer() - t0 > kWaitLimitNs) { flag_error(1); break; }
         }
+    } else if (warp == kMxSchedWarp) {
+        // =================================================== item scheduler
+        if (lane == 0) {
+            const int F = IP ? p.pipes : 1;   // static items of each CTA
+            const int L = IP ? p.pipes : 1;   // claim entry j once the producers took entry j - L
+            int j = 0;
+            bool ok = true;
+            auto publish = [&](int item) {
+                const int e = j % kMxQ;
+                if (j >= kMxQ && !mbar_wait(&sm.qempty[e], (uint32_t)(((j / kMxQ) & 1) ^ 1), abort_flag)) {
+                    ok = false;
+                    return;
+                }
+                *reinterpret_cast<volatile int *>(&sm.qitem[e]) = item;
+                mbar_arrive(&sm.qfull[e]);
+                ++j;
+            };
+            for (int f = 0; f < F && ok; ++f) {
+                const int item = blockIdx.x + f * gridDim.x;
+                if (item >= total) break;
+                publish(item);
+            }
+            if (p.sched) {
+                pdl_wait();   // the counter was zeroed by the kernel before this one
+                int next = F * gridDim.x;
+                while (ok && next < total) {
+                    if (j >= L && !mbar_wait(&sm.qtake[(j - L) % kMxQ], (uint32_t)(((j - L) / kMxQ) & 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    next = F * gridDim.x + (int)atomicAdd(reinterpret_cast<unsigned int *>(p.sched), 1u);
+                    if (next < total) publish(next);
+                }
+            } else {   // no counter: the static order, blockIdx.x + j gridDim.x
+                for (int item = blockIdx.x + F * gridDim.x; item < total && ok; item += gridDim.x) publish(item);
+            }
+            // end markers: a reader takes every entry (producers and MMA warps of the stage-parallel
+            // modes), every NP-th (item-parallel) or every other one (epilogue groups), so each
+            // residue meets one among max(2, NP) consecutive entries
+            const int S = IP && p.pipes > 2 ? p.pipes : 2;
+            for (int e = 0; e < S && ok; ++e) publish(-1);
+        }
     } else if (warp >= 12) {
         // =================================================== MMA issuer of pipeline w
         const int w = warp - 12;
@@ -836,7 +923,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             int loc = 0, lt = 0;
             bool ok = true;
             const uint32_t base_u32 = smem_u32(base);
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++lt) {
+            for (int jq = 0; ok; ++jq, ++lt) {
+                if (mx_q_get(sm, jq, abort_flag, ok) < 0) break;
+                mbar_arrive(&sm.qempty[jq % kMxQ]);
                 const int a = lt & 1;
                 if (!mbar_wait(&sm.accempty[a], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -870,9 +959,11 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             int loc = 0, lt = 0, sc = 0;
             bool ok = true;
             const uint32_t base_u32 = smem_u32(base);
-            for (int item = blockIdx.x + j0 * gridDim.x; item < total && ok; item += dj * gridDim.x, ++lt) {
-                const int a = lt & 1, bi = IP ? 2 * w + a : a;   // lt: this pipeline's items so far
-                if (!mbar_wait(&sm.accempty[bi], ((lt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            for (int jq = j0; ok; jq += dj, ++lt) {   // this pipeline's queue entries
+                if (mx_q_get(sm, jq, abort_flag, ok) < 0) break;
+                mbar_arrive(&sm.qempty[jq % kMxQ]);
+                const int a = lt % NB, bi = IP ? 2 * w + a : a;   // lt: this pipeline's items so far
+                if (!mbar_wait(&sm.accempty[bi], ((lt / NB) & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)((a * NW + w) * N);
                 for (int k = 0; k < PER; ++k, ++loc) {
@@ -920,7 +1011,12 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         float *xg = xch + grp * 128 * kMxXch;
         int lt = grp, xc = 0;
         bool ok = true;
-        for (int item = blockIdx.x + grp * gridDim.x; item < total && ok; item += 2 * gridDim.x, lt += 2) {
+        for (; ok; lt += 2) {   // queue entries grp, grp + 2, ...: lt is the item's place in the CTA
+            int item = 0;
+            if (lane == 0) item = mx_q_get(sm, lt, abort_flag, ok);
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (item < 0) break;   // the end, or lane 0 gave up (the abort flag is set)
+            if (lane == 0) mbar_arrive(&sm.qempty[lt % kMxQ]);
             const MxItem it = mx_item(tab, p, item, BN);
             // NVFP4: the expert's tensor scale (static data), loaded once per item while the
             // accumulators are still being computed
@@ -928,9 +1024,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             if constexpr (FMT == kBsNv) iscale = p.tscale[it.e];
             // lt: the item's index in this CTA. Item-parallel: pipeline lt % NP, its item lt / NP.
             const int wi = IP ? lt % NP : 0, li = IP ? lt / NP : lt;
-            const int a = li & 1, bi = IP ? 2 * wi + a : a;
+            const int a = li % NB, bi = IP ? 2 * wi + a : a;
             const int wlo = IP ? wi : 0, whi = IP ? wi + 1 : NP;   // accumulators to add
-            if (!mbar_wait(&sm.accfull[bi], (li >> 1) & 1, abort_flag)) break;
+            if (!mbar_wait(&sm.accfull[bi], (li / NB) & 1, abort_flag)) break;
             tc_fence_after();
             // A4 UP: the tensor scale of x comes from the quantiser just before this kernel. It is
             // read only now: the accumulators hold its output, so the producer has passed the wait
@@ -1274,6 +1370,10 @@ bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl, int planes) {
         pl->pipes = np;
         pl->stages = np * nsw;
         pl->itempar = np > 1 && KST / np == 1;
+        // a third accumulator buffer lets the MMAs run up to two items ahead of the epilogue,
+        // so a slow epilogue does not stop the weight stream (the ring holds about one item)
+        const bool tm = planes == 1 && BN == 128;
+        pl->nbuf = (!pl->itempar && !tm && 3 * nw * N + nw * 16 * bs_atoms(fmt) <= 512) ? 3 : 2;
         return true;
     }
     return false;
@@ -1289,6 +1389,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
     p.pipes = pl.pipes;
     p.stages = pl.stages;
     p.itempar = pl.itempar;
+    p.nbuf = pl.nbuf;
     size_t smem = mx_smem_bytes(fmt, phase, BN, pl.stages, p.E, planes);
     if (smem < 120 * 1024) smem = 120 * 1024;   // one CTA per SM: it allocates all 512 TMEM columns
     const int64_t items_ub = ((int64_t)p.n_rows / BN + p.E) * p.m_tiles;
@@ -1308,7 +1409,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
 
 moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
-                           cudaStream_t st) {
+                           cudaStream_t st, int *sched_zero) {
     if (P == 0) return MOE_OK;
     if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
@@ -1316,13 +1417,13 @@ moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *so
     if (fmt == kBsNv) {   // one block per row
         const int blocks = P < num_sms * 8 ? P : num_sms * 8;
         e = launch_pdl(nv_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
-                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp);
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), rowexp, sched_zero);
     } else {              // one warp per (row, stage)
         if (mode == 2) return set_error(MOE_ERR_UNSUPPORTED, "MXFP4 quantiser mode 2");
         const int64_t units = (int64_t)P * (K / kMxStageK);
         const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
         e = launch_pdl(mx_quant_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src), mode,
-                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob));
+                       sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob), sched_zero);
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "block-scaled quantiser launch");
@@ -1332,10 +1433,10 @@ moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *so
 
 namespace moe {
 
-moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cudaStream_t st) {
+moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, int *sched_zero, cudaStream_t st) {
     const int64_t n8 = n_elems / 8;
     cudaError_t e = launch_pdl(a4_amax_kernel, dim3(kA4Parts), dim3(256), 0, st, reinterpret_cast<const uint4 *>(src),
-                               n8, partials);
+                               n8, partials, sched_zero);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 amax launch");
 }

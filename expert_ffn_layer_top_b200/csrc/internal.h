@@ -65,6 +65,7 @@ struct MxParams {
     int stages;                 // shared-memory slots, set by the launcher
     int pipes;                  // independent producer/MMA pipelines, set by the launcher
     int itempar;                // pipelines take whole items (else stages of every item), set by the launcher
+    int nbuf;                   // accumulator buffers per pipeline (2, or 3 where TMEM has room), set by the launcher
     int n_rows;
     const uint8_t *wbase;       // this phase's prepacked tensor: [m_tiles][K/256] weight blobs
     int64_t w_estride;          // bytes between experts (or cache slots)
@@ -76,6 +77,7 @@ struct MxParams {
     uint8_t *bblob_out;         // MXFP4 and A4 up: blobs of h for the down pass [tiles][I/256]
     void *hout;                 // NVFP4 up: h bf16 [n_rows][I]
     const float *xscale;        // A4 up: device word with the per-tensor scale of x
+    int *sched;                 // item claim counter of this phase (zero at launch), or null: static order
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -95,7 +97,7 @@ moe_status launch_ffn_phase(int phase, int fmt, int BN, const CUtensorMap &wmap,
 
 int choose_bn_mx(int n_rows, int E);
 struct MxPlan {
-    int pipes, stages, itempar;
+    int pipes, stages, itempar, nbuf;
 };
 bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl, int planes = kMxPlanes);
 size_t mx_tiles_ub(int n_rows, int E);
@@ -107,7 +109,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
 // partial maxima of |x| and the quantiser (src rows as launch_mx_quant modes 1 and 2).
 int choose_bn_a4(int n_rows, int E);
 size_t a4_blob_bytes(int n_rows, int K, int E);
-moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, cudaStream_t st);
+moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, int *sched_zero, cudaStream_t st);
 // Token-major A4 rows of x [T][K] (codes [T][K/2], scales [T][K/16]), then their scatter into
 // the blobs of the pairs (the layer forward's path: each token quantised once, not k times).
 moe_status launch_a4_token_quant(const void *x, int T, int K, const float *partials, float *xscale, void *codes,
@@ -121,7 +123,7 @@ moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair
 // order), 2 src[r] (natural order; NVFP4 only). rowexp: NVFP4 only.
 moe_status launch_mx_quant(int fmt, const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, void *bblob, int32_t *rowexp, int num_sms,
-                           cudaStream_t st);
+                           cudaStream_t st, int *sched_zero = nullptr);
 
 moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscale, int rows, int K, void *out,
                           cudaStream_t st);
