@@ -716,7 +716,8 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
         else
             r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
     }
-    if (r == MOE_OK) r = moe_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, stream);
+    // the combine reads prow and w, written by the routing, before its wait for y
+    if (r == MOE_OK) r = launch_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, st, 1);
     if (cache) cache_compute_end(cache, st);   // closes the call's timing record in every case
     return r;
 }

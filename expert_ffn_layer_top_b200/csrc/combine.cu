@@ -2,6 +2,10 @@
 // accumulated in fp32 in order of j and rounded once to bf16. The pages give no
 // combine formula; this is the standard weighted sum of the k expert outputs.
 // One block per token, 8 channels (16-byte bf16 / 32-byte fp32 loads) per thread.
+// early != 0: pair_row and w were complete before the previous kernel let this one
+// start (the layer forward: they come from the routing, several kernels back, and every
+// kernel of the library lets its successor start only after its own wait), so they
+// are read before the wait for y_perm.
 #include "common.cuh"
 #include "internal.h"
 
@@ -11,9 +15,8 @@ template <bool Y32>
 __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y_perm,
                                                      const int32_t *__restrict__ pair_row,
                                                      const float *__restrict__ w, int k, int H,
-                                                     __nv_bfloat16 *__restrict__ out) {
-    pdl_wait();
-    pdl_release();
+                                                     __nv_bfloat16 *__restrict__ out, int early) {
+    if (!early) pdl_wait();
     const int t = blockIdx.x;
     __shared__ int rows[kMaxTopK];
     __shared__ float ws[kMaxTopK];
@@ -27,6 +30,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
         rows[threadIdx.x] = r;
         ws[threadIdx.x] = w[(int64_t)t * k + threadIdx.x];
     }
+    if (early) pdl_wait();
+    pdl_release();
     __syncthreads();
     for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
         float acc[8];
@@ -80,14 +85,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
 }
 
 moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
-                          int H, void *out, cudaStream_t st) {
+                          int H, void *out, cudaStream_t st, int early) {
     if (T == 0) return MOE_OK;
     int threads = H / 8;
     if (threads > 256) threads = 256;
     threads = (threads + 31) / 32 * 32;
     __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out);
-    cudaError_t e = y_is_fp32 ? launch_pdl(combine_kernel<true>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o)
-                              : launch_pdl(combine_kernel<false>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o);
+    cudaError_t e = y_is_fp32
+                        ? launch_pdl(combine_kernel<true>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o, early)
+                        : launch_pdl(combine_kernel<false>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o,
+                                     early);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "combine launch");
 }

@@ -307,16 +307,23 @@ __global__ void __launch_bounds__(256) mx_quant_kernel(const uint4 *__restrict__
     pdl_release();
     if (sched_zero && blockIdx.x == 0 && threadIdx.x < 2) sched_zero[threadIdx.x] = 0;   // the FFN's claim counters
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     const int K8 = K / 8, KST = K / kMxStageK, NROW = kMxPlanes * BN, BB = bs_bblob_bytes(kBsMx, BN);
     const int64_t units = (int64_t)P * KST;
     const int64_t nw = (int64_t)gridDim.x * 8;
-    for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += nw) {
+    const int64_t u0 = (int64_t)blockIdx.x * 8 + warp;
+    // the first unit's row goes out before the tile prefix, which it does not need
+    uint4 uv0 = make_uint4(0, 0, 0, 0);
+    if (u0 < units) {
+        const int r = (int)(u0 / KST), st = (int)(u0 - (int64_t)r * KST);
+        uv0 = src[(int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8 + st * 32 + lane];
+    }
+    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
+    for (int64_t u = u0; u < units; u += nw) {
         const int r = (int)(u / KST), st = (int)(u - (int64_t)r * KST);
         const int e = expert_of_row(s_off, E, r);
         const int rel = r - s_off[e];
         const int tile = s_tile[e] + rel / BN, n = rel % BN;
-        uint4 uv = src[(int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8 + st * 32 + lane];
+        uint4 uv = u == u0 ? uv0 : src[(int64_t)(mode == 1 ? sorted_pair[r] / k : r) * K8 + st * 32 + lane];
         if (mode == 0) uv = deinterleave8(uv);
         float v[8];
         bf16x8_to_float(uv, v);

@@ -156,7 +156,7 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
 
 // combine (combine.cu)
 moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
-                          int H, void *out, cudaStream_t st);
+                          int H, void *out, cudaStream_t st, int early = 0);
 
 // tensor maps (api.cu)
 moe_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,

@@ -124,9 +124,10 @@ __global__ void __launch_bounds__(kChunk) perm_small_kernel(const int32_t *__res
                                                            int32_t *__restrict__ sorted_pair,
                                                            int32_t *__restrict__ pair_row) {
     __shared__ SmallPermuteSmem<kChunk> sm;
+    extern __shared__ int32_t sidx[];   // [P]
     pdl_wait();
     pdl_release();
-    small_permute<kChunk>(idx, P, E, offsets, sorted_pair, pair_row, sm);
+    small_permute<kChunk>(idx, P, E, offsets, sorted_pair, pair_row, sm, sidx);
 }
 
 // Workspace bytes launch_permute actually uses for these sizes: none on the
@@ -163,7 +164,10 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
     }
     cudaError_t e;
     if (P <= kSmallP && E <= kSmallE) {
-        e = launch_pdl(perm_small_kernel, dim3(1), dim3(kChunk), 0, st, idx, P, E, offsets, sorted_pair, pair_row);
+        e = ensure_max_smem<perm_small_kernel>((int)(kSmallP * sizeof(int32_t)));
+        if (e == cudaSuccess)
+            e = launch_pdl(perm_small_kernel, dim3(1), dim3(kChunk), (size_t)P * sizeof(int32_t), st, idx, P, E,
+                           offsets, sorted_pair, pair_row);
         if (e != cudaSuccess) return set_cuda_error(e, "permute launch");
     } else {
         const int C = (P + kChunk - 1) / kChunk;

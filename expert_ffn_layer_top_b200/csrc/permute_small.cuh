@@ -4,8 +4,8 @@
 // and by the router's last cluster when the layer fuses routing and
 // permutation.
 //
-// Histogram, exclusive scan over the experts, then the pairs in chunks of NT in
-// order: each pair lands at its expert's running position + its rank among the
+// idx is read from global memory once, into sidx (shared, P entries). Histogram,
+// exclusive scan over the experts, then the pairs in chunks of NT in order: each pair lands at its expert's running position + its rank among the
 // equal experts of earlier warps of the chunk + its rank inside its warp, which
 // is the stable order (by pair index) within every expert.
 #pragma once
@@ -28,19 +28,38 @@ struct SmallPermuteSmem {
 
 // idx is read through L2 (__ldcg): in the fused case other CTAs of the same
 // kernel wrote it. Entries outside [0, E) set the device error word and are
-// left out.
+// left out (sidx holds -1 for them).
 template <int NT>
 __device__ void small_permute(const int32_t *idx, int P, int E, int32_t *__restrict__ offsets,
                               int32_t *__restrict__ sorted_pair, int32_t *__restrict__ pair_row,
-                              SmallPermuteSmem<NT> &s) {
+                              SmallPermuteSmem<NT> &s, int32_t *sidx) {
     static_assert(NT % 32 == 0 && NT >= kSmallE && NT <= 1024, "block size");
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    // into shared memory, up to 8 loads per thread in flight; the counters are cleared
+    // meanwhile (the histogram starts after the barrier)
+    for (int p0 = 0; p0 < P; p0 += 8 * NT) {
+        int ev[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int p = p0 + tid + i * NT;
+            ev[i] = p < P ? __ldcg(idx + p) : 0;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int p = p0 + tid + i * NT;
+            if (p < P) sidx[p] = ev[i];
+        }
+    }
     for (int e = tid; e < E; e += NT) s.cnt[e] = 0;
     __syncthreads();
     for (int p = tid; p < P; p += NT) {
-        const int e = __ldcg(idx + p);
-        if (e >= 0 && e < E) atomicAdd(&s.cnt[e], 1);
-        else flag_error(2);
+        const int e = sidx[p];
+        if (e >= 0 && e < E) {
+            atomicAdd(&s.cnt[e], 1);
+        } else {
+            flag_error(2);
+            sidx[p] = -1;
+        }
     }
     __syncthreads();
     // exclusive scan over experts (E <= NT: one expert per thread)
@@ -73,8 +92,8 @@ __device__ void small_permute(const int32_t *idx, int P, int E, int32_t *__restr
         for (int i = tid; i < (NT / 32) * E; i += NT) s.wcnt[i / E][i % E] = 0;
         __syncthreads();
         const int p = c0 + tid;
-        int e = (p < P) ? __ldcg(idx + p) : -1 - lane;
-        if (p < P && (e < 0 || e >= E)) e = -1 - lane;   // never matches a real expert
+        int e = (p < P) ? sidx[p] : -1;
+        if (e < 0) e = -1 - lane;   // never matches a real expert
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int rank_w = __popc(peers & ((1u << lane) - 1u));
         if (e >= 0 && rank_w == 0) s.wcnt[wid][e] = __popc(peers);

@@ -575,7 +575,8 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
         __syncthreads();
         if (s_last) {   // the ring and the sums are no longer needed: their space is the scratch
             auto &ps = *reinterpret_cast<SmallPermuteSmem<kRClThreads> *>(rsm + 64);
-            small_permute<kRClThreads>(idx, T * k, E, fz.offsets, fz.sorted_pair, fz.pair_row, ps);
+            int32_t *sidx = reinterpret_cast<int32_t *>(rsm + 64 + sizeof(SmallPermuteSmem<kRClThreads>));
+            small_permute<kRClThreads>(idx, T * k, E, fz.offsets, fz.sorted_pair, fz.pair_row, ps, sidx);
             if (tid == 0) atomicExch(fz.ticket, 0u);   // ready for the next launch on this counter
         }
     }
@@ -587,7 +588,8 @@ static cudaError_t launch_router_cluster_t(const RouterClusterShape &sh, const v
                                            const RouterFuse &fz, cudaStream_t st) {
     auto kern = router_cluster_kernel<WR32, TT>;
     size_t smem = sh.smem;
-    if (fz.ticket && smem < 64 + sizeof(SmallPermuteSmem<kRClThreads>)) smem = 64 + sizeof(SmallPermuteSmem<kRClThreads>);
+    const size_t perm_smem = 64 + sizeof(SmallPermuteSmem<kRClThreads>) + (size_t)T * k * sizeof(int32_t);
+    if (fz.ticket && smem < perm_smem) smem = perm_smem;
     if (smem > 48 * 1024) {
         cudaError_t e = ensure_max_smem<router_cluster_kernel<WR32, TT>>((int)smem);
         if (e != cudaSuccess) return e;
