@@ -252,11 +252,21 @@ static bool use_bs(int fmt, int layout, int n_rows, int E) {
 }
 static bool is_mx(const moe_experts &x, int n_rows) { return use_bs(x.fmt, x.layout, n_rows, x.E); }
 
+// Activations already in the slot layout (the router wrote them; see RouterFuse).
+struct SlotInput {
+    const int32_t *cnt;
+    uint8_t *blob;
+    int T, mt;
+    int32_t *cprefix;
+};
+
 // Block-scaled FP4 grouped FFN. The activations are quantised first: gathered
-// from token rows x[sorted_pair[r] / k] (gather != 0) or read from x_perm.
+// from token rows x[sorted_pair[r] / k] (gather != 0) or read from x_perm; or
+// they are in the slot layout already (slot non-null: MXFP4; no quantiser runs,
+// and the router cleared the claim counters).
 static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sorted_pair, int k, int n_rows,
                               const int32_t *offsets, const moe_experts *x, void *y_perm, int y_is_fp32, void *ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, const SlotInput *slot = nullptr) {
     if (n_rows == 0) return MOE_OK;
     const int E = x->E, H = x->H, I = x->I;
     const int fmt = x->fmt == MOE_NVFP4 ? kBsNv : kBsMx;
@@ -267,8 +277,11 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     uint8_t *b = reinterpret_cast<uint8_t *>(ws);
     int32_t *re1 = reinterpret_cast<int32_t *>(b + W.re1), *re2 = reinterpret_cast<int32_t *>(b + W.re2);
     int *sched = reinterpret_cast<int *>(b + W.sched);
-    moe_status r = launch_mx_quant(fmt, x_src, gather ? 1 : 0, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1,
-                                   re1, nsm, st, sched);
+    moe_status r = MOE_OK;
+    if (slot && fmt != kBsMx) return set_error(MOE_ERR_UNSUPPORTED, "the slot layout carries MXFP4 activations");
+    if (!slot)
+        r = launch_mx_quant(fmt, x_src, gather ? 1 : 0, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1, re1, nsm,
+                            st, sched);
     if (r != MOE_OK) return r;
     MxParams p;
     memset(&p, 0, sizeof(p));
@@ -289,6 +302,14 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.bblob_out = b + W.b2;
     p.hout = b + W.h;
     p.sched = sched;
+    if (slot) {
+        p.bblob = slot->blob;
+        p.slab_cnt = slot->cnt;
+        p.slab_T = slot->T;
+        p.slab_mt = slot->mt;
+        p.cprefix = slot->cprefix;
+        p.slab_wait = 1;   // the counts may come from the kernel just before
+    }
     if ((r = launch_mx_phase(fmt, kPhaseUp, BN, p, nsm, st)) != MOE_OK) return r;
     if (fmt == kBsNv &&
         (r = launch_mx_quant(fmt, b + W.h, 2, nullptr, 1, n_rows, I, offsets, E, BN, b + W.b2, re2, nsm, st)) !=
@@ -307,6 +328,9 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.out = y_perm;
     p.out_fp32 = y_is_fp32;
     p.sched = sched + 1;
+    p.slab_mt = 0;         // h is in compact tiles
+    p.cprefix = nullptr;
+    p.slab_wait = 0;       // the counts come from two kernels back
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 
@@ -435,8 +459,20 @@ static moe_status grouped_ffn_impl(const void *x_perm, int n_rows, const int32_t
 
 // workspace layout of moe_layer_forward
 struct LayerWs {
-    size_t router, idx, w, offsets, sorted, pair_row, perm, x_perm, h, y, total;
+    size_t router, idx, w, offsets, sorted, pair_row, perm, x_perm, h, y, slot, cprefix, total;
 };
+
+// Bytes of the slot layout's activation tiles (MXFP4, four planes) for a decode-sized
+// batch: every expert gets room for T rows, ceil(T / BN) tiles. 0 where the layout is not
+// used (large batches, or more than 64 MiB of tiles).
+static size_t slot_blob_bytes(int T, int H, int E, int k) {
+    // the router's 8 CTAs each write whole 256-wide stages of the rows: H % 2048 == 0
+    if ((int64_t)T * k > 8192 || T > 256 || E > kMaxRouterExperts || H % (8 * kMxStageK)) return 0;
+    const int BN = choose_bn_mx(T * k, E);
+    const int64_t mt = (T + BN - 1) / BN;
+    const int64_t bytes = (int64_t)E * mt * (H / kMxStageK) * bs_bblob_bytes(kBsMx, BN);
+    return bytes <= (64ll << 20) ? align_up((size_t)bytes, 256) : 0;
+}
 
 static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
     LayerWs L;
@@ -452,6 +488,8 @@ static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
     L.x_perm = o; o += align_up(P * H * 2, 256);
     L.h = o; o += ffn_ws_bytes((int)P, H, I, E);
     L.y = o; o += align_up(P * H * (y32 ? 4 : 2), 256);
+    L.slot = o; o += slot_blob_bytes(T, H, E, k);
+    L.cprefix = o; o += align_up((size_t)E * 4, 256);
     L.total = o;
     return L;
 }
@@ -668,6 +706,7 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     const bool mx = a4 || use_bs(experts->fmt, layout, T * k, E);
     moe_status r;
     int fused = 0;
+    int32_t *slot_cnt = nullptr;   // the slot layout's row counts when the router wrote it
     if (mx) {
         if (H % 8 || E < 1 || E > kMaxRouterExperts || k < 1 || k > kMaxTopK || k > E)
             return set_error(MOE_ERR_UNSUPPORTED, "router needs 1<=k<=%d, k<=E<=%d (E=%d k=%d)", kMaxTopK,
@@ -687,9 +726,27 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
             pfb = std::min<int64_t>(kPrefetchL2, ss.w13 * (E - 1) +
                                                      (int64_t)prepacked_expert_bytes(experts->fmt, H, I, 0));
         }
-        const RouterFuse fz{offsets, sorted, prow, nullptr, pf, pfb};
+        RouterFuse fz{};
+        fz.offsets = offsets;
+        fz.sorted_pair = sorted;
+        fz.pair_row = prow;
+        fz.pf_base = pf;
+        fz.pf_bytes = pfb;
+        // Decode-sized MXFP4 batches: the router writes the slot layout itself (pair rows by
+        // atomic claims in per-expert slots, activation rows quantised straight into their
+        // tiles), so neither the permutation nor the quantiser runs.
+        if (!a4 && experts->fmt == MOE_MXFP4 && L.cprefix > L.slot && router_cluster_ok(T, H, E, wr_is_fp32, wr) &&
+            (slot_cnt = route_slot_counts(st)) != nullptr) {
+            const int BN = choose_bn_mx(T * k, E);
+            fz.cnt = slot_cnt;
+            fz.bslab = b + L.slot;
+            fz.BN = BN;
+            fz.mt = (T + BN - 1) / BN;
+            fz.sched_zero = reinterpret_cast<int *>(b + L.h + ffn_ws(T * k, H, I, E).sched);
+        }
         r = launch_router(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router, L.idx - L.router,
                           num_sms(current_device()), st, &fz, &fused);
+        if (fused != 2) slot_cnt = nullptr;
     } else {
         r = moe_route_topk(x, T, H, wr, wr_is_fp32, bias, E, k, idx, w, nullptr, b + L.router, L.idx - L.router,
                            stream);
@@ -708,16 +765,23 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     r = check_experts(&view);
     if (r == MOE_OK && !a4 && is_mx(view, T * k) != mx)
         r = set_error(MOE_ERR_INVALID_ARG, "cache layout differs from the layer's");
+    const int BNs = choose_bn_mx(T * k, E);
+    const SlotInput si{slot_cnt, b + L.slot, T, (T + BNs - 1) / BNs, reinterpret_cast<int32_t *>(b + L.cprefix)};
     if (r == MOE_OK) {
         if (a4)
             r = a4_ffn_impl(x, 1, x, (int64_t)T * H, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
         else if (mx)
-            r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+            r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st,
+                            slot_cnt ? &si : nullptr);
         else
             r = grouped_ffn_impl(b + L.x_perm, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
     }
-    // the combine reads prow and w, written by the routing, before its wait for y
-    if (r == MOE_OK) r = launch_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, st, 1);
+    // the combine reads prow and w, written by the routing, before its wait for y; in the
+    // slot layout it also maps the slot rows to y's rows and clears the counts
+    if (r == MOE_OK)
+        r = launch_combine(b + L.y, y_is_fp32, prow, w, T, k, H, out, st, 1, slot_cnt ? si.cprefix : nullptr, T,
+                           slot_cnt, E);
+    if (r != MOE_OK && slot_cnt) cudaMemsetAsync(slot_cnt, 0, sizeof(int32_t) * E, st);   // for the next call
     if (cache) cache_compute_end(cache, st);   // closes the call's timing record in every case
     return r;
 }

@@ -5,7 +5,9 @@
 // early != 0: pair_row and w were complete before the previous kernel let this one
 // start (the layer forward: they come from the routing, several kernels back, and every
 // kernel of the library lets its successor start only after its own wait), so they
-// are read before the wait for y_perm.
+// are read before the wait for y_perm. Slot layout (cprefix non-null): pair_row holds
+// e slab_T + pos and the row of y is cprefix[e] + pos (cprefix comes from the UP kernel,
+// also several kernels back); block 0 then clears the layer's slot counts for the next call.
 #include "common.cuh"
 #include "internal.h"
 
@@ -15,13 +17,19 @@ template <bool Y32>
 __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y_perm,
                                                      const int32_t *__restrict__ pair_row,
                                                      const float *__restrict__ w, int k, int H,
-                                                     __nv_bfloat16 *__restrict__ out, int early) {
+                                                     __nv_bfloat16 *__restrict__ out, int early,
+                                                     const int32_t *__restrict__ cprefix, int slab_T,
+                                                     int32_t *__restrict__ cnt_zero, int E) {
     if (!early) pdl_wait();
     const int t = blockIdx.x;
     __shared__ int rows[kMaxTopK];
     __shared__ float ws[kMaxTopK];
     if (threadIdx.x < k) {
         int r = pair_row[(int64_t)t * k + threadIdx.x];
+        if (cprefix) {
+            const int e = r / slab_T;
+            r = (r >= 0 && e < E) ? __ldcg(cprefix + e) + (r - e * slab_T) : -1;
+        }
         // a row outside y_perm's T*k rows is reported, and row 0 read in its place
         if (r < 0 || (int64_t)r >= (int64_t)gridDim.x * k) {
             flag_error(2);
@@ -32,6 +40,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
     }
     if (early) pdl_wait();
     pdl_release();
+    if (cnt_zero && blockIdx.x == 0)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_zero[e] = 0;
     __syncthreads();
     for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
         float acc[8];
@@ -85,16 +95,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
 }
 
 moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
-                          int H, void *out, cudaStream_t st, int early) {
+                          int H, void *out, cudaStream_t st, int early, const int32_t *cprefix, int slab_T,
+                          int32_t *cnt_zero, int E) {
     if (T == 0) return MOE_OK;
     int threads = H / 8;
     if (threads > 256) threads = 256;
     threads = (threads + 31) / 32 * 32;
     __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out);
     cudaError_t e = y_is_fp32
-                        ? launch_pdl(combine_kernel<true>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o, early)
+                        ? launch_pdl(combine_kernel<true>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o,
+                                     early, cprefix, slab_T, cnt_zero, E)
                         : launch_pdl(combine_kernel<false>, dim3(T), dim3(threads), 0, st, y_perm, pair_row, w, k, H, o,
-                                     early);
+                                     early, cprefix, slab_T, cnt_zero, E);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "combine launch");
 }

@@ -78,6 +78,14 @@ struct MxParams {
     void *hout;                 // NVFP4 up: h bf16 [n_rows][I]
     const float *xscale;        // A4 up: device word with the per-tensor scale of x
     int *sched;                 // item claim counter of this phase (zero at launch), or null: static order
+    // Slot layout of decode-sized batches (routing wrote the rows; no permutation ran):
+    // expert e owns pair rows [e slab_T, (e + 1) slab_T), slab_cnt[e] of them used, and
+    // its UP input tiles are e slab_mt ... (compact tiles otherwise). Rows of h and y stay
+    // compact: expert e's start at the prefix of the counts, published in cprefix.
+    const int32_t *slab_cnt;    // null: offsets describe the rows
+    int slab_T, slab_mt;
+    int32_t *cprefix;           // [E] written by the UP kernel in the slot layout
+    int slab_wait;              // slab_cnt comes from the previous kernel: read it after the wait
 };
 
 // error reporting (thread-local message), defined in api.cu
@@ -135,12 +143,23 @@ size_t router_ws_bytes(int T, int H, int E);
 struct RouterFuse {
     int32_t *offsets, *sorted_pair, *pair_row;
     unsigned int *ticket;
+    // Slot layout (cnt non-null, MXFP4 FFN of a decode-sized batch): pair j of token t takes
+    // row e T + atomicAdd(cnt + e, 1) of its expert e (pair_row), and the token's activation
+    // row is written in the four-plane MXFP4 form into row pos % BN of tile e mt + pos / BN of
+    // bslab. No permutation runs; cnt starts at zero (the layer's combine clears it again).
+    int32_t *cnt;
+    uint8_t *bslab;
+    int BN, mt;
+    int *sched_zero;   // the FFN's claim counters, zeroed here
     // L2 prefetch of the expert weights the grouped FFN reads first (static data, issued
     // before the router waits on its predecessor): pf_bytes from pf_base, 0 = none
     const uint8_t *pf_base;
     int64_t pf_bytes;
 };
-// fuse may be null; *fused (if given) tells whether the permutation was done.
+// fuse may be null; *fused (if given): 1 the permutation was done, 2 the slot layout was
+// written (fuse->cnt set; the cluster router must apply: router_cluster_ok).
+int32_t *route_slot_counts(cudaStream_t st);
+bool router_cluster_ok(int T, int H, int E, int wr_is_fp32, const void *wr);
 moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,
                          int k, int32_t *idx, float *w, float *logits, void *ws, size_t ws_bytes, int nsm,
                          cudaStream_t st, const RouterFuse *fuse = nullptr, int *fused = nullptr);
@@ -156,7 +175,9 @@ moe_status launch_permute(const int32_t *idx, int T, int k, int E, const void *x
 
 // combine (combine.cu)
 moe_status launch_combine(const void *y_perm, int y_is_fp32, const int32_t *pair_row, const float *w, int T, int k,
-                          int H, void *out, cudaStream_t st, int early = 0);
+                          int H, void *out, cudaStream_t st, int early = 0,
+                          const int32_t *cprefix = nullptr, int slab_T = 1, int32_t *cnt_zero = nullptr,
+                          int E = 0);
 
 // tensor maps (api.cu)
 moe_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,

@@ -22,6 +22,7 @@
 
 #include "internal.h"
 #include "permute_small.cuh"
+#include "mx_codec.cuh"
 
 namespace moe {
 
@@ -382,6 +383,9 @@ static bool router_cluster_shape(int T, int H, int E, int wr_is_fp32, RouterClus
 // counter at zero again (the last cluster resets it), so a launch counts from 0.
 constexpr int kTicketSlots = 256;
 __device__ unsigned int g_route_ticket[kTicketSlots];
+// Per-expert row counts of the slot layout, one set per stream slot: zero when the module
+// loads; the layer's combine clears them after the grouped FFN has read them.
+__device__ int32_t g_slot_count[kTicketSlots * kMaxRouterExperts];
 
 template <bool WR32, int TT>
 __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
@@ -392,6 +396,7 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     constexpr int eb = WR32 ? 4 : 2;
+    __shared__ int2 s_dest[16][kMaxTopK];   // slot layout: (tile, row) of each pair of the tile's tokens
     extern __shared__ __align__(128) uint8_t rsm[];
     uint64_t *full = reinterpret_cast<uint64_t *>(rsm);            // [kRClRing]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(rsm + 48);
@@ -432,12 +437,24 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     // Wr is static and already on its way; x comes from the previous kernel
     pdl_wait();
     pdl_release();
-    // x tile -> shared, as fp64 (exact), layout [h][tt]; tokens past T are zero
-    for (int i = tid; i < hs * TT; i += kRClThreads) {
-        const int tt = i / hs, h = i - tt * hs;
-        const int t = t0 + tt;
-        xs[h * TT + tt] =
-            t < T ? bf16_bits_to_f64(reinterpret_cast<const uint16_t *>(x)[(int64_t)t * H + h0 + h]) : 0.0;
+    if (fz.sched_zero && blockIdx.x == 0 && blockIdx.y == 0 && tid < 2) fz.sched_zero[tid] = 0;
+    // x tile -> shared, as fp64 (exact), layout [h][tt]; tokens past T are zero. Up to 8
+    // loads per thread are in flight before the first conversion.
+    for (int i0 = 0; i0 < hs * TT; i0 += 8 * kRClThreads) {
+        uint16_t xv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRClThreads + tid;
+            const int tt = i / hs, h = i - tt * hs;
+            xv[u] = (i < hs * TT && t0 + tt < T) ? reinterpret_cast<const uint16_t *>(x)[(int64_t)(t0 + tt) * H + h0 + h]
+                                                  : (uint16_t)0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRClThreads + tid;
+            const int tt = i / hs, h = i - tt * hs;
+            if (i < hs * TT) xs[h * TT + tt] = bf16_bits_to_f64(xv[u]);
+        }
     }
     __syncthreads();
 
@@ -564,8 +581,57 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
         }
         topk_softmax_warp(v, E, k, lane, idx + (int64_t)t * k, w + (int64_t)t * k);
         if (fz.ticket) __threadfence();   // the top-k is visible before this cluster's ticket
+        if (fz.cnt) {
+            // slot layout: each pair takes the next row of its expert's slot (the experts of a
+            // token are distinct, so a slot never holds more than T rows); the tile and row it
+            // lands in are left for the cluster's CTAs, which write the activation rows below
+            if (lane < k) {
+                const int e = idx[(int64_t)t * k + lane];   // written by this lane just above
+                const int pos = atomicAdd(fz.cnt + e, 1);
+                fz.pair_row[(int64_t)t * k + lane] = e * T + pos;
+                s_dest[tt][lane] = make_int2(e * fz.mt + pos / fz.BN, pos % fz.BN);
+            }
+        }
     }
     cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
+    if (fz.cnt) {
+        // Slot layout: every CTA writes its own slice of H (whole 256-wide stages, still in
+        // shared memory as exact fp64) of each token's activation row, in the four-plane MXFP4
+        // form, into the tiles of the token's k rows; the destinations come from the CTA that
+        // finished the token (rank tt % 8).
+        const int nls = hs / kMxStageK, st0 = h0 / kMxStageK, KST = H / kMxStageK;
+        const int BB = bs_bblob_bytes(kBsMx, fz.BN), NROW = kMxPlanes * fz.BN;
+        for (int item = warp; item < TT * nls; item += kRClThreads / 32) {
+            const int tt2 = item / nls, ls = item - tt2 * nls;
+            if (t0 + tt2 >= T) continue;   // warp-uniform
+            const int2 *rd = cluster.map_shared_rank(&s_dest[0][0], tt2 % kRCl) + tt2 * kMaxTopK;
+            const int2 dj = lane < k ? rd[lane] : make_int2(0, 0);
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = (float)xs[(ls * kMxStageK + lane * 8 + i) * TT + tt2];
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // 4 lanes hold one 32-block
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            const int s = mx_plane0_exp(amax);
+            uint32_t pw[kMxPlanes];
+            mx_planes8(v, s, pw);
+            const int c16 = lane >> 2, st = st0 + ls;
+            for (int j = 0; j < k; ++j) {
+                const int tile = __shfl_sync(0xffffffffu, dj.x, j), n = __shfl_sync(0xffffffffu, dj.y, j);
+                uint8_t *blob = fz.bslab + ((int64_t)tile * KST + st) * BB;
+#pragma unroll
+                for (int pl = 0; pl < kMxPlanes; ++pl) {
+                    const int Rw = pl * fz.BN + n;
+                    *reinterpret_cast<uint32_t *>(blob + sw128_chunk(Rw, c16) + (lane & 3) * 4) = pw[pl];
+                    if ((lane & 3) == 0)
+                        blob[NROW * 128 + (c16 >> 2) * 512 + atom_offset(Rw, c16 & 3)] = (uint8_t)(s - 3 * pl);
+                }
+            }
+        }
+        cluster.sync();   // every peer has read this CTA's destinations
+    }
     if (fz.ticket && rank == 0) {
         __shared__ int s_last;
         if (tid == 0) {
@@ -618,6 +684,32 @@ static cudaError_t launch_router_cluster(const RouterClusterShape &sh, const voi
 // handed out per (device, stream) on first use; a device holds kTicketSlots of
 // them. Null once a device's slots are all taken (its later streams route and
 // permute in two launches) or if the counters cannot be found.
+static unsigned int *route_ticket(cudaStream_t st);
+
+// The slot-layout row counts of stream st (kMaxRouterExperts of them), or null.
+int32_t *route_slot_counts(cudaStream_t st) {
+    static std::mutex mu;
+    static int32_t *base[64] = {};
+    static unsigned int *tbase[64] = {};
+    unsigned int *tk = route_ticket(st);
+    int dev = 0;
+    if (!tk || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!base[dev]) {
+        void *p = nullptr, *q = nullptr;
+        if (cudaGetSymbolAddress(&p, g_slot_count) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&q, g_route_ticket) != cudaSuccess) return nullptr;
+        base[dev] = reinterpret_cast<int32_t *>(p);
+        tbase[dev] = reinterpret_cast<unsigned int *>(q);
+    }
+    return base[dev] + (size_t)(tk - tbase[dev]) * kMaxRouterExperts;
+}
+
+bool router_cluster_ok(int T, int H, int E, int wr_is_fp32, const void *wr) {
+    RouterClusterShape sh;
+    return router_cluster_shape(T, H, E, wr_is_fp32, &sh) && (reinterpret_cast<uintptr_t>(wr) & 15) == 0;
+}
+
 static unsigned int *route_ticket(cudaStream_t st) {
     struct Slot { int dev; cudaStream_t st; int idx; };
     static std::mutex mu;
@@ -656,15 +748,19 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
             fz.pf_base = fuse->pf_base;
             fz.pf_bytes = fuse->pf_bytes;
         }
-        if (fuse && (int64_t)T * k <= kSmallP && E <= kSmallE) {
+        if (fuse && fuse->cnt) {   // slot layout: no permutation
             fz = *fuse;
+            fz.ticket = nullptr;
+        } else if (fuse && (int64_t)T * k <= kSmallP && E <= kSmallE) {
+            fz = *fuse;
+            fz.cnt = nullptr;
             fz.ticket = route_ticket(st);
         }
         cudaError_t e = wr_is_fp32
                             ? launch_router_cluster<true>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st)
                             : launch_router_cluster<false>(sh, x, T, H, wr, E, bias, k, idx, w, logits, fz, st);
         if (e != cudaSuccess) return set_cuda_error(e, "router_cluster launch");
-        if (fused) *fused = fz.ticket != nullptr;
+        if (fused) *fused = fz.cnt ? 2 : (fz.ticket != nullptr);
         return MOE_OK;
     }
     int S, slice;

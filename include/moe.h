@@ -284,6 +284,13 @@ struct expert_cache;
  *     (one host synchronisation per call to read the miss list).
  *   idx_out, w_out: nullable copies of the routing.
  *   y_is_fp32: keep the expert outputs in fp32 before the combine.
+ * Decode-sized MXFP4 batches (T <= 256, T k <= 8192, the activation tiles below
+ * 64 MiB) skip the separate permutation and quantiser: the router gives each
+ * pair a row in a per-expert slot of T rows by an atomic claim and writes the
+ * token's four-plane activation rows straight into those rows' tiles. The order
+ * of rows inside an expert then depends on timing, but every row's result does
+ * not, so `out` is the same as on the other paths. The slots' row counts are
+ * per stream and cleared by the call's last kernel.
  * T == 0 is a no-op. Errors: INVALID_ARG for NULL experts, x, wr, out or ws,
  * T < 0, an unknown af, k outside 1..min(16, E), x, wr or out not 16-byte
  * aligned, bias, idx_out or w_out not 4-byte aligned, or ws not 256-byte
@@ -299,7 +306,9 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
 /* Scratch bytes needed by moe_layer_forward / moe_route_topk / moe_permute /
  * moe_grouped_ffn for these sizes and activation format (an upper bound that
  * covers every path the sizes can take: the router's fp64 partial sums, the
- * routing, the permutation, x_perm, h or the FP4 activation blobs, y). No
+ * routing, the permutation, x_perm, h or the FP4 activation blobs, y, and for
+ * decode-sized batches the slot layout's tiles, which make the size larger at
+ * T = 64 than at T = 128, where that layout is not used). No
  * counterpart in the pages: it is what lets every call run without allocating.
  * Host-only, no CUDA call; 0 for non-positive sizes or an unknown af. */
 size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32, int af);

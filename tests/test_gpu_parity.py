@@ -284,10 +284,11 @@ def test_layer_decode_mxfp4(moe, decode_layer, T):
 
 
 def test_layer_fused_routing_and_permutation(moe, decode_layer):
-    """On the block-scaled path a small batch routes and permutes in one router
-    launch (the last cluster to finish sorts the pairs by expert), so a layer
-    call is 5 kernels: router, quantiser, UP, DOWN, combine. CUDA-graph replays reuse one launch's arguments, the
-    ticket epoch included; each replay must give the eager result."""
+    """A decode-sized MXFP4 batch takes the slot layout: the router claims each pair's
+    row in its expert's slot and writes the activation rows itself, so a layer call is
+    4 kernels: router, UP, DOWN, combine. CUDA-graph replays reuse one launch's
+    arguments and the slot counts must be back at zero after every call; each replay
+    (and a call on another stream, with its own counts) must give the eager result."""
     L = decode_layer.to("cuda")
     ex = moe.moe_prepack(moe.Experts.from_layer(L))
     T = 64
@@ -296,7 +297,7 @@ def test_layer_fused_routing_and_permutation(moe, decode_layer):
     out = torch.empty(T, L.H, dtype=torch.bfloat16, device="cuda")
     n0 = moe.moe_kernel_launch_count()
     ref = moe.moe_layer_forward(x, L.wr, L.k, ex, bias=L.bias, ws=ws, out=out).clone()
-    assert moe.moe_kernel_launch_count() - n0 == 5
+    assert moe.moe_kernel_launch_count() - n0 == 4
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -528,8 +529,8 @@ def test_layer_block_scaled_unfused_routing(moe):
 
 
 def test_layer_on_more_streams_than_ticket_counters(moe, decode_layer):
-    """Each stream gets one of 256 ticket counters for the fused routing + permutation;
-    calls on further streams permute in their own launch. Every stream's output must equal
+    """Each stream gets one of 256 sets of slot counts (and ticket counters); calls on
+    further streams permute and quantise in their own launches. Every stream's output must equal
     the default stream's, bit for bit, on both sides of that limit."""
     from cuda.bindings import runtime as rt
 
@@ -561,8 +562,9 @@ def test_layer_on_more_streams_than_ticket_counters(moe, decode_layer):
         torch.cuda.synchronize()
         for h in handles:
             rt.cudaStreamDestroy(h)
-    # fused (5 launches) while counters last, then routing and permutation apart (6)
-    assert launches[-1] == 6 and set(launches) <= {5, 6}
+    # slot layout (4 launches: router, UP, DOWN, combine) while the per-stream counts last,
+    # then routing, permutation and quantiser apart (6)
+    assert launches[-1] == 6 and set(launches) <= {4, 6}
     assert launches == sorted(launches)
     assert moe.moe_device_error() == 0
 
