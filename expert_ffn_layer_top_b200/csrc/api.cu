@@ -713,25 +713,10 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
                              kMaxRouterExperts, E, k);
         if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(wr)) & 15)
             return set_error(MOE_ERR_INVALID_ARG, "x and wr must be 16-byte aligned");
-        // With most experts routed to (T k >= E), the FFN reads nearly every expert in id order: the
-        // first ones' gate/up blobs are pulled into L2 while the router runs (at most kPrefetchL2
-        // bytes, half of L2). Not with a cache, whose slots are known only after routing.
-        constexpr int64_t kPrefetchL2 = 64ll << 20;
-        const uint8_t *pf = nullptr;
-        int64_t pfb = 0;
-        if (!cache && layout == MOE_LAYOUT_TILED && (int64_t)T * k >= E && !experts->expert_map) {
-            const Strides ss = default_strides(*experts);
-            pf = reinterpret_cast<const uint8_t *>(experts->w13);
-            // within the last expert's bytes (the array may end right after them)
-            pfb = std::min<int64_t>(kPrefetchL2, ss.w13 * (E - 1) +
-                                                     (int64_t)prepacked_expert_bytes(experts->fmt, H, I, 0));
-        }
         RouterFuse fz{};
         fz.offsets = offsets;
         fz.sorted_pair = sorted;
         fz.pair_row = prow;
-        fz.pf_base = pf;
-        fz.pf_bytes = pfb;
         // Decode-sized MXFP4 batches: the router writes the slot layout itself (pair rows by
         // atomic claims in per-expert slots, activation rows quantised straight into their
         // tiles), so neither the permutation nor the quantiser runs.

@@ -151,10 +151,6 @@ struct RouterFuse {
     uint8_t *bslab;
     int BN, mt;
     int *sched_zero;   // the FFN's claim counters, zeroed here
-    // L2 prefetch of the expert weights the grouped FFN reads first (static data, issued
-    // before the router waits on its predecessor): pf_bytes from pf_base, 0 = none
-    const uint8_t *pf_base;
-    int64_t pf_bytes;
 };
 // fuse may be null; *fused (if given): 1 the permutation was done, 2 the slot layout was
 // written (fuse->cnt set; the cluster router must apply: router_cluster_ok).

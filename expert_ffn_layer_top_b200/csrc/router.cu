@@ -85,19 +85,8 @@ __device__ __forceinline__ double f32_bits_to_f64(uint32_t f) {
 template <bool WR32>
 __global__ void __launch_bounds__(kDThreads) router_dmma_kernel(const __nv_bfloat16 *__restrict__ x, int T, int H,
                                                                const void *__restrict__ wr, int E, int slice,
-                                                               int wvec, double *__restrict__ part,
-                                                               const uint8_t *__restrict__ pf_base, int64_t pf_bytes) {
+                                                               int wvec, double *__restrict__ part) {
     extern __shared__ __align__(16) double dsm[];
-    if (pf_bytes > 0 && threadIdx.x == 0) {
-        // the expert weights the grouped FFN reads first, into L2 while the batch routes
-        constexpr int64_t kPiece = 64 * 1024;
-        const int64_t nb = (int64_t)gridDim.x * gridDim.y * gridDim.z;
-        const int64_t me = ((int64_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-        for (int64_t o = me * kPiece; o < pf_bytes; o += nb * kPiece) {
-            const int64_t n = pf_bytes - o < kPiece ? pf_bytes - o : kPiece;
-            bulk_prefetch_l2(pf_base + o, (uint32_t)(n & ~int64_t(15)));
-        }
-    }
     pdl_wait();
     pdl_release();
     double *xs = dsm;                        // [2][kDT * kXS]
@@ -424,16 +413,6 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
             bulk_load(wring + c * chunk_bytes, wsrc + c * chunk_bytes, (uint32_t)chunk_bytes, &full[c]);
         }
     }
-    if (fz.pf_bytes > 0 && tid == 32) {
-        // While the batch routes, pull the expert weights the grouped FFN reads first into L2:
-        // 64 KiB pieces dealt round-robin over the CTAs, so the earliest bytes arrive first.
-        constexpr int64_t kPiece = 64 * 1024;
-        const int64_t ncta = (int64_t)gridDim.x * gridDim.y, me = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
-        for (int64_t o = me * kPiece; o < fz.pf_bytes; o += ncta * kPiece) {
-            const int64_t n = fz.pf_bytes - o < kPiece ? fz.pf_bytes - o : kPiece;
-            bulk_prefetch_l2(fz.pf_base + o, (uint32_t)(n & ~int64_t(15)));
-        }
-    }
     // Wr is static and already on its way; x comes from the previous kernel
     pdl_wait();
     pdl_release();
@@ -744,10 +723,6 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
     if (router_cluster_shape(T, H, E, wr_is_fp32, &sh) && (reinterpret_cast<uintptr_t>(wr) & 15) == 0) {
         // the permutation joins this kernel when asked for and small enough for one block
         RouterFuse fz{};
-        if (fuse) {
-            fz.pf_base = fuse->pf_base;
-            fz.pf_bytes = fuse->pf_bytes;
-        }
         if (fuse && fuse->cnt) {   // slot layout: no permutation
             fz = *fuse;
             fz.ticket = nullptr;
@@ -777,7 +752,7 @@ moe_status launch_router(const void *x, int T, int H, const void *wr, int wr_is_
     if (e != cudaSuccess) return set_cuda_error(e, "router smem attribute");
     const int wvec = (E * (wr_is_fp32 ? 4 : 2)) % 16 == 0;
     e = launch_pdl(kfn, grid, dim3(kDThreads), smem, st, reinterpret_cast<const __nv_bfloat16 *>(x), T, H, wr, E, slice,
-                   wvec, part, fuse ? fuse->pf_base : nullptr, fuse ? fuse->pf_bytes : (int64_t)0);
+                   wvec, part);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_cuda_error(e, "router_dmma launch");
     e = launch_pdl(router_finish_kernel, dim3((T + 7) / 8), dim3(256), 0, st, (const double *)part, S, T, E, bias, k,
