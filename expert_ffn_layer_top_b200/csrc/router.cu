@@ -397,6 +397,12 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     uint8_t *wring = rsm + 64;
     double *red = reinterpret_cast<double *>(rsm + 64);              // aliases the ring after the loop
     double *xs = reinterpret_cast<double *>(rsm + 64 + (ring > red_bytes ? ring : red_bytes));   // [hs][TT]
+    // slot layout: the four-plane codes and plane scales of this CTA's slice of each token's row,
+    // [TT][hs / 256 stages][4 planes] x (32 words, 8 scale bytes), after the x tile
+    const int nls = hs / kMxStageK;
+    uint32_t *pcode = reinterpret_cast<uint32_t *>(
+        (reinterpret_cast<uintptr_t>(xs + (size_t)hs * TT) + 15) & ~uintptr_t(15));
+    uint8_t *pscale = reinterpret_cast<uint8_t *>(pcode + (size_t)TT * nls * kMxPlanes * 32);
 
     const int tid = threadIdx.x;
     const int rank = (int)cluster.block_rank();
@@ -436,6 +442,31 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
         }
     }
     __syncthreads();
+    if (fz.cnt) {
+        // The activation rows in the four-plane MXFP4 form do not depend on the routing: this CTA's
+        // slice of them is made now, while the Wr slices stream in. One warp per (token, stage),
+        // 8 elements per lane, 4 lanes per 32-block.
+        const int wq = tid >> 5, lq = tid & 31;
+        for (int item = wq; item < TT * nls; item += kRClThreads / 32) {
+            const int tt2 = item / nls, ls = item - tt2 * nls;
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = (float)xs[(ls * kMxStageK + lq * 8 + i) * TT + tt2];
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            const int s = mx_plane0_exp(amax);
+            uint32_t pw[kMxPlanes];
+            mx_planes8(v, s, pw);
+#pragma unroll
+            for (int pl = 0; pl < kMxPlanes; ++pl) {
+                pcode[(item * kMxPlanes + pl) * 32 + lq] = pw[pl];
+                if ((lq & 3) == 0) pscale[(item * kMxPlanes + pl) * 8 + (lq >> 2)] = (uint8_t)(s - 3 * pl);
+            }
+        }
+    }
 
     // thread (g, ep) owns experts 4 ep .. 4 ep + 3 for every token of the tile over
     // rows [g rows_g, (g + 1) rows_g) of each chunk (a row group is whole warps, so
@@ -574,39 +605,27 @@ __global__ void __cluster_dims__(kRCl, 1, 1) __launch_bounds__(kRClThreads)
     }
     cluster.sync();   // keep this CTA's shared memory alive until every peer has read it
     if (fz.cnt) {
-        // Slot layout: every CTA writes its own slice of H (whole 256-wide stages, still in
-        // shared memory as exact fp64) of each token's activation row, in the four-plane MXFP4
-        // form, into the tiles of the token's k rows; the destinations come from the CTA that
-        // finished the token (rank tt % 8).
-        const int nls = hs / kMxStageK, st0 = h0 / kMxStageK, KST = H / kMxStageK;
+        // Slot layout: every CTA copies its slice of each token's activation row (the codes made
+        // above: whole 256-wide stages) into the tiles of the token's k rows; the destinations come
+        // from the CTA that finished the token (rank tt % 8). Lane L moves 16-byte chunk L % 8 of
+        // plane L / 8 and that 32-block's plane scale.
+        const int st0 = h0 / kMxStageK, KST = H / kMxStageK;
         const int BB = bs_bblob_bytes(kBsMx, fz.BN), NROW = kMxPlanes * fz.BN;
+        const int pl = lane >> 3, c = lane & 7;
         for (int item = warp; item < TT * nls; item += kRClThreads / 32) {
             const int tt2 = item / nls, ls = item - tt2 * nls;
             if (t0 + tt2 >= T) continue;   // warp-uniform
             const int2 *rd = cluster.map_shared_rank(&s_dest[0][0], tt2 % kRCl) + tt2 * kMaxTopK;
             const int2 dj = lane < k ? rd[lane] : make_int2(0, 0);
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = (float)xs[(ls * kMxStageK + lane * 8 + i) * TT + tt2];
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // 4 lanes hold one 32-block
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            const int s = mx_plane0_exp(amax);
-            uint32_t pw[kMxPlanes];
-            mx_planes8(v, s, pw);
-            const int c16 = lane >> 2, st = st0 + ls;
+            const uint4 cw = *reinterpret_cast<const uint4 *>(pcode + (item * kMxPlanes + pl) * 32 + c * 4);
+            const uint8_t sc = pscale[(item * kMxPlanes + pl) * 8 + c];
+            const int st = st0 + ls;
             for (int j = 0; j < k; ++j) {
                 const int tile = __shfl_sync(0xffffffffu, dj.x, j), n = __shfl_sync(0xffffffffu, dj.y, j);
                 uint8_t *blob = fz.bslab + ((int64_t)tile * KST + st) * BB;
-#pragma unroll
-                for (int pl = 0; pl < kMxPlanes; ++pl) {
-                    const int Rw = pl * fz.BN + n;
-                    *reinterpret_cast<uint32_t *>(blob + sw128_chunk(Rw, c16) + (lane & 3) * 4) = pw[pl];
-                    if ((lane & 3) == 0)
-                        blob[NROW * 128 + (c16 >> 2) * 512 + atom_offset(Rw, c16 & 3)] = (uint8_t)(s - 3 * pl);
-                }
+                const int Rw = pl * fz.BN + n;
+                *reinterpret_cast<uint4 *>(blob + sw128_chunk(Rw, c)) = cw;
+                blob[NROW * 128 + (c >> 2) * 512 + atom_offset(Rw, c & 3)] = sc;
             }
         }
         cluster.sync();   // every peer has read this CTA's destinations
@@ -635,6 +654,8 @@ static cudaError_t launch_router_cluster_t(const RouterClusterShape &sh, const v
     size_t smem = sh.smem;
     const size_t perm_smem = 64 + sizeof(SmallPermuteSmem<kRClThreads>) + (size_t)T * k * sizeof(int32_t);
     if (fz.ticket && smem < perm_smem) smem = perm_smem;
+    // slot layout: the plane codes and scales after the x tile (16-byte aligned)
+    if (fz.cnt) smem += 16 + (size_t)TT * (sh.hs / kMxStageK) * kMxPlanes * (32 * 4 + 8);
     if (smem > 48 * 1024) {
         cudaError_t e = ensure_max_smem<router_cluster_kernel<WR32, TT>>((int)smem);
         if (e != cudaSuccess) return e;
