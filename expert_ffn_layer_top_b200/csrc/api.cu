@@ -216,7 +216,7 @@ static moe_status act_tmap(CUtensorMap *m, const void *base, int rows, int K, in
 // atoms) of x and of h; NVFP4 also keeps h in bf16 at offset 0 and the per-row
 // exponent offsets of x and h.
 struct FfnWs {
-    size_t h, re1, re2, a4, tq, b1, b2, sched, total;
+    size_t h, re1, re2, a4, b1, b2, sched, total;
 };
 
 // h: bf16 [n][I] (the decoding paths' h buffer; NVFP4: h before its
@@ -232,7 +232,6 @@ static FfnWs ffn_ws(int n, int H, int I, int E) {
     W.re1 = o; o += align_up((size_t)n * 4, 256);
     W.re2 = o; o += align_up((size_t)n * 4, 256);
     W.a4 = o; o += align_up((size_t)(1 + kA4Parts) * 4, 256);
-    W.tq = o; o += align_up((size_t)n * H / 2, 256) + align_up((size_t)n * H / 16, 256);   // A4 token rows
     W.b1 = o; o += std::max(mx_blob_bytes(n, H, E), a4_blob_bytes(n, H, E));
     W.b2 = o; o += std::max(mx_blob_bytes(n, I, E), a4_blob_bytes(n, I, E));
     W.sched = o; o += 256;
@@ -338,8 +337,9 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
 // scale of x comes from the rows the maxima are taken over: the token rows x [T][H]
 // when gathering (every token appears k times among the pairs), else x_perm.
 static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_src, int64_t amax_elems,
-                              const int32_t *sorted_pair, int k, int n_rows, const int32_t *offsets,
-                              const moe_experts *x, void *y_perm, int y_is_fp32, void *ws, cudaStream_t st) {
+                              const int32_t *sorted_pair, const int32_t *pair_row, int k, int n_rows,
+                              const int32_t *offsets, const moe_experts *x, void *y_perm, int y_is_fp32, void *ws,
+                              cudaStream_t st) {
     if (n_rows == 0) return MOE_OK;
     if (x->fmt != MOE_NVFP4 || x->layout != MOE_LAYOUT_TILED)
         return set_error(MOE_ERR_UNSUPPORTED, "A4 activations need prepacked NVFP4 experts");
@@ -353,12 +353,9 @@ static moe_status a4_ffn_impl(const void *x_src, int gather, const void *amax_sr
     int *sched = reinterpret_cast<int *>(b + W.sched);
     moe_status r = launch_a4_amax(amax_src, amax_elems, parts, sched, st);
     if (r == MOE_OK && gather) {
-        // token rows: quantise each token once (amax_elems / H of them), then place its k pairs
+        // token rows (amax_elems / H of them): each quantised once and placed in its k pairs' rows
         const int T = (int)(amax_elems / H);
-        uint8_t *codes = b + W.tq, *scales = codes + align_up((size_t)n_rows * H / 2, 256);
-        r = launch_a4_token_quant(x_src, T, H, parts, xscale, codes, scales, nsm, st);
-        if (r == MOE_OK)
-            r = launch_a4_scatter(codes, scales, sorted_pair, k, n_rows, H, offsets, E, BN, b + W.b1, nsm, st);
+        r = launch_a4_token_rows(x_src, T, H, k, pair_row, offsets, E, BN, parts, xscale, b + W.b1, nsm, st);
     } else if (r == MOE_OK) {
         r = launch_a4_quant(x_src, 2, sorted_pair, k, n_rows, H, offsets, E, BN, parts, xscale, b + W.b1, nsm, st);
     }
@@ -613,8 +610,8 @@ moe_status moe_grouped_ffn(const void *x_perm, int n_rows, const int32_t *offset
     if (misaligned(y_perm, 16) || misaligned(offsets, 4))
         return set_error(MOE_ERR_INVALID_ARG, "y_perm must be 16-byte aligned, offsets 4-byte aligned");
     if (af == MOE_ACT_A4)
-        return a4_ffn_impl(x_perm, 0, x_perm, (int64_t)n_rows * experts->H, nullptr, 1, n_rows, offsets, experts, y_perm,
-                           y_is_fp32, ws, (cudaStream_t)stream);
+        return a4_ffn_impl(x_perm, 0, x_perm, (int64_t)n_rows * experts->H, nullptr, nullptr, 1, n_rows, offsets, experts,
+                           y_perm, y_is_fp32, ws, (cudaStream_t)stream);
     if (is_mx(*experts, n_rows))
         return mx_ffn_impl(x_perm, 0, nullptr, 1, n_rows, offsets, experts, y_perm, y_is_fp32, ws,
                            (cudaStream_t)stream);
@@ -754,7 +751,8 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
     const SlotInput si{slot_cnt, b + L.slot, T, (T + BNs - 1) / BNs, reinterpret_cast<int32_t *>(b + L.cprefix)};
     if (r == MOE_OK) {
         if (a4)
-            r = a4_ffn_impl(x, 1, x, (int64_t)T * H, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st);
+            r = a4_ffn_impl(x, 1, x, (int64_t)T * H, sorted, prow, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h,
+                            st);
         else if (mx)
             r = mx_ffn_impl(x, 1, sorted, k, T * k, offsets, &view, b + L.y, y_is_fp32, b + L.h, st,
                             slot_cnt ? &si : nullptr);

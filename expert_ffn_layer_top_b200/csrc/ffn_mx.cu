@@ -407,17 +407,31 @@ __global__ void __launch_bounds__(256) a4_quant_kernel(const uint4 *__restrict__
     }
 }
 
-// A4 form of the token rows, once per token (the layer forward, where each token is
-// in k pairs): the same arithmetic as a4_quant_kernel, one warp per (token t, 256-wide
-// stage), written token-major: codes[t][stage] 128 bytes (natural order, low nibble =
-// lower K index), scales[t][stage] 16 E4M3 bytes. Block 0 also stores s_g in *xscale.
-__global__ void __launch_bounds__(256) a4_token_kernel(const uint4 *__restrict__ x, int T, int K,
-                                                       const float *__restrict__ part, float *__restrict__ xscale,
-                                                       uint8_t *__restrict__ codes, uint8_t *__restrict__ scales) {
+// A4 form of the token rows straight into the activation blobs of the FFN's token tiles
+// (the layer forward, where each token is in k pairs): the arithmetic of a4_quant_kernel,
+// once per (token t, 256-wide stage), one warp each, then stored into the rows of the
+// token's k pairs (row r = pair_row[t k + j] of its expert's tile, as in a4_quant_kernel).
+// The next unit's x and pair_row loads are issued before this unit's arithmetic. Block 0 also stores s_g
+// in *xscale.
+__global__ void __launch_bounds__(256) a4_token_rows_kernel(const uint4 *__restrict__ x, int T, int K, int k,
+                                                            const int32_t *__restrict__ pair_row,
+                                                            const int32_t *__restrict__ offsets, int E, int BN,
+                                                            const float *__restrict__ part, float *__restrict__ xscale,
+                                                            uint8_t *__restrict__ bblob) {
+    __shared__ int s_off[kMaxExperts + 1];
+    __shared__ int s_tile[kMaxExperts + 1];
+    __shared__ int s_wsum[8];
     __shared__ float s_sg;
     pdl_wait();
     pdl_release();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int K8 = K / 8, KST = K / kMxStageK, BB = bs_bblob_bytes(kBsNv, BN, 1);
+    const int64_t units = (int64_t)T * KST;
+    const int64_t nw = (int64_t)gridDim.x * 8;
+    int64_t u = (int64_t)blockIdx.x * 8 + warp;
+    uint4 cur = u < units ? x[(u / KST) * K8 + (u % KST) * 32 + lane] : make_uint4(0, 0, 0, 0);
+    int pr = (u < units && lane < k) ? pair_row[(u / KST) * k + lane] : 0;   // lane j < k: row of pair j
+    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
     if (warp == 0) {
         uint32_t m = 0u;
         for (int i = lane; i < kA4Parts; i += 32) m = max(m, __float_as_uint(__ldcg(part + i)));
@@ -431,59 +445,42 @@ __global__ void __launch_bounds__(256) a4_token_kernel(const uint4 *__restrict__
     }
     __syncthreads();
     const float sg = s_sg;
-    const int K8 = K / 8, KST = K / kMxStageK;
-    const int64_t units = (int64_t)T * KST;
-    for (int64_t u = (int64_t)blockIdx.x * 8 + warp; u < units; u += (int64_t)gridDim.x * 8) {
+    for (; u < units; u += nw) {
         const int t = (int)(u / KST), st = (int)(u - (int64_t)t * KST);
+        const int64_t un = u + nw;
+        const uint4 nxt = un < units ? x[(un / KST) * K8 + (un % KST) * 32 + lane] : cur;   // in flight
+        const int prn = (un < units && lane < k) ? pair_row[(un / KST) * k + lane] : 0;
+        // the token's pairs: lane j < k holds pair j's tile and row in it
+        int tile_j = 0, n_j = 0;
+        if (lane < k) {
+            const int r = pr;
+            const int e = expert_of_row(s_off, E, r);
+            const int rel = r - s_off[e];
+            tile_j = s_tile[e] + rel / BN;
+            n_j = rel % BN;
+        }
         float v[8];
-        bf16x8_to_float(x[(int64_t)t * K8 + st * 32 + lane], v);
+        bf16x8_to_float(cur, v);
+        cur = nxt;
+        pr = prn;
         float bmax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));   // two lanes per 16-block
         const uint32_t sc = e4m3_code(__fdiv_rn(__fdiv_rn(bmax, 6.0f), sg));
         const float den = __fmul_rn(e4m3_value(sc), sg);
         float tq[8], q[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) tq[i] = den > 0.0f ? __fdiv_rn(v[i], den) : 0.0f;
-        reinterpret_cast<uint32_t *>(codes)[u * 32 + lane] = e2m1x8(tq, q);
-        if ((lane & 1) == 0) scales[u * 16 + (lane >> 1)] = (uint8_t)sc;
-    }
-}
-
-// The token-major A4 rows into the activation blobs of the FFN's token tiles: one warp
-// per permuted row r = a pair of token t = sorted_pair[r] / k; per stage, its 8 16-byte
-// code chunks go to row n of the blob (128-byte swizzle) and its 16 scales, 4 per atom,
-// to the atoms (row n of atom a: byte (n % 32) 16 + (n / 32) 4).
-__global__ void __launch_bounds__(256) a4_scatter_kernel(const uint8_t *__restrict__ codes,
-                                                         const uint8_t *__restrict__ scales,
-                                                         const int32_t *__restrict__ sorted_pair, int k, int P, int K,
-                                                         const int32_t *__restrict__ offsets, int E, int BN,
-                                                         uint8_t *__restrict__ bblob) {
-    __shared__ int s_off[kMaxExperts + 1];
-    __shared__ int s_tile[kMaxExperts + 1];
-    __shared__ int s_wsum[8];
-    pdl_wait();
-    pdl_release();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    quant_tile_prefix(offsets, E, BN, s_off, s_tile, s_wsum);
-    const int KST = K / kMxStageK, BB = bs_bblob_bytes(kBsNv, BN, 1);
-    for (int r = blockIdx.x * 8 + warp; r < P; r += gridDim.x * 8) {
-        const int e = expert_of_row(s_off, E, r);
-        const int rel = r - s_off[e];
-        const int tile = s_tile[e] + rel / BN, n = rel % BN;
-        const int64_t t = sorted_pair[r] / k;
-        for (int i = lane; i < KST * 12; i += 32) {
-            const int st = i / 12, q = i - st * 12;
+        const uint32_t word = e2m1x8(tq, q);
+        // the 4 scales of atom a (16-blocks 4a..4a+3, lanes 8a, 8a+2, 8a+4, 8a+6) as one word
+        const uint32_t sw = sc | (__shfl_down_sync(0xffffffffu, sc, 2) << 8) |
+                            (__shfl_down_sync(0xffffffffu, sc, 4) << 16) | (__shfl_down_sync(0xffffffffu, sc, 6) << 24);
+        for (int j = 0; j < k; ++j) {
+            const int tile = __shfl_sync(0xffffffffu, tile_j, j), n = __shfl_sync(0xffffffffu, n_j, j);
             uint8_t *blob = bblob + ((int64_t)tile * KST + st) * BB;
-            const int64_t u = t * KST + st;
-            if (q < 8) {
-                *reinterpret_cast<uint4 *>(blob + sw128_chunk(n, q)) = reinterpret_cast<const uint4 *>(codes)[u * 8 + q];
-            } else {
-                const int a = q - 8;
-                *reinterpret_cast<uint32_t *>(blob + BN * 128 + a * 512 + atom_offset(n, 0)) =
-                    reinterpret_cast<const uint32_t *>(scales)[u * 4 + a];
-            }
+            *reinterpret_cast<uint32_t *>(blob + sw128_chunk(n, lane >> 2) + (lane & 3) * 4) = word;
+            if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(blob + BN * 128 + (lane >> 3) * 512 + atom_offset(n, 0)) = sw;
         }
     }
 }
@@ -1370,28 +1367,19 @@ moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair
 
 namespace moe {
 
-moe_status launch_a4_token_quant(const void *x, int T, int K, const float *partials, float *xscale, void *codes,
-                                 void *scales, int num_sms, cudaStream_t st) {
+moe_status launch_a4_token_rows(const void *x, int T, int K, int k, const int32_t *pair_row, const int32_t *offsets,
+                                int E, int BN, const float *partials, float *xscale, void *bblob, int num_sms,
+                                cudaStream_t st) {
+    if (T == 0) return MOE_OK;
+    if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
     if (K % kMxStageK) return set_error(MOE_ERR_UNSUPPORTED, "K=%d is not a multiple of %d", K, kMxStageK);
     const int64_t units = (int64_t)T * (K / kMxStageK);
     const int blocks = (int)((units + 7) / 8 < (int64_t)num_sms * 8 ? (units + 7) / 8 : (int64_t)num_sms * 8);
-    cudaError_t e = launch_pdl(a4_token_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st,
-                               reinterpret_cast<const uint4 *>(x), T, K, partials, xscale,
-                               reinterpret_cast<uint8_t *>(codes), reinterpret_cast<uint8_t *>(scales));
+    cudaError_t e = launch_pdl(a4_token_rows_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st,
+                               reinterpret_cast<const uint4 *>(x), T, K, k, pair_row, offsets, E, BN, partials, xscale,
+                               reinterpret_cast<uint8_t *>(bblob));
     if (e == cudaSuccess) e = cudaGetLastError();
-    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 token quantiser launch");
-}
-
-moe_status launch_a4_scatter(const void *codes, const void *scales, const int32_t *sorted_pair, int k, int P, int K,
-                             const int32_t *offsets, int E, int BN, void *bblob, int num_sms, cudaStream_t st) {
-    if (P == 0) return MOE_OK;
-    if (E > kMaxExperts) return set_error(MOE_ERR_UNSUPPORTED, "E=%d above %d", E, kMaxExperts);
-    const int blocks = (P + 7) / 8 < num_sms * 8 ? (P + 7) / 8 : num_sms * 8;
-    cudaError_t e = launch_pdl(a4_scatter_kernel, dim3(blocks), dim3(256), 0, st,
-                               reinterpret_cast<const uint8_t *>(codes), reinterpret_cast<const uint8_t *>(scales),
-                               sorted_pair, k, P, K, offsets, E, BN, reinterpret_cast<uint8_t *>(bblob));
-    if (e == cudaSuccess) e = cudaGetLastError();
-    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 scatter launch");
+    return e == cudaSuccess ? MOE_OK : set_cuda_error(e, "A4 token rows launch");
 }
 
 }  // namespace moe

@@ -118,12 +118,11 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
 int choose_bn_a4(int n_rows, int E);
 size_t a4_blob_bytes(int n_rows, int K, int E);
 moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, int *sched_zero, cudaStream_t st);
+moe_status launch_a4_token_rows(const void *x, int T, int K, int k, const int32_t *pair_row, const int32_t *offsets,
+                                int E, int BN, const float *partials, float *xscale, void *bblob, int num_sms,
+                                cudaStream_t st);
 // Token-major A4 rows of x [T][K] (codes [T][K/2], scales [T][K/16]), then their scatter into
 // the blobs of the pairs (the layer forward's path: each token quantised once, not k times).
-moe_status launch_a4_token_quant(const void *x, int T, int K, const float *partials, float *xscale, void *codes,
-                                 void *scales, int num_sms, cudaStream_t st);
-moe_status launch_a4_scatter(const void *codes, const void *scales, const int32_t *sorted_pair, int k, int P, int K,
-                             const int32_t *offsets, int E, int BN, void *bblob, int num_sms, cudaStream_t st);
 moe_status launch_a4_quant(const void *src, int mode, const int32_t *sorted_pair, int k, int P, int K,
                            const int32_t *offsets, int E, int BN, const float *partials, float *xscale, void *bblob,
                            int num_sms, cudaStream_t st);
