@@ -18,6 +18,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -42,10 +43,24 @@ constexpr int kTargetBlocks = 444;   // three blocks per SM of a 148-SM B200
 
 static void router_split(int T, int H, int E, int *S, int *slice) {
     const int tiles = ((T + kDT - 1) / kDT) * ((E + kDE - 1) / kDE);
-    int s = (kTargetBlocks + tiles - 1) / tiles;
-    const int maxs = (H + kDK - 1) / kDK;
-    if (s > maxs) s = maxs;
-    if (s < 1) s = 1;
+    // The split of H with the shortest estimated time, among splits up to about two waves of
+    // blocks (at least 4; this bounds the fp64 partial sums): an SM runs 3 blocks at once at the
+    // full fp64 tensor rate, 2 at about 80% of it, 1 at about half, so a block count just above
+    // a multiple of 3 per SM leaves a slow tail (at prefill, 4 slices give 512 blocks: 68 SMs
+    // run a 4th block alone).
+    const int maxs = std::min(std::max(4, (2 * kTargetBlocks + tiles - 1) / tiles), (H + kDK - 1) / kDK);
+    int s = 1;
+    double best = 0.0;
+    for (int c = 1; c <= maxs; ++c) {
+        const int64_t blocks = (int64_t)tiles * c;
+        const int64_t per_sm = (blocks + kTargetBlocks / 3 - 1) / (kTargetBlocks / 3);
+        const double rounds = 3.0 * (double)(per_sm / 3) + (per_sm % 3 == 1 ? 2.0 : (per_sm % 3 == 2 ? 2.5 : 0.0));
+        const double t = rounds / (double)blocks;   // in units of the whole router's work
+        if (c == 1 || t < best - 1e-12) {
+            best = t;
+            s = c;
+        }
+    }
     int sl = (H + s - 1) / s;
     sl = (sl + kDK - 1) / kDK * kDK;
     *slice = sl;
