@@ -254,7 +254,7 @@ def time_ffn_only(moe, lb: LayerBench, K: int, W: int, device):
 
 def source_sha():
     h = hashlib.sha256()
-    for f in ("ffn_tc.cu", "ffn_mx.cu", "common.cuh"):
+    for f in ("ffn_tc.cu", "ffn_mx.cu", "mx_codec.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "expert_ffn_layer_top_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
