@@ -225,15 +225,19 @@ struct FfnWs {
 // x and h for the block-scaled FP4 path (four planes, or one in A4 form: the
 // larger of the two sizes); sched: the block-scaled kernels' item claim counters (UP,
 // DOWN), zeroed by the quantiser that runs first.
-static FfnWs ffn_ws(int n, int H, int I, int E) {
+// bound: size the activation blobs for the largest need over all row counts up to n
+// (the layout itself is always the one for n).
+static FfnWs ffn_ws(int n, int H, int I, int E, bool bound = false) {
     FfnWs W;
     size_t o = 0;
     W.h = o; o += align_up((size_t)n * I * 2, 256);
     W.re1 = o; o += align_up((size_t)n * 4, 256);
     W.re2 = o; o += align_up((size_t)n * 4, 256);
     W.a4 = o; o += align_up((size_t)(1 + kA4Parts) * 4, 256);
-    W.b1 = o; o += std::max(mx_blob_bytes(n, H, E), a4_blob_bytes(n, H, E));
-    W.b2 = o; o += std::max(mx_blob_bytes(n, I, E), a4_blob_bytes(n, I, E));
+    W.b1 = o; o += bound ? std::max(mx_blob_bound(n, H, E), a4_blob_bound(n, H, E))
+                         : std::max(mx_blob_bytes(n, H, E), a4_blob_bytes(n, H, E));
+    W.b2 = o; o += bound ? std::max(mx_blob_bound(n, I, E), a4_blob_bound(n, I, E))
+                         : std::max(mx_blob_bytes(n, I, E), a4_blob_bytes(n, I, E));
     W.sched = o; o += 256;
     W.total = o;
     return W;
@@ -471,11 +475,22 @@ static size_t slot_blob_bytes(int T, int H, int E, int k) {
     return bytes <= (64ll << 20) ? align_up((size_t)bytes, 256) : 0;
 }
 
-static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
+// The largest slot region over all batches up to T (it depends on the tile height and
+// stops above 256 tokens or 64 MiB).
+static size_t slot_blob_bound(int T, int H, int E, int k) {
+    size_t m = 0;
+    for (int t = 1; t <= std::min(T, 256); ++t) m = std::max(m, slot_blob_bytes(t, H, E, k));
+    return m;
+}
+
+// bound: every term that can shrink as T grows (the router's H split, the FP4
+// activation blobs, the slot region) taken at its largest over all batches up to T,
+// so the total never decreases with T. With bound set only the total is meaningful.
+static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32, bool bound = false) {
     LayerWs L;
     const size_t P = (size_t)T * k;
     size_t o = 0;
-    L.router = o; o += align_up(router_ws_bytes(T, H, E), 256);
+    L.router = o; o += align_up(bound ? router_ws_bound(T, H, E) : router_ws_bytes(T, H, E), 256);
     L.idx = o; o += align_up(P * 4, 256);
     L.w = o; o += align_up(P * 4, 256);
     L.offsets = o; o += align_up((size_t)(E + 1) * 4, 256);
@@ -483,9 +498,9 @@ static LayerWs layer_ws(int T, int H, int I, int E, int k, int y32) {
     L.pair_row = o; o += align_up(P * 4, 256);
     L.perm = o; o += align_up(permute_ws_bytes(T, k, E), 256);
     L.x_perm = o; o += align_up(P * H * 2, 256);
-    L.h = o; o += ffn_ws_bytes((int)P, H, I, E);
+    L.h = o; o += ffn_ws((int)P, H, I, E, bound).total;
     L.y = o; o += align_up(P * H * (y32 ? 4 : 2), 256);
-    L.slot = o; o += slot_blob_bytes(T, H, E, k);
+    L.slot = o; o += bound ? slot_blob_bound(T, H, E, k) : slot_blob_bytes(T, H, E, k);
     L.cprefix = o; o += align_up((size_t)E * 4, 256);
     L.total = o;
     return L;
@@ -537,7 +552,7 @@ moe_status moe_device_error(int *code) {
 
 size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32, int af) {
     if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || (af != MOE_ACT_A16 && af != MOE_ACT_A4)) return 0;
-    return layer_ws(T, H, I, E, k, y_is_fp32).total;
+    return layer_ws(T, H, I, E, k, y_is_fp32, true).total;
 }
 
 moe_status moe_route_topk(const void *x, int T, int H, const void *wr, int wr_is_fp32, const float *bias, int E,

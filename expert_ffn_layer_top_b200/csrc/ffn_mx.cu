@@ -1226,6 +1226,24 @@ size_t mx_blob_bytes(int n_rows, int K, int E) {
     return align_up(mx_tiles_ub(n_rows, E) * (K / kMxStageK) * bs_bblob_bytes(kBsNv, choose_bn_mx(n_rows, E)), 256);
 }
 
+// The largest blob over all row counts up to n_rows. Each size grows with the rows
+// while the tile height stays put; it can drop where the height steps up (the mean
+// rows per expert passing 8 and 16, or 32 and 64), so the last row count before each
+// step is a candidate.
+size_t mx_blob_bound(int n_rows, int K, int E) {
+    size_t m = mx_blob_bytes(n_rows, K, E);
+    for (int avg : {8, 16})
+        if ((int64_t)avg * E < n_rows) m = std::max(m, mx_blob_bytes(avg * E, K, E));
+    return m;
+}
+
+size_t a4_blob_bound(int n_rows, int K, int E) {
+    size_t m = a4_blob_bytes(n_rows, K, E);
+    for (int avg : {32, 64})
+        if ((int64_t)avg * E < n_rows) m = std::max(m, a4_blob_bytes(avg * E, K, E));
+    return m;
+}
+
 static size_t mx_smem_bytes(int fmt, int phase, int BN, int stages, int E, int planes) {
     const size_t stage = (size_t)bs_ablob_bytes(fmt) + bs_bblob_bytes(fmt, BN, planes);
     return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 128 * kMxXch * 4 : 0) + sizeof(MxSmem) +

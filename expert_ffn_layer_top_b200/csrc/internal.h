@@ -110,6 +110,7 @@ struct MxPlan {
 bool mx_plan(int fmt, int phase, int BN, int K, int E, MxPlan *pl, int planes = kMxPlanes);
 size_t mx_tiles_ub(int n_rows, int E);
 size_t mx_blob_bytes(int n_rows, int K, int E);
+size_t mx_blob_bound(int n_rows, int K, int E);   // max of mx_blob_bytes over row counts <= n_rows
 // planes: kMxPlanes (A16 activations) or 1 (A4, NVFP4 only)
 moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, cudaStream_t st,
                            int planes = kMxPlanes);
@@ -117,6 +118,7 @@ moe_status launch_mx_phase(int fmt, int phase, int BN, MxParams p, int num_sms, 
 // partial maxima of |x| and the quantiser (src rows as launch_mx_quant modes 1 and 2).
 int choose_bn_a4(int n_rows, int E);
 size_t a4_blob_bytes(int n_rows, int K, int E);
+size_t a4_blob_bound(int n_rows, int K, int E);   // max of a4_blob_bytes over row counts <= n_rows
 moe_status launch_a4_amax(const void *src, int64_t n_elems, float *partials, int *sched_zero, cudaStream_t st);
 moe_status launch_a4_token_rows(const void *x, int T, int K, int k, const int32_t *pair_row, const int32_t *offsets,
                                 int E, int BN, const float *partials, float *xscale, void *bblob, int num_sms,
@@ -137,6 +139,7 @@ moe_status launch_dequant(int fmt, const void *w, const void *scale, float tscal
 
 // router (router.cu)
 size_t router_ws_bytes(int T, int H, int E);
+size_t router_ws_bound(int T, int H, int E);   // max of router_ws_bytes over batches <= T
 // Outputs of the permutation for a router launch that also permutes (the
 // layer forward); the launcher fills in the ticket counter.
 struct RouterFuse {

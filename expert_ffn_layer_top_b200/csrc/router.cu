@@ -74,6 +74,14 @@ size_t router_ws_bytes(int T, int H, int E) {
     return align_up((size_t)S * T * E * sizeof(double), 256);
 }
 
+size_t router_ws_bound(int T, int H, int E) {
+    // The split depends only on the tile count, so between tile boundaries the partials grow
+    // with T; the largest over smaller batches sits at one of the boundaries below T.
+    size_t m = router_ws_bytes(T, H, E);
+    for (int t = kDT; t < T; t += kDT) m = std::max(m, router_ws_bytes(t, H, E));
+    return m;
+}
+
 __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
     asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
                  : "+d"(d[0]), "+d"(d[1])

@@ -304,13 +304,14 @@ moe_status moe_layer_forward(const void *x, int T, const void *wr, int wr_is_fp3
                              moe_stream_t stream);
 
 /* Scratch bytes needed by moe_layer_forward / moe_route_topk / moe_permute /
- * moe_grouped_ffn for these sizes and activation format (an upper bound that
- * covers every path the sizes can take: the router's fp64 partial sums, the
+ * moe_grouped_ffn for these sizes and activation format: an upper bound that
+ * covers every path the sizes can take (the router's fp64 partial sums, the
  * routing, the permutation, x_perm, h or the FP4 activation blobs, y, and for
- * decode-sized batches the slot layout's tiles, which make the size larger at
- * T = 64 than at T = 128, where that layout is not used). No
- * counterpart in the pages: it is what lets every call run without allocating.
- * Host-only, no CUDA call; 0 for non-positive sizes or an unknown af. */
+ * decode-sized batches the slot layout's tiles). The bound never decreases as T
+ * grows, with the other sizes fixed, so a workspace sized for the largest batch
+ * serves every smaller one. No counterpart in the pages: it is what lets every
+ * call run without allocating. Host-only, no CUDA call; 0 for non-positive sizes
+ * or an unknown af. */
 size_t moe_workspace_size(int T, int H, int I, int E, int k, int y_is_fp32, int af);
 
 /* ---------------------------------------------------------------- cache */

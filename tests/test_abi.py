@@ -42,12 +42,10 @@ def test_library_loads_and_host_only_calls_work():
 
     L = moe.lib()
     assert moe.moe_version().startswith("libmoe")
-    # workspace sizing is host arithmetic only; it grows with T outside the decode sizes,
-    # whose slot layout adds its own tiles
+    # workspace sizing is host arithmetic only
     a = moe.moe_workspace_size(1024, 2048, 768, 128, 8)
     b = moe.moe_workspace_size(2048, 2048, 768, 128, 8)
     assert 0 < a < b
-    assert moe.moe_workspace_size(64, 2048, 768, 128, 8) > moe.moe_workspace_size(128, 2048, 768, 128, 8) > 0
     assert moe.moe_workspace_size(-1, 2048, 768, 128, 8) == 0
     assert L.moe_last_error_string() is not None
 

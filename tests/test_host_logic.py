@@ -179,6 +179,16 @@ def test_workspace_size_is_monotone_and_rejects_bad_sizes():
         H, I, E, k = cfg
         sizes = [ws(T, H, I, E, k) for T in (1, 8, 64, 512, 4096)]
         assert all(0 < a < b for a, b in zip(sizes, sizes[1:]))
+    # never smaller for a larger batch, across every step of the terms that depend on a tile
+    # choice: the slot layout's tile height and its 256-token and 64 MiB limits, the activation
+    # blobs' tile height (mean rows per expert past 8, 16, 32, 64), the router's H split per
+    # 64-token tile
+    for H, I, E, k in ((4096, 2048, 256, 6), (2048, 768, 128, 8), (2048, 1024, 32, 4), (6144, 1536, 160, 8)):
+        prev = 0
+        for T in list(range(1, 300)) + list(range(300, 2200, 7)):
+            s = ws(T, H, I, E, k)
+            assert s >= prev, (H, I, E, k, T, s, prev)
+            prev = s
         assert ws(64, H, I, E, k, 1) > ws(64, H, I, E, k, 0)
         assert ws(64, H, I, E, k) < ws(64, H, I, E, k + 1)
         # at least the permuted activations and the expert outputs of every pair
