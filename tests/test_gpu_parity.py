@@ -283,6 +283,23 @@ def test_layer_decode_mxfp4(moe, decode_layer, T):
     _layer_check(moe, decode_layer, x)
 
 
+@pytest.mark.parametrize("T,y_fp32", [(1, True), (37, False), (64, True), (256, False)])
+def test_layer_decode_mxfp4_combine_in_down(moe, decode_layer, T, y_fp32):
+    """Slot layout (the router claims the rows and writes the activation tiles; the combine
+    maps slot rows to y rows through UP's count prefix): a ragged batch, the largest batch
+    the layout takes, and y kept in fp32, against the oracle."""
+    x = synthetic.make_tokens(T, 2048, seed=300 + T)
+    _layer_check(moe, decode_layer, x, y_fp32=y_fp32)
+
+
+def test_layer_top16_slot_layout(moe):
+    """k = 16 through the slot layout (H a multiple of 2048): 16 claims per token in the
+    router, 16 rows per token in the combine."""
+    cfg = dict(H=2048, E=64, k=16, I=256, fmt="mxfp4", wr_fp32=False)
+    L = synthetic.make_layer(cfg, seed=27)
+    _layer_check(moe, L, synthetic.make_tokens(40, 2048, seed=27))
+
+
 def test_layer_fused_routing_and_permutation(moe, decode_layer):
     """A decode-sized MXFP4 batch takes the slot layout: the router claims each pair's
     row in its expert's slot and writes the activation rows itself, so a layer call is
