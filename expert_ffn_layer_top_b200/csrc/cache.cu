@@ -174,17 +174,82 @@ __device__ void lru_predict_warp(const LruTable &t, int layer, int depth, bool f
     __syncwarp();
 }
 
-// mode 0: resolve `layer` from idx[P]; then, unless pf_mode is 0, prefetch layer+1
-//         (pf_mode 1: the first `depth` of its prediction, depth < 0 all; 2: every expert)
-// mode 1: prefetch `layer` with the explicit ids in io (count io[0], ids io[1..])
-// Output in io: [0] status (0 ok, 6 cache full), [1] n resolve loads, [2] n prefetch loads
-// (-1 = not run or full), then the pairs.
-__global__ void __launch_bounds__(32) lru_kernel(LruTable t, int layer, const int32_t *idx, int P, int mode,
-                                                  int pf_mode, int depth, int32_t *io) {
-    __shared__ uint32_t req[kMaxExperts / 32];
-    __shared__ uint32_t pf[kMaxExperts / 32];
-    __shared__ int32_t cnt[kMaxExperts];
-    __shared__ uint32_t keys[kMaxExperts];
+// Shared-memory image of the table for one update: the parts a call can touch (every
+// layer's slot_of, last and lastcnt; owner, prev, next, ref and the free bitmap of the S
+// slots in use; the state and counters), each padded to 16 bytes. The update then makes
+// its dependent reads (about ten per requested expert) in shared memory.
+struct LruStage {
+    int n[10];        // words of each part: slot_of owner prev next ref freeb last lastcnt st counts
+    int off[10];      // word offset of each part in the image
+    int total;        // words
+};
+constexpr int kLruStageThreads = 512;
+constexpr int kLruStageMaxBytes = 200 * 1024;
+
+__host__ __device__ inline LruStage lru_stage(int L, int E, int S) {
+    LruStage g;
+    const int lw = (E + 31) / 32;
+    const int n[10] = {L * E, S, S, S, S, (S + 31) / 32, L * lw, L * E, ST_N, 4};
+    int o = 0;
+    for (int i = 0; i < 10; ++i) {
+        g.n[i] = (n[i] + 3) & ~3;
+        g.off[i] = o;
+        o += g.n[i];
+    }
+    g.total = o;
+    return g;
+}
+
+// The table's arrays in the order of LruStage (base pointers).
+__device__ inline void lru_parts(const LruTable &t, uint32_t **p) {
+    p[0] = reinterpret_cast<uint32_t *>(t.slot_of);
+    p[1] = reinterpret_cast<uint32_t *>(t.owner);
+    p[2] = reinterpret_cast<uint32_t *>(t.prev);
+    p[3] = reinterpret_cast<uint32_t *>(t.next);
+    p[4] = reinterpret_cast<uint32_t *>(t.ref);
+    p[5] = t.freeb;
+    p[6] = t.last;
+    p[7] = reinterpret_cast<uint32_t *>(t.lastcnt);
+    p[8] = reinterpret_cast<uint32_t *>(t.st);
+    p[9] = reinterpret_cast<uint32_t *>(t.counts);
+}
+
+// Global address of 16-byte chunk j of the image (j < g.total / 4).
+__device__ inline uint4 *lru_stage_src(const LruStage &g, uint32_t *const *gp, int j) {
+    int i = 0;
+    while (i < 9 && j >= g.off[i + 1] / 4) ++i;
+    return reinterpret_cast<uint4 *>(gp[i]) + (j - g.off[i] / 4);
+}
+
+// Copies the image in (in = true) or back, over all parts as one range of 16-byte chunks,
+// eight in flight per thread. The parts start 256-byte aligned in global memory with room
+// past each used end (their allocations are padded to 256 bytes, or hold max_slots >= S
+// entries), and a word read past the end is written back unchanged.
+__device__ inline void lru_stage_copy(const LruStage &g, uint32_t *const *gp, uint4 *img, bool in) {
+    constexpr int kU = 8;
+    const int n4 = g.total / 4;
+    for (int j0 = threadIdx.x; j0 < n4; j0 += kU * blockDim.x) {
+        uint4 v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int j = j0 + u * blockDim.x;
+            if (j < n4) v[u] = in ? *lru_stage_src(g, gp, j) : img[j];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int j = j0 + u * blockDim.x;
+            if (j < n4) {
+                if (in) img[j] = v[u];
+                else *lru_stage_src(g, gp, j) = v[u];
+            }
+        }
+    }
+}
+
+// The update by one warp (lane = thread index): the request bitmap and pair counts of the
+// call, the prediction of the next layer, then lane 0 runs the table's policy.
+__device__ void lru_update_warp(LruTable &t, int layer, const int32_t *idx, int P, int mode, int pf_mode,
+                                int depth, int32_t *io, uint32_t *req, uint32_t *pf, int32_t *cnt, uint32_t *keys) {
     const int lane = threadIdx.x;
     const int words = (t.E + 31) / 32;
     for (int w = lane; w < words; w += 32) req[w] = 0;
@@ -211,8 +276,53 @@ __global__ void __launch_bounds__(32) lru_kernel(LruTable t, int layer, const in
     const bool pfn = mode == 0 && pf_mode != 0 && layer + 1 < t.L;
     if (pfn) lru_predict_warp(t, layer + 1, depth, pf_mode == 2, pf, keys);
     __syncwarp();
-    if (lane != 0) return;
-    lru_run(t, layer, req, mode == 0 ? cnt : nullptr, mode, pfn ? pf : nullptr, io);
+    if (lane == 0) lru_run(t, layer, req, mode == 0 ? cnt : nullptr, mode, pfn ? pf : nullptr, io);
+}
+
+// mode 0: resolve `layer` from idx[P]; then, unless pf_mode is 0, prefetch layer+1
+//         (pf_mode 1: the first `depth` of its prediction, depth < 0 all; 2: every expert)
+// mode 1: prefetch `layer` with the explicit ids in io (count io[0], ids io[1..])
+// Output in io: [0] status (0 ok, 6 cache full), [1] n resolve loads, [2] n prefetch loads
+// (-1 = not run or full), then the pairs.
+// staged: the block (kLruStageThreads threads) copies the table into dynamic shared
+// memory (lru_stage), warp 0 updates it there, and the block copies it back; otherwise
+// one warp updates the table in global memory. The table was last written by the update
+// before (several kernels back), so it is read before the wait on the kernel just before,
+// which writes idx.
+__global__ void __launch_bounds__(kLruStageThreads) lru_kernel(LruTable tg, int layer, const int32_t *idx, int P,
+                                                               int mode, int pf_mode, int depth, int32_t *io,
+                                                               int staged) {
+    __shared__ uint32_t req[kMaxExperts / 32];
+    __shared__ uint32_t pf[kMaxExperts / 32];
+    __shared__ int32_t cnt[kMaxExperts];
+    __shared__ uint32_t keys[kMaxExperts];
+    extern __shared__ uint4 img[];
+    LruTable t = tg;
+    LruStage g;
+    uint32_t *gp[10];
+    if (staged) {
+        g = lru_stage(tg.L, tg.E, tg.S);
+        lru_parts(tg, gp);
+        lru_stage_copy(g, gp, img, true);
+        uint32_t *w = reinterpret_cast<uint32_t *>(img);
+        t.slot_of = reinterpret_cast<int32_t *>(w + g.off[0]);
+        t.owner = reinterpret_cast<int32_t *>(w + g.off[1]);
+        t.prev = reinterpret_cast<int32_t *>(w + g.off[2]);
+        t.next = reinterpret_cast<int32_t *>(w + g.off[3]);
+        t.ref = reinterpret_cast<int32_t *>(w + g.off[4]);
+        t.freeb = w + g.off[5];
+        t.last = w + g.off[6];
+        t.lastcnt = reinterpret_cast<int32_t *>(w + g.off[7]);
+        t.st = reinterpret_cast<int32_t *>(w + g.off[8]);
+        t.counts = reinterpret_cast<unsigned long long *>(w + g.off[9]);
+    }
+    pdl_wait();
+    if (staged) __syncthreads();
+    if (threadIdx.x < 32) lru_update_warp(t, layer, idx, P, mode, pf_mode, depth, io, req, pf, cnt, keys);
+    if (staged) {
+        __syncthreads();
+        lru_stage_copy(g, gp, img, false);
+    }
 }
 
 __global__ void lru_init_kernel(LruTable t) { lru_init_one(t, blockIdx.x * blockDim.x + threadIdx.x); }
@@ -259,6 +369,21 @@ static size_t table_block_bytes(int L, int E, int Smax) {
 }
 
 static LruTable table_of(expert_cache *c) { return table_at(c, reinterpret_cast<uint8_t *>(c->d_slot_of)); }
+
+// Launches the table update: staged in shared memory when the image fits, else one warp
+// on the table in global memory.
+static cudaError_t launch_lru(expert_cache *c, int layer, const int32_t *idx, int P, int mode, int pf_mode,
+                              int depth, cudaStream_t st) {
+    const LruTable t = table_of(c);
+    const size_t bytes = (size_t)lru_stage(t.L, t.E, t.S).total * 4;
+    cudaError_t e;
+    if (bytes <= (size_t)kLruStageMaxBytes && ensure_max_smem<lru_kernel>((int)bytes) == cudaSuccess)
+        e = launch_pdl(lru_kernel, dim3(1), dim3(kLruStageThreads), bytes, st, t, layer, idx, P, mode, pf_mode, depth,
+                       c->d_io, 1);
+    else
+        e = launch_pdl(lru_kernel, dim3(1), dim3(32), 0, st, t, layer, idx, P, mode, pf_mode, depth, c->d_io, 0);
+    return e == cudaSuccess ? cudaGetLastError() : e;
+}
 
 static size_t part_bytes(int fmt, int rows, int K, bool scale) {
     if (scale) return (size_t)rows * scale_rowbytes(fmt, K);
@@ -477,9 +602,7 @@ moe_status cache_resolve_and_map(expert_cache *c, int layer, const int32_t *idx,
     timer_open(c);
     ++c->calls;
     timer_mark(c, TK_TABLE_B, st);
-    count_launch();
-    lru_kernel<<<1, 32, 0, st>>>(table_of(c), layer, idx, T * k, 0, pf_mode, depth, c->d_io);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_lru(c, layer, idx, T * k, 0, pf_mode, depth, st);
     timer_mark(c, TK_TABLE_E, st);
     const double t0 = now_s();
     if (e == cudaSuccess) e = cudaEventRecord(c->ev_lru, st);
@@ -700,9 +823,7 @@ moe_status expert_cache_prefetch(struct expert_cache *c, int layer, const int32_
     // the previous call's readback is complete (it was synchronised), so io is free
     c->h_io[0] = n;
     memcpy(c->h_io + 1, ids, sizeof(int32_t) * n);
-    count_launch();
-    lru_kernel<<<1, 32, 0, st>>>(table_of(c), layer, nullptr, 0, 1, 0, 0, c->d_io);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_lru(c, layer, nullptr, 0, 1, 0, 0, st);
     if (e == cudaSuccess) e = cudaEventRecord(c->ev_lru, st);
     if (e == cudaSuccess) e = cudaEventSynchronize(c->ev_lru);
     if (e != cudaSuccess) return set_cuda_error(e, "prefetch table update");
