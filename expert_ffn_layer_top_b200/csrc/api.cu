@@ -312,6 +312,9 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
         p.slab_mt = slot->mt;
         p.cprefix = slot->cprefix;
         p.slab_wait = 1;   // the counts may come from the kernel just before
+        // with at least 4 pairs per expert on average few experts are without rows (uniform
+        // routing: under 2%), so an empty head tile rarely streams an unused expert's weights
+        p.slab_head = n_rows >= 4 * E;
     }
     if ((r = launch_mx_phase(fmt, kPhaseUp, BN, p, nsm, st)) != MOE_OK) return r;
     if (fmt == kBsNv &&
@@ -334,6 +337,7 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.slab_mt = 0;         // h is in compact tiles
     p.cprefix = nullptr;
     p.slab_wait = 0;       // the counts come from two kernels back
+    p.slab_head = 0;
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 

@@ -509,22 +509,42 @@ struct MxSmem {
 
 struct MxItem {
     int e, rt, row0, nvalid, m, slot;
-    int rtin;   // the tile of the phase's input blob (rt, or the expert's slot tile)
+    int rtin;     // the tile of the phase's input blob (rt, or the expert's slot tile)
+    int rt_out;   // the tile of the output blob (h for the down pass): the compact tile in expert order
 };
 
-// tab = tile_start[E + 1], then off[E + 1] (a copy of offsets), then slot[E].
+// Head mode (p.slab_head): the experts whose first tile leads the item order, enough for
+// every CTA's static first items.
+__device__ __forceinline__ int mx_head_experts(const MxParams &p) {
+    const int F = p.itempar ? p.pipes : 1;
+    const int h = ((int)gridDim.x * F + p.m_tiles - 1) / p.m_tiles;
+    return h < p.E ? h : p.E;
+}
+
+// tab = tile_start[E + 1], then off[E + 1] (a copy of offsets), then slot[E], then std_start[E + 1].
+// tile_start: the prefix of each expert's tiles in item order (head mode: of the tiles after
+// the head ones); std_start: the prefix of all its tiles (the compact order of the outputs).
 __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int item, int BN) {
     const int *tile_start = tab, *off = tab + p.E + 1, *slot = tab + 2 * (p.E + 1);
+    const int *std_start = tab + 3 * p.E + 2;
     MxItem it;
     it.rt = item / p.m_tiles;
     it.m = item - it.rt * p.m_tiles;
-    int lo = 0, hi = p.E - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tile_start[mid] <= it.rt) lo = mid; else hi = mid - 1;
+    const int SH = p.slab_head ? mx_head_experts(p) : 0;
+    int lo = 0, t = 0;
+    if (it.rt < SH) {
+        lo = it.rt;   // the expert's first tile, possibly without rows
+    } else {
+        const int x = it.rt - SH;
+        int hi = p.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tile_start[mid] <= x) lo = mid; else hi = mid - 1;
+        }
+        t = x - tile_start[lo] + (lo < SH ? 1 : 0);
     }
+    it.rt_out = p.slab_head ? std_start[lo] + t : it.rt;
     it.e = lo;
-    const int t = it.rt - tile_start[lo];
     const int beg = off[lo];
     it.row0 = beg + t * BN;
     it.nvalid = min(BN, off[lo + 1] - beg - t * BN);
@@ -636,6 +656,24 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    // Head mode: the static first item of each pipeline is an expert's first tile whatever the
+    // routing (item = blockIdx.x + j0 gridDim.x, expert item / m_tiles), so its weights go out
+    // now, while the routing kernel is still running and before the tile prefix waits on it.
+    int pre_head = 0;
+    if (p.slab_head) {
+        __syncthreads();   // the barriers are initialised
+        const int item = blockIdx.x + j0 * gridDim.x;
+        if (warp < 4 && lane == 0 && warp < NP && item < mx_head_experts(p) * p.m_tiles) {
+            const int e = item / p.m_tiles, m = item - e * p.m_tiles;
+            const int slot = p.expert_map ? p.expert_map[e] : e;
+            for (int st = st0; st < KST && pre_head < NSW; st += dst, ++pre_head) {
+                const int s = warp * NSW + pre_head;
+                mbar_expect_tx(&sm.full[s], (uint32_t)STAGE);
+                bulk_load(base + s * STAGE, p.wbase + (int64_t)slot * p.w_estride + ((int64_t)m * KST + st) * ABLOB,
+                          ABLOB, &sm.full[s]);
+            }
+        }
+    }
     if (warp == 12) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
@@ -644,11 +682,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
         // Offsets come from the permutation, two launches back, so they are
         // complete before this kernel's predecessor could let it start. In the slot
         // layout the counts may come from the kernel just before (then: wait first).
-        int *tile_start = tab, *off = tab + p.E + 1, *slot = tab + 2 * (p.E + 1);
+        int *tile_start = tab, *off = tab + p.E + 1, *slot = tab + 2 * (p.E + 1), *std_start = tab + 3 * p.E + 2;
         if (p.slab_cnt && p.slab_wait) pdl_wait();
-        int run = 0, rrun = 0;
+        const int SH = p.slab_head ? mx_head_experts(p) : 0;   // head mode: experts whose first tile leads
+        int run = 0, rrun = 0, srun = 0;
         if (lane == 0) {
             tile_start[0] = 0;
+            std_start[0] = 0;
             off[0] = p.slab_cnt ? 0 : p.offsets[0];
         }
         for (int e0 = 0; e0 < p.E; e0 += 32) {
@@ -664,18 +704,22 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                 slot[e] = p.expert_map ? p.expert_map[e] : e;
                 nt = (nr + BN - 1) / BN;
             }
-            int incl = nt, rincl = nr;
+            // tiles in the item order after the head ones, rows, and all tiles (the compact order)
+            int incl = e < SH ? (nt > 1 ? nt - 1 : 0) : nt, rincl = nr, sincl = nt;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, incl, d);
                 const int vr = __shfl_up_sync(0xffffffffu, rincl, d);
+                const int vs = __shfl_up_sync(0xffffffffu, sincl, d);
                 if (lane >= d) {
                     incl += v;
                     rincl += vr;
+                    sincl += vs;
                 }
             }
             if (e < p.E) {
                 tile_start[e + 1] = run + incl;
+                std_start[e + 1] = srun + sincl;
                 if (p.slab_cnt) {   // compact rows of h and y
                     off[e + 1] = rrun + rincl;
                     if (p.cprefix && blockIdx.x == 0) p.cprefix[e] = rrun + rincl - nr;
@@ -683,8 +727,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             }
             run += __shfl_sync(0xffffffffu, incl, 31);
             rrun += __shfl_sync(0xffffffffu, rincl, 31);
+            srun += __shfl_sync(0xffffffffu, sincl, 31);
         }
-        if (lane == 0) sm.total_items = run * p.m_tiles;
+        if (lane == 0) sm.total_items = (SH + run) * p.m_tiles;
     }
     tc_fence_before();
     __syncthreads();
@@ -708,8 +753,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             // The slots start empty: the weights of this pipeline's first stages go out before
             // waiting for the kernel that writes the activations. Its first item is static
             // (queue entry j0), so they stay within that item.
-            int pre = 0;
-            if (blockIdx.x + j0 * gridDim.x < total) {
+            int pre = pre_head;
+            if (!p.slab_head && blockIdx.x + j0 * gridDim.x < total) {
                 const MxItem it = mx_item(tab, p, blockIdx.x + j0 * gridDim.x, BN);
                 for (int st = st0; st < KST && pre < NSW; st += dst, ++pre) issue_weights(it, st, w * NSW + pre);
             }
@@ -947,7 +992,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                 if constexpr (PHASE == kPhaseUp) {
                     // columns 0..63: gate of channels 64 m ..; 64..127: up of the same channels. h
                     // goes out in A4 form, 16 channels (one scale block) at a time.
-                    uint8_t *blob = p.bblob_out + ((int64_t)it.rt * (p.I / kMxStageK) + ((it.m * 64) >> 8)) * BBLOB;
+                    uint8_t *blob = p.bblob_out + ((int64_t)it.rt_out * (p.I / kMxStageK) + ((it.m * 64) >> 8)) * BBLOB;
 #pragma unroll 1
                     for (int blk = 0; blk < 4; ++blk) {
                         uint32_t G[16], U[16];
@@ -1103,7 +1148,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                         // A4: h in NVFP4 form with tensor scale 1. A 16-block of channels is 16 lanes:
                         // scale E4M3(amax / 6), codes E2M1(h / scale); lane pairs share a byte.
                         const int c16 = (ch >> 5) & 7, b16 = (ch & 255) >> 4;
-                        uint8_t *blob = p.bblob_out + ((int64_t)it.rt * (p.I / kMxStageK) + (ch >> 8)) * BBLOB;
+                        uint8_t *blob = p.bblob_out + ((int64_t)it.rt_out * (p.I / kMxStageK) + (ch >> 8)) * BBLOB;
 #pragma unroll
                         for (int j = 0; j < HCH; ++j) {
                             const float g = gate ? val[j] : other[j];
@@ -1142,7 +1187,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
                         continue;
                     }
                     const int c16 = (ch >> 5) & 7;   // 32-block within the 256-wide stage
-                    uint8_t *blob = p.bblob_out + ((int64_t)it.rt * (p.I / kMxStageK) + (ch >> 8)) * BBLOB;
+                    uint8_t *blob = p.bblob_out + ((int64_t)it.rt_out * (p.I / kMxStageK) + (ch >> 8)) * BBLOB;
 #pragma unroll
                     for (int j = 0; j < HCH; ++j) {
                         const float g = gate ? val[j] : other[j];
@@ -1247,7 +1292,7 @@ size_t a4_blob_bound(int n_rows, int K, int E) {
 static size_t mx_smem_bytes(int fmt, int phase, int BN, int stages, int E, int planes) {
     const size_t stage = (size_t)bs_ablob_bytes(fmt) + bs_bblob_bytes(fmt, BN, planes);
     return 1024 + stages * stage + (phase == kPhaseUp ? 2 * 128 * kMxXch * 4 : 0) + sizeof(MxSmem) +
-           (size_t)(3 * E + 2) * sizeof(int);
+           (size_t)(4 * E + 3) * sizeof(int);
 }
 
 template <int FMT, int PHASE, int BN, int PL>
