@@ -128,7 +128,9 @@ def active_expert_bytes(idx: torch.Tensor, layer) -> int:
 
 
 class LayerBench:
-    """One layer configuration: NSETS weight copies, NSETS token batches, a graph per pair."""
+    """One layer configuration: NSETS weight copies, NSETS token batches, a graph per pair, and
+    one graph of all NSETS calls in order (consecutive layer calls in one graph, as a serving
+    engine captures a whole decode step: no graph launch between the layers)."""
 
     def __init__(self, moe, cfg: str, T: int, device, seed: int = 0, nsets: int = NSETS, act: str = "a16"):
         self.moe, self.cfg, self.T, self.dev, self.act = moe, cfg, T, device, act
@@ -178,10 +180,27 @@ class LayerBench:
             with torch.cuda.graph(g):
                 self.call(j)
             self.graphs.append(g)
+        self.seq = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.seq):
+            for j in range(len(self.sets)):
+                self.call(j)
         torch.cuda.synchronize(self.dev)
 
     def step(self, i: int):
         self.graphs[i % len(self.graphs)].replay()
+
+    def run(self, i0: int, n: int):
+        """Steps i0 .. i0 + n - 1: whole replays of the sequence graph where a block of NSETS
+        steps starts at a multiple of NSETS, single-call graphs for the rest."""
+        ns = len(self.graphs)
+        i, end = i0, i0 + n
+        while i < end:
+            if i % ns == 0 and end - i >= ns:
+                self.seq.replay()
+                i += ns
+            else:
+                self.graphs[i % ns].replay()
+                i += 1
 
     def algorithmic_bytes(self, i: int) -> int:
         """Algorithmic bytes of one layer: router weights + experts with >= 1 token + x in + out."""
@@ -195,9 +214,14 @@ class LayerBench:
         return 2.0 * self.T * s.H * s.E + self.T * self.k * 6.0 * s.H * s.I
 
 
-def time_steps(fn, K: int, W: int, device, barrier=None):
-    for i in range(W):
-        fn(i)
+def time_steps(fn, K: int, W: int, device, barrier=None, run=None):
+    """W untimed steps, then exactly K timed steps (fn(i) runs step i; run(i0, n), when
+    given, runs steps i0 .. i0 + n - 1 instead)."""
+    if run:
+        run(0, W)
+    else:
+        for i in range(W):
+            fn(i)
     torch.cuda.synchronize(device)
     if barrier:
         barrier()
@@ -205,8 +229,11 @@ def time_steps(fn, K: int, W: int, device, barrier=None):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(st)
-    for i in range(K):
-        fn(W + i)
+    if run:
+        run(W, K)
+    else:
+        for i in range(K):
+            fn(W + i)
     e1.record(st)
     torch.cuda.synchronize(device)
     if barrier:
@@ -214,16 +241,16 @@ def time_steps(fn, K: int, W: int, device, barrier=None):
     return e0.elapsed_time(e1) / 1e3
 
 
-def time_passes(fn, K: int, W: int, device, barrier, world, min_s: float = 0.5, max_passes: int = 400):
+def time_passes(fn, K: int, W: int, device, barrier, world, min_s: float = 0.5, max_passes: int = 400, run=None):
     """Timed regions of exactly K steps each (barrier + synchronise on both sides, CUDA
     events on the launching stream, max over ranks), repeated until together they span
     min_s, so the clock sampler sees the load; returns the per-pass seconds. Every rank
     runs the same number of passes (decided from the slowest rank's first pass)."""
-    first = max_over_ranks(time_steps(fn, K, W, device, barrier), world, device)
+    first = max_over_ranks(time_steps(fn, K, W, device, barrier, run), world, device)
     n = int(max(1, min(max_passes, math.ceil(min_s / max(first, 1e-9)))))
     out = [first]
     for p in range(1, n):
-        out.append(max_over_ranks(time_steps(fn, K, 0, device, barrier), world, device))
+        out.append(max_over_ranks(time_steps(fn, K, 0, device, barrier, run), world, device))
     return out
 
 
@@ -513,7 +540,7 @@ def run_ours(args, rank, world, device):
     extra = {}
     launches_per_step = lb.launches_per_call
     with ClockSampler(device) as clk:
-        passes = time_passes(lb.step, args.steps, args.warmup, device, barrier, world)
+        passes = time_passes(lb.step, args.steps, args.warmup, device, barrier, world, run=lb.run)
     clocks = clk.summary()
     sec = statistics.median(passes)
     tokens = lb.T * args.steps * world
@@ -602,7 +629,7 @@ def run_ours(args, rank, world, device):
             b = lb if (cfg == "decode" and T == 64) else LayerBench(moe, cfg, T, device, nsets=nsets, act=act)
             b.capture()
             nsteps = max(10, args.steps // 2) if T < 8192 else max(10, min(args.steps // 2, 40))
-            s = time_steps(b.step, nsteps, args.warmup, device, barrier)
+            s = time_steps(b.step, nsteps, args.warmup, device, barrier, run=b.run)
             ms_b = s / nsteps * 1e3
             n_alg = [b.algorithmic_bytes(args.warmup + i) for i in range(min(8, len(b.sets)))]
             gbs = sum(n_alg) / len(n_alg) / (ms_b * 1e-3) / 1e9
@@ -644,7 +671,8 @@ def run_ours(args, rank, world, device):
         "config": dict(HEADLINE_CONFIG, parallelism=f"replicas x{world}",
                        l2=f"{NSETS} rotating weight copies + activation batches (weights touched per step > L2)",
                        timing=f"median of {len(passes)} timed regions of exactly {args.steps} steps each "
-                              f"(repeated until they span 0.5 s)"),
+                              f"(repeated until they span 0.5 s); a CUDA graph holds {NSETS} consecutive layer "
+                              f"calls, one per weight copy, as a serving engine captures a decode step"),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clocks, "extra": extra,
     }
