@@ -332,6 +332,39 @@ def test_layer_fused_routing_and_permutation(moe, decode_layer):
     assert moe.moe_device_error() == 0
 
 
+def test_layer_consecutive_calls_in_one_graph(moe, decode_layer):
+    """Several layer calls captured in one CUDA graph, sharing one workspace (each layer's router
+    starts its weight loads while the layer before finishes): every replay gives each call's eager
+    output bit for bit: decode batches on the slot layout (T = 64 with head tiles, 37 and 1 without)
+    and off it (T = 300: separate permutation, quantiser and combine launches)."""
+    L = decode_layer.to("cuda")
+    ex = [moe.moe_prepack(moe.Experts.from_layer(L)) for _ in range(2)]
+    for T in (64, 37, 1, 300):
+        xs = [synthetic.make_tokens(T, L.H, seed=700 + 10 * T + i).cuda() for i in range(4)]
+        ws = torch.empty(moe.moe_workspace_size(T, L.H, L.I, L.E, L.k), dtype=torch.uint8, device="cuda")
+        outs = [torch.empty(T, L.H, dtype=torch.bfloat16, device="cuda") for _ in xs]
+        calls = [(xs[i], ex[i % 2], outs[i]) for i in range(len(xs))]
+        refs = []
+        for x, e, o in calls:
+            moe.moe_layer_forward(x, L.wr, L.k, e, bias=L.bias, ws=ws, out=o)
+            refs.append(o.clone())
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for x, e, o in calls:
+                moe.moe_layer_forward(x, L.wr, L.k, e, bias=L.bias, ws=ws, out=o)
+        for _ in range(3):
+            for o in outs:
+                o.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            for o, r in zip(outs, refs):
+                assert torch.equal(o, r)
+    assert moe.moe_device_error() == 0
+
+
 def test_layer_decode_mxfp4_standard_layout(moe, decode_layer):
     x = synthetic.make_tokens(64, 2048, seed=9)
     _layer_check(moe, decode_layer, x, tiled=False)
