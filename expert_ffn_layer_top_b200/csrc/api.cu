@@ -337,7 +337,8 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.slab_mt = 0;         // h is in compact tiles
     p.cprefix = nullptr;
     p.slab_wait = 0;       // the counts come from two kernels back
-    p.slab_head = 0;
+    // head tiles as in UP: the first items' weights go out before the tile prefix reads the counts
+    p.slab_head = slot && n_rows >= 4 * E;
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 

@@ -549,7 +549,7 @@ __device__ __forceinline__ MxItem mx_item(const int *tab, const MxParams &p, int
     it.row0 = beg + t * BN;
     it.nvalid = min(BN, off[lo + 1] - beg - t * BN);
     it.slot = slot[lo];
-    it.rtin = p.slab_mt ? lo * p.slab_mt + t : it.rt;
+    it.rtin = p.slab_mt ? lo * p.slab_mt + t : it.rt_out;
     return it;
 }
 
