@@ -337,8 +337,10 @@ static moe_status mx_ffn_impl(const void *x_src, int gather, const int32_t *sort
     p.slab_mt = 0;         // h is in compact tiles
     p.cprefix = nullptr;
     p.slab_wait = 0;       // the counts come from two kernels back
-    // head tiles as in UP: the first items' weights go out before the tile prefix reads the counts
-    p.slab_head = slot && n_rows >= 4 * E;
+    // no head tiles: DOWN reads the counts before its wait, so its first weights go out early
+    // anyway, and with three static items per CTA its head would span 28 experts (at decode
+    // dims one of them often without rows, whose weights it would read for nothing)
+    p.slab_head = 0;
     return launch_mx_phase(fmt, kPhaseDown, BN, p, nsm, st);
 }
 

@@ -88,8 +88,8 @@ struct MxParams {
     int slab_wait;              // slab_cnt comes from the previous kernel: read it after the wait
     // Slot layout with most experts routed to: the first tile of each of the first experts
     // (enough for every CTA's static first items) leads the item order, present even when the
-    // expert has no rows, so those items' weights go out before the tile prefix (UP: before the
-    // wait on the router). Outputs (h, y rows) and DOWN's input tiles keep the compact order.
+    // expert has no rows, so those items' weights go out before the tile prefix and the wait
+    // on the router. Outputs (h, y rows) and input tiles read by index keep the compact order.
     int slab_head;
 };
 
