@@ -752,7 +752,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_kernel(const __grid_cons
             };
             // The slots start empty: the weights of this pipeline's first stages go out before
             // waiting for the kernel that writes the activations. Its first item is static
-            // (queue entry j0), so they stay within that item.
+            // (queue entry j0), so they stay within that item. In head mode they went out
+            // already, before the tile prefix.
             int pre = pre_head;
             if (!p.slab_head && blockIdx.x + j0 * gridDim.x < total) {
                 const MxItem it = mx_item(tab, p, blockIdx.x + j0 * gridDim.x, BN);
