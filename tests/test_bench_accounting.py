@@ -51,3 +51,27 @@ def test_active_expert_bytes_count_each_used_expert_once():
     g = np.random.default_rng(0)
     idx = torch.from_numpy(np.stack([g.choice(8, 2, replace=False) for _ in range(50)]).astype(np.int32))
     assert bench.active_expert_bytes(idx, L) == len(set(idx.flatten().tolist())) * per
+
+
+class _Replay:
+    """Stands in for a CUDA graph: records the layer calls a replay would run."""
+
+    def __init__(self, log, calls):
+        self.log, self.calls = log, calls
+
+    def replay(self):
+        self.log.extend(self.calls)
+
+
+@pytest.mark.parametrize("i0,n", [(0, 20), (20, 2000), (0, 3), (5, 16), (16, 32), (7, 41)])
+def test_layer_bench_runs_exactly_the_steps_asked_for(i0, n):
+    """bench.LayerBench.run(i0, n) replays the 16-call sequence graph only where a block of 16
+    steps starts at a multiple of 16 and single-call graphs elsewhere: the layer calls it runs
+    are exactly steps i0 .. i0 + n - 1, each on weight set step % 16, in order."""
+    log = []
+    lb = bench.LayerBench.__new__(bench.LayerBench)
+    ns = bench.NSETS
+    lb.graphs = [_Replay(log, [j]) for j in range(ns)]
+    lb.seq = _Replay(log, list(range(ns)))
+    lb.run(i0, n)
+    assert log == [i % ns for i in range(i0, i0 + n)]
