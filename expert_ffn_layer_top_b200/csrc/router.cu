@@ -320,15 +320,34 @@ __global__ void __launch_bounds__(256) router_finish_kernel(const double *__rest
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
     constexpr int kPer = kMaxRouterExperts / 32;
+    // the partial sums of four slices for all of this lane's experts are loaded at once, then
+    // added in slice order (the same fp64 order as one slice at a time)
+    double sum[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) sum[i] = 0.0;
+    for (int s0 = 0; s0 < S; s0 += 4) {
+        double a[4][kPer];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int e = lane + 32 * i;
+                a[j][i] = (s0 + j < S && e < E) ? __ldg(part + ((int64_t)(s0 + j) * T + t) * E + e) : 0.0;
+            }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (s0 + j < S) {
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) sum[i] += a[j][i];
+            }
+    }
     float v[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
         v[i] = 0.0f;
         if (e < E) {
-            double sum = 0.0;
-            for (int s = 0; s < S; ++s) sum += part[((int64_t)s * T + t) * E + e];
-            float l = (float)sum;
+            float l = (float)sum[i];
             if (bias) l = l + bias[e];
             v[i] = l;
             if (logits) logits[(int64_t)t * E + e] = l;
