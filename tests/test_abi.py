@@ -13,7 +13,8 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 
 
 def _declared():
-    src = open(HEADER).read()
+    with open(HEADER) as fh:
+        src = fh.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z_0-9]*\s*\**\s*\**([a-z_][a-z_0-9]*)\s*\(", src, flags=re.M)
     return sorted(set(n for n in names if n.startswith(("moe_", "expert_cache_"))))
@@ -63,5 +64,6 @@ def test_product_package_does_not_touch_the_oracle():
     for dirpath, _, files in os.walk(pkg):
         for f in files:
             if f.endswith((".py", ".cu", ".cuh", ".h")):
-                txt = open(os.path.join(dirpath, f)).read()
+                with open(os.path.join(dirpath, f)) as fh:
+                    txt = fh.read()
                 assert "oracle" not in txt.lower().replace("oracle.", "oracle"), f
